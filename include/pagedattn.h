@@ -1,0 +1,257 @@
+/*
+ * pagedattn.h -- C ABI of the B200 paged-KV decode library (libpagedattn.so).
+ *
+ * The hot path of PagedAttention for single-query decode: a KV cache held in
+ * fixed-size physical blocks, a per-sequence block table that maps logical
+ * blocks to physical ones, the append of new tokens' K/V into their slots,
+ * the copy-on-write block copy, and the host-side block allocator that hands
+ * out slots, shares blocks and decides copies.
+ *
+ * Sources (the PagedAttention pages):
+ *   [P1] paweldubiel.com "PagedAttention" -- blocks of a fixed number of
+ *        positions; a block table gives the physical place of each logical
+ *        block; appending never moves the prefix; paging does not change the
+ *        attention result ("Text order is not a memory address").
+ *   [P2] sanketn26 "PagedAttention -- grow the allocation with the sequence" --
+ *        "Separate logical order from physical location", "Sharing needs
+ *        ownership rules" (copy-on-write), "Exercise and checkpoint" (release
+ *        on completion), "What this does not solve" (admission can fail).
+ *   [P3] mbrenndoerfer.com "Paged Attention > Summary" -- bullet 2 (block
+ *        table, one partial block per sequence), bullet 3 (K/V gathered
+ *        through the table, block at a time, online softmax), bullet 4
+ *        (copy-on-write sharing for beams).
+ *
+ * Conventions for every call:
+ *   - Returns a pa_status (0 = PA_OK).  Nothing throws across the ABI.  On an
+ *     error, pa_last_error() gives a message for the calling thread.
+ *   - Device pointers are plain CUDA device addresses owned by the caller
+ *     (e.g. allocated by PyTorch); the library allocates no device memory and
+ *     keeps no pointer after a call returns.  Host pointers are plain host
+ *     memory owned by the caller.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Device
+ *     work is enqueued on it and the call returns without synchronising;
+ *     argument checks that need no device data happen before anything is
+ *     enqueued, so an error return means nothing was launched.
+ *   - Faults found on the device (a block-table entry, slot or copy pair out
+ *     of range, a pipeline wait that timed out) never trap: the kernel skips
+ *     the access, sets a bit in the library's device error word and carries
+ *     on.  pa_device_errors() reads that word.
+ *   - All device buffers must be 16-byte aligned and contiguous in the
+ *     layouts given below.
+ *   - Supported: head_dim D in {64, 128}; block_size bs in {4, 8, 16, 32};
+ *     num_heads / num_kv_heads = G in 1..8; dtype f32, bf16, f16.  Anything
+ *     else returns PA_ERR_UNSUPPORTED.
+ */
+#ifndef PAGEDATTN_H
+#define PAGEDATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { PA_F32 = 0, PA_BF16 = 1, PA_F16 = 2 } pa_dtype;
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = -1,   /* null/unaligned pointer, bad size, bad id     */
+    PA_ERR_UNSUPPORTED = -2,   /* dtype, head_dim, block_size or G not built   */
+    PA_ERR_OUT_OF_BLOCKS = -3, /* allocator: not enough free blocks            */
+    PA_ERR_UNKNOWN_SEQ = -4,   /* allocator: no such sequence                  */
+    PA_ERR_CUDA = -5,          /* a CUDA runtime call or launch failed         */
+    PA_ERR_DEVICE_BOUNDS = -6, /* pa_device_errors(): the device word is set   */
+    PA_ERR_SEQ_TOO_LONG = -7   /* allocator: table would exceed max_blocks     */
+} pa_status;
+
+/* Device error word bits (pa_device_errors). */
+#define PA_DEVERR_TABLE 0x1u   /* block-table entry outside [0, num_blocks)   */
+#define PA_DEVERR_SEQLEN 0x2u  /* seq_len < 0, > max_seq_len or > table width */
+#define PA_DEVERR_SLOT 0x4u    /* slot >= num_blocks * block_size             */
+#define PA_DEVERR_PAIR 0x8u    /* copy pair block outside [0, num_blocks)     */
+#define PA_DEVERR_TIMEOUT 0x10u/* a pipeline wait gave up after ~2 s          */
+
+/* Message of the last failed call on this thread ("" if none). */
+const char *pa_last_error(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int pa_version(void);
+
+/*
+ * Reads (and, if `clear`, zeroes) the device error word of the current device.
+ * Synchronises the device.  Returns PA_OK when the word is 0,
+ * PA_ERR_DEVICE_BOUNDS when any bit is set (bits in *flags_out if non-NULL),
+ * PA_ERR_CUDA if the copy fails.
+ */
+int pa_device_errors(uint32_t *flags_out, int clear);
+
+/*
+ * KV append [P1 "Mechanism and details"; P2 "Separate logical order from
+ * physical location"]: writes each new token's K and V rows into its slot.
+ *   for t < num_tokens, h < num_kv_heads, with slot = slot_mapping[t] >= 0:
+ *     k_cache[slot / bs][h][slot % bs][:] = k[t][h][:]   (same for v)
+ * A negative slot skips the token.  Slots must be distinct (else which write
+ * lands is unspecified).  The copy is bitwise.
+ *   k, v          device, [num_tokens][num_kv_heads][head_dim], `dtype`
+ *   k_cache,v_cache device, [num_blocks][num_kv_heads][block_size][head_dim]
+ *   slot_mapping  device, int64 [num_tokens]
+ * A slot >= num_blocks*block_size is skipped and sets PA_DEVERR_SLOT.
+ */
+int pa_reshape_and_cache(const void *k, const void *v, void *k_cache, void *v_cache,
+                         const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                         int head_dim, int block_size, int num_blocks, int dtype, void *stream);
+
+/*
+ * Bytes of device workspace pa_decode needs for the split-context partials:
+ * 0 when max_seq_len fits one partition.  partition_size 0 means 512.
+ */
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim, int max_seq_len,
+                                int partition_size);
+
+/*
+ * Paged decode attention [P1 "Text order is not a memory address"; P3 bullet
+ * 3]: for sequence s and query head h (KV head g = h / G, G = num_heads /
+ * num_kv_heads), over its tokens t < L_s = seq_lens[s]:
+ *   pb = block_tables[s][t / bs], off = t % bs
+ *   x_t = scale * <q[s][h], k_cache[pb][g][off]>
+ *   out[s][h][:] = sum_t softmax(x)_t * v_cache[pb][g][off][:]
+ * L_s == 0 gives zeros.  The context is cut into partitions of
+ * `partition_size` tokens (512 by default) processed by separate CTAs; their
+ * (max, sum, weighted sum) partials are merged by a second kernel.
+ *   out           device, float32 [num_seqs][num_heads][head_dim]
+ *   q             device, [num_seqs][num_heads][head_dim], `dtype`
+ *   k_cache,v_cache device, [num_blocks][num_kv_heads][block_size][head_dim]
+ *   block_tables  device, int32 [num_seqs][max_blocks_per_seq]
+ *   seq_lens      device, int32 [num_seqs]; each <= max_seq_len
+ *   max_seq_len   host bound on seq_lens; sizes the grid and the workspace;
+ *                 must be <= max_blocks_per_seq * block_size
+ *   workspace     device, >= pa_decode_workspace_size(...) bytes (NULL if 0)
+ * A seq_len above max_seq_len or the table width, or a table entry outside
+ * [0, num_blocks), sets a PA_DEVERR_* bit; such a sequence's output is zero
+ * (bad length) or computed with zero rows for the bad block (bad entry).
+ */
+int pa_decode(float *out, const void *q, const void *k_cache, const void *v_cache,
+              const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
+              int num_heads, int num_kv_heads, int head_dim, int block_size,
+              int max_blocks_per_seq, int num_blocks, int max_seq_len, float scale, int dtype,
+              void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * pa_decode with two tuning knobs: partition_size (0 = 512; else a multiple
+ * of 64 in [64, 1024]) and variant (0 = automatic; 1 = the CUDA-core kernel,
+ * any dtype; 2 = the tensor-core kernel, bf16/f16 with block_size >= 8).
+ */
+int pa_decode_ex(float *out, const void *q, const void *k_cache, const void *v_cache,
+                 const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
+                 int num_heads, int num_kv_heads, int head_dim, int block_size,
+                 int max_blocks_per_seq, int num_blocks, int max_seq_len, float scale,
+                 int dtype, void *workspace, size_t workspace_bytes, int partition_size,
+                 int variant, void *stream);
+
+/*
+ * Copy-on-write block copy [P2 "Sharing needs ownership rules"; P3 bullet 4]:
+ * for each pair i, copies physical block src_dst_pairs[2i] onto block
+ * src_dst_pairs[2i+1] in both caches, all heads and positions, bitwise.
+ * Pairs act together: no destination may also be a source or repeat.
+ *   src_dst_pairs device, int64 [num_pairs][2]
+ *   block_bytes   num_kv_heads * block_size * head_dim * element size
+ * A block id outside [0, num_blocks) skips the pair and sets PA_DEVERR_PAIR.
+ */
+int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pairs, int num_pairs,
+                   size_t block_bytes, int num_blocks, void *stream);
+
+/*
+ * Measurement hook: when both events are non-NULL, the next pa_decode /
+ * pa_decode_ex calls on this thread record ev_begin (a cudaEvent_t) before
+ * their main kernel and ev_end after it, on the call's stream.  Pass NULLs
+ * to stop.
+ */
+int pa_set_profile_events(void *ev_begin, void *ev_end);
+
+/* ------------------------------------------------------------------------
+ * Host block allocator [P1 "Mechanism and details"; P2 "Separate logical
+ * order from physical location", "Sharing needs ownership rules", "Exercise
+ * and checkpoint", "What this does not solve"; P3 bullets 2 and 4].
+ * Pure host code: no CUDA call, usable without a GPU.  Not thread-safe: one
+ * handle per thread, or external locking.
+ *
+ * Policy (what the pages leave open is fixed here):
+ *   - free list: FIFO queue initialised with free_order (NULL = 0..n-1);
+ *     blocks are taken from the head and returned to the tail;
+ *   - append: a block is taken when a token lands at position p with
+ *     p % bs == 0; slot = table[p / bs] * bs + p % bs;
+ *   - copy-on-write: at the first token of an append, if the last block is
+ *     partially filled and shared (refcount > 1), the sequence takes a fresh
+ *     block (before any other block of that append), the pair (old, new) is
+ *     reported and the old block's refcount drops; the last owner writes in
+ *     place;
+ *   - fork: the child shares the parent's blocks (refcounts + 1);
+ *   - free: blocks are released in ascending logical order; a block whose
+ *     refcount reaches 0 goes to the free-list tail;
+ *   - an append needing more free blocks than exist returns
+ *     PA_ERR_OUT_OF_BLOCKS, one needing more than max_blocks_per_seq table
+ *     entries returns PA_ERR_SEQ_TOO_LONG; neither changes any state.
+ * ---------------------------------------------------------------------- */
+typedef struct pa_alloc pa_alloc;
+
+typedef struct {
+    int64_t num_blocks;
+    int64_t free_blocks;
+    int64_t used_blocks;     /* refcount > 0              */
+    int64_t shared_blocks;   /* refcount > 1              */
+    int64_t num_seqs;
+    int64_t table_entries;   /* sum of table lengths      */
+    int64_t logical_tokens;  /* sum of sequence lengths   */
+    int64_t reserved_slots;  /* used_blocks * block_size  */
+} pa_alloc_stats_t;
+
+/* max_blocks_per_seq 0 = unlimited.  free_order: host int32[num_blocks], a
+ * permutation of 0..num_blocks-1, copied; NULL = identity. */
+int pa_alloc_create(pa_alloc **out, int num_blocks, int block_size, int max_blocks_per_seq,
+                    const int32_t *free_order);
+void pa_alloc_destroy(pa_alloc *a);
+
+/* New empty sequence; PA_ERR_INVALID_ARG if the id exists. */
+int pa_seq_add(pa_alloc *a, int64_t seq_id);
+
+/* Reserves slots for the next n_tokens positions.  slots_out: host
+ * int64[n_tokens].  cow_pair_out: host int64[2] or NULL; *n_cow_out (if
+ * non-NULL) receives 0 or 1.  n_tokens == 0 does nothing. */
+int pa_seq_append(pa_alloc *a, int64_t seq_id, int n_tokens, int64_t *slots_out,
+                  int64_t *cow_pair_out, int *n_cow_out);
+
+/* Appends n_tokens[i] (all 1 if n_tokens is NULL) to seq_ids[i], in order.
+ * slots_out: host int64[sum of tokens], in order; cow_pairs_out: host
+ * int64[2*n_seqs] or NULL; *n_cow_out receives the pair count.  All or
+ * nothing: on an error every earlier append of the batch is undone. */
+int pa_batch_append(pa_alloc *a, const int64_t *seq_ids, int n_seqs, const int32_t *n_tokens,
+                    int64_t *slots_out, int64_t *cow_pairs_out, int *n_cow_out);
+
+int pa_seq_fork(pa_alloc *a, int64_t parent, int64_t child);
+int pa_seq_free(pa_alloc *a, int64_t seq_id);
+
+/* Copies up to `cap` table entries into out (host int32); *n_out = table
+ * length, *len_out = sequence length (either may be NULL). */
+int pa_seq_block_table(const pa_alloc *a, int64_t seq_id, int32_t *out, int cap, int *n_out,
+                       int64_t *len_out);
+
+/* Rows of a decode batch: tables_out host int32[n_seqs][width], entries past
+ * a table's length set to 0; seq_lens_out host int32[n_seqs].  Returns
+ * PA_ERR_SEQ_TOO_LONG if a table is longer than width. */
+int pa_block_tables(const pa_alloc *a, const int64_t *seq_ids, int n_seqs, int32_t *tables_out,
+                    int width, int32_t *seq_lens_out);
+
+int pa_alloc_stats(const pa_alloc *a, pa_alloc_stats_t *out);
+
+/* Free list from head to tail into out (host int32, up to cap); *n_out =
+ * its length. */
+int pa_alloc_free_list(const pa_alloc *a, int32_t *out, int cap, int *n_out);
+
+/* Refcount of one physical block (-1 if out of range). */
+int pa_alloc_refcount(const pa_alloc *a, int block);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* PAGEDATTN_H */

@@ -1,0 +1,300 @@
+// The C ABI of pagedattn.h for the device calls: argument checks, workspace
+// layout, kernel choice and launch.  The allocator's half of the ABI is in
+// allocator.cpp.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/pagedattn.h"
+#include "launch.h"
+#include "status.h"
+
+namespace pa {
+
+char *error_buffer() {
+    static thread_local char buf[512];
+    return buf;
+}
+
+// The device error word (one per device that loads the library).
+__device__ unsigned int g_device_error = 0;
+
+constexpr int kMaxDevices = 64;
+
+static int current_device() {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return dev;
+}
+
+static unsigned int *device_error_ptr() {
+    static std::atomic<unsigned int *> ptrs[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    unsigned int *p = ptrs[dev].load(std::memory_order_acquire);
+    if (!p) {
+        void *a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_device_error) != cudaSuccess) return nullptr;
+        p = static_cast<unsigned int *>(a);
+        ptrs[dev].store(p, std::memory_order_release);
+    }
+    return p;
+}
+
+int num_sms() {
+    static std::atomic<int> cache[kMaxDevices];
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return 148;
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
+struct ProfileEvents {
+    cudaEvent_t begin = nullptr, end = nullptr;
+};
+static thread_local ProfileEvents t_prof;
+
+static int elem_bytes(int dtype) { return dtype == PA_F32 ? 4 : 2; }
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static int cuda_fail(cudaError_t e, const char *what) {
+    return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+static int check_shape(int num_kv_heads, int head_dim, int block_size, int dtype) {
+    if (dtype != PA_F32 && dtype != PA_BF16 && dtype != PA_F16)
+        return fail(PA_ERR_UNSUPPORTED, "dtype %d not supported", dtype);
+    if (head_dim != 64 && head_dim != 128)
+        return fail(PA_ERR_UNSUPPORTED, "head_dim %d not supported (64, 128)", head_dim);
+    if (block_size != 4 && block_size != 8 && block_size != 16 && block_size != 32)
+        return fail(PA_ERR_UNSUPPORTED, "block_size %d not supported (4, 8, 16, 32)", block_size);
+    if (num_kv_heads <= 0 || num_kv_heads > 65535)
+        return fail(PA_ERR_INVALID_ARG, "num_kv_heads %d", num_kv_heads);
+    return PA_OK;
+}
+
+constexpr int kDefaultPartition = 512;
+
+static int partition_or_default(int partition_size) {
+    return partition_size == 0 ? kDefaultPartition : partition_size;
+}
+
+static int splits_for(int max_seq_len, int partition) {
+    return max_seq_len <= 0 ? 1 : (max_seq_len + partition - 1) / partition;
+}
+
+static size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Workspace: part_o [B][Hq][S][D] float, then part_ml [B][Hq][S][2] float.
+static size_t workspace_bytes_for(int num_seqs, int num_heads, int head_dim, int splits) {
+    if (splits <= 1) return 0;
+    const size_t units = (size_t)num_seqs * num_heads * splits;
+    return round256(units * head_dim * sizeof(float)) + round256(units * 2 * sizeof(float));
+}
+
+}  // namespace pa
+
+using namespace pa;
+
+extern "C" {
+
+const char *pa_last_error(void) { return error_buffer(); }
+
+int pa_version(void) { return 10000; }
+
+int pa_device_errors(uint32_t *flags_out, int clear) {
+    clear_error();
+    unsigned int v = 0;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+    e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+    if (e != cudaSuccess) return cuda_fail(e, "reading the device error word");
+    if (clear && v) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+        if (e != cudaSuccess) return cuda_fail(e, "clearing the device error word");
+    }
+    if (flags_out) *flags_out = v;
+    if (v) return fail(PA_ERR_DEVICE_BOUNDS, "device error bits 0x%x", v);
+    return PA_OK;
+}
+
+int pa_reshape_and_cache(const void *k, const void *v, void *k_cache, void *v_cache,
+                         const int64_t *slot_mapping, int num_tokens, int num_kv_heads,
+                         int head_dim, int block_size, int num_blocks, int dtype, void *stream) {
+    clear_error();
+    int rc = check_shape(num_kv_heads, head_dim, block_size, dtype);
+    if (rc) return rc;
+    if (num_tokens < 0 || num_blocks <= 0)
+        return fail(PA_ERR_INVALID_ARG, "num_tokens %d, num_blocks %d", num_tokens, num_blocks);
+    if (num_tokens == 0) return PA_OK;
+    if (!k || !v || !k_cache || !v_cache || !slot_mapping)
+        return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(k) || !aligned16(v) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(slot_mapping) & 7u))
+        return fail(PA_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+    unsigned int *err = device_error_ptr();
+    if (!err) return fail(PA_ERR_CUDA, "no CUDA device");
+    cudaError_t e = launch_reshape_and_cache(k, v, k_cache, v_cache, slot_mapping, num_tokens,
+                                             num_kv_heads, head_dim * elem_bytes(dtype),
+                                             block_size, num_blocks, err,
+                                             static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "reshape_and_cache launch");
+    return PA_OK;
+}
+
+size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim, int max_seq_len,
+                                int partition_size) {
+    const int part = partition_or_default(partition_size);
+    if (num_seqs <= 0 || num_heads <= 0 || head_dim <= 0 || part <= 0) return 0;
+    return workspace_bytes_for(num_seqs, num_heads, head_dim, splits_for(max_seq_len, part));
+}
+
+int pa_decode_ex(float *out, const void *q, const void *k_cache, const void *v_cache,
+                 const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
+                 int num_heads, int num_kv_heads, int head_dim, int block_size,
+                 int max_blocks_per_seq, int num_blocks, int max_seq_len, float scale,
+                 int dtype, void *workspace, size_t workspace_bytes, int partition_size,
+                 int variant, void *stream) {
+    clear_error();
+    int rc = check_shape(num_kv_heads, head_dim, block_size, dtype);
+    if (rc) return rc;
+    if (num_heads <= 0 || num_heads % num_kv_heads != 0)
+        return fail(PA_ERR_INVALID_ARG, "num_heads %d not a multiple of num_kv_heads %d",
+                    num_heads, num_kv_heads);
+    const int G = num_heads / num_kv_heads;
+    if (G > 8) return fail(PA_ERR_UNSUPPORTED, "GQA group %d > 8", G);
+    if (num_seqs < 0 || num_seqs > 65535)
+        return fail(PA_ERR_INVALID_ARG, "num_seqs %d outside [0, 65535]", num_seqs);
+    if (num_blocks <= 0 || max_blocks_per_seq < 0 || max_seq_len < 0)
+        return fail(PA_ERR_INVALID_ARG, "bad sizes");
+    if ((int64_t)max_seq_len > (int64_t)max_blocks_per_seq * block_size)
+        return fail(PA_ERR_INVALID_ARG, "max_seq_len %d > max_blocks_per_seq * block_size",
+                    max_seq_len);
+    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
+    const int part = partition_or_default(partition_size);
+    if (part < 64 || part > 1024 || part % 64 != 0)
+        return fail(PA_ERR_INVALID_ARG, "partition_size %d: a multiple of 64 in [64, 1024]",
+                    partition_size);
+    if (variant < 0 || variant > 2) return fail(PA_ERR_INVALID_ARG, "variant %d", variant);
+    if (variant == 2 && (dtype == PA_F32 || block_size < 8))
+        return fail(PA_ERR_UNSUPPORTED, "the tensor-core kernel takes bf16/f16, block_size >= 8");
+    if (num_seqs == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens)
+        return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+        (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+        return fail(PA_ERR_INVALID_ARG, "misaligned pointer");
+    const int splits = splits_for(max_seq_len, part);
+    const size_t need = workspace_bytes_for(num_seqs, num_heads, head_dim, splits);
+    if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+        return fail(PA_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", need,
+                    workspace ? workspace_bytes : (size_t)0);
+    unsigned int *err = device_error_ptr();
+    if (!err) return fail(PA_ERR_CUDA, "no CUDA device");
+
+    DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.out = out;
+    if (need > 0) {
+        const size_t units = (size_t)num_seqs * num_heads * splits;
+        p.part_o = static_cast<float *>(workspace);
+        p.part_ml = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                              round256(units * head_dim * sizeof(float)));
+    }
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.err = err;
+    p.num_seqs = num_seqs;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.head_dim = head_dim;
+    p.block_size = block_size;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_blocks = num_blocks;
+    p.max_seq_len = max_seq_len;
+    p.partition_size = part;
+    p.max_splits = splits;
+    p.scale_log2 = scale * 1.4426950408889634f;
+
+    // 16-bit caches with blocks of 8+ rows go to the tensor-core kernel (it
+    // needs the cache to fit 2^31 TMA rows); fp32 and block size 4 to the
+    // CUDA-core kernel.
+    const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
+    const bool tc_ok = dtype != PA_F32 && block_size >= 8 && rows + 64 < (int64_t(1) << 31);
+    if (variant == 2 && !tc_ok)
+        return fail(PA_ERR_UNSUPPORTED, "cache too large for the tensor-core kernel");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const ProfileEvents prof = t_prof;
+    cudaError_t e;
+    if (prof.begin && prof.end) {
+        e = cudaEventRecord(prof.begin, st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    }
+    if ((variant == 0 && tc_ok) || variant == 2)
+        e = launch_decode_tc(p, dtype, st);
+    else
+        e = launch_decode_simt(p, dtype, st);
+    if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+    if (prof.begin && prof.end) {
+        e = cudaEventRecord(prof.end, st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
+    }
+    e = launch_decode_reduce(p, st);
+    if (e != cudaSuccess) return cuda_fail(e, "reduce launch");
+    return PA_OK;
+}
+
+int pa_decode(float *out, const void *q, const void *k_cache, const void *v_cache,
+              const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
+              int num_heads, int num_kv_heads, int head_dim, int block_size,
+              int max_blocks_per_seq, int num_blocks, int max_seq_len, float scale, int dtype,
+              void *workspace, size_t workspace_bytes, void *stream) {
+    return pa_decode_ex(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads,
+                        num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                        max_seq_len, scale, dtype, workspace, workspace_bytes, 0, 0, stream);
+}
+
+int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pairs, int num_pairs,
+                   size_t block_bytes, int num_blocks, void *stream) {
+    clear_error();
+    if (num_pairs < 0 || num_blocks <= 0)
+        return fail(PA_ERR_INVALID_ARG, "num_pairs %d, num_blocks %d", num_pairs, num_blocks);
+    if (num_pairs == 0) return PA_OK;
+    if (!k_cache || !v_cache || !src_dst_pairs) return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+    if (block_bytes == 0 || block_bytes % 16 != 0)
+        return fail(PA_ERR_INVALID_ARG, "block_bytes %zu must be a positive multiple of 16",
+                    block_bytes);
+    if (!aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(src_dst_pairs) & 7u))
+        return fail(PA_ERR_INVALID_ARG, "misaligned pointer");
+    unsigned int *err = device_error_ptr();
+    if (!err) return fail(PA_ERR_CUDA, "no CUDA device");
+    cudaError_t e = launch_copy_blocks(k_cache, v_cache, src_dst_pairs, num_pairs, block_bytes,
+                                       num_blocks, err, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "copy_blocks launch");
+    return PA_OK;
+}
+
+int pa_set_profile_events(void *ev_begin, void *ev_end) {
+    clear_error();
+    t_prof.begin = static_cast<cudaEvent_t>(ev_begin);
+    t_prof.end = static_cast<cudaEvent_t>(ev_end);
+    return PA_OK;
+}
+
+}  // extern "C"

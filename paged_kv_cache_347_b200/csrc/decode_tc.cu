@@ -1,0 +1,428 @@
+// Tensor-core paged decode for 16-bit caches (bf16 / f16), sm_100a.
+//
+// What it computes is the attention of mbrenndoerfer.com "Paged Attention >
+// Summary", bullet 3: keys and values read through the block table one block
+// at a time, no gather into a contiguous buffer, softmax kept online.  It is a
+// memory-bound kernel: every K/V byte is read once, and the design is about
+// keeping enough bytes in flight.
+//
+// Work unit: one CTA per (split of `partition_size` tokens, KV head g,
+// sequence s); 4 consumer warps + 1 producer warp.
+//
+//  * Producer (one thread): copies the CTA's slice of the block table into
+//    shared memory, then streams the split in stages of 64 tokens.  For each
+//    physical block of a stage it issues TMA tensor loads (no multicast) of the
+//    block's K and V rows for head g -- a (block, head) run is bs*D contiguous
+//    elements in the [NB][Hkv][bs][D] cache -- as 128-byte-wide boxes with the
+//    128B swizzle, completion counted in bytes on the stage's "full" mbarrier.
+//    A stage buffer is refilled after the 4 consumer warps release it on its
+//    "empty" mbarrier.
+//
+//  * Consumers: warp w owns tokens [16w, 16w+16) of every stage.  The GQA
+//    group is a genuine dense tile, so both products run on mma.sync
+//    m16n8k16 (fp32 accumulate):
+//      S^T[16 tok x 8 heads] = K[16 x D] . Q^T[D x 8]      (A = K via ldmatrix)
+//      O^T[D x 8 heads]     += V^T[D x 16] . P^T[16 x 8]    (A = V via ldmatrix.trans)
+//    The QK accumulator fragment holds, per lane, 2 tokens x 2 heads; it is
+//    rounded to 16 bits and transposed in registers with movmatrix into the
+//    B fragment of the PV product, so P never touches shared memory.  Heads
+//    beyond G are zero rows of Q.  Each lane's O fragment covers the same 2
+//    heads as its S fragment, so the online-softmax rescale is per lane.
+//    Running max (log2 units) and the running sum stay in fp32; the sum is
+//    taken over the same 16-bit-rounded weights that enter the PV product.
+//
+//  * End: the 4 warps' (m, l, O) are merged through shared memory and the
+//    CTA writes either the normalised output (one split) or the partial for
+//    the reduce kernel.
+//
+// All pipeline waits are bounded (~2 s); a wait that gives up sets
+// PA_DEVERR_TIMEOUT and an abort flag the other warps observe, and the
+// producer waits for its own copies in flight before the CTA exits.
+#include <math.h>
+
+#include <mutex>
+
+#include "decode_common.cuh"
+
+namespace pa {
+
+namespace tc {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kStageTokens = 16 * kConsumerWarps;  // 64
+constexpr int kRowBytes = 128;                       // one swizzled box row
+constexpr int kMaxPartition = 1024;
+
+template <typename T, int D, int BS, int NS>
+struct Cfg {
+    static constexpr int kPieces = D / 64;                        // 128-byte pieces of a row
+    static constexpr int kPieceBytes = kStageTokens * kRowBytes;  // 8 KB
+    static constexpr int kKBytes = kPieces * kPieceBytes;         // K of one stage
+    static constexpr int kStageBytes = 2 * kKBytes;               // K + V
+    static constexpr int kBlocksPerStage = kStageTokens / BS;
+    static constexpr int kMaxTable = kMaxPartition / BS;
+    static constexpr int kMergeStride = D + 4;                    // floats per head row
+    static constexpr int kMergeBytes = kConsumerWarps * 8 * kMergeStride * 4;
+    static constexpr int kBarOffset = NS * kStageBytes;
+    static constexpr int kTableOffset = kBarOffset + 2 * NS * 8;
+    static constexpr int kAbortOffset = kTableOffset + kMaxTable * 4;
+    static constexpr int kMlOffset = kAbortOffset + 16;           // m, l of the merge
+    static constexpr int kSmemBytes = kMlOffset + 2 * kConsumerWarps * 8 * 4;
+    static constexpr int kDynSmem = kSmemBytes + 1024;            // room to align to 1 KB
+    static_assert(kMergeBytes <= NS * kStageBytes, "merge area reuses the stage buffers");
+    static_assert(kStageTokens % BS == 0, "block size divides a stage");
+    static_assert(sizeof(T) == 2, "16-bit caches");
+};
+
+// Waits, as a whole warp, for the phase of `bar` with parity `parity`; the
+// decision to give up is lane 0's, so the outcome is warp-uniform.
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                          int lane) {
+    uint64_t t0 = 0;
+    for (uint32_t it = 0;; ++it) {
+        const bool ok = mbar_try_wait(bar, parity);
+        if (__all_sync(0xffffffffu, ok)) return true;
+        if ((it & 63u) == 63u) {
+            int quit = 0;
+            if (lane == 0) {
+                const uint64_t now = global_timer_ns();
+                if (t0 == 0) t0 = now;
+                quit = (*abort_flag != 0) || (now - t0 > 2000000000ull);
+            }
+            if (__shfl_sync(0xffffffffu, quit, 0)) return false;
+        }
+    }
+}
+
+template <typename T, int D, int BS, int NS>
+__global__ void __launch_bounds__(kThreads) decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                                                            const __grid_constant__ CUtensorMap tmap_v,
+                                                            const DecodeParams p) {
+    using C = Cfg<T, D, BS, NS>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+    const int split = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+    const int L = checked_seq_len(p, s, split == 0 && g == 0 && threadIdx.x == 0);
+    const int nsplit = num_splits_for(L, p.partition_size);
+    if (split >= nsplit) return;  // uniform over the CTA, before any barrier
+
+    const int G = p.num_heads / p.num_kv_heads;
+    const int t0 = split * p.partition_size;
+    const int t1 = min(L, t0 + p.partition_size);
+    const int ntok = max(0, t1 - t0);
+    const int nstages = (ntok + kStageTokens - 1) / kStageTokens;
+    const int blk0 = t0 / BS;
+    const int nblk = (ntok + BS - 1) / BS;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kBarOffset);
+    const uint32_t full0 = smem_u32(bars), empty0 = smem_u32(bars + NS);
+    int32_t *table = reinterpret_cast<int32_t *>(smem + C::kTableOffset);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kAbortOffset);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NS; ++i) {
+            mbar_init(full0 + 8 * i, 1);
+            mbar_init(empty0 + 8 * i, kConsumerWarps);
+        }
+        *abort_flag = 0;
+        fence_mbarrier_init();
+    }
+    if (warp == kConsumerWarps) {
+        for (int i = lane; i < nblk; i += 32) {
+            const int b = checked_block(p, s, blk0 + i);
+            // an entry out of range reads rows past the tensor: TMA fills zeros
+            table[i] = b < 0 ? p.num_blocks : b;
+        }
+    }
+    __syncthreads();
+
+    // ------------------------------------------------------------ producer
+    if (warp == kConsumerWarps) {
+        if (lane == 0) {
+            prefetch_tensormap(&tmap_k);
+            prefetch_tensormap(&tmap_v);
+            const uint64_t policy = l2_policy_evict_first();
+            const uint32_t stage0 = smem_u32(smem);
+            int issued = 0;
+            for (int i = 0; i < nstages; ++i) {
+                const int buf = i % NS;
+                if (i >= NS && !mbar_wait_bounded(empty0 + 8 * buf, ((i / NS) - 1) & 1, abort_flag)) {
+                    raise_device_error(p.err, PA_DEVERR_TIMEOUT);
+                    *abort_flag = 1;
+                    break;
+                }
+                const int jb = i * C::kBlocksPerStage;
+                const int jn = min(C::kBlocksPerStage, nblk - jb);
+                const uint32_t full = full0 + 8 * buf;
+                mbar_arrive_expect_tx(full, (uint32_t)(jn * 2 * BS * D * (int)sizeof(T)));
+                const uint32_t kdst = stage0 + buf * C::kStageBytes;
+                const uint32_t vdst = kdst + C::kKBytes;
+                for (int j = 0; j < jn; ++j) {
+                    const int y = (table[jb + j] * p.num_kv_heads + g) * BS;
+#pragma unroll
+                    for (int pc = 0; pc < C::kPieces; ++pc) {
+                        const uint32_t off = pc * C::kPieceBytes + j * BS * kRowBytes;
+                        tma_load_2d(kdst + off, &tmap_k, pc * 64, y, full, policy);
+                        tma_load_2d(vdst + off, &tmap_v, pc * 64, y, full, policy);
+                    }
+                }
+                issued = i + 1;
+            }
+            // copies still in flight must land before the CTA may exit
+            for (int i = max(0, issued - NS); i < issued; ++i)
+                mbar_wait_bounded(full0 + 8 * (i % NS), (i / NS) & 1, nullptr);
+        }
+        return;
+    }
+
+    // ------------------------------------------------------------ consumers
+    const int gid = lane >> 2, tig = lane & 3;
+    uint32_t qb[D / 16][2];
+    {
+        const T *qrow = static_cast<const T *>(p.q) + ((int64_t)s * p.num_heads + g * G + gid) * D;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            if (gid < G) {
+                qb[kk][0] = __ldg(reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 2 * tig));
+                qb[kk][1] = __ldg(reinterpret_cast<const uint32_t *>(qrow + 16 * kk + 8 + 2 * tig));
+            } else {
+                qb[kk][0] = qb[kk][1] = 0u;
+            }
+        }
+    }
+
+    float m_run[2] = {-INFINITY, -INFINITY};
+    float l_run[2] = {0.f, 0.f};
+    float o[D / 16][4];
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.f;
+
+    // ldmatrix row addresses: rows are tokens of this warp's 16-token tile
+    const int r7 = lane & 7;
+    const int row_k = 16 * warp + r7 + ((lane >> 3) & 1) * 8;
+    const int chk_k = lane >> 4;
+    const int row_v = 16 * warp + r7 + (lane >> 4) * 8;
+    const int chk_v = (lane >> 3) & 1;
+    const float sl2 = p.scale_log2;
+    const uint32_t stage0 = smem_u32(smem);
+
+    for (int i = 0; i < nstages; ++i) {
+        const int buf = i % NS;
+        if (!warp_wait(full0 + 8 * buf, (i / NS) & 1, abort_flag, lane)) {
+            if (lane == 0) {
+                raise_device_error(p.err, PA_DEVERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+            break;
+        }
+        const int tb = t0 + i * kStageTokens + 16 * warp;
+        if (tb < t1) {
+            const uint32_t kbase = stage0 + buf * C::kStageBytes;
+            const uint32_t vbase = kbase + C::kKBytes;
+            // ---- S^T = K Q^T
+            float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const int chunk = ((kk & 3) << 1) + chk_k;
+                const uint32_t addr = kbase + (kk >> 2) * C::kPieceBytes + row_k * kRowBytes +
+                                      ((chunk ^ r7) << 4);
+                uint32_t a[4];
+                ldmatrix_x4(addr, a[0], a[1], a[2], a[3]);
+                Mma<T>::run(c, a, qb[kk][0], qb[kk][1]);
+            }
+            // ---- online softmax (log2 domain); tokens past the end -> -inf
+            const bool ok_lo = tb + gid < t1, ok_hi = tb + gid + 8 < t1;
+            const float x0 = ok_lo ? c[0] * sl2 : -INFINITY;
+            const float x1 = ok_lo ? c[1] * sl2 : -INFINITY;
+            const float x2 = ok_hi ? c[2] * sl2 : -INFINITY;
+            const float x3 = ok_hi ? c[3] * sl2 : -INFINITY;
+            float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+            }
+            const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+            const float al0 = exp2f(m_run[0] - mn0), al1 = exp2f(m_run[1] - mn1);
+            m_run[0] = mn0;
+            m_run[1] = mn1;
+            const uint32_t plo = Mma<T>::pack(exp2f(x0 - mn0), exp2f(x1 - mn1));
+            const uint32_t phi = Mma<T>::pack(exp2f(x2 - mn0), exp2f(x3 - mn1));
+            // the sum takes the same rounded weights the PV product uses
+            l_run[0] = l_run[0] * al0 + (Mma<T>::lo(plo) + Mma<T>::lo(phi));
+            l_run[1] = l_run[1] * al1 + (Mma<T>::hi(plo) + Mma<T>::hi(phi));
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) {
+                o[mt][0] *= al0;
+                o[mt][1] *= al1;
+                o[mt][2] *= al0;
+                o[mt][3] *= al1;
+            }
+            const uint32_t pb0 = movmatrix_trans(plo);  // tokens 0-7 of the tile
+            const uint32_t pb1 = movmatrix_trans(phi);  // tokens 8-15
+            // rows past the end may hold stale data: zero them so 0 * x stays 0
+            const bool tail = tb + 16 > t1;
+            uint32_t vm0 = 0xffffffffu, vm1 = 0xffffffffu;
+            if (tail) {
+                const int te = t1 - tb;
+                vm0 = (2 * tig < te ? 0x0000ffffu : 0u) | (2 * tig + 1 < te ? 0xffff0000u : 0u);
+                vm1 = (2 * tig + 8 < te ? 0x0000ffffu : 0u) | (2 * tig + 9 < te ? 0xffff0000u : 0u);
+            }
+            // ---- O^T += V^T P^T
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) {
+                const int chunk = ((mt & 3) << 1) + chk_v;
+                const uint32_t addr = vbase + (mt >> 2) * C::kPieceBytes + row_v * kRowBytes +
+                                      ((chunk ^ r7) << 4);
+                uint32_t a[4];
+                ldmatrix_x4_trans(addr, a[0], a[1], a[2], a[3]);
+                a[0] &= vm0;
+                a[1] &= vm0;
+                a[2] &= vm1;
+                a[3] &= vm1;
+                Mma<T>::run(o[mt], a, pb0, pb1);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * buf);
+    }
+
+    // ------------------------------------------------------------ merge
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+        l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
+        l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
+    }
+    named_barrier_sync(1, kConsumerWarps * 32);  // every stage buffer has been read
+    float *mo = reinterpret_cast<float *>(smem);  // [warp][8 heads][D + 4]
+    float *mml = reinterpret_cast<float *>(smem + C::kMlOffset);  // [warp][8] m, then l
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt) {
+        float *w0 = mo + (warp * 8 + 2 * tig) * C::kMergeStride + 16 * mt + gid;
+        float *w1 = w0 + C::kMergeStride;
+        w0[0] = o[mt][0];
+        w1[0] = o[mt][1];
+        w0[8] = o[mt][2];
+        w1[8] = o[mt][3];
+    }
+    if (gid == 0) {
+        mml[warp * 8 + 2 * tig] = m_run[0];
+        mml[warp * 8 + 2 * tig + 1] = m_run[1];
+        mml[kConsumerWarps * 8 + warp * 8 + 2 * tig] = l_run[0];
+        mml[kConsumerWarps * 8 + warp * 8 + 2 * tig + 1] = l_run[1];
+    }
+    named_barrier_sync(1, kConsumerWarps * 32);
+    for (int idx = threadIdx.x; idx < G * D; idx += kConsumerWarps * 32) {
+        const int h = idx / D, d = idx - (idx / D) * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, mml[w * 8 + h]);
+        float num = 0.f, den = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kConsumerWarps; ++w) {
+                const float sc = exp2f(mml[w * 8 + h] - M);
+                num = fmaf(sc, mo[(w * 8 + h) * C::kMergeStride + d], num);
+                den = fmaf(sc, mml[kConsumerWarps * 8 + w * 8 + h], den);
+            }
+        }
+        store_unit(p, s, g * G + h, split, nsplit, d, M, den, num);
+    }
+}
+
+// ------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(ptr);
+    }();
+    return fn;
+}
+
+// Rows of 128 bytes (64 elements), `box_rows` rows per box, over the cache
+// viewed as a [NB*Hkv*bs][D] matrix.
+static bool make_map(CUtensorMap *m, const void *base, int dtype, int D, int64_t rows,
+                     int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1u, 1u};
+    const CUtensorMapDataType dt =
+        dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    return enc(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <typename T, int D, int BS, int NS>
+static cudaError_t launch_tc_inst(const DecodeParams &p, const CUtensorMap &mk,
+                                  const CUtensorMap &mv, cudaStream_t stream) {
+    using C = Cfg<T, D, BS, NS>;
+    static std::once_flag once[64];
+    static cudaError_t attr_err[64];
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::call_once(once[dev], [&] {
+        attr_err[dev] = cudaFuncSetAttribute(decode_tc_kernel<T, D, BS, NS>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kDynSmem);
+    });
+    if (attr_err[dev] != cudaSuccess) return attr_err[dev];
+    const dim3 grid(p.max_splits, p.num_kv_heads, p.num_seqs);
+    decode_tc_kernel<T, D, BS, NS><<<grid, kThreads, C::kDynSmem, stream>>>(mk, mv, p);
+    return cudaGetLastError();
+}
+
+template <typename T, int D>
+static cudaError_t launch_tc_d(const DecodeParams &p, const CUtensorMap &mk,
+                               const CUtensorMap &mv, cudaStream_t stream) {
+    constexpr int NS = D == 128 ? 3 : 4;
+    switch (p.block_size) {
+    case 8: return launch_tc_inst<T, D, 8, NS>(p, mk, mv, stream);
+    case 16: return launch_tc_inst<T, D, 16, NS>(p, mk, mv, stream);
+    case 32: return launch_tc_inst<T, D, 32, NS>(p, mk, mv, stream);
+    default: return cudaErrorNotSupported;
+    }
+}
+
+}  // namespace tc
+
+cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, cudaStream_t stream) {
+    if (dtype != PA_BF16 && dtype != PA_F16) return cudaErrorNotSupported;
+    if (p.block_size < 8 || p.block_size > 32) return cudaErrorNotSupported;
+    if (p.head_dim != 64 && p.head_dim != 128) return cudaErrorNotSupported;
+    if (p.partition_size % tc::kStageTokens != 0 || p.partition_size > tc::kMaxPartition)
+        return cudaErrorNotSupported;
+    if (p.num_heads / p.num_kv_heads > 8) return cudaErrorNotSupported;
+    if (p.num_seqs == 0) return cudaSuccess;
+    const int64_t rows = (int64_t)p.num_blocks * p.num_kv_heads * p.block_size;
+    CUtensorMap mk, mv;
+    if (!tc::make_map(&mk, p.k_cache, dtype, p.head_dim, rows, p.block_size) ||
+        !tc::make_map(&mv, p.v_cache, dtype, p.head_dim, rows, p.block_size))
+        return cudaErrorInvalidValue;
+    if (dtype == PA_BF16)
+        return p.head_dim == 128 ? tc::launch_tc_d<__nv_bfloat16, 128>(p, mk, mv, stream)
+                                 : tc::launch_tc_d<__nv_bfloat16, 64>(p, mk, mv, stream);
+    return p.head_dim == 128 ? tc::launch_tc_d<__half, 128>(p, mk, mv, stream)
+                             : tc::launch_tc_d<__half, 64>(p, mk, mv, stream);
+}
+
+}  // namespace pa

@@ -1,0 +1,47 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pa {
+
+// Everything a decode kernel needs; passed by value.
+struct DecodeParams {
+    float *out;        // [B][Hq][D]
+    float *part_o;     // [B][Hq][S][D]  unnormalised partial sums (S > 1 only)
+    float *part_ml;    // [B][Hq][S][2]  (running max in log2 units, sum of weights)
+    const void *q;     // [B][Hq][D]
+    const void *k_cache, *v_cache;  // [NB][Hkv][bs][D]
+    const int32_t *block_tables;    // [B][max_blocks_per_seq]
+    const int32_t *seq_lens;        // [B]
+    unsigned int *err;              // device error word
+    int num_seqs, num_heads, num_kv_heads, head_dim, block_size;
+    int max_blocks_per_seq, num_blocks, max_seq_len;
+    int partition_size;  // tokens per split
+    int max_splits;      // S = ceil(max_seq_len / partition_size), >= 1
+    float scale_log2;    // softmax scale * log2(e)
+};
+
+int num_sms();  // SMs of the current device (cached per device)
+
+cudaError_t launch_reshape_and_cache(const void *k, const void *v, void *k_cache, void *v_cache,
+                                     const int64_t *slot_mapping, int num_tokens,
+                                     int num_kv_heads, int row_bytes, int block_size,
+                                     int num_blocks, unsigned int *err, cudaStream_t stream);
+
+cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *pairs, int num_pairs,
+                               size_t block_bytes, int num_blocks, unsigned int *err,
+                               cudaStream_t stream);
+
+// CUDA-core decode (any dtype, any supported block size).  dtype: pa_dtype.
+cudaError_t launch_decode_simt(const DecodeParams &p, int dtype, cudaStream_t stream);
+
+// Tensor-core decode (bf16/f16, block_size >= 8): TMA-staged K/V, mma.sync.
+// Returns cudaErrorNotSupported for shapes it does not cover.
+cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, cudaStream_t stream);
+
+// Merge of split partials into out; a no-op when max_splits == 1.
+cudaError_t launch_decode_reduce(const DecodeParams &p, cudaStream_t stream);
+
+}  // namespace pa

@@ -1,0 +1,303 @@
+"""Python binding of libpagedattn.so (include/pagedattn.h).
+
+Argument marshalling only: torch tensors become device pointers and sizes,
+the current CUDA stream is passed through, and a non-zero status becomes a
+``PagedAttnError`` carrying ``pa_last_error()``.  Every step of the path runs
+in the library's CUDA kernels or its C++ allocator; there is no fallback.
+If the shared library is missing this module fails to import.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, List, Optional, Sequence, Tuple
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedattn.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_347_b200.build` "
+        "(nvcc, sm_100a); there is no non-CUDA implementation")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+PA_F32, PA_BF16, PA_F16 = 0, 1, 2
+DTYPE_CODE = {torch.float32: PA_F32, torch.bfloat16: PA_BF16, torch.float16: PA_F16}
+STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID_ARG", -2: "PA_ERR_UNSUPPORTED",
+          -3: "PA_ERR_OUT_OF_BLOCKS", -4: "PA_ERR_UNKNOWN_SEQ", -5: "PA_ERR_CUDA",
+          -6: "PA_ERR_DEVICE_BOUNDS", -7: "PA_ERR_SEQ_TOO_LONG"}
+DEVERR = {0x1: "table", 0x2: "seqlen", 0x4: "slot", 0x8: "pair", 0x10: "timeout"}
+
+_c = ctypes
+_vp, _i, _i64, _sz, _f = _c.c_void_p, _c.c_int, _c.c_int64, _c.c_size_t, _c.c_float
+
+
+def _sig(name, res, *args):
+    fn = getattr(_lib, name)
+    fn.restype = res
+    fn.argtypes = list(args)
+    return fn
+
+
+class pa_alloc_stats_t(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in (
+        "num_blocks", "free_blocks", "used_blocks", "shared_blocks", "num_seqs",
+        "table_entries", "logical_tokens", "reserved_slots")]
+
+
+_sig("pa_last_error", _c.c_char_p)
+_sig("pa_version", _i)
+_sig("pa_device_errors", _i, _vp, _i)
+_sig("pa_reshape_and_cache", _i, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp)
+_sig("pa_decode_workspace_size", _sz, _i, _i, _i, _i, _i)
+_sig("pa_decode", _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i,
+     _vp, _sz, _vp)
+_sig("pa_decode_ex", _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i,
+     _vp, _sz, _i, _i, _vp)
+_sig("pa_copy_blocks", _i, _vp, _vp, _vp, _i, _sz, _i, _vp)
+_sig("pa_set_profile_events", _i, _vp, _vp)
+_sig("pa_alloc_create", _i, _c.POINTER(_vp), _i, _i, _i, _vp)
+_sig("pa_alloc_destroy", None, _vp)
+_sig("pa_seq_add", _i, _vp, _i64)
+_sig("pa_seq_append", _i, _vp, _i64, _i, _vp, _vp, _vp)
+_sig("pa_batch_append", _i, _vp, _vp, _i, _vp, _vp, _vp, _vp)
+_sig("pa_seq_fork", _i, _vp, _i64, _i64)
+_sig("pa_seq_free", _i, _vp, _i64)
+_sig("pa_seq_block_table", _i, _vp, _i64, _vp, _i, _vp, _vp)
+_sig("pa_block_tables", _i, _vp, _vp, _i, _vp, _i, _vp)
+_sig("pa_alloc_stats", _i, _vp, _c.POINTER(pa_alloc_stats_t))
+_sig("pa_alloc_free_list", _i, _vp, _vp, _i, _vp)
+_sig("pa_alloc_refcount", _i, _vp, _i)
+
+
+class PagedAttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        msg = _lib.pa_last_error().decode(errors="replace")
+        super().__init__(f"{where}: {STATUS.get(code, code)}: {msg}")
+        self.code = code
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != 0:
+        raise PagedAttnError(rc, where)
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _dev(t: torch.Tensor, name: str, dtype=None) -> int:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def version() -> int:
+    return _lib.pa_version()
+
+
+def device_errors(clear: bool = True) -> List[str]:
+    """Names of the device error bits set since the last clear (synchronises)."""
+    flags = ctypes.c_uint32(0)
+    rc = _lib.pa_device_errors(ctypes.addressof(flags), 1 if clear else 0)
+    if rc not in (0, -6):
+        _check(rc, "pa_device_errors")
+    return [n for b, n in DEVERR.items() if flags.value & b]
+
+
+def set_profile_events(begin: Optional[torch.cuda.Event], end: Optional[torch.cuda.Event]) -> None:
+    """Record `begin`/`end` around the main decode kernel of later pa_decode calls."""
+    if begin is None or end is None:
+        _check(_lib.pa_set_profile_events(None, None), "pa_set_profile_events")
+    else:
+        _check(_lib.pa_set_profile_events(begin.cuda_event, end.cuda_event),
+               "pa_set_profile_events")
+
+
+# ----------------------------------------------------------------- kernels
+def pa_reshape_and_cache(k: torch.Tensor, v: torch.Tensor, k_cache: torch.Tensor,
+                         v_cache: torch.Tensor, slot_mapping: torch.Tensor) -> None:
+    """k, v [N, Hkv, D]; caches [NB, Hkv, bs, D]; slot_mapping int64 [N]."""
+    NB, Hkv, bs, D = k_cache.shape
+    dt = DTYPE_CODE[k_cache.dtype]
+    n = slot_mapping.numel()
+    if tuple(k.shape) != (n, Hkv, D) or tuple(v.shape) != (n, Hkv, D):
+        raise ValueError(f"k/v must be [{n}, {Hkv}, {D}]")
+    if tuple(v_cache.shape) != tuple(k_cache.shape):
+        raise ValueError("k_cache and v_cache shapes differ")
+    _check(_lib.pa_reshape_and_cache(
+        _dev(k, "k", k_cache.dtype), _dev(v, "v", k_cache.dtype), _dev(k_cache, "k_cache"),
+        _dev(v_cache, "v_cache", k_cache.dtype), _dev(slot_mapping, "slot_mapping", torch.int64),
+        n, Hkv, D, bs, NB, dt, _stream(k_cache)), "pa_reshape_and_cache")
+
+
+_ws_cache: Dict[Tuple[int, int], torch.Tensor] = {}
+
+
+def decode_workspace_size(num_seqs: int, num_heads: int, head_dim: int, max_seq_len: int,
+                          partition_size: int = 0) -> int:
+    return _lib.pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_seq_len,
+                                         partition_size)
+
+
+def _workspace(device: torch.device, nbytes: int) -> torch.Tensor:
+    key = (device.index or 0, 0)
+    ws = _ws_cache.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _ws_cache[key] = ws
+    return ws
+
+
+def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+              block_tables: torch.Tensor, seq_lens: torch.Tensor, scale: float,
+              block_size: Optional[int] = None, num_kv_heads: Optional[int] = None,
+              max_seq_len: Optional[int] = None, workspace: Optional[torch.Tensor] = None,
+              partition_size: int = 0, variant: int = 0) -> torch.Tensor:
+    """out float32 [B, Hq, D] <- paged attention of q [B, Hq, D] over the caches.
+
+    max_seq_len (a host bound on seq_lens) defaults to the table width times
+    the block size.  The workspace for split partials is taken from a cached
+    device buffer unless one is given."""
+    NB, Hkv, bs, D = k_cache.shape
+    if block_size is not None and block_size != bs:
+        raise ValueError(f"block_size {block_size} != cache block size {bs}")
+    if num_kv_heads is not None and num_kv_heads != Hkv:
+        raise ValueError(f"num_kv_heads {num_kv_heads} != cache heads {Hkv}")
+    B, Hq, Dq = q.shape
+    if Dq != D or tuple(out.shape) != (B, Hq, D):
+        raise ValueError("q/out shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.numel() != B:
+        raise ValueError("block_tables must be [B, W] and seq_lens [B]")
+    W = block_tables.shape[1]
+    if max_seq_len is None:
+        max_seq_len = W * bs
+    need = decode_workspace_size(B, Hq, D, max_seq_len, partition_size)
+    if workspace is None and need:
+        workspace = _workspace(q.device, need)
+    ws_ptr = 0 if workspace is None else _dev(workspace, "workspace")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(_lib.pa_decode_ex(
+        _dev(out, "out", torch.float32), _dev(q, "q", k_cache.dtype), _dev(k_cache, "k_cache"),
+        _dev(v_cache, "v_cache", k_cache.dtype), _dev(block_tables, "block_tables", torch.int32),
+        _dev(seq_lens, "seq_lens", torch.int32), B, Hq, Hkv, D, bs, W, NB, int(max_seq_len),
+        float(scale), DTYPE_CODE[k_cache.dtype], ws_ptr, ws_bytes, int(partition_size),
+        int(variant), _stream(q)), "pa_decode")
+    return out
+
+
+def pa_copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, src_dst_pairs: torch.Tensor) -> None:
+    """src_dst_pairs int64 [n, 2] on the device."""
+    NB, Hkv, bs, D = k_cache.shape
+    n = src_dst_pairs.shape[0] if src_dst_pairs.numel() else 0
+    if n == 0:
+        return
+    block_bytes = Hkv * bs * D * k_cache.element_size()
+    _check(_lib.pa_copy_blocks(
+        _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache", k_cache.dtype),
+        _dev(src_dst_pairs, "src_dst_pairs", torch.int64), n, block_bytes, NB,
+        _stream(k_cache)), "pa_copy_blocks")
+
+
+# ----------------------------------------------------------------- allocator
+def _np_ptr(a: np.ndarray) -> int:
+    return a.ctypes.data
+
+
+class BlockAllocator:
+    """Handle on the C++ host allocator (pa_alloc_*, pa_seq_*)."""
+
+    def __init__(self, num_blocks: int, block_size: int,
+                 free_order: Optional[Sequence[int]] = None, max_blocks_per_seq: int = 0):
+        self._h = ctypes.c_void_p()
+        fo = None
+        if free_order is not None:
+            fo = np.ascontiguousarray(free_order, dtype=np.int32)
+            if fo.shape != (num_blocks,):
+                raise ValueError("free_order must have num_blocks entries")
+        _check(_lib.pa_alloc_create(ctypes.byref(self._h), num_blocks, block_size,
+                                    max_blocks_per_seq, None if fo is None else _np_ptr(fo)),
+               "pa_alloc_create")
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def __del__(self):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            _lib.pa_alloc_destroy(h)
+            self._h = ctypes.c_void_p()
+
+    def seq_add(self, seq_id: int) -> None:
+        _check(_lib.pa_seq_add(self._h, seq_id), "pa_seq_add")
+
+    def seq_append(self, seq_id: int, n: int) -> Tuple[np.ndarray, Optional[Tuple[int, int]]]:
+        slots = np.empty(max(n, 1), np.int64)
+        pair = np.empty(2, np.int64)
+        ncow = ctypes.c_int(0)
+        _check(_lib.pa_seq_append(self._h, seq_id, n, _np_ptr(slots), _np_ptr(pair),
+                                  ctypes.addressof(ncow)), "pa_seq_append")
+        return slots[:n], ((int(pair[0]), int(pair[1])) if ncow.value else None)
+
+    def batch_append(self, seq_ids: Sequence[int], n_tokens: Optional[Sequence[int]] = None,
+                     slots_out: Optional[np.ndarray] = None
+                     ) -> Tuple[np.ndarray, np.ndarray]:
+        """Returns (slots int64 [sum n], cow pairs int64 [k, 2])."""
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        nt = None if n_tokens is None else np.ascontiguousarray(n_tokens, dtype=np.int32)
+        total = ids.shape[0] if nt is None else int(nt.sum())
+        slots = slots_out if slots_out is not None else np.empty(max(total, 1), np.int64)
+        pairs = np.empty((max(ids.shape[0], 1), 2), np.int64)
+        ncow = ctypes.c_int(0)
+        _check(_lib.pa_batch_append(self._h, _np_ptr(ids), ids.shape[0],
+                                    None if nt is None else _np_ptr(nt), _np_ptr(slots),
+                                    _np_ptr(pairs), ctypes.addressof(ncow)), "pa_batch_append")
+        return slots[:total], pairs[:ncow.value]
+
+    def seq_fork(self, parent: int, child: int) -> None:
+        _check(_lib.pa_seq_fork(self._h, parent, child), "pa_seq_fork")
+
+    def seq_free(self, seq_id: int) -> None:
+        _check(_lib.pa_seq_free(self._h, seq_id), "pa_seq_free")
+
+    def seq_block_table(self, seq_id: int) -> Tuple[List[int], int]:
+        n = ctypes.c_int(0)
+        L = ctypes.c_int64(0)
+        _check(_lib.pa_seq_block_table(self._h, seq_id, None, 0, ctypes.addressof(n),
+                                       ctypes.addressof(L)), "pa_seq_block_table")
+        buf = np.empty(max(n.value, 1), np.int32)
+        _check(_lib.pa_seq_block_table(self._h, seq_id, _np_ptr(buf), n.value, None, None),
+               "pa_seq_block_table")
+        return buf[:n.value].tolist(), L.value
+
+    def block_tables(self, seq_ids: Sequence[int], width: int,
+                     tables_out: Optional[np.ndarray] = None,
+                     lens_out: Optional[np.ndarray] = None) -> Tuple[np.ndarray, np.ndarray]:
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int64)
+        tables = tables_out if tables_out is not None else np.empty((ids.shape[0], width), np.int32)
+        lens = lens_out if lens_out is not None else np.empty(ids.shape[0], np.int32)
+        _check(_lib.pa_block_tables(self._h, _np_ptr(ids), ids.shape[0], _np_ptr(tables), width,
+                                    _np_ptr(lens)), "pa_block_tables")
+        return tables, lens
+
+    def stats(self) -> dict:
+        st = pa_alloc_stats_t()
+        _check(_lib.pa_alloc_stats(self._h, ctypes.byref(st)), "pa_alloc_stats")
+        return {n: getattr(st, n) for n, _ in pa_alloc_stats_t._fields_}
+
+    def free_list(self) -> List[int]:
+        n = ctypes.c_int(0)
+        _check(_lib.pa_alloc_free_list(self._h, None, 0, ctypes.addressof(n)), "pa_alloc_free_list")
+        buf = np.empty(max(n.value, 1), np.int32)
+        _check(_lib.pa_alloc_free_list(self._h, _np_ptr(buf), n.value, None), "pa_alloc_free_list")
+        return buf[:n.value].tolist()
+
+    def refcount(self, block: int) -> int:
+        return _lib.pa_alloc_refcount(self._h, block)

@@ -1,0 +1,148 @@
+"""A decode-step driver over the C ABI: device caches plus the host allocator.
+
+A step is a list of sequence events -- ("add", sid), ("fork", parent, child),
+("free", sid), ("append", sid, n), ("decode", [sid, ...]) -- with the K/V
+rows of its appends (in op order) and the queries of its decode.  The
+runner turns a step into device actions in two phases:
+
+* ``plan``: the C++ allocator runs every event on the host.  Consecutive
+  appends become one ``write`` action (their slots and copy-on-write pairs,
+  from ``pa_batch_append``); a decode becomes a ``decode`` action carrying the
+  block-table rows and lengths of its batch.  Any other event ends a run of
+  appends, so the batched copies-then-writes of one action equal applying the
+  appends one at a time.
+* ``execute``: ``pa_copy_blocks`` (when the write has pairs), then
+  ``pa_reshape_and_cache``, and for a decode ``pa_decode``; all on the
+  current stream, nothing synchronised.
+
+``run`` does both for one step, moving the host arrays to the device on the
+way.  Planning ahead lets a caller stage a whole run of steps in device
+memory before timing it.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+from typing import List, Optional, Sequence
+
+import numpy as np
+import torch
+
+from . import pagedattn as pa
+
+
+@dataclass
+class Action:
+    kind: str                            # "write" | "decode"
+    slots: Optional[np.ndarray] = None   # int64 [n]
+    pairs: Optional[np.ndarray] = None   # int64 [k, 2]
+    row0: int = 0
+    nrows: int = 0
+    tables: Optional[np.ndarray] = None  # int32 [b, width]
+    lens: Optional[np.ndarray] = None    # int32 [b]
+    max_len: int = 0
+    dev: dict = field(default_factory=dict)
+
+
+class PagedKVRunner:
+    def __init__(self, num_blocks: int, block_size: int, num_heads: int, num_kv_heads: int,
+                 head_dim: int, dtype: torch.dtype, scale: float, table_width: int,
+                 free_order: Optional[Sequence[int]] = None, max_blocks_per_seq: int = 0,
+                 device: str = "cuda", partition_size: int = 0, variant: int = 0):
+        self.alloc = pa.BlockAllocator(num_blocks, block_size, free_order, max_blocks_per_seq)
+        self.device = torch.device(device)
+        dims = (num_blocks, num_kv_heads, block_size, head_dim)
+        self.k_cache = torch.zeros(dims, dtype=dtype, device=self.device)
+        self.v_cache = torch.zeros(dims, dtype=dtype, device=self.device)
+        self.num_heads, self.num_kv_heads, self.head_dim = num_heads, num_kv_heads, head_dim
+        self.block_size, self.num_blocks = block_size, num_blocks
+        self.dtype, self.scale, self.width = dtype, scale, table_width
+        self.partition_size, self.variant = partition_size, variant
+
+    @classmethod
+    def for_shape(cls, shape, table_width: int, **kw) -> "PagedKVRunner":
+        dt = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[shape.dtype]
+        return cls(shape.num_blocks, shape.block_size, shape.num_heads, shape.num_kv_heads,
+                   shape.head_dim, dt, shape.scale, table_width, shape.free_order, **kw)
+
+    # ------------------------------------------------------------ plan
+    def plan(self, ops) -> List[Action]:
+        acts: List[Action] = []
+        row = 0
+        i = 0
+        while i < len(ops):
+            op = ops[i]
+            kind = op[0]
+            if kind == "append":
+                ids, ns = [], []
+                while i < len(ops) and ops[i][0] == "append":
+                    ids.append(ops[i][1])
+                    ns.append(ops[i][2])
+                    i += 1
+                slots, pairs = self.alloc.batch_append(ids, ns)
+                n = int(sum(ns))
+                acts.append(Action("write", slots=slots.copy(), pairs=pairs.copy(), row0=row,
+                                   nrows=n))
+                row += n
+                continue
+            if kind == "add":
+                self.alloc.seq_add(op[1])
+            elif kind == "fork":
+                self.alloc.seq_fork(op[1], op[2])
+            elif kind == "free":
+                self.alloc.seq_free(op[1])
+            elif kind == "decode":
+                tables, lens = self.alloc.block_tables(list(op[1]), self.width)
+                acts.append(Action("decode", tables=tables, lens=lens,
+                                   max_len=int(lens.max()) if lens.size else 0))
+            else:
+                raise ValueError(f"unknown op {op!r}")
+            i += 1
+        return acts
+
+    # ------------------------------------------------------------ device side
+    def upload(self, acts: List[Action], pin: bool = False) -> None:
+        """Copy each action's host arrays to the device (async from pinned
+        memory when ``pin``)."""
+        def put(a: np.ndarray) -> torch.Tensor:
+            t = torch.from_numpy(np.ascontiguousarray(a))
+            if pin:
+                t = t.pin_memory()
+            return t.to(self.device, non_blocking=pin)
+
+        for a in acts:
+            if a.kind == "write":
+                a.dev["slots"] = put(a.slots)
+                if len(a.pairs):
+                    a.dev["pairs"] = put(a.pairs)
+            else:
+                a.dev["tables"] = put(a.tables)
+                a.dev["lens"] = put(a.lens)
+
+    def execute(self, acts: List[Action], k_new: Optional[torch.Tensor],
+                v_new: Optional[torch.Tensor], q: Optional[torch.Tensor],
+                out: Optional[torch.Tensor] = None) -> Optional[torch.Tensor]:
+        res = None
+        for a in acts:
+            if a.kind == "write":
+                if "pairs" in a.dev:
+                    pa.pa_copy_blocks(self.k_cache, self.v_cache, a.dev["pairs"])
+                if a.nrows:
+                    pa.pa_reshape_and_cache(k_new[a.row0:a.row0 + a.nrows],
+                                            v_new[a.row0:a.row0 + a.nrows], self.k_cache,
+                                            self.v_cache, a.dev["slots"])
+            else:
+                b = a.tables.shape[0]
+                o = out if out is not None else torch.empty(
+                    (b, self.num_heads, self.head_dim), dtype=torch.float32, device=self.device)
+                pa.pa_decode(o, q, self.k_cache, self.v_cache, a.dev["tables"], a.dev["lens"],
+                             self.scale, max_seq_len=a.max_len,
+                             partition_size=self.partition_size, variant=self.variant)
+                res = o
+        return res
+
+    def run(self, step) -> Optional[torch.Tensor]:
+        """Plan, upload and execute one step whose tensors may live on the host."""
+        acts = self.plan(step.ops)
+        self.upload(acts)
+        to = lambda t: None if t is None else t.to(self.device)
+        return self.execute(acts, to(step.k_new), to(step.v_new), to(step.q))

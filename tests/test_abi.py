@@ -1,0 +1,89 @@
+"""The C ABI library loads without a GPU and exports what the header declares;
+argument checks that need no device return their status codes."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+from conftest import ROOT
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "pagedattn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared()
+    for n in ("pa_reshape_and_cache", "pa_decode", "pa_copy_blocks", "pa_alloc_create",
+              "pa_seq_append", "pa_seq_fork", "pa_seq_free", "pa_last_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    lib = ctypes.CDLL(pa.LIB_PATH)
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert pa.version() >= 10000
+
+
+def test_checks_before_any_device_work():
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    L = pa._lib
+    # unsupported head_dim / block_size / dtype / GQA group
+    args = dict(out=None, q=None, kc=None, vc=None, bt=None, sl=None)
+    rc = L.pa_decode(None, None, None, None, None, None, 1, 8, 8, 96, 16, 4, 64, 64, 1.0, 1,
+                     None, 0, None)
+    assert rc == -2
+    rc = L.pa_decode(None, None, None, None, None, None, 1, 8, 8, 128, 12, 4, 64, 48, 1.0, 1,
+                     None, 0, None)
+    assert rc == -2 and b"block_size" in L.pa_last_error()
+    rc = L.pa_decode(None, None, None, None, None, None, 1, 18, 2, 128, 16, 4, 64, 64, 1.0, 1,
+                     None, 0, None)
+    assert rc == -2 and b"GQA" in L.pa_last_error()
+    rc = L.pa_decode(None, None, None, None, None, None, 1, 8, 8, 128, 16, 4, 64, 64, 1.0, 7,
+                     None, 0, None)
+    assert rc == -2
+    # max_seq_len beyond the table, bad partition, NULL pointers
+    rc = L.pa_decode(None, None, None, None, None, None, 1, 8, 8, 128, 16, 4, 64, 65, 1.0, 1,
+                     None, 0, None)
+    assert rc == -1
+    rc = L.pa_decode_ex(None, None, None, None, None, None, 1, 8, 8, 128, 16, 4, 64, 64, 1.0, 1,
+                        None, 0, 100, 0, None)
+    assert rc == -1 and b"partition" in L.pa_last_error()
+    rc = L.pa_decode(None, None, None, None, None, None, 1, 8, 8, 128, 16, 4, 64, 64, 1.0, 1,
+                     None, 0, None)
+    assert rc == -1 and b"NULL" in L.pa_last_error()
+    # the tensor-core kernel does not take fp32
+    rc = L.pa_decode_ex(None, None, None, None, None, None, 1, 8, 8, 128, 16, 4, 64, 64, 1.0, 0,
+                        None, 0, 0, 2, None)
+    assert rc == -2
+    # nothing to do is success without a device
+    assert L.pa_decode(None, None, None, None, None, None, 0, 8, 8, 128, 16, 4, 64, 64, 1.0, 1,
+                       None, 0, None) == 0
+    assert L.pa_reshape_and_cache(None, None, None, None, None, 0, 8, 128, 16, 64, 1, None) == 0
+    assert L.pa_copy_blocks(None, None, None, 0, 4096, 64, None) == 0
+    assert L.pa_copy_blocks(1, 1, 8, 1, 15, 64, None) == -1
+    assert L.pa_reshape_and_cache(None, None, None, None, None, 3, 8, 128, 16, 64, 1, None) == -1
+
+
+def test_workspace_size():
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    assert pa.decode_workspace_size(8, 64, 128, 512) == 0
+    n = pa.decode_workspace_size(8, 64, 128, 32768)
+    units = 8 * 64 * 64
+    assert n == units * 128 * 4 + units * 2 * 4
+    assert pa.decode_workspace_size(8, 64, 128, 32768, 1024) < n
+
+
+def test_python_binding_rejects_cpu_tensors():
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    kc = torch.zeros(4, 1, 16, 128, dtype=torch.bfloat16)
+    with pytest.raises(TypeError):
+        pa.pa_reshape_and_cache(torch.zeros(1, 1, 128, dtype=torch.bfloat16),
+                                torch.zeros(1, 1, 128, dtype=torch.bfloat16), kc, kc.clone(),
+                                torch.zeros(1, dtype=torch.int64))
