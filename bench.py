@@ -1,0 +1,510 @@
+#!/usr/bin/env python
+"""Benchmark of the paged decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload long32k]
+                    [--impl ours|reference]
+
+One step = one decode step of the workload through every piece of the path:
+the host allocator's slots and tables (a1), the copy-on-write block copy when
+the step has one (a2), the KV append of the new tokens (a3), the paged decode
+main kernel (a4) and the split reduce (a5).  Default workload: the
+long-context batch (8 sequences x 32768 tokens, 64/8 heads, head_dim 128,
+bf16 KV, block size 16, 512-token splits); each step appends one token per
+sequence and decodes; the last planned step decodes exactly 32768 tokens.
+
+* ``value``: KV bytes read by the decode per step (sum over sequences of
+  L_s * Hkv * D * 2 * 2 bytes) / device step time, with the step's inputs
+  (queries, new K/V rows, slots, tables, lengths) already in HBM, timed with
+  CUDA events over K steps (K cycles through up to 64 distinct planned steps;
+  re-running a planned step rewrites the same slots with the same bytes, so
+  every pass does identical work).  The KV cache (1.07 GB) is larger than
+  L2, so no flush is needed between steps.
+* ``e2e``: the same metric through the public API with host buffers: the
+  allocator runs live, inputs are copied from pinned host memory, the output
+  is read back, each step synchronised.
+* ``roofline``: the main decode kernel's algorithmic bytes per launch over
+  its own CUDA-event time (events recorded by the library around that launch
+  on the launching stream), against the measured HBM copy bandwidth.
+* ``cpu_baseline``: the fp64 oracle on the host cores on a bounded sample of
+  the same workload.
+
+``--impl reference`` times the oracle alone (the CPU arm).  With N > 1 GPUs
+(torchrun) every rank runs its own batch (a different seed) with no
+collective on the data path; times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ----------------------------------------------------------------- distributed
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    group = None
+    if ws > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=timedelta(seconds=120))
+        group = dist.group.WORLD
+    return ws, rank, local, group
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def aggregate(elapsed_s: float, units: float, ws: int, device=None):
+    """(max elapsed over ranks, sum of units over ranks)."""
+    if ws <= 1:
+        return elapsed_s, units
+    import torch.distributed as dist
+    t = torch.tensor([elapsed_s], dtype=torch.float64, device=device)
+    u = torch.tensor([units], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(u, op=dist.ReduceOp.SUM)
+    return float(t.item()), float(u.item())
+
+
+def rank_seed(base: int, rank: int) -> int:
+    return base + 1000 * rank
+
+
+# ----------------------------------------------------------------- workloads
+def make_workload(name: str, n_steps: int, seed: int):
+    if name == "long32k":
+        return workloads.long_context(seed=seed, steps=n_steps), 2048
+    if name == "llama8b":
+        return workloads.llama(seed=seed, steps=n_steps), 4096 // 16 + 1 + (n_steps + 15) // 16
+    if name.startswith("mix"):
+        bs = int(name[len("mix_bs"):]) if name.startswith("mix_bs") else 16
+        return workloads.mix(seed=seed, block_size=bs, steps=n_steps), (8192 + n_steps) // bs + 2
+    if name == "beam":
+        return workloads.beam(seed=seed, steps=n_steps), (2050 + n_steps) // 16 + 2
+    raise SystemExit(f"unknown workload {name}")
+
+
+DESCR = {
+    "long32k": "long context: B 8, Hq 64 / Hkv 8, D 128, bf16 KV, block 16, seq_len 32768, "
+               "split 512 + reduce, 32768-block pool in a seeded permutation",
+    "llama8b": "Llama-8B-shaped decode: B 32, Hq 32 / Hkv 8, D 128, bf16 KV, block 16, "
+               "seq_len U[512, 4096], 16384-block pool in a seeded permutation",
+}
+
+
+def kv_bytes(lens, hkv, d, e) -> int:
+    return int(sum(int(x) for x in lens)) * hkv * d * 2 * e
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+        self.gpu = gpu_index
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "50"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def mark(self, which):
+        setattr(self, which, time.time())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = []
+        for line in self.f.read().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                rows.append((ts, float(parts[2]), float(parts[3]), parts[5:]))
+            except ValueError:
+                continue
+        os.unlink(self.f.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        lo, hi = (self.t0 or 0) - 1, (self.t1 or 1e18) + 1
+        win = [r for r in rows if lo <= r[0] <= hi] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in win:
+            for n, v in zip(names, r[3][1:]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median([r[1] for r in win])),
+                "sm_max_mhz": float(max(r[2] for r in win)),
+                "reasons": sorted(reasons), "samples": len(win)}
+
+
+# ----------------------------------------------------------------- peaks
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured (MEASURED_PEAKS.json hbm_gbs, torch copy read+write)"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s"
+
+
+def traffic_from_profile(kernel_src: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the kernel source as it is now; else None."""
+    path = os.path.join(ROOT, "profiles", f"decode_tc_{workload}.json")
+    try:
+        with open(path) as f:
+            prof = json.load(f)
+        with open(kernel_src, "rb") as f:
+            h = hashlib.sha256(f.read()).hexdigest()[:16]
+    except (OSError, ValueError):
+        return None
+    if prof.get("kernel_src_sha256_16") != h:
+        return None
+    return prof.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------- CPU oracle
+class OracleSampler:
+    """The fp64 oracle on sequence 0 of the workload's shape (same seed):
+    state built once, then timed head by head.  A (sequence, head) pair is
+    credited 1/G of its KV head's bytes, so a whole sequence counts its KV
+    bytes once, as the device metric does."""
+
+    def __init__(self, wl_name: str, seed: int):
+        from oracle.run import OracleRun
+        from oracle import attn
+        self.attn = attn
+        if wl_name == "long32k":
+            wl = workloads.long_context(seed=seed, steps=1, batch=1)
+        else:
+            wl, _ = make_workload(wl_name, 1, seed)
+        sh = self.sh = wl.shape
+        self.orc = OracleRun(sh)
+        steps = list(wl.steps)
+        for st in steps[:-1]:
+            self.orc.step(st, decode=False)
+        self.last = steps[-1]
+        res = self.orc.step(self.last, decode=False)
+        self.bt, self.lens = res["block_tables"][:1], res["seq_lens"][:1]
+        self.L = int(self.lens[0])
+        self.G = sh.num_heads // sh.num_kv_heads
+        self.threads = attn.max_threads()
+        self.h = 0
+
+    def run(self, budget_s: float, min_pairs: int = 1):
+        sh = self.sh
+        done_bytes, done_pairs, spent = 0.0, 0, 0.0
+        while spent < budget_s or done_pairs < min_pairs:
+            chunk = [(0, (self.h + i) % sh.num_heads) for i in range(self.threads)]
+            t = time.perf_counter()
+            self.attn.paged_decode(self.last.q[:1], self.orc.k_cache, self.orc.v_cache, self.bt,
+                                   self.lens, sh.scale, sel=chunk)
+            spent += time.perf_counter() - t
+            done_pairs += len(chunk)
+            done_bytes += len(chunk) * self.L * sh.head_dim * 2 * sh.elem_bytes / self.G
+            self.h += len(chunk)
+        return done_bytes, spent, done_pairs
+
+
+# ----------------------------------------------------------------- main arm
+def run_ours(args, ws, rank, local):
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    from paged_kv_cache_347_b200.runner import PagedKVRunner
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    seed = rank_seed({"long32k": 2, "llama8b": 1}.get(args.workload, 4), rank)
+    n_plan = min(args.steps + args.warmup, 64)
+    wl, width = make_workload(args.workload, n_plan, seed)
+    sh = wl.shape
+    runner = PagedKVRunner.for_shape(sh, width, device=str(dev))
+    steps = list(wl.steps)
+    prefill, dec = steps[0], steps[1:]
+    runner.run(prefill)                                   # untimed prefill
+    torch.cuda.synchronize()
+
+    # plan every decode step (host allocator) and stage its inputs in HBM
+    plans = []
+    alloc_t = time.perf_counter()
+    for st in dec:
+        plans.append(runner.plan(st.ops))
+    alloc_us = (time.perf_counter() - alloc_t) / len(dec) * 1e6
+    for acts, st in zip(plans, dec):
+        runner.upload(acts)
+    dev_in = [(st.k_new.to(dev), st.v_new.to(dev), st.q.to(dev)) for st in dec]
+    b = dec[0].q.shape[0]
+    out = torch.empty((b, sh.num_heads, sh.head_dim), dtype=torch.float32, device=dev)
+    step_bytes = []
+    for acts in plans:
+        d = [a for a in acts if a.kind == "decode"][0]
+        step_bytes.append(kv_bytes(d.lens, sh.num_kv_heads, sh.head_dim, sh.elem_bytes))
+    launches_per = []
+    for acts in plans:
+        n = 0
+        for a in acts:
+            if a.kind == "write":
+                n += (1 if len(a.pairs) else 0) + (1 if a.nrows else 0)
+            else:
+                n += 1 + (1 if math.ceil(a.max_len / 512) > 1 else 0)
+        launches_per.append(n)
+
+    def step(i):
+        j = i % len(plans)
+        k, v, q = dev_in[j]
+        runner.execute(plans[j], k, v, q, out=out)
+
+    # warm-up (the first W planned steps, then cycling)
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    n_ev = args.steps
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
+                          if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit()
+                          else local)
+    clocks.start()
+    barrier(ws)
+    torch.cuda.synchronize()
+    clocks.mark("t0")
+    t_start.record()
+    total_bytes = 0
+    launches = 0
+    for i in range(args.steps):
+        pa.set_profile_events(ev_b[i], ev_e[i])
+        step(args.warmup + i)
+        total_bytes += step_bytes[(args.warmup + i) % len(plans)]
+        launches += launches_per[(args.warmup + i) % len(plans)]
+    pa.set_profile_events(None, None)
+    t_end.record()
+    torch.cuda.synchronize()
+    clocks.mark("t1")
+    barrier(ws)
+    clk = clocks.stop()
+    elapsed = t_start.elapsed_time(t_end) / 1e3
+    main_ms = [ev_b[i].elapsed_time(ev_e[i]) for i in range(args.steps)]
+    errs = pa.device_errors(clear=True)
+    if errs:
+        raise SystemExit(f"device errors during the bench: {errs}")
+
+    elapsed_max, bytes_all = aggregate(elapsed, float(total_bytes), ws, dev)
+    value = bytes_all / elapsed_max / 1e9
+    ms_per_step = elapsed_max / args.steps * 1e3
+
+    # roofline of the main decode kernel
+    peak, peak_src = hbm_peak()
+    d0 = [a for a in plans[0] if a.kind == "decode"][0]
+    mean_main_s = float(np.mean(main_ms)) / 1e3
+    alg = []
+    for i in range(args.steps):
+        acts = plans[(args.warmup + i) % len(plans)]
+        d = [a for a in acts if a.kind == "decode"][0]
+        nb = int(sum(-(-int(x) // sh.block_size) for x in d.lens))
+        alg.append(kv_bytes(d.lens, sh.num_kv_heads, sh.head_dim, sh.elem_bytes)
+                   + b * sh.num_heads * sh.head_dim * sh.elem_bytes + nb * 4 + b * 4)
+    alg_per_launch = float(np.mean(alg))
+    achieved = alg_per_launch / mean_main_s / 1e9
+    traffic = traffic_from_profile(os.path.join(ROOT, "paged_kv_cache_347_b200", "csrc",
+                                                "decode_tc.cu"), args.workload)
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "kernel": "pa_decode main (decode_tc_kernel)", "peak_source": peak_src,
+            "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+            "main_us_per_launch": round(mean_main_s * 1e6, 2),
+            "algorithmic_bytes_per_launch": int(alg_per_launch)}
+
+    # end to end through the public API with host buffers
+    e2e = run_e2e(args, sh, width, seed, prefill, dev, ws)
+
+    res = {
+        "metric": "paged decode attention: KV-read GB/s (% of B200 HBM peak), us/step",
+        "value": round(value, 1), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "us_per_step": round(ms_per_step * 1e3, 2),
+        "tokens_per_s": round(b * ws / (ms_per_step / 1e3), 1),
+        "frac_of_peak": round(value / peak, 4), "frac_of_nominal_8tbs": round(value / NOMINAL_HBM_GBS, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1), numpy PCG64, rounded to bf16)",
+        "config": {"workload": f"{args.workload}: {DESCR.get(args.workload, args.workload)}",
+                   "global_batch": b * ws, "seq_len": int(max(d0.lens)),
+                   "parallelism": f"dp{ws} (independent batches, no collective)",
+                   "l2": "inputs larger than L2 (KV cache 1.07 GB per step), no flush",
+                   "planned_steps": len(plans), "host_alloc_us_per_step": round(alloc_us, 2)},
+        "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
+    }
+    if rank == 0 and ws == 1 and not args.no_cpu:
+        smp = OracleSampler(args.workload, seed)
+        nb, secs, pairs = smp.run(args.cpu_budget)
+        res["cpu_baseline"] = {"value": round(nb / secs / 1e9, 4), "unit": "GB/s",
+                               "cores": smp.threads, "kind": "oracle",
+                               "sample": f"sequence 0 of the workload's shape ({smp.L} tokens), "
+                                         f"{pairs} (sequence, head) pairs, fp64 C loop, "
+                                         f"{secs:.1f} s"}
+    return res
+
+
+def run_e2e(args, sh, width, seed, prefill, dev, ws):
+    """Live steps through the public API, inputs from pinned host memory."""
+    from paged_kv_cache_347_b200.runner import PagedKVRunner
+    n = max(1, min(args.steps, args.e2e_steps))
+    w = min(args.warmup, 3)
+    wl, _ = make_workload(args.workload, n + w, seed)
+    steps = list(wl.steps)
+    r = PagedKVRunner.for_shape(sh, width, device=str(dev))
+    r.run(steps[0])
+    torch.cuda.synchronize()
+    host = [(st, st.k_new.pin_memory(), st.v_new.pin_memory(), st.q.pin_memory())
+            for st in steps[1:]]
+    b = steps[1].q.shape[0]
+    out_host = torch.empty((b, sh.num_heads, sh.head_dim), dtype=torch.float32).pin_memory()
+    h2d = d2h = 0
+    total = 0
+
+    def one(st, k, v, q):
+        nonlocal h2d, d2h, total
+        acts = r.plan(st.ops)
+        r.upload(acts, pin=True)
+        kd, vd, qd = (x.to(dev, non_blocking=True) for x in (k, v, q))
+        o = r.execute(acts, kd, vd, qd)
+        out_host.copy_(o, non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+        ab = 0
+        for a in acts:
+            ab += a.slots.nbytes + a.pairs.nbytes if a.kind == "write" else (
+                a.tables.nbytes + a.lens.nbytes)
+        d = [a for a in acts if a.kind == "decode"][0]
+        return ab + k.nbytes + v.nbytes + q.nbytes, out_host.nbytes, kv_bytes(
+            d.lens, sh.num_kv_heads, sh.head_dim, sh.elem_bytes)
+
+    for i in range(w):
+        one(*host[i])
+    barrier(ws)
+    t = time.perf_counter()
+    for i in range(n):
+        hb, db, kb = one(*host[w + i])
+        h2d += hb
+        d2h += db
+        total += kb
+    el = time.perf_counter() - t
+    el, total = aggregate(el, float(total), ws, dev)
+    return {"value": round(total / el / 1e9, 1), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d / n), "d2h_bytes_per_step": int(d2h / n),
+            "steps": n, "us_per_step": round(el / n * 1e6, 2)}
+
+
+def run_reference(args, ws, rank):
+    """The oracle as it stands on the host cores, on a bounded sample per step."""
+    if rank != 0:
+        return None
+    seed = {"long32k": 2, "llama8b": 1}.get(args.workload, 4)
+    smp = OracleSampler(args.workload, seed)
+    # calibrate, then size each step so the whole run takes about two minutes
+    _, secs1, pairs1 = smp.run(0.0)
+    per_step_budget = max(secs1, 120.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        smp.run(per_step_budget)
+    nb_all = secs_all = 0.0
+    pairs_all = 0
+    for _ in range(args.steps):
+        nb, secs, pairs = smp.run(per_step_budget)
+        nb_all += nb
+        secs_all += secs
+        pairs_all += pairs
+    v = nb_all / secs_all / 1e9
+    return {
+        "impl": "reference",
+        "metric": "paged decode attention: KV-read GB/s (% of B200 HBM peak), us/step",
+        "value": round(v, 4), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(secs_all / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1), numpy PCG64, rounded to bf16)",
+        "config": {"workload": f"{args.workload}: {DESCR.get(args.workload, args.workload)}",
+                   "global_batch": 8, "seq_len": smp.L,
+                   "parallelism": f"host cores (OpenMP, {smp.threads} threads)"},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": smp.threads,
+                         "kind": "oracle",
+                         "sample": f"per step {pairs_all / args.steps:.0f} (sequence 0, head) "
+                                   f"pairs of {smp.L} tokens, fp64 C loop"},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="long32k")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    ws, rank, local, _ = dist_setup()
+    try:
+        if args.impl == "reference":
+            res = run_reference(args, ws, rank)
+        else:
+            res = run_ours(args, ws, rank, local)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -235,7 +235,8 @@ int pa_decode_ex(float *out, const void *q, const void *k_cache, const void *v_c
     // needs the cache to fit 2^31 TMA rows); fp32 and block size 4 to the
     // CUDA-core kernel.
     const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
-    const bool tc_ok = dtype != PA_F32 && block_size >= 8 && rows + 64 < (int64_t(1) << 31);
+    const bool tc_ok = dtype != PA_F32 && block_size >= 8 &&
+                       rows + (int64_t)(num_kv_heads + 1) * block_size < (int64_t(1) << 31);
     if (variant == 2 && !tc_ok)
         return fail(PA_ERR_UNSUPPORTED, "cache too large for the tensor-core kernel");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
