@@ -96,9 +96,9 @@ def rank_seed(base: int, rank: int) -> int:
 
 
 # ----------------------------------------------------------------- workloads
-def make_workload(name: str, n_steps: int, seed: int):
+def make_workload(name: str, n_steps: int, seed: int, batch: int = 0):
     if name == "long32k":
-        return workloads.long_context(seed=seed, steps=n_steps), 2048
+        return workloads.long_context(seed=seed, steps=n_steps, batch=batch or 8), 2048
     if name == "llama8b":
         return workloads.llama(seed=seed, steps=n_steps), 4096 // 16 + 1 + (n_steps + 15) // 16
     if name.startswith("mix"):
@@ -261,7 +261,7 @@ def run_ours(args, ws, rank, local):
     torch.cuda.set_device(dev)
     seed = rank_seed({"long32k": 2, "llama8b": 1}.get(args.workload, 4), rank)
     n_plan = min(args.steps + args.warmup, 64)
-    wl, width = make_workload(args.workload, n_plan, seed)
+    wl, width = make_workload(args.workload, n_plan, seed, args.batch)
     sh = wl.shape
     runner = PagedKVRunner.for_shape(sh, width, device=str(dev))
     steps = list(wl.steps)
@@ -396,7 +396,7 @@ def run_e2e(args, sh, width, seed, prefill, dev, ws):
     from paged_kv_cache_347_b200.runner import PagedKVRunner
     n = max(1, min(args.steps, args.e2e_steps))
     w = min(args.warmup, 3)
-    wl, _ = make_workload(args.workload, n + w, seed)
+    wl, _ = make_workload(args.workload, n + w, seed, args.batch)
     steps = list(wl.steps)
     r = PagedKVRunner.for_shape(sh, width, device=str(dev))
     r.run(steps[0])
@@ -489,6 +489,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override the workload's batch (small cases for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -22,6 +22,9 @@ __global__ void __launch_bounds__(256) reshape_and_cache_kernel(
     uint4 *__restrict__ v_cache, const int64_t *__restrict__ slot_mapping, int num_tokens,
     int num_kv_heads, int words_per_row, int block_size, int64_t num_slots,
     unsigned int *err) {
+    // a decode launched after this kernel may start its prologue now; it
+    // waits for this grid's writes before reading the cache
+    pdl_launch_dependents();
     const int64_t words_per_token = (int64_t)num_kv_heads * words_per_row;
     const int64_t total = (int64_t)num_tokens * words_per_token;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;

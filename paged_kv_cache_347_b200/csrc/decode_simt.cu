@@ -153,24 +153,72 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
     }
 }
 
-// One CTA per (query head, sequence) with more than one split.
-__global__ void __launch_bounds__(128) decode_reduce_kernel(DecodeParams p) {
+// Merge of the split partials: one CTA per (query head, sequence) with more
+// than one split.  out = sum_x 2^(m_x - M) o_x / sum_x 2^(m_x - M) l_x with
+// M = max_x m_x (m in log2 units).  The partials were just written by the main
+// kernel and are read from L2; the CTA's threads split the splits between
+// them (kReduceThreads / D groups) so many loads are in flight at once.
+constexpr int kReduceThreads = 256;
+
+__global__ void __launch_bounds__(kReduceThreads) decode_reduce_kernel(DecodeParams p) {
+    // launched as a programmatic dependent of the main kernel: wait for its
+    // partials to be complete and visible
+    pdl_wait_prior_grid();
     const int h = blockIdx.x, s = blockIdx.y;
     const int L = checked_seq_len(p, s, false);
     const int nsplit = num_splits_for(L, p.partition_size);
     if (nsplit <= 1) return;
+    __shared__ float red[kReduceThreads / 32];
+    __shared__ float part[kReduceThreads];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int64_t u0 = ((int64_t)s * p.num_heads + h) * p.max_splits;
     const float *ml = p.part_ml + 2 * u0;
+
     float M = -INFINITY;
-    for (int x = 0; x < nsplit; ++x) M = fmaxf(M, ml[2 * x]);
-    for (int d = threadIdx.x; d < p.head_dim; d += blockDim.x) {
-        float num = 0.f, den = 0.f;
-        for (int x = 0; x < nsplit; ++x) {
-            const float w = exp2f(ml[2 * x] - M);
-            num = fmaf(w, p.part_o[(u0 + x) * p.head_dim + d], num);
-            den = fmaf(w, ml[2 * x + 1], den);
-        }
-        p.out[((int64_t)s * p.num_heads + h) * p.head_dim + d] = den > 0.f ? num / den : 0.f;
+    for (int x = tid; x < nsplit; x += kReduceThreads) M = fmaxf(M, __ldg(ml + 2 * x));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    if (lane == 0) red[wid] = M;
+    __syncthreads();
+    M = red[0];
+#pragma unroll
+    for (int w = 1; w < kReduceThreads / 32; ++w) M = fmaxf(M, red[w]);
+    __syncthreads();
+
+    float den = 0.f;
+    for (int x = tid; x < nsplit; x += kReduceThreads)
+        den = fmaf(exp2f(__ldg(ml + 2 * x) - M), __ldg(ml + 2 * x + 1), den);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
+    if (lane == 0) red[wid] = den;
+
+    const int D = p.head_dim;
+    const int groups = kReduceThreads / D;
+    const int grp = tid / D, d = tid - grp * D;
+    const float *po = p.part_o + u0 * D + d;
+    float num = 0.f;
+    int x = grp;
+    for (; x + 3 * groups < nsplit; x += 4 * groups) {
+        const float w0 = exp2f(__ldg(ml + 2 * x) - M);
+        const float w1 = exp2f(__ldg(ml + 2 * (x + groups)) - M);
+        const float w2 = exp2f(__ldg(ml + 2 * (x + 2 * groups)) - M);
+        const float w3 = exp2f(__ldg(ml + 2 * (x + 3 * groups)) - M);
+        const float a0 = __ldg(po + (int64_t)x * D);
+        const float a1 = __ldg(po + (int64_t)(x + groups) * D);
+        const float a2 = __ldg(po + (int64_t)(x + 2 * groups) * D);
+        const float a3 = __ldg(po + (int64_t)(x + 3 * groups) * D);
+        num = fmaf(w0, a0, fmaf(w1, a1, fmaf(w2, a2, fmaf(w3, a3, num))));
+    }
+    for (; x < nsplit; x += groups) num = fmaf(exp2f(__ldg(ml + 2 * x) - M), __ldg(po + (int64_t)x * D), num);
+    part[tid] = num;
+    __syncthreads();
+    if (tid < D) {
+        float tot = 0.f;
+        for (int gq = 0; gq < groups; ++gq) tot += part[gq * D + tid];
+        float dsum = 0.f;
+#pragma unroll
+        for (int w = 0; w < kReduceThreads / 32; ++w) dsum += red[w];
+        p.out[((int64_t)s * p.num_heads + h) * D + tid] = dsum > 0.f ? tot / dsum : 0.f;
     }
 }
 
@@ -206,8 +254,17 @@ cudaError_t launch_decode_simt(const DecodeParams &p, int dtype, cudaStream_t st
 
 cudaError_t launch_decode_reduce(const DecodeParams &p, cudaStream_t stream) {
     if (p.max_splits <= 1 || p.num_seqs == 0) return cudaSuccess;
-    decode_reduce_kernel<<<dim3(p.num_heads, p.num_seqs), 128, 0, stream>>>(p);
-    return cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.num_heads, p.num_seqs);
+    cfg.blockDim = dim3(kReduceThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, decode_reduce_kernel, p);
 }
 
 }  // namespace pa

@@ -114,10 +114,16 @@ def device_errors(clear: bool = True) -> List[str]:
 
 
 def set_profile_events(begin: Optional[torch.cuda.Event], end: Optional[torch.cuda.Event]) -> None:
-    """Record `begin`/`end` around the main decode kernel of later pa_decode calls."""
+    """Record `begin`/`end` around the main decode kernel of later pa_decode calls.
+
+    torch creates its events lazily and only lets elapsed_time() read events it
+    recorded itself, so both are recorded once here (on the current stream,
+    before any later call re-records them through the library)."""
     if begin is None or end is None:
         _check(_lib.pa_set_profile_events(None, None), "pa_set_profile_events")
     else:
+        begin.record()
+        end.record()
         _check(_lib.pa_set_profile_events(begin.cuda_event, end.cuda_event),
                "pa_set_profile_events")
 

@@ -33,7 +33,7 @@ def _rand_bits(shape, dtype, seed):
 @pytest.mark.parametrize("D,bs,Hkv", [(64, 4, 1), (128, 16, 8), (128, 32, 2), (64, 8, 3)])
 def test_reshape_and_cache_bit_exact(dtype, D, bs, Hkv):
     from paged_kv_cache_347_b200 import pagedattn as pa
-    NB, N = 37, 300
+    NB, N = 160, 300
     r = np.random.default_rng(D + bs)
     slots = r.choice(NB * bs, size=N, replace=False).astype(np.int64)
     slots[r.random(N) < 0.1] = -1
