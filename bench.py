@@ -374,7 +374,9 @@ def run_ours(args, ws, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1), numpy PCG64, rounded to bf16)",
         "config": {"workload": f"{args.workload}: {DESCR.get(args.workload, args.workload)}",
-                   "global_batch": b * ws, "seq_len": int(max(d0.lens)),
+                   "global_batch": b * ws,
+                   "seq_len": int(max(int(max(a.lens)) for acts in plans for a in acts
+                                      if a.kind == "decode")),
                    "parallelism": f"dp{ws} (independent batches, no collective)",
                    "l2": "inputs larger than L2 (KV cache 1.07 GB per step), no flush",
                    "planned_steps": len(plans), "host_alloc_us_per_step": round(alloc_us, 2)},

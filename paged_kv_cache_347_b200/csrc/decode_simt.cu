@@ -156,9 +156,12 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
 // Merge of the split partials: one CTA per (query head, sequence) with more
 // than one split.  out = sum_x 2^(m_x - M) o_x / sum_x 2^(m_x - M) l_x with
 // M = max_x m_x (m in log2 units).  The partials were just written by the main
-// kernel and are read from L2; the CTA's threads split the splits between
-// them (kReduceThreads / D groups) so many loads are in flight at once.
+// kernel and are read from L2, so the kernel is latency-bound: the weights go
+// to shared memory in one pass, then each thread owns 4 consecutive d of one
+// group of splits (kReduceThreads / (D/4) groups) and keeps its float4 loads
+// independent so they are all in flight at once.
 constexpr int kReduceThreads = 256;
+constexpr int kReduceMaxSplits = 2048;
 
 __global__ void __launch_bounds__(kReduceThreads) decode_reduce_kernel(DecodeParams p) {
     // launched as a programmatic dependent of the main kernel: wait for its
@@ -168,14 +171,20 @@ __global__ void __launch_bounds__(kReduceThreads) decode_reduce_kernel(DecodePar
     const int L = checked_seq_len(p, s, false);
     const int nsplit = num_splits_for(L, p.partition_size);
     if (nsplit <= 1) return;
+    __shared__ float w_s[kReduceMaxSplits];
     __shared__ float red[kReduceThreads / 32];
-    __shared__ float part[kReduceThreads];
+    __shared__ float4 part[kReduceThreads];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int64_t u0 = ((int64_t)s * p.num_heads + h) * p.max_splits;
-    const float *ml = p.part_ml + 2 * u0;
+    const float2 *ml = reinterpret_cast<const float2 *>(p.part_ml + 2 * u0);
 
+    // max of the split maxima
     float M = -INFINITY;
-    for (int x = tid; x < nsplit; x += kReduceThreads) M = fmaxf(M, __ldg(ml + 2 * x));
+    for (int x = tid; x < nsplit; x += kReduceThreads) {
+        const float2 v = __ldg(ml + x);
+        w_s[x] = v.x;
+        M = fmaxf(M, v.x);
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
     if (lane == 0) red[wid] = M;
@@ -184,41 +193,63 @@ __global__ void __launch_bounds__(kReduceThreads) decode_reduce_kernel(DecodePar
 #pragma unroll
     for (int w = 1; w < kReduceThreads / 32; ++w) M = fmaxf(M, red[w]);
     __syncthreads();
-
+    // weights and the denominator
     float den = 0.f;
-    for (int x = tid; x < nsplit; x += kReduceThreads)
-        den = fmaf(exp2f(__ldg(ml + 2 * x) - M), __ldg(ml + 2 * x + 1), den);
+    for (int x = tid; x < nsplit; x += kReduceThreads) {
+        const float wgt = exp2f(w_s[x] - M);
+        w_s[x] = wgt;
+        den = fmaf(wgt, __ldg(ml + x).y, den);
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
     if (lane == 0) red[wid] = den;
-
-    const int D = p.head_dim;
-    const int groups = kReduceThreads / D;
-    const int grp = tid / D, d = tid - grp * D;
-    const float *po = p.part_o + u0 * D + d;
-    float num = 0.f;
-    int x = grp;
-    for (; x + 3 * groups < nsplit; x += 4 * groups) {
-        const float w0 = exp2f(__ldg(ml + 2 * x) - M);
-        const float w1 = exp2f(__ldg(ml + 2 * (x + groups)) - M);
-        const float w2 = exp2f(__ldg(ml + 2 * (x + 2 * groups)) - M);
-        const float w3 = exp2f(__ldg(ml + 2 * (x + 3 * groups)) - M);
-        const float a0 = __ldg(po + (int64_t)x * D);
-        const float a1 = __ldg(po + (int64_t)(x + groups) * D);
-        const float a2 = __ldg(po + (int64_t)(x + 2 * groups) * D);
-        const float a3 = __ldg(po + (int64_t)(x + 3 * groups) * D);
-        num = fmaf(w0, a0, fmaf(w1, a1, fmaf(w2, a2, fmaf(w3, a3, num))));
-    }
-    for (; x < nsplit; x += groups) num = fmaf(exp2f(__ldg(ml + 2 * x) - M), __ldg(po + (int64_t)x * D), num);
-    part[tid] = num;
     __syncthreads();
-    if (tid < D) {
-        float tot = 0.f;
-        for (int gq = 0; gq < groups; ++gq) tot += part[gq * D + tid];
+
+    // numerator: thread = (group of splits, 4 consecutive d)
+    const int D4 = p.head_dim / 4;
+    const int groups = kReduceThreads / D4;
+    const int grp = tid / D4, c4 = tid - grp * D4;
+    const float4 *po = reinterpret_cast<const float4 *>(p.part_o + u0 * p.head_dim) + c4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    int x = grp;
+    for (; x + 7 * groups < nsplit; x += 8 * groups) {
+        float4 v[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) v[k] = __ldg(po + (int64_t)(x + k * groups) * D4);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float wgt = w_s[x + k * groups];
+            acc.x = fmaf(wgt, v[k].x, acc.x);
+            acc.y = fmaf(wgt, v[k].y, acc.y);
+            acc.z = fmaf(wgt, v[k].z, acc.z);
+            acc.w = fmaf(wgt, v[k].w, acc.w);
+        }
+    }
+    for (; x < nsplit; x += groups) {
+        const float4 v = __ldg(po + (int64_t)x * D4);
+        const float wgt = w_s[x];
+        acc.x = fmaf(wgt, v.x, acc.x);
+        acc.y = fmaf(wgt, v.y, acc.y);
+        acc.z = fmaf(wgt, v.z, acc.z);
+        acc.w = fmaf(wgt, v.w, acc.w);
+    }
+    part[tid] = acc;
+    __syncthreads();
+    if (tid < D4) {
+        float4 tot = part[tid];
+        for (int gq = 1; gq < groups; ++gq) {
+            const float4 v = part[gq * D4 + tid];
+            tot.x += v.x;
+            tot.y += v.y;
+            tot.z += v.z;
+            tot.w += v.w;
+        }
         float dsum = 0.f;
 #pragma unroll
         for (int w = 0; w < kReduceThreads / 32; ++w) dsum += red[w];
-        p.out[((int64_t)s * p.num_heads + h) * D + tid] = dsum > 0.f ? tot / dsum : 0.f;
+        const float inv = dsum > 0.f ? 1.f / dsum : 0.f;
+        float4 *dst = reinterpret_cast<float4 *>(p.out + ((int64_t)s * p.num_heads + h) * p.head_dim);
+        dst[tid] = make_float4(tot.x * inv, tot.y * inv, tot.z * inv, tot.w * inv);
     }
 }
 
