@@ -150,6 +150,36 @@ int pa_decode_ex(float *out, const void *q, const void *k_cache, const void *v_c
                  int variant, void *stream);
 
 /*
+ * pa_decode for callers that cannot allocate device memory.  The paper has no
+ * counterpart: this is a deployment variant of pa_decode.
+ *
+ * Some callers can't call cudaMalloc or take a caller-sized workspace: code
+ * inside a host runtime that owns every device allocation, plug-ins for which
+ * an allocation (and the synchronisation it may imply) mid-step is not
+ * allowed, or paths where an out-of-memory error cannot be handled.  This
+ * call takes the same arguments as pa_decode minus the workspace and keeps
+ * the split partials in a fixed 32 MiB array inside the library's device
+ * image (a file-scope __device__ array, held by every GPU that loads the
+ * library until the process exits).  It calls no cudaMalloc, cudaFree or
+ * other allocating routine.
+ *   - Limit: pa_decode_workspace_size(num_seqs, num_heads, head_dim,
+ *     max_seq_len, 0) must be <= 32 MiB (e.g. 8 sequences x 64 heads x 32768
+ *     tokens at head_dim 128 need 17 MB); larger requests return
+ *     PA_ERR_INVALID_ARG before anything is launched.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - Every call shares the one array and it keeps the last call's contents;
+ *     nothing in it needs to start at zero.  Calls that overlap on the GPU
+ *     (e.g. on two streams at once) race on it: serialise them.
+ * Output and device error behaviour are those of pa_decode.
+ */
+int pa_decode_static(float *out, const void *q, const void *k_cache, const void *v_cache,
+                     const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
+                     int num_heads, int num_kv_heads, int head_dim, int block_size,
+                     int max_blocks_per_seq, int num_blocks, int max_seq_len, float scale,
+                     int dtype, void *stream);
+
+/*
  * Copy-on-write block copy [P2 "Sharing needs ownership rules"; P3 bullet 4]:
  * for each pair i, copies physical block src_dst_pairs[2i] onto block
  * src_dst_pairs[2i+1] in both caches, all heads and positions, bitwise.

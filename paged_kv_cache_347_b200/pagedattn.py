@@ -59,6 +59,8 @@ _sig("pa_decode", _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, 
 _sig("pa_decode_ex", _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i,
      _vp, _sz, _i, _i, _vp)
 _sig("pa_copy_blocks", _i, _vp, _vp, _vp, _i, _sz, _i, _vp)
+_sig("pa_decode_static", _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
+     _i, _vp)
 _sig("pa_set_profile_events", _i, _vp, _vp)
 _sig("pa_alloc_create", _i, _c.POINTER(_vp), _i, _i, _i, _vp)
 _sig("pa_alloc_destroy", None, _vp)
@@ -197,6 +199,29 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
         _dev(seq_lens, "seq_lens", torch.int32), B, Hq, Hkv, D, bs, W, NB, int(max_seq_len),
         float(scale), DTYPE_CODE[k_cache.dtype], ws_ptr, ws_bytes, int(partition_size),
         int(variant), _stream(q)), "pa_decode")
+    return out
+
+
+def pa_decode_static(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,
+                     v_cache: torch.Tensor, block_tables: torch.Tensor, seq_lens: torch.Tensor,
+                     scale: float, max_seq_len: Optional[int] = None) -> torch.Tensor:
+    """pa_decode without a workspace, for callers that cannot allocate device
+    memory: the split partials live in the library's fixed 32 MiB device
+    array (shared by all calls; serialise calls that could overlap)."""
+    NB, Hkv, bs, D = k_cache.shape
+    B, Hq, Dq = q.shape
+    if Dq != D or tuple(out.shape) != (B, Hq, D):
+        raise ValueError("q/out shape mismatch")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.numel() != B:
+        raise ValueError("block_tables must be [B, W] and seq_lens [B]")
+    W = block_tables.shape[1]
+    if max_seq_len is None:
+        max_seq_len = W * bs
+    _check(_lib.pa_decode_static(
+        _dev(out, "out", torch.float32), _dev(q, "q", k_cache.dtype), _dev(k_cache, "k_cache"),
+        _dev(v_cache, "v_cache", k_cache.dtype), _dev(block_tables, "block_tables", torch.int32),
+        _dev(seq_lens, "seq_lens", torch.int32), B, Hq, Hkv, D, bs, W, NB, int(max_seq_len),
+        float(scale), DTYPE_CODE[k_cache.dtype], _stream(q)), "pa_decode_static")
     return out
 
 
