@@ -260,10 +260,10 @@ class BlockAllocator:
         self.num_blocks = num_blocks
         self.block_size = block_size
 
-    def __del__(self):
+    def __del__(self, _destroy=_lib.pa_alloc_destroy):
         h = getattr(self, "_h", None)
         if h is not None and h.value:
-            _lib.pa_alloc_destroy(h)
+            _destroy(h)
             self._h = ctypes.c_void_p()
 
     def seq_add(self, seq_id: int) -> None:

@@ -140,6 +140,65 @@ class PagedKVRunner:
                 res = o
         return res
 
+    # ------------------------------------------------------------ host-fed steps
+    def _staging(self, nbytes: int):
+        """Persistent pinned host buffer and device buffer for a step's small
+        arrays (slots, copy pairs, tables, lengths), grown on demand."""
+        cur = getattr(self, "_stage_h", None)
+        if cur is None or cur.numel() < nbytes:
+            n = max(nbytes, 1 << 20)
+            self._stage_h = torch.empty(n, dtype=torch.uint8).pin_memory()
+            self._stage_d = torch.empty(n, dtype=torch.uint8, device=self.device)
+            self._stage_ev = None
+        if self._stage_ev is not None:
+            self._stage_ev.synchronize()   # the previous step's copy has left the buffer
+        return self._stage_h, self._stage_d
+
+    def upload_packed(self, acts: List[Action]) -> int:
+        """Pack every action's host arrays into one pinned buffer and move them
+        with a single host-to-device copy; returns the bytes copied."""
+        arrays = []
+        for a in acts:
+            if a.kind == "write":
+                arrays.append((a, "slots", a.slots))
+                if len(a.pairs):
+                    arrays.append((a, "pairs", a.pairs))
+            else:
+                arrays.append((a, "tables", a.tables))
+                arrays.append((a, "lens", a.lens))
+        offs, total = [], 0
+        for _, _, arr in arrays:
+            offs.append(total)
+            total += (arr.nbytes + 15) & ~15
+        host, devb = self._staging(total)
+        hb = host.numpy()
+        for (a, name, arr), off in zip(arrays, offs):
+            hb[off:off + arr.nbytes] = np.ascontiguousarray(arr).view(np.uint8).reshape(-1)
+        if total:
+            devb[:total].copy_(host[:total], non_blocking=True)
+            self._stage_ev = torch.cuda.Event()
+            self._stage_ev.record()
+        for (a, name, arr), off in zip(arrays, offs):
+            dt = torch.int64 if arr.dtype == np.int64 else torch.int32
+            a.dev[name] = devb[off:off + arr.nbytes].view(dt).view(arr.shape)
+        return total
+
+    def run_pinned(self, ops, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,
+                   out_host: torch.Tensor) -> dict:
+        """One step fed from pinned host memory: the allocator runs on the
+        host, the step's small arrays go to the device in one copy, the new
+        K/V rows and queries in one copy each, the kernels run, and the
+        output is copied back into ``out_host`` (pinned).  Synchronises the
+        stream before returning.  Returns the bytes moved each way."""
+        acts = self.plan(ops)
+        h2d = self.upload_packed(acts)
+        dev = [t.to(self.device, non_blocking=True) for t in (k_new, v_new, q)]
+        h2d += sum(t.nbytes for t in (k_new, v_new, q))
+        o = self.execute(acts, *dev)
+        out_host.copy_(o, non_blocking=True)
+        torch.cuda.current_stream(self.device).synchronize()
+        return {"h2d": h2d, "d2h": out_host.nbytes, "acts": acts}
+
     def run(self, step) -> Optional[torch.Tensor]:
         """Plan, upload and execute one step whose tensors may live on the host."""
         acts = self.plan(step.ops)
