@@ -420,21 +420,28 @@ def run_e2e(args, sh, width, seed, prefill, dev, ws):
     h2d = d2h = 0
     total = 0
 
-    def one(ops, k, v, q):
-        res = r.run_pinned(ops, k, v, q, out_host)
-        d = [a for a in res["acts"] if a.kind == "decode"][0]
-        return res["h2d"], res["d2h"], kv_bytes(d.lens, sh.num_kv_heads, sh.head_dim,
-                                                sh.elem_bytes)
+    # the allocator work of step i+1 runs on the host while the GPU runs step
+    # i; every step still copies its inputs in and its output back before the
+    # next step's inputs go out
+    def loop(first, count):
+        nonlocal h2d, d2h, total
+        if count <= 0:
+            return
+        prep = r.prepare(host[first][0])
+        for i in range(first, first + count):
+            res = r.launch(prep, *host[i][1:], out_host)
+            prep = r.prepare(host[i + 1][0]) if i + 1 < first + count else None
+            r.wait()
+            if first >= w:
+                d = [a for a in res["acts"] if a.kind == "decode"][0]
+                h2d += res["h2d"]
+                d2h += res["d2h"]
+                total += kv_bytes(d.lens, sh.num_kv_heads, sh.head_dim, sh.elem_bytes)
 
-    for i in range(w):
-        one(*host[i])
+    loop(0, w)
     barrier(ws)
     t = time.perf_counter()
-    for i in range(n):
-        hb, db, kb = one(*host[w + i])
-        h2d += hb
-        d2h += db
-        total += kb
+    loop(w, n)
     el = time.perf_counter() - t
     el, total = aggregate(el, float(total), ws, dev)
     return {"value": round(total / el / 1e9, 1), "unit": "GB/s",

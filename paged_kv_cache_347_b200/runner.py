@@ -141,22 +141,36 @@ class PagedKVRunner:
         return res
 
     # ------------------------------------------------------------ host-fed steps
-    def _staging(self, nbytes: int):
-        """Persistent pinned host buffer and device buffer for a step's small
-        arrays (slots, copy pairs, tables, lengths), grown on demand."""
-        cur = getattr(self, "_stage_h", None)
-        if cur is None or cur.numel() < nbytes:
+    # A step fed from host memory is split in two so that the host work of the
+    # next step (allocator, packing) can run while the GPU works on this one:
+    #   prepare(ops)  -> host only: plan, pack the small arrays into one of two
+    #                    pinned staging buffers;
+    #   launch(...)   -> one copy of the packed arrays, one copy each of the new
+    #                    K/V rows and queries, the kernels, the output copied
+    #                    back into pinned memory -- all asynchronous;
+    #   wait()        -> synchronise the stream (the output is then readable).
+    def _staging(self, slot: int, nbytes: int):
+        """Pinned host / device buffer pair number ``slot`` (of 2), grown on demand."""
+        if not hasattr(self, "_stage"):
+            self._stage = [None, None]
+            self._stage_ev = [None, None]
+        cur = self._stage[slot]
+        if cur is None or cur[0].numel() < nbytes:
             n = max(nbytes, 1 << 20)
-            self._stage_h = torch.empty(n, dtype=torch.uint8).pin_memory()
-            self._stage_d = torch.empty(n, dtype=torch.uint8, device=self.device)
-            self._stage_ev = None
-        if self._stage_ev is not None:
-            self._stage_ev.synchronize()   # the previous step's copy has left the buffer
-        return self._stage_h, self._stage_d
+            if self._stage_ev[slot] is not None:
+                self._stage_ev[slot].synchronize()
+            cur = (torch.empty(n, dtype=torch.uint8).pin_memory(),
+                   torch.empty(n, dtype=torch.uint8, device=self.device))
+            self._stage[slot] = cur
+            self._stage_ev[slot] = None
+        if self._stage_ev[slot] is not None:
+            self._stage_ev[slot].synchronize()  # its previous copy has left the host buffer
+        return cur
 
-    def upload_packed(self, acts: List[Action]) -> int:
-        """Pack every action's host arrays into one pinned buffer and move them
-        with a single host-to-device copy; returns the bytes copied."""
+    def prepare(self, ops) -> dict:
+        """Host half of a step: run the allocator and pack every action's
+        arrays (slots, copy pairs, tables, lengths) into a pinned buffer."""
+        acts = self.plan(ops)
         arrays = []
         for a in acts:
             if a.kind == "write":
@@ -170,34 +184,42 @@ class PagedKVRunner:
         for _, _, arr in arrays:
             offs.append(total)
             total += (arr.nbytes + 15) & ~15
-        host, devb = self._staging(total)
+        slot = getattr(self, "_next_slot", 0)
+        self._next_slot = 1 - slot
+        host, devb = self._staging(slot, total)
         hb = host.numpy()
-        for (a, name, arr), off in zip(arrays, offs):
+        for (_, _, arr), off in zip(arrays, offs):
             hb[off:off + arr.nbytes] = np.ascontiguousarray(arr).view(np.uint8).reshape(-1)
+        return {"acts": acts, "arrays": arrays, "offs": offs, "bytes": total, "slot": slot,
+                "host": host, "dev": devb}
+
+    def launch(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,
+               out_host: torch.Tensor) -> dict:
+        """Device half of a step, all asynchronous on the current stream."""
+        total, host, devb = prep["bytes"], prep["host"], prep["dev"]
         if total:
             devb[:total].copy_(host[:total], non_blocking=True)
-            self._stage_ev = torch.cuda.Event()
-            self._stage_ev.record()
-        for (a, name, arr), off in zip(arrays, offs):
+            ev = torch.cuda.Event()
+            ev.record()
+            self._stage_ev[prep["slot"]] = ev
+        for (a, name, arr), off in zip(prep["arrays"], prep["offs"]):
             dt = torch.int64 if arr.dtype == np.int64 else torch.int32
             a.dev[name] = devb[off:off + arr.nbytes].view(dt).view(arr.shape)
-        return total
+        dev = [t.to(self.device, non_blocking=True) for t in (k_new, v_new, q)]
+        o = self.execute(prep["acts"], *dev)
+        out_host.copy_(o, non_blocking=True)
+        h2d = total + sum(t.nbytes for t in (k_new, v_new, q))
+        return {"h2d": h2d, "d2h": out_host.nbytes, "acts": prep["acts"]}
+
+    def wait(self) -> None:
+        torch.cuda.current_stream(self.device).synchronize()
 
     def run_pinned(self, ops, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,
                    out_host: torch.Tensor) -> dict:
-        """One step fed from pinned host memory: the allocator runs on the
-        host, the step's small arrays go to the device in one copy, the new
-        K/V rows and queries in one copy each, the kernels run, and the
-        output is copied back into ``out_host`` (pinned).  Synchronises the
-        stream before returning.  Returns the bytes moved each way."""
-        acts = self.plan(ops)
-        h2d = self.upload_packed(acts)
-        dev = [t.to(self.device, non_blocking=True) for t in (k_new, v_new, q)]
-        h2d += sum(t.nbytes for t in (k_new, v_new, q))
-        o = self.execute(acts, *dev)
-        out_host.copy_(o, non_blocking=True)
-        torch.cuda.current_stream(self.device).synchronize()
-        return {"h2d": h2d, "d2h": out_host.nbytes, "acts": acts}
+        """prepare + launch + wait for one step fed from pinned host memory."""
+        res = self.launch(self.prepare(ops), k_new, v_new, q, out_host)
+        self.wait()
+        return res
 
     def run(self, step) -> Optional[torch.Tensor]:
         """Plan, upload and execute one step whose tensors may live on the host."""
