@@ -264,7 +264,7 @@ def run_ours(args, ws, rank, local):
     n_plan = min(args.steps + args.warmup, 64)
     wl, width = make_workload(args.workload, n_plan, seed, args.batch)
     sh = wl.shape
-    runner = PagedKVRunner.for_shape(sh, width, device=str(dev))
+    runner = PagedKVRunner.for_shape(sh, width, device=str(dev), partition_size=args.partition)
     steps = list(wl.steps)
     prefill, dec = steps[0], steps[1:]
     runner.run(prefill)                                   # untimed prefill
@@ -292,7 +292,7 @@ def run_ours(args, ws, rank, local):
             if a.kind == "write":
                 n += (1 if len(a.pairs) else 0) + (1 if a.nrows else 0)
             else:
-                n += 1 + (1 if math.ceil(a.max_len / 512) > 1 else 0)
+                n += 1 + (1 if math.ceil(a.max_len / (args.partition or 512)) > 1 else 0)
         launches_per.append(n)
 
     def step(i):
@@ -387,7 +387,8 @@ def run_ours(args, ws, rank, local):
                                       if a.kind == "decode")),
                    "parallelism": f"dp{ws} (independent batches, no collective)",
                    "l2": "inputs larger than L2 (KV cache 1.07 GB per step), no flush",
-                   "planned_steps": len(plans), "host_alloc_us_per_step": round(alloc_us, 2)},
+                   "planned_steps": len(plans), "host_alloc_us_per_step": round(alloc_us, 2),
+                   "partition_tokens": args.partition or 512},
         "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
     }
     if rank == 0 and ws == 1 and not args.no_cpu:
@@ -410,7 +411,7 @@ def run_e2e(args, sh, width, seed, prefill, dev, ws):
     w = min(args.warmup, 3)
     wl, _ = make_workload(args.workload, n + w, seed, args.batch)
     steps = list(wl.steps)
-    r = PagedKVRunner.for_shape(sh, width, device=str(dev))
+    r = PagedKVRunner.for_shape(sh, width, device=str(dev), partition_size=args.partition)
     r.run(steps[0])
     torch.cuda.synchronize()
     host = [(st.ops, st.k_new.pin_memory(), st.v_new.pin_memory(), st.q.pin_memory())
@@ -498,6 +499,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--partition", type=int, default=0,
+                    help="split length in tokens (0: the library default, 512)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (small cases for profiling)")
     args = ap.parse_args()
