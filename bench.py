@@ -269,6 +269,11 @@ def run_ours(args, ws, rank, local):
     prefill, dec = steps[0], steps[1:]
     runner.run(prefill)                                   # untimed prefill
     torch.cuda.synchronize()
+    ast = runner.alloc.stats()
+    alloc_info = {"block_size": sh.block_size, "used_blocks": ast["used_blocks"],
+                  "reserved_slots": ast["reserved_slots"], "logical_tokens": ast["logical_tokens"],
+                  "tail_waste_frac": round(1 - ast["logical_tokens"] / max(1, ast["reserved_slots"]),
+                                           5)}
 
     # plan every decode step (host allocator) and stage its inputs in HBM
     plans = []
@@ -388,7 +393,7 @@ def run_ours(args, ws, rank, local):
                    "parallelism": f"dp{ws} (independent batches, no collective)",
                    "l2": "inputs larger than L2 (KV cache 1.07 GB per step), no flush",
                    "planned_steps": len(plans), "host_alloc_us_per_step": round(alloc_us, 2),
-                   "partition_tokens": args.partition or 512},
+                   "partition_tokens": args.partition or 512, "allocator_after_prefill": alloc_info},
         "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
     }
     if rank == 0 and ws == 1 and not args.no_cpu:

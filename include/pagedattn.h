@@ -38,7 +38,7 @@
  *     on.  pa_device_errors() reads that word.
  *   - All device buffers must be 16-byte aligned and contiguous in the
  *     layouts given below.
- *   - Supported: head_dim D in {64, 128}; block_size bs in {4, 8, 16, 32};
+ *   - Supported: head_dim D in {64, 128}; block_size bs in {4, 8, 16, 32, 64};
  *     num_heads / num_kv_heads = G in 1..8; dtype f32, bf16, f16.  Anything
  *     else returns PA_ERR_UNSUPPORTED.
  */

@@ -76,8 +76,10 @@ static int check_shape(int num_kv_heads, int head_dim, int block_size, int dtype
         return fail(PA_ERR_UNSUPPORTED, "dtype %d not supported", dtype);
     if (head_dim != 64 && head_dim != 128)
         return fail(PA_ERR_UNSUPPORTED, "head_dim %d not supported (64, 128)", head_dim);
-    if (block_size != 4 && block_size != 8 && block_size != 16 && block_size != 32)
-        return fail(PA_ERR_UNSUPPORTED, "block_size %d not supported (4, 8, 16, 32)", block_size);
+    if (block_size != 4 && block_size != 8 && block_size != 16 && block_size != 32 &&
+        block_size != 64)
+        return fail(PA_ERR_UNSUPPORTED, "block_size %d not supported (4, 8, 16, 32, 64)",
+                    block_size);
     if (num_kv_heads <= 0 || num_kv_heads > 65535)
         return fail(PA_ERR_INVALID_ARG, "num_kv_heads %d", num_kv_heads);
     return PA_OK;

@@ -436,6 +436,8 @@ static cudaError_t launch_tc_d(const DecodeParams &p, const CUtensorMap &mk,
     case 8: return launch_tc_inst<T, D, 8, W, NS>(p, mk, mv, stream);
     case 16: return launch_tc_inst<T, D, 16, W, NS>(p, mk, mv, stream);
     case 32: return launch_tc_inst<T, D, 32, W, NS>(p, mk, mv, stream);
+    // a 64-token block fills a 4-warp stage (64 KB at D = 128: 3 CTAs per SM)
+    case 64: return launch_tc_inst<T, D, 64, 4, D == 128 ? 2 : 4>(p, mk, mv, stream);
     default: return cudaErrorNotSupported;
     }
 }
@@ -444,7 +446,7 @@ static cudaError_t launch_tc_d(const DecodeParams &p, const CUtensorMap &mk,
 
 cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, cudaStream_t stream) {
     if (dtype != PA_BF16 && dtype != PA_F16) return cudaErrorNotSupported;
-    if (p.block_size < 8 || p.block_size > 32) return cudaErrorNotSupported;
+    if (p.block_size < 8 || p.block_size > 64) return cudaErrorNotSupported;
     if (p.head_dim != 64 && p.head_dim != 128) return cudaErrorNotSupported;
     if (p.partition_size % 64 != 0 || p.partition_size > tc::kMaxPartition)
         return cudaErrorNotSupported;

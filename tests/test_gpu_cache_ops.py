@@ -30,7 +30,8 @@ def _rand_bits(shape, dtype, seed):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
-@pytest.mark.parametrize("D,bs,Hkv", [(64, 4, 1), (128, 16, 8), (128, 32, 2), (64, 8, 3)])
+@pytest.mark.parametrize("D,bs,Hkv", [(64, 4, 1), (128, 16, 8), (128, 32, 2), (64, 8, 3),
+                                      (128, 64, 2)])
 def test_reshape_and_cache_bit_exact(dtype, D, bs, Hkv):
     from paged_kv_cache_347_b200 import pagedattn as pa
     NB, N = 160, 300

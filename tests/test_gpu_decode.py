@@ -104,7 +104,7 @@ def test_beam_cow_and_decode():
     assert st["used_blocks"] == 4 * (128 + 4 * 1) == orc.alloc.stats()["used_blocks"]
 
 
-@pytest.mark.parametrize("bs", [8, 16, 32])
+@pytest.mark.parametrize("bs", [8, 16, 32, 64])
 def test_mix_reduced(bs):
     wl = workloads.mix(block_size=bs, steps=4, batch=24, hi=1500, pool_slots=65536)
     errs, _, _ = run_parity(wl, table_width=1600 // bs + 2)
@@ -145,7 +145,9 @@ def test_placement_permutation_gives_bit_identical_outputs():
 @pytest.mark.parametrize("dtype,G,D,bs", [("bf16", 1, 128, 16), ("bf16", 3, 64, 8),
                                           ("f16", 8, 64, 32), ("f32", 4, 128, 16),
                                           ("f32", 8, 64, 8), ("bf16", 5, 128, 4),
-                                          ("f16", 2, 128, 8), ("f32", 1, 64, 32)])
+                                          ("f16", 2, 128, 8), ("f32", 1, 64, 32),
+                                          ("bf16", 4, 128, 64), ("f16", 8, 64, 64),
+                                          ("f32", 2, 64, 64)])
 def test_shapes_and_ragged_lengths(dtype, G, D, bs):
     lens = [0, 1, 15, 16, 17, 63, 64, 65, 127, 511, 512, 513, 1100]
     wl = workloads.custom(f"ragged", lens, 2 * G, 2, D, dtype, bs, 4096 // bs * 4, seed=5,
