@@ -192,6 +192,21 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pairs, i
                    size_t block_bytes, int num_blocks, void *stream);
 
 /*
+ * Block copy between two caches of the same block shape [P2 "What this does
+ * not solve": preemption; the swap of a sequence's blocks]: for each pair i,
+ * block src_dst_pairs[2i] of (src_k, src_v) is copied onto block
+ * src_dst_pairs[2i+1] of (dst_k, dst_v), bitwise.  Each cache may be device
+ * memory or page-locked host memory (pinned with cudaHostAlloc /
+ * cudaHostRegister and mapped: the kernel reads or writes it over the bus);
+ * src_dst_pairs likewise.  Any other host pointer returns PA_ERR_INVALID_ARG.
+ * A block id outside [0, num_src_blocks) / [0, num_dst_blocks) skips the pair
+ * and sets PA_DEVERR_PAIR.
+ */
+int pa_swap_blocks(void *dst_k, void *dst_v, const void *src_k, const void *src_v,
+                   const int64_t *src_dst_pairs, int num_pairs, size_t block_bytes,
+                   int num_src_blocks, int num_dst_blocks, void *stream);
+
+/*
  * Measurement hook: when both events are non-NULL, the next pa_decode /
  * pa_decode_ex calls on this thread record ev_begin (a cudaEvent_t) before
  * their main kernel and ev_end after it, on the call's stream.  Pass NULLs
@@ -234,6 +249,13 @@ typedef struct {
     int64_t table_entries;   /* sum of table lengths      */
     int64_t logical_tokens;  /* sum of sequence lengths   */
     int64_t reserved_slots;  /* used_blocks * block_size  */
+    int64_t cached_blocks;        /* full blocks in the prefix index       */
+    int64_t prefix_hit_blocks;    /* blocks reused by pa_seq_add_cached    */
+    int64_t prefix_query_blocks;  /* full blocks looked up by it           */
+    int64_t evicted_blocks;       /* indexed blocks handed out again       */
+    int64_t host_blocks;          /* host pool size (pa_alloc_set_host_pool) */
+    int64_t host_free_blocks;
+    int64_t swapped_seqs;
 } pa_alloc_stats_t;
 
 /* max_blocks_per_seq 0 = unlimited.  free_order: host int32[num_blocks], a
@@ -280,6 +302,62 @@ int pa_alloc_free_list(const pa_alloc *a, int32_t *out, int cap, int *n_out);
 
 /* Refcount of one physical block (-1 if out of range). */
 int pa_alloc_refcount(const pa_alloc *a, int block);
+
+/* ------------------------------------------------------------------------
+ * Prefix caching [P1 "Text order is not a memory address", last paragraph:
+ * block sharing is useful for prefix caching; P2 "Use a runtime that owns the
+ * blocks": prefix reuse inside a paged runtime].
+ *
+ * A full block whose token ids are known is indexed by (the physical block
+ * holding the preceding tokens, or -1 for the first block; its bs token ids).
+ * Matching is exact (no hash collisions).  A block enters the index when an
+ * append by pa_seq_append_tokens fills it, unless an identical block is
+ * indexed already.  Released blocks stay indexed while they wait in the free
+ * list; taking a block from the free list for new use drops it from the
+ * index ("evicted").  A prefix match on a block in the free list takes it
+ * out of the free list (wherever it is) and gives it refcount 1.
+ * ---------------------------------------------------------------------- */
+
+/* New sequence whose first n_tokens token ids are token_ids: shares the
+ * longest chain of indexed full blocks matching its leading tokens (at most
+ * n_tokens / bs blocks) and starts with that many tokens in place;
+ * *n_cached_out = matched blocks * bs.  The caller appends the rest with
+ * pa_seq_append_tokens (and writes their K/V).  Never allocates, never fails
+ * for lack of blocks. */
+int pa_seq_add_cached(pa_alloc *a, int64_t seq_id, const int64_t *token_ids, int n_tokens,
+                      int *n_cached_out);
+
+/* pa_seq_append for a sequence made by pa_seq_add_cached (or forked from
+ * one): same slots and copy-on-write rule, and every block the append fills
+ * enters the prefix index.  PA_ERR_INVALID_ARG for other sequences.  (A plain
+ * pa_seq_append on such a sequence ends its token history.) */
+int pa_seq_append_tokens(pa_alloc *a, int64_t seq_id, const int64_t *token_ids, int n_tokens,
+                         int64_t *slots_out, int64_t *cow_pair_out, int *n_cow_out);
+
+/* ------------------------------------------------------------------------
+ * Preemption by swap [P2 "What this does not solve": excess admission can
+ * cause preemption; P3 bullet 5].  A pool of host blocks (same block shape)
+ * with its own FIFO free list (identity order).  Swapping a sequence out
+ * moves every block of its table to a host block, in logical order, and
+ * releases the device blocks (a block shared with another sequence keeps its
+ * other owners); swapping in takes fresh device blocks from the free list.
+ * Swapped-out sequences can only be swapped in or freed.  The data moves with
+ * pa_swap_blocks, using the returned pairs; run the swap-out copy before any
+ * later write can reuse the released device blocks (same stream).
+ * ---------------------------------------------------------------------- */
+
+/* Sets the host pool size (host blocks 0..n-1, all free).  Fails while a
+ * sequence is swapped out. */
+int pa_alloc_set_host_pool(pa_alloc *a, int num_host_blocks);
+
+/* pairs_out: host int64[cap][2] of (device block, host block), one per table
+ * entry in logical order; PA_ERR_OUT_OF_BLOCKS (no change) when the host
+ * pool is short. */
+int pa_seq_swap_out(pa_alloc *a, int64_t seq_id, int64_t *pairs_out, int cap, int *n_pairs_out);
+
+/* pairs_out: host int64[cap][2] of (host block, device block); PA_ERR_OUT_OF_
+ * BLOCKS (no change) when the device free list is short. */
+int pa_seq_swap_in(pa_alloc *a, int64_t seq_id, int64_t *pairs_out, int cap, int *n_pairs_out);
 
 #ifdef __cplusplus
 }

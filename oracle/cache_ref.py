@@ -52,3 +52,16 @@ def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor,
     v_src = v_cache[src].clone()
     k_cache[dst] = k_src
     v_cache[dst] = v_src
+
+
+def copy_between(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor,
+                 src_v: torch.Tensor, pairs: Iterable[Tuple[int, int]]) -> None:
+    """Swap copy: block a of the source caches onto block b of the
+    destination caches for each (a, b), bitwise."""
+    pairs = [(int(a), int(b)) for a, b in pairs]
+    if not pairs:
+        return
+    src = torch.tensor([a for a, _ in pairs], dtype=torch.int64)
+    dst = torch.tensor([b for _, b in pairs], dtype=torch.int64)
+    dst_k[dst] = src_k[src]
+    dst_v[dst] = src_v[src]

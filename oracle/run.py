@@ -54,9 +54,19 @@ class OracleRun:
                 self.alloc.fork(op[1], op[2])
             elif kind == "free":
                 self.alloc.free_seq(op[1])
-            elif kind == "append":
-                sid, n = op[1], op[2]
-                slots, pair = self.alloc.append(sid, n)
+            elif kind in ("append", "append_tokens", "admit"):
+                sid = op[1]
+                if kind == "append":
+                    n = op[2]
+                    slots, pair = self.alloc.append(sid, n)
+                elif kind == "append_tokens":
+                    n = len(op[2])
+                    slots, pair = self.alloc.append_tokens(sid, op[2])
+                else:
+                    n = len(op[2])
+                    c = self.alloc.add_cached(sid, op[2])
+                    slots, pair = self.alloc.append_tokens(sid, op[2][c:])
+                    slots = [-1] * c + list(slots)   # cached rows are not written
                 res["slots"] += slots
                 if pair is not None:
                     res["pairs"].append(pair)
@@ -66,6 +76,24 @@ class OracleRun:
                     cache_ref.reshape_and_cache(st.k_new[row:row + n], st.v_new[row:row + n],
                                                 self.k_cache, self.v_cache, slots)
                 row += n
+            elif kind == "host_pool":
+                self.alloc.set_host_pool(op[1])
+                if self.keep_cache:
+                    dims = (max(op[1], 1),) + tuple(self.k_cache.shape[1:])
+                    self.k_host = torch.zeros(dims, dtype=self.k_cache.dtype)
+                    self.v_host = torch.zeros(dims, dtype=self.k_cache.dtype)
+            elif kind == "swap_out":
+                pairs = self.alloc.swap_out(op[1])
+                res.setdefault("swaps", []).append(("out", pairs))
+                if self.keep_cache:
+                    cache_ref.copy_between(self.k_host, self.v_host, self.k_cache, self.v_cache,
+                                           pairs)
+            elif kind == "swap_in":
+                pairs = self.alloc.swap_in(op[1])
+                res.setdefault("swaps", []).append(("in", pairs))
+                if self.keep_cache:
+                    cache_ref.copy_between(self.k_cache, self.v_cache, self.k_host, self.v_host,
+                                           pairs)
             elif kind == "decode":
                 sids = list(op[1])
                 bt, lens = self.tables(sids)

@@ -296,6 +296,57 @@ int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pairs, i
     return PA_OK;
 }
 
+// Device-usable address of a device or page-locked (mapped) host pointer;
+// nullptr for memory the GPU cannot reach.
+static const void *device_view(const void *p) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();  // clear the sticky-free error of an unknown pointer
+        return nullptr;
+    }
+    switch (at.type) {
+    case cudaMemoryTypeDevice:
+    case cudaMemoryTypeManaged: return p;
+    case cudaMemoryTypeHost: return at.devicePointer;
+    default: return nullptr;
+    }
+}
+
+int pa_swap_blocks(void *dst_k, void *dst_v, const void *src_k, const void *src_v,
+                   const int64_t *src_dst_pairs, int num_pairs, size_t block_bytes,
+                   int num_src_blocks, int num_dst_blocks, void *stream) {
+    clear_error();
+    if (num_pairs < 0 || num_src_blocks <= 0 || num_dst_blocks <= 0)
+        return fail(PA_ERR_INVALID_ARG, "num_pairs %d, blocks %d / %d", num_pairs,
+                    num_src_blocks, num_dst_blocks);
+    if (num_pairs == 0) return PA_OK;
+    if (!dst_k || !dst_v || !src_k || !src_v || !src_dst_pairs)
+        return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+    if (block_bytes == 0 || block_bytes % 16 != 0)
+        return fail(PA_ERR_INVALID_ARG, "block_bytes %zu must be a positive multiple of 16",
+                    block_bytes);
+    const void *v[5] = {dst_k, dst_v, src_k, src_v, src_dst_pairs};
+    const void *d[5];
+    for (int i = 0; i < 5; ++i) {
+        d[i] = device_view(v[i]);
+        if (!d[i])
+            return fail(PA_ERR_INVALID_ARG,
+                        "pointer %d is neither device memory nor mapped page-locked host memory",
+                        i);
+    }
+    if (!aligned16(d[0]) || !aligned16(d[1]) || !aligned16(d[2]) || !aligned16(d[3]) ||
+        (reinterpret_cast<uintptr_t>(d[4]) & 7u))
+        return fail(PA_ERR_INVALID_ARG, "misaligned pointer");
+    unsigned int *err = device_error_ptr();
+    if (!err) return fail(PA_ERR_CUDA, "no CUDA device");
+    cudaError_t e = launch_swap_blocks(const_cast<void *>(d[0]), const_cast<void *>(d[1]), d[2],
+                                       d[3], static_cast<const int64_t *>(d[4]), num_pairs,
+                                       block_bytes, num_src_blocks, num_dst_blocks, err,
+                                       static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "swap_blocks launch");
+    return PA_OK;
+}
+
 int pa_set_profile_events(void *ev_begin, void *ev_end) {
     clear_error();
     t_prof.begin = static_cast<cudaEvent_t>(ev_begin);

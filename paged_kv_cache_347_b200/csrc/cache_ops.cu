@@ -73,6 +73,53 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(
     }
 }
 
+// Pair p copies block src of (src_k, src_v) onto block dst of (dst_k, dst_v);
+// either side may be mapped host memory, so this is also the swap path.
+__global__ void __launch_bounds__(256) swap_blocks_kernel(
+    const uint4 *__restrict__ src_k, const uint4 *__restrict__ src_v, uint4 *__restrict__ dst_k,
+    uint4 *__restrict__ dst_v, const int64_t *__restrict__ pairs, int num_pairs,
+    int64_t words_per_block, int num_src_blocks, int num_dst_blocks, unsigned int *err) {
+    for (int p = blockIdx.y; p < num_pairs; p += gridDim.y) {
+        const int64_t src = pairs[2 * p];
+        const int64_t dst = pairs[2 * p + 1];
+        if (src < 0 || src >= num_src_blocks || dst < 0 || dst >= num_dst_blocks) {
+            if (blockIdx.x == 0 && threadIdx.x == 0) raise_device_error(err, PA_DEVERR_PAIR);
+            continue;
+        }
+        const uint4 *ks = src_k + src * words_per_block;
+        const uint4 *vs = src_v + src * words_per_block;
+        uint4 *kd = dst_k + dst * words_per_block;
+        uint4 *vd = dst_v + dst * words_per_block;
+        for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < words_per_block;
+             w += (int64_t)gridDim.x * blockDim.x) {
+            const uint4 a = ks[w];
+            const uint4 b = vs[w];
+            kd[w] = a;
+            vd[w] = b;
+        }
+    }
+}
+
+cudaError_t launch_swap_blocks(void *dst_k, void *dst_v, const void *src_k, const void *src_v,
+                               const int64_t *pairs, int num_pairs, size_t block_bytes,
+                               int num_src_blocks, int num_dst_blocks, unsigned int *err,
+                               cudaStream_t stream) {
+    if (num_pairs == 0) return cudaSuccess;
+    const int64_t words = (int64_t)(block_bytes / 16);
+    const int threads = 256;
+    int64_t bx = (words + threads - 1) / threads;
+    if (bx > 64) bx = 64;
+    int64_t by = num_pairs;
+    const int64_t cap = (int64_t)num_sms() * 8;
+    if (bx * by > cap) by = cap / bx > 0 ? cap / bx : 1;
+    if (by > 65535) by = 65535;
+    swap_blocks_kernel<<<dim3((unsigned)bx, (unsigned)by), threads, 0, stream>>>(
+        static_cast<const uint4 *>(src_k), static_cast<const uint4 *>(src_v),
+        static_cast<uint4 *>(dst_k), static_cast<uint4 *>(dst_v), pairs, num_pairs, words,
+        num_src_blocks, num_dst_blocks, err);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_reshape_and_cache(const void *k, const void *v, void *k_cache, void *v_cache,
                                      const int64_t *slot_mapping, int num_tokens,
                                      int num_kv_heads, int row_bytes, int block_size,

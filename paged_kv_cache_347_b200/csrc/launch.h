@@ -34,6 +34,11 @@ cudaError_t launch_copy_blocks(void *k_cache, void *v_cache, const int64_t *pair
                                size_t block_bytes, int num_blocks, unsigned int *err,
                                cudaStream_t stream);
 
+cudaError_t launch_swap_blocks(void *dst_k, void *dst_v, const void *src_k, const void *src_v,
+                               const int64_t *pairs, int num_pairs, size_t block_bytes,
+                               int num_src_blocks, int num_dst_blocks, unsigned int *err,
+                               cudaStream_t stream);
+
 // CUDA-core decode (any dtype, any supported block size).  dtype: pa_dtype.
 cudaError_t launch_decode_simt(const DecodeParams &p, int dtype, cudaStream_t stream);
 

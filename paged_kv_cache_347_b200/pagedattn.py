@@ -46,7 +46,9 @@ def _sig(name, res, *args):
 class pa_alloc_stats_t(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in (
         "num_blocks", "free_blocks", "used_blocks", "shared_blocks", "num_seqs",
-        "table_entries", "logical_tokens", "reserved_slots")]
+        "table_entries", "logical_tokens", "reserved_slots", "cached_blocks",
+        "prefix_hit_blocks", "prefix_query_blocks", "evicted_blocks", "host_blocks",
+        "host_free_blocks", "swapped_seqs")]
 
 
 _sig("pa_last_error", _c.c_char_p)
@@ -74,6 +76,12 @@ _sig("pa_block_tables", _i, _vp, _vp, _i, _vp, _i, _vp)
 _sig("pa_alloc_stats", _i, _vp, _c.POINTER(pa_alloc_stats_t))
 _sig("pa_alloc_free_list", _i, _vp, _vp, _i, _vp)
 _sig("pa_alloc_refcount", _i, _vp, _i)
+_sig("pa_seq_add_cached", _i, _vp, _i64, _vp, _i, _vp)
+_sig("pa_seq_append_tokens", _i, _vp, _i64, _vp, _i, _vp, _vp, _vp)
+_sig("pa_alloc_set_host_pool", _i, _vp, _i)
+_sig("pa_seq_swap_out", _i, _vp, _i64, _vp, _i, _vp)
+_sig("pa_seq_swap_in", _i, _vp, _i64, _vp, _i, _vp)
+_sig("pa_swap_blocks", _i, _vp, _vp, _vp, _vp, _vp, _i, _sz, _i, _i, _vp)
 
 
 class PagedAttnError(RuntimeError):
@@ -238,6 +246,33 @@ def pa_copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, src_dst_pairs: 
         _stream(k_cache)), "pa_copy_blocks")
 
 
+def pa_swap_blocks(dst_k: torch.Tensor, dst_v: torch.Tensor, src_k: torch.Tensor,
+                   src_v: torch.Tensor, src_dst_pairs: torch.Tensor) -> None:
+    """Copy blocks between two caches of one block shape; a side may be pinned
+    host memory (``tensor.pin_memory()``).  src_dst_pairs int64 [n, 2], on the
+    device or pinned."""
+    n = src_dst_pairs.shape[0] if src_dst_pairs.numel() else 0
+    if n == 0:
+        return
+    if tuple(dst_k.shape[1:]) != tuple(src_k.shape[1:]) or dst_k.dtype != src_k.dtype:
+        raise ValueError("caches differ in block shape or dtype")
+    for name, t in (("dst_k", dst_k), ("dst_v", dst_v), ("src_k", src_k), ("src_v", src_v),
+                    ("src_dst_pairs", src_dst_pairs)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+        if not (t.is_cuda or t.is_pinned()):
+            raise TypeError(f"{name} must be a CUDA tensor or pinned host memory")
+    if src_dst_pairs.dtype != torch.int64:
+        raise TypeError("src_dst_pairs must be int64")
+    NBd, Hkv, bs, D = dst_k.shape
+    block_bytes = Hkv * bs * D * dst_k.element_size()
+    dev = dst_k.device if dst_k.is_cuda else src_k.device
+    _check(_lib.pa_swap_blocks(dst_k.data_ptr(), dst_v.data_ptr(), src_k.data_ptr(),
+                               src_v.data_ptr(), src_dst_pairs.data_ptr(), n, block_bytes,
+                               src_k.shape[0], NBd, torch.cuda.current_stream(dev).cuda_stream),
+           "pa_swap_blocks")
+
+
 # ----------------------------------------------------------------- allocator
 def _np_ptr(a: np.ndarray) -> int:
     return a.ctypes.data
@@ -332,3 +367,43 @@ class BlockAllocator:
 
     def refcount(self, block: int) -> int:
         return _lib.pa_alloc_refcount(self._h, block)
+
+    # prefix caching
+    def seq_add_cached(self, seq_id: int, token_ids: Sequence[int]) -> int:
+        """New sequence sharing the longest indexed prefix; returns the number
+        of cached tokens (a multiple of the block size)."""
+        t = np.ascontiguousarray(token_ids, dtype=np.int64)
+        n = ctypes.c_int(0)
+        _check(_lib.pa_seq_add_cached(self._h, seq_id, _np_ptr(t) if t.size else None, t.size,
+                                      ctypes.addressof(n)), "pa_seq_add_cached")
+        return n.value
+
+    def seq_append_tokens(self, seq_id: int, token_ids: Sequence[int]
+                          ) -> Tuple[np.ndarray, Optional[Tuple[int, int]]]:
+        t = np.ascontiguousarray(token_ids, dtype=np.int64)
+        slots = np.empty(max(t.size, 1), np.int64)
+        pair = np.empty(2, np.int64)
+        ncow = ctypes.c_int(0)
+        _check(_lib.pa_seq_append_tokens(self._h, seq_id, _np_ptr(t) if t.size else None, t.size,
+                                         _np_ptr(slots), _np_ptr(pair), ctypes.addressof(ncow)),
+               "pa_seq_append_tokens")
+        return slots[:t.size], ((int(pair[0]), int(pair[1])) if ncow.value else None)
+
+    # swap
+    def set_host_pool(self, num_host_blocks: int) -> None:
+        _check(_lib.pa_alloc_set_host_pool(self._h, num_host_blocks), "pa_alloc_set_host_pool")
+
+    def _swap(self, fn, name, seq_id: int) -> np.ndarray:
+        n = ctypes.c_int(0)
+        cap = max(self.num_blocks, 1)
+        pairs = np.empty((cap, 2), np.int64)
+        _check(fn(self._h, seq_id, _np_ptr(pairs), cap, ctypes.addressof(n)), name)
+        return pairs[:n.value].copy()
+
+    def seq_swap_out(self, seq_id: int) -> np.ndarray:
+        """(device block, host block) pairs, in logical order."""
+        return self._swap(_lib.pa_seq_swap_out, "pa_seq_swap_out", seq_id)
+
+    def seq_swap_in(self, seq_id: int) -> np.ndarray:
+        """(host block, device block) pairs, in logical order."""
+        return self._swap(_lib.pa_seq_swap_in, "pa_seq_swap_in", seq_id)

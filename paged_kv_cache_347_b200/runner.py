@@ -6,11 +6,13 @@ rows of its appends (in op order) and the queries of its decode.  The
 runner turns a step into device actions in two phases:
 
 * ``plan``: the C++ allocator runs every event on the host.  Consecutive
-  appends become one ``write`` action (their slots and copy-on-write pairs,
-  from ``pa_batch_append``); a decode becomes a ``decode`` action carrying the
-  block-table rows and lengths of its batch.  Any other event ends a run of
-  appends, so the batched copies-then-writes of one action equal applying the
-  appends one at a time.
+  appends (plain, with token ids, or the uncached part of an admitted
+  sequence, whose cached rows get slot -1) become one ``write`` action: their
+  slots and copy-on-write pairs.  A decode becomes a ``decode`` action
+  carrying the block-table rows and lengths of its batch; a swap becomes a
+  ``swap_out``/``swap_in`` action with its block pairs.  Any other event ends
+  a run of appends, so the batched copies-then-writes of one action equal
+  applying the appends one at a time.
 * ``execute``: ``pa_copy_blocks`` (when the write has pairs), then
   ``pa_reshape_and_cache``, and for a decode ``pa_decode``; all on the
   current stream, nothing synchronised.
@@ -32,7 +34,7 @@ from . import pagedattn as pa
 
 @dataclass
 class Action:
-    kind: str                            # "write" | "decode"
+    kind: str                            # "write" | "decode" | "swap_out" | "swap_in"
     slots: Optional[np.ndarray] = None   # int64 [n]
     pairs: Optional[np.ndarray] = None   # int64 [k, 2]
     row0: int = 0
@@ -65,9 +67,35 @@ class PagedKVRunner:
                    shape.head_dim, dt, shape.scale, table_width, shape.free_order, **kw)
 
     # ------------------------------------------------------------ plan
+    def enable_swap(self, num_host_blocks: int) -> None:
+        """Host pool for swapped-out sequences: the allocator's host blocks and
+        page-locked host caches of the same block shape."""
+        self.alloc.set_host_pool(num_host_blocks)
+        dims = (max(num_host_blocks, 1), self.num_kv_heads, self.block_size, self.head_dim)
+        self.k_host = torch.zeros(dims, dtype=self.dtype).pin_memory()
+        self.v_host = torch.zeros(dims, dtype=self.dtype).pin_memory()
+
     def plan(self, ops) -> List[Action]:
         acts: List[Action] = []
         row = 0
+        pend = {"slots": [], "pairs": [], "row0": 0, "nrows": 0}
+
+        def add_rows(slots, pairs, n):
+            if pend["nrows"] == 0:
+                pend["row0"] = row
+            pend["slots"].append(np.asarray(slots, dtype=np.int64))
+            if pairs is not None and len(pairs):
+                pend["pairs"].append(np.asarray(pairs, dtype=np.int64).reshape(-1, 2))
+            pend["nrows"] += n
+
+        def flush():
+            if pend["nrows"]:
+                pairs = (np.concatenate(pend["pairs"]) if pend["pairs"]
+                         else np.empty((0, 2), np.int64))
+                acts.append(Action("write", slots=np.concatenate(pend["slots"]), pairs=pairs,
+                                   row0=pend["row0"], nrows=pend["nrows"]))
+            pend.update(slots=[], pairs=[], nrows=0)
+
         i = 0
         while i < len(ops):
             op = ops[i]
@@ -80,23 +108,43 @@ class PagedKVRunner:
                     i += 1
                 slots, pairs = self.alloc.batch_append(ids, ns)
                 n = int(sum(ns))
-                acts.append(Action("write", slots=slots.copy(), pairs=pairs.copy(), row0=row,
-                                   nrows=n))
+                add_rows(slots.copy(), pairs.copy(), n)
                 row += n
                 continue
-            if kind == "add":
-                self.alloc.seq_add(op[1])
-            elif kind == "fork":
-                self.alloc.seq_fork(op[1], op[2])
-            elif kind == "free":
-                self.alloc.seq_free(op[1])
-            elif kind == "decode":
-                tables, lens = self.alloc.block_tables(list(op[1]), self.width)
-                acts.append(Action("decode", tables=tables, lens=lens,
-                                   max_len=int(lens.max()) if lens.size else 0))
+            if kind == "append_tokens":
+                slots, pair = self.alloc.seq_append_tokens(op[1], op[2])
+                add_rows(slots.copy(), [pair] if pair else None, len(op[2]))
+                row += len(op[2])
+            elif kind == "admit":
+                toks = op[2]
+                c = self.alloc.seq_add_cached(op[1], toks)
+                slots, pair = self.alloc.seq_append_tokens(op[1], toks[c:])
+                # rows of cached tokens are skipped (slot -1)
+                add_rows(np.concatenate([np.full(c, -1, np.int64), slots]),
+                         [pair] if pair else None, len(toks))
+                row += len(toks)
             else:
-                raise ValueError(f"unknown op {op!r}")
+                flush()
+                if kind == "add":
+                    self.alloc.seq_add(op[1])
+                elif kind == "fork":
+                    self.alloc.seq_fork(op[1], op[2])
+                elif kind == "free":
+                    self.alloc.seq_free(op[1])
+                elif kind == "decode":
+                    tables, lens = self.alloc.block_tables(list(op[1]), self.width)
+                    acts.append(Action("decode", tables=tables, lens=lens,
+                                       max_len=int(lens.max()) if lens.size else 0))
+                elif kind == "host_pool":
+                    self.enable_swap(op[1])
+                elif kind == "swap_out":
+                    acts.append(Action("swap_out", pairs=self.alloc.seq_swap_out(op[1])))
+                elif kind == "swap_in":
+                    acts.append(Action("swap_in", pairs=self.alloc.seq_swap_in(op[1])))
+                else:
+                    raise ValueError(f"unknown op {op!r}")
             i += 1
+        flush()
         return acts
 
     # ------------------------------------------------------------ device side
@@ -114,9 +162,11 @@ class PagedKVRunner:
                 a.dev["slots"] = put(a.slots)
                 if len(a.pairs):
                     a.dev["pairs"] = put(a.pairs)
-            else:
+            elif a.kind == "decode":
                 a.dev["tables"] = put(a.tables)
                 a.dev["lens"] = put(a.lens)
+            elif len(a.pairs):
+                a.dev["pairs"] = put(a.pairs)
 
     def execute(self, acts: List[Action], k_new: Optional[torch.Tensor],
                 v_new: Optional[torch.Tensor], q: Optional[torch.Tensor],
@@ -130,6 +180,14 @@ class PagedKVRunner:
                     pa.pa_reshape_and_cache(k_new[a.row0:a.row0 + a.nrows],
                                             v_new[a.row0:a.row0 + a.nrows], self.k_cache,
                                             self.v_cache, a.dev["slots"])
+            elif a.kind == "swap_out":
+                if "pairs" in a.dev:
+                    pa.pa_swap_blocks(self.k_host, self.v_host, self.k_cache, self.v_cache,
+                                      a.dev["pairs"])
+            elif a.kind == "swap_in":
+                if "pairs" in a.dev:
+                    pa.pa_swap_blocks(self.k_cache, self.v_cache, self.k_host, self.v_host,
+                                      a.dev["pairs"])
             else:
                 b = a.tables.shape[0]
                 o = out if out is not None else torch.empty(
@@ -177,9 +235,11 @@ class PagedKVRunner:
                 arrays.append((a, "slots", a.slots))
                 if len(a.pairs):
                     arrays.append((a, "pairs", a.pairs))
-            else:
+            elif a.kind == "decode":
                 arrays.append((a, "tables", a.tables))
                 arrays.append((a, "lens", a.lens))
+            elif len(a.pairs):
+                arrays.append((a, "pairs", a.pairs))
         offs, total = [], 0
         for _, _, arr in arrays:
             offs.append(total)

@@ -156,3 +156,71 @@ def test_create_validates_free_order():
         pa.BlockAllocator(4, 4, [0, 1, 1, 2])
     with pytest.raises(pa.PagedAttnError):
         pa.BlockAllocator(0, 4)
+
+
+def _apply_ext(ref, nat, op):
+    """Prefix-cache and swap events on both allocators; results must agree."""
+    kind = op[0]
+    r = n = None
+    try:
+        if kind == "add_cached": r = ref.add_cached(op[1], op[2])
+        elif kind == "admit":
+            c = ref.add_cached(op[1], op[2])
+            sl, p = ref.append_tokens(op[1], op[2][c:]); r = (c, list(sl), p)
+        elif kind == "append_tokens":
+            s, p = ref.append_tokens(op[1], op[2]); r = (list(s), p)
+        elif kind == "swap_out": r = [tuple(x) for x in ref.swap_out(op[1])]
+        elif kind == "swap_in": r = [tuple(x) for x in ref.swap_in(op[1])]
+        else:
+            return _apply(ref, nat, op)
+    except AllocError as e:
+        r = type(e).code
+    try:
+        if kind == "add_cached": n = nat.seq_add_cached(op[1], op[2])
+        elif kind == "admit":
+            c = nat.seq_add_cached(op[1], op[2])
+            sl, p = nat.seq_append_tokens(op[1], op[2][c:]); n = (c, sl.tolist(), p)
+        elif kind == "append_tokens":
+            s, p = nat.seq_append_tokens(op[1], op[2]); n = (s.tolist(), p)
+        elif kind == "swap_out": n = [tuple(x) for x in nat.seq_swap_out(op[1]).tolist()]
+        elif kind == "swap_in": n = [tuple(x) for x in nat.seq_swap_in(op[1]).tolist()]
+    except pa.PagedAttnError as e:
+        n = e.code
+    assert r == n, (op, r, n)
+
+
+@pytest.mark.parametrize("seed", range(8))
+def test_prefix_cache_and_swap_ops_bit_exact(seed):
+    rr = random.Random(1000 + seed)
+    nb = rr.choice([16, 32, 64])
+    bs = rr.choice([1, 2, 4, 8])
+    order = list(np.random.default_rng(seed).permutation(nb))
+    ref = RefAllocator(nb, bs, order)
+    nat = pa.BlockAllocator(nb, bs, order)
+    hp = rr.choice([0, 8, 32])
+    ref.set_host_pool(hp)
+    nat.set_host_pool(hp)
+    # a few shared "system prompts" so prefix hits happen
+    prompts = [[rr.randrange(4) for _ in range(rr.randrange(bs, 5 * bs))] for _ in range(3)]
+    live, nxt = [], 0
+    for _ in range(500):
+        x = rr.random()
+        if x < 0.2 or not live:
+            toks = rr.choice(prompts) + [rr.randrange(4) for _ in range(rr.randrange(0, 2 * bs))]
+            op = (rr.choice(["admit", "admit", "add_cached"]), nxt, toks)
+            live.append(nxt); nxt += 1
+        elif x < 0.5:
+            op = ("append_tokens", rr.choice(live), [rr.randrange(4) for _ in range(rr.choice([1, 1, 2, bs + 1]))])
+        elif x < 0.6:
+            op = ("append", rr.choice(live), rr.choice([1, 3]))
+        elif x < 0.68:
+            op = ("fork", rr.choice(live), nxt); live.append(nxt); nxt += 1
+        elif x < 0.78:
+            op = ("swap_out", rr.choice(live))
+        elif x < 0.88:
+            op = ("swap_in", rr.choice(live))
+        else:
+            s = rr.choice(live); op = ("free", s); live.remove(s)
+        _apply_ext(ref, nat, op)
+        _same_state(ref, nat)
+    assert ref.stats()["prefix_hit_blocks"] > 0

@@ -106,3 +106,42 @@ def test_beam_first_step_copies_twelve_blocks():
     assert len(errs) == 1
     st = gpu.alloc.stats()
     assert st["used_blocks"] == 4 * (129 + 3) == orc.alloc.stats()["used_blocks"]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_swap_blocks_device_host_round_trip_bit_exact(dtype):
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    NB, NH, Hkv, bs, D = 48, 20, 4, 16, 128
+    dk = _rand_bits((NB, Hkv, bs, D), dtype, 7).cuda()
+    dv = _rand_bits((NB, Hkv, bs, D), dtype, 8).cuda()
+    hk = torch.zeros((NH, Hkv, bs, D), dtype=DT[dtype]).pin_memory()
+    hv = torch.zeros((NH, Hkv, bs, D), dtype=DT[dtype]).pin_memory()
+    r = np.random.default_rng(3)
+    out_pairs = np.stack([r.choice(NB, 12, replace=False), r.choice(NH, 12, replace=False)], 1)
+    pa.pa_swap_blocks(hk, hv, dk, dv, torch.from_numpy(out_pairs).cuda())
+    torch.cuda.synchronize()
+    b = BITS[dtype]
+    ref_k = torch.zeros_like(hk).view(b); ref_v = torch.zeros_like(hv).view(b)
+    cache_ref.copy_between(ref_k, ref_v, dk.cpu().view(b), dv.cpu().view(b), out_pairs.tolist())
+    assert torch.equal(hk.view(b), ref_k) and torch.equal(hv.view(b), ref_v)
+    # back into other device blocks, pairs given in pinned host memory
+    in_pairs = np.stack([out_pairs[:, 1], r.choice(NB, 12, replace=False)], 1)
+    dk2, dv2 = dk.clone(), dv.clone()
+    pa.pa_swap_blocks(dk2, dv2, hk, hv, torch.from_numpy(in_pairs.copy()).pin_memory())
+    torch.cuda.synchronize()
+    ek, ev = dk.cpu().view(b).clone(), dv.cpu().view(b).clone()
+    cache_ref.copy_between(ek, ev, hk.view(b), hv.view(b), in_pairs.tolist())
+    assert torch.equal(dk2.cpu().view(b), ek) and torch.equal(dv2.cpu().view(b), ev)
+
+
+def test_swap_blocks_rejects_pageable_host_memory():
+    import ctypes
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    dk = torch.zeros(4, 1, 16, 64, dtype=torch.bfloat16, device="cuda")
+    hk = torch.zeros(4, 1, 16, 64, dtype=torch.bfloat16)          # not pinned
+    pairs = torch.tensor([[0, 1]], dtype=torch.int64, device="cuda")
+    rc = pa._lib.pa_swap_blocks(hk.data_ptr(), hk.data_ptr(), dk.data_ptr(), dk.data_ptr(),
+                                pairs.data_ptr(), 1, 16 * 64 * 2, 4, 4, None)
+    assert rc == -1 and b"page-locked" in pa._lib.pa_last_error()
+    with pytest.raises(TypeError):
+        pa.pa_swap_blocks(hk, hk, dk, dk, pairs)

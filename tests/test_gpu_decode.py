@@ -238,3 +238,21 @@ def test_pinned_host_fed_steps_match_oracle():
         assert res["h2d"] > 0 and res["d2h"] == out.nbytes
         err = float(np.abs(out.double().numpy() - ref["out"]).max())
         assert err <= TOL["f16"], (i, err)
+
+
+def test_prefix_cached_requests_decode_like_the_oracle():
+    """Requests sharing a cached system prompt reuse its blocks (fewer rows
+    written) and decode exactly as if each had its own copy."""
+    wl = workloads.prefix_share(requests=8, prompt=300, suffix_hi=40, steps=3)
+    errs, gpu, orc = run_parity(wl, table_width=32, compare_cache=True)
+    assert max(errs) <= TOL["bf16"], errs
+    st = gpu.alloc.stats()
+    assert st["prefix_hit_blocks"] == 7 * (300 // 16) == orc.alloc.stats()["prefix_hit_blocks"]
+
+
+def test_preempted_sequence_swaps_out_and_back_and_decodes_on():
+    wl = workloads.preempt(batch=4, lo=100, hi=600, steps=6, host_blocks=64, num_blocks=256)
+    errs, gpu, orc = run_parity(wl, table_width=48, compare_cache=True)
+    assert len(errs) == 6 and max(errs) <= TOL["bf16"], errs
+    # the victim's rows came back from host blocks into fresh device blocks
+    assert gpu.alloc.stats()["swapped_seqs"] == 0 and gpu.alloc.stats()["host_free_blocks"] == 64

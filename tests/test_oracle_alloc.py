@@ -230,3 +230,112 @@ def _ops_only(wl):
     # the beam generator draws values lazily per step; pull ops step by step
     for st in wl.steps:
         yield st.ops
+
+
+# ---------------------------------------------------------------- prefix caching
+def _tok(n, base=0):
+    return list(range(base, base + n))
+
+
+def test_prefix_blocks_are_shared_and_partial_blocks_are_not():
+    bs = 4
+    a = RefAllocator(32, bs)
+    T = _tok(10)                        # 2 full blocks + 2 tokens
+    assert a.add_cached(1, T) == 0      # empty index
+    a.append_tokens(1, T)
+    assert a.stats()["cached_blocks"] == 2
+    # same first 8 tokens, different tail: both full blocks are shared
+    assert a.add_cached(2, T[:8] + [99, 98, 97]) == 8
+    assert a.table(2) == a.table(1)[:2]
+    assert [a.ref[b] for b in a.table(1)[:2]] == [2, 2]
+    # diverging inside block 1: only block 0 is shared
+    assert a.add_cached(3, T[:5] + [77, 76, 75]) == 4
+    assert a.table(3) == a.table(1)[:1] and a.ref[a.table(1)[0]] == 3
+    # the same tokens under a different parent block never match
+    assert a.add_cached(4, [50, 51, 52, 53] + T[4:8]) == 0
+    st = a.stats()
+    assert st["prefix_hit_blocks"] == 3 and st["prefix_query_blocks"] == 2 + 2 + 2 + 2
+
+
+def test_prefix_cache_survives_release_and_is_evicted_in_fifo_order():
+    bs = 4
+    a = RefAllocator(8, bs, list(range(8)))
+    T = _tok(8)
+    a.add_cached(1, T)
+    a.append_tokens(1, T)               # blocks 0, 1 indexed
+    a.free_seq(1)
+    assert a.free_list() == [2, 3, 4, 5, 6, 7, 0, 1]
+    assert a.stats()["cached_blocks"] == 2
+    # a hit takes the cached blocks out of the free list, wherever they are
+    assert a.add_cached(2, T + [9]) == 8
+    assert a.table(2) == [0, 1] and 0 not in a.free_list() and 1 not in a.free_list()
+    assert a.stats()["free_blocks"] == 6
+    a.free_seq(2)
+    # new allocations walk the FIFO: blocks 2..7 first, then the cached 0 and 1
+    a.add(3)
+    a.append(3, 6 * bs)
+    assert a.stats()["cached_blocks"] == 2 and a.stats()["evicted_blocks"] == 0
+    a.append(3, 1)                      # takes block 0: evicted from the index
+    st = a.stats()
+    assert st["cached_blocks"] == 1 and st["evicted_blocks"] == 1
+    # block 1 is still indexed but its parent (block 0) is gone: no chain match
+    assert a.add_cached(4, T) == 0
+
+
+def test_identical_blocks_are_indexed_once():
+    bs = 4
+    a = RefAllocator(16, bs)
+    T = _tok(8)
+    a.add_cached(1, T)
+    a.append_tokens(1, T)
+    assert a.add_cached(2, T[:3]) == 0  # no full block to match
+    a.append_tokens(2, T[3:8])          # fills two blocks with seq 1's tokens
+    # block 0's key (-1, T[0:4]) is taken, so it is not indexed; block 1's key
+    # has seq 2's own block 0 as parent, a different key: it is indexed
+    assert a.stats()["cached_blocks"] == 3
+    assert a.table(2) != a.table(1)
+    # a new request follows the first chain
+    assert a.add_cached(3, T) == 8 and a.table(3) == a.table(1)
+    with pytest.raises(InvalidArg):
+        a.add(9); a.append(9, 1); a.append_tokens(9, [1])   # no token history
+
+
+# ---------------------------------------------------------------- swap
+def test_swap_out_and_in_move_blocks_in_logical_order():
+    bs = 4
+    a = RefAllocator(8, bs, [7, 6, 5, 4, 3, 2, 1, 0])
+    a.set_host_pool(4)
+    a.add(1); a.append(1, 10)           # blocks 7, 6, 5
+    a.add(2); a.append(2, 4)            # block 4
+    pairs = a.swap_out(1)
+    assert pairs == [(7, 0), (6, 1), (5, 2)]
+    assert a.free_list() == [3, 2, 1, 0, 7, 6, 5]
+    assert a.table(1) == [0, 1, 2] and a.length(1) == 10
+    st = a.stats()
+    assert st["host_free_blocks"] == 1 and st["swapped_seqs"] == 1 and st["used_blocks"] == 1
+    with pytest.raises(InvalidArg):
+        a.append(1, 1)
+    with pytest.raises(InvalidArg):
+        a.fork(1, 5)
+    a.append(2, 8)                      # seq 2 now has 3 blocks, the host pool 1 free
+    before = (list(a.free), list(a.host_free), a.table(2))
+    with pytest.raises(OutOfBlocks):
+        a.swap_out(2)
+    assert before == (list(a.free), list(a.host_free), a.table(2))
+    back = a.swap_in(1)                 # seq 2 took blocks 3, 2; the head is now 1, 0, 7
+    assert back == [(0, 1), (1, 0), (2, 7)]
+    assert a.table(1) == [1, 0, 7] and a.stats()["host_free_blocks"] == 4
+    assert list(a.host_free) == [3, 0, 1, 2]
+
+
+def test_swap_of_a_shared_block_keeps_the_other_owner():
+    bs = 4
+    a = RefAllocator(8, bs)
+    a.set_host_pool(4)
+    a.add(1); a.append(1, 6)
+    a.fork(1, 2)
+    pairs = a.swap_out(2)
+    assert [d for d, _ in pairs] == a.table(1)
+    assert all(a.ref[b] == 1 for b in a.table(1))
+    a.free_seq(2)                       # a swapped sequence returns its host blocks
+    assert a.stats()["host_free_blocks"] == 4 and a.stats()["swapped_seqs"] == 0

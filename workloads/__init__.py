@@ -99,6 +99,9 @@ class Shape:
 # An event on the sequences, applied in list order.
 #   ("add", sid) ("append", sid, n) ("fork", parent, child) ("free", sid)
 #   ("decode", [sid, ...])
+#   ("admit", sid, token_ids)        new sequence with token ids (prefix cache)
+#   ("append_tokens", sid, token_ids)
+#   ("host_pool", n_blocks) ("swap_out", sid) ("swap_in", sid)
 Op = Tuple
 
 
@@ -119,7 +122,15 @@ class Step:
 
     @property
     def n_new_tokens(self) -> int:
-        return sum(op[2] for op in self.ops if op[0] == "append")
+        """K/V rows the step carries: every appended token, and every token of
+        an admitted sequence (the prefix cache may make some rows unused)."""
+        n = 0
+        for op in self.ops:
+            if op[0] == "append":
+                n += op[2]
+            elif op[0] in ("admit", "append_tokens"):
+                n += len(op[2])
+        return n
 
     @property
     def decode_seqs(self) -> List[int]:
@@ -308,12 +319,88 @@ def custom(name: str, lens: Sequence[int], num_heads: int, num_kv_heads: int, he
     return Workload(sh, gen(), name, {"lens": list(lens)})
 
 
+def prefix_share(seed: int = 5, requests: int = 16, prompt: int = 1000, suffix_lo: int = 1,
+                 suffix_hi: int = 200, steps: int = 2, block_size: int = 16,
+                 num_blocks: int = 4096, vocab: int = 32000) -> Workload:
+    """Prefix caching: ``requests`` sequences share a ``prompt``-token system
+    prompt (same token ids, hence the same K/V rows) followed by their own
+    suffix; they are admitted one by one with their token ids ("admit"), then
+    decode ``steps`` tokens each ("append_tokens" + "decode").  32/8 heads,
+    D 128, bf16.  The K/V rows of an admit op cover all of its tokens; the
+    runner writes only the ones the prefix cache does not already hold."""
+    sh = Shape("prefix", 32, 8, 128, "bf16", block_size, num_blocks, seed)
+    sh.free_order = permutation(seed, num_blocks)
+    r = rng_for(seed, (5,))
+    sys_ids = r.integers(0, vocab, size=prompt).tolist()
+    sfx = r.integers(suffix_lo, suffix_hi, size=requests, endpoint=True).tolist()
+    pk, pv = _kv(sh, (40,), prompt)
+    sids = list(range(requests))
+
+    def gen():
+        ops: List[Op] = []
+        ks, vs = [], []
+        for i in sids:
+            ids = sys_ids + r.integers(0, vocab, size=sfx[i]).tolist()
+            ops.append(("admit", i, ids))
+            k2, v2 = _kv(sh, (41, i), sfx[i])
+            ks += [pk, k2]
+            vs += [pv, v2]
+        yield Step(ops, torch.cat(ks), torch.cat(vs), tag="admit")
+        for t in range(steps):
+            ops = [("append_tokens", i, [int(r.integers(0, vocab))]) for i in sids]
+            ops.append(("decode", sids))
+            k, v = _kv(sh, (20, t), len(sids))
+            yield Step(ops, k, v, _q(sh, (20, t), len(sids)), tag="decode")
+
+    return Workload(sh, gen(), "prefix sharing with a cached system prompt",
+                    {"prompt": prompt, "suffix": sfx})
+
+
+def preempt(seed: int = 6, batch: int = 8, lo: int = 200, hi: int = 3000, steps: int = 6,
+            victim: int = 0, out_step: int = 1, in_step: int = 4, host_blocks: int = 512,
+            block_size: int = 16, num_blocks: int = 2048) -> Workload:
+    """Preemption by swap: a batch decodes; at ``out_step`` one sequence is
+    swapped out to host blocks and a newcomer is admitted into the freed
+    device blocks; at ``in_step`` the newcomer finishes and the preempted
+    sequence is swapped back in and decodes on.  32/8 heads, D 128, bf16."""
+    sh = Shape("preempt", 32, 8, 128, "bf16", block_size, num_blocks, seed)
+    sh.free_order = permutation(seed, num_blocks)
+    lens = rng_for(seed, (2,)).integers(lo, hi, size=batch, endpoint=True).tolist()
+    newcomer = batch
+
+    def gen():
+        st = _prefill_step(sh, [int(x) - 1 for x in lens], list(range(batch)), (10,), decode=False)
+        st.ops.insert(0, ("host_pool", host_blocks))
+        yield st
+        live = list(range(batch))
+        for t in range(steps):
+            pre: List[Op] = []
+            k0 = v0 = None
+            if t == out_step:
+                pre = [("swap_out", victim), ("add", newcomer), ("append", newcomer, lens[victim])]
+                live = [s for s in live if s != victim] + [newcomer]
+                k0, v0 = _kv(sh, (50,), lens[victim])
+            elif t == in_step:
+                pre = [("free", newcomer), ("swap_in", victim)]
+                live = [s for s in live if s != newcomer] + [victim]
+            st = _decode_step(sh, live, (20, t))
+            st.ops = pre + st.ops
+            if k0 is not None:
+                st.k_new = torch.cat([k0, st.k_new])
+                st.v_new = torch.cat([v0, st.v_new])
+            yield st
+
+    return Workload(sh, gen(), "preemption by swap", {"lens": lens, "victim": victim})
+
+
 WORKLOADS = {
     "tiny": tiny,
     "llama8b": llama,
     "long32k": long_context,
     "beam": beam,
     "mix": mix,
+    "prefix": prefix_share,
+    "preempt": preempt,
 }
 
 
