@@ -494,6 +494,108 @@ def run_reference(args, ws, rank):
     }
 
 
+# ----------------------------------------------------------------- studies
+def _events_ms(fn, reps=20):
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    fn()
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(reps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / reps
+
+
+def study_prefix(args):
+    """Prefix caching on vs off for requests sharing a system prompt: K/V rows
+    written at admission, admission time (allocator + append kernel), hits."""
+    from paged_kv_cache_347_b200.runner import PagedKVRunner
+    res = {"study": "prefix_cache", "requests": 64, "prompt_tokens": 2048}
+    for mode in ("on", "off"):
+        wl = workloads.prefix_share(requests=64, prompt=2048, suffix_lo=16, suffix_hi=256,
+                                    steps=1, num_blocks=16384)
+        steps = list(wl.steps)
+        admit = steps[0]
+        if mode == "off":   # same tokens, no index: plain add + append of every token
+            ops = []
+            for op in admit.ops:
+                ops += [("add", op[1]), ("append", op[1], len(op[2]))]
+            admit = workloads.Step(ops, admit.k_new, admit.v_new, None, tag="admit")
+        r = PagedKVRunner.for_shape(wl.shape, 160)
+        k, v = admit.k_new.cuda(), admit.v_new.cuda()
+        t = time.perf_counter()
+        acts = r.plan(admit.ops)
+        host_us = (time.perf_counter() - t) * 1e6
+        r.upload(acts)
+        rows = int(sum(int((a.slots >= 0).sum()) for a in acts if a.kind == "write"))
+        ms = _events_ms(lambda: r.execute(acts, k, v, None), reps=10)
+        st = r.alloc.stats()
+        res[mode] = {"rows_written": rows, "kv_bytes_written": rows * 8 * 128 * 2 * 2,
+                     "append_kernel_us": round(ms * 1e3, 2), "allocator_us": round(host_us, 1),
+                     "used_blocks": st["used_blocks"], "prefix_hit_blocks": st["prefix_hit_blocks"],
+                     "prefix_query_blocks": st["prefix_query_blocks"]}
+        del r
+        torch.cuda.empty_cache()
+    return res
+
+
+def study_swap(args):
+    """pa_swap_blocks bandwidth between HBM and pinned host memory for one
+    32768-token sequence (2048 blocks of 8 heads x 16 x 128 bf16, K and V)."""
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    NB, Hkv, bs, D, n = 4096, 8, 16, 128, 2048
+    dk = torch.randn(NB, Hkv, bs, D, device="cuda").to(torch.bfloat16)
+    dv = torch.randn(NB, Hkv, bs, D, device="cuda").to(torch.bfloat16)
+    hk = torch.empty(n, Hkv, bs, D, dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty(n, Hkv, bs, D, dtype=torch.bfloat16).pin_memory()
+    r = np.random.default_rng(0)
+    out_p = torch.from_numpy(np.stack([r.permutation(NB)[:n], np.arange(n)], 1)).cuda()
+    in_p = torch.from_numpy(np.stack([np.arange(n), r.permutation(NB)[:n]], 1)).cuda()
+    nbytes = n * Hkv * bs * D * 2 * 2
+    out_ms = _events_ms(lambda: pa.pa_swap_blocks(hk, hv, dk, dv, out_p), reps=10)
+    in_ms = _events_ms(lambda: pa.pa_swap_blocks(dk, dv, hk, hv, in_p), reps=10)
+    errs = pa.device_errors()
+    return {"study": "swap", "bytes": nbytes, "blocks": n,
+            "swap_out_ms": round(out_ms, 3), "swap_out_GBs": round(nbytes / out_ms / 1e6, 1),
+            "swap_in_ms": round(in_ms, 3), "swap_in_GBs": round(nbytes / in_ms / 1e6, 1),
+            "device_errors": errs}
+
+
+def study_blocksize(args):
+    """Block-size trade-off on the continuous-batching mix: decode kernel
+    bandwidth and the tail waste of partially filled last blocks."""
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    from paged_kv_cache_347_b200.runner import PagedKVRunner
+    out = {"study": "block_size", "rows": []}
+    for bs in (4, 8, 16, 32, 64):
+        wl = workloads.mix(block_size=bs, steps=1)
+        steps = list(wl.steps)
+        r = PagedKVRunner.for_shape(wl.shape, 8256 // bs + 2)
+        r.run(steps[0])
+        acts = r.plan(steps[1].ops)
+        r.upload(acts)
+        dev = [t.cuda() for t in (steps[1].k_new, steps[1].v_new, steps[1].q)]
+        d = [a for a in acts if a.kind == "decode"][0]
+        o = torch.empty(dev[2].shape, dtype=torch.float32, device="cuda")
+        r.execute(acts, *dev)
+        ms = _events_ms(lambda: pa.pa_decode(o, dev[2], r.k_cache, r.v_cache, d.dev["tables"],
+                                             d.dev["lens"], r.scale, max_seq_len=d.max_len),
+                        reps=20)
+        kvb = kv_bytes(d.lens, 8, 128, 2)
+        st = r.alloc.stats()
+        out["rows"].append({"block_size": bs, "decode_us": round(ms * 1e3, 2),
+                            "kv_GBs": round(kvb / ms / 1e6, 1),
+                            "kernel": "tensor-core" if bs >= 8 else "cuda-core",
+                            "reserved_slots": st["reserved_slots"],
+                            "logical_tokens": st["logical_tokens"],
+                            "tail_waste_frac": round(1 - st["logical_tokens"] / st["reserved_slots"], 5),
+                            "table_entries": st["table_entries"]})
+        del r
+        torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -504,6 +606,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--study", default="", choices=["", "prefix", "swap", "blocksize"],
+                    help="print one of the side studies instead of the bench line")
     ap.add_argument("--partition", type=int, default=0,
                     help="split length in tokens (0: the library default, 512)")
     ap.add_argument("--batch", type=int, default=0,
@@ -511,6 +615,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
+    if args.study:
+        fn = {"prefix": study_prefix, "swap": study_swap, "blocksize": study_blocksize}[args.study]
+        print(json.dumps(fn(args)), flush=True)
+        return
     ws, rank, local, _ = dist_setup()
     try:
         if args.impl == "reference":
