@@ -6,7 +6,9 @@ Plain, slow, obviously correct CPU code that states what the path computes:
   copy-on-write on append to a shared block) as a Python model;
 * ``attn_ref.c`` -- single-query attention over a block-paged KV cache in
   fp64 C: every token is gathered through the block table and the softmax is
-  the exact two-pass one (max, then exp-sum), no online recurrence;
+  the exact two-pass one (max, then exp-sum), no online recurrence; and the
+  same for several new tokens per sequence under a causal mask (chunked
+  prefill);
 * ``attn``       -- ctypes entry to ``attn_ref.c``, a numpy fp64 brute force
   over contiguous (already gathered) K/V, the split-partial merge, and the
   storage-dtype decoders;

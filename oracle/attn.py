@@ -44,6 +44,12 @@ def lib() -> ctypes.CDLL:
         L.attn_ref_decode_value.restype = ctypes.c_double
         L.attn_ref_decode_value.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_longlong]
         L.attn_ref_max_threads.restype = ctypes.c_int
+        L.attn_ref_prefill.restype = ctypes.c_int
+        L.attn_ref_prefill.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_double, ctypes.c_int]
         _lib = L
     return _lib
 
@@ -91,6 +97,32 @@ def paged_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
         n_sel, int(n_threads))
     if rc != 0:
         raise ValueError("oracle: bad argument or block-table entry out of range")
+    return out
+
+
+def paged_prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                  block_tables: np.ndarray, seq_lens: np.ndarray, cu_q: np.ndarray,
+                  scale: float, n_threads: int = 0) -> np.ndarray:
+    """fp64 causal attention of chunk rows over the paged cache.
+
+    q [total, Hq, D] holds, for sequence s, rows cu_q[s]..cu_q[s+1]-1 at
+    positions L_s - n_s .. L_s - 1 (n_s = cu_q[s+1] - cu_q[s]); each attends to
+    tokens 0..its position.  Returns float64 [total, Hq, D]."""
+    q = q.contiguous(); k_cache = k_cache.contiguous(); v_cache = v_cache.contiguous()
+    total, Hq, D = q.shape
+    NB, Hkv, bs, _ = k_cache.shape
+    bt = np.ascontiguousarray(block_tables, dtype=np.int32)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int32)
+    cu = np.ascontiguousarray(cu_q, dtype=np.int32)
+    B = sl.shape[0]
+    assert cu.shape == (B + 1,) and int(cu[-1]) == total and bt.shape[0] == B
+    out = np.zeros((total, Hq, D), np.float64)
+    rc = lib().attn_ref_prefill(out.ctypes.data, q.data_ptr(), k_cache.data_ptr(),
+                                v_cache.data_ptr(), _DT[_dtype_name(q)], bt.ctypes.data,
+                                sl.ctypes.data, cu.ctypes.data, B, Hq, Hkv, D, bs, bt.shape[1],
+                                NB, float(scale), int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle: bad prefill argument or table entry out of range")
     return out
 
 

@@ -161,3 +161,78 @@ int attn_ref_decode(double *out, const void *q, const void *k_cache, const void 
     }
     return bad ? -1 : 0;
 }
+
+/*
+ * Oracle for multi-token (chunked prefill) attention over the paged cache.
+ * The query rows of sequence s are q[cu_q[s] .. cu_q[s+1]): the last
+ * n_s = cu_q[s+1] - cu_q[s] positions of the sequence, L_s - n_s .. L_s - 1,
+ * whose K/V are already in the cache.  Row r at position p attends, causally,
+ * to tokens 0..p, gathered through the block table exactly as in the decode
+ * oracle (the decode is the case n_s = 1).
+ * Layouts: q [total][Hq][D]; out [total][Hq][D] double.  Returns 0, or -1 on a
+ * bad argument (n_s < 0, n_s > L_s, a table entry out of range).
+ */
+static int prefill_row(double *o, const void *q, size_t qbase, const void *kc, const void *vc,
+                       dec_fn dec, const int32_t *table, int L, int g, int num_kv_heads,
+                       int head_dim, int block_size, int num_blocks, double scale) {
+    const int D = head_dim;
+    double *x, m, den;
+    int t, d;
+    for (d = 0; d < D; d++) o[d] = 0.0;
+    x = (double *)malloc(sizeof(double) * (size_t)L);
+    if (!x) return -1;
+    m = -INFINITY;
+    for (t = 0; t < L; t++) {
+        int pb = table[t / block_size], off = t % block_size;
+        size_t kbase;
+        double acc = 0.0;
+        if (pb < 0 || pb >= num_blocks) { free(x); return -1; }
+        kbase = (((size_t)pb * num_kv_heads + g) * block_size + off) * D;
+        for (d = 0; d < D; d++) acc += dec(q, qbase + d) * dec(kc, kbase + d);
+        x[t] = scale * acc;
+        if (x[t] > m) m = x[t];
+    }
+    den = 0.0;
+    for (t = 0; t < L; t++) {
+        int pb = table[t / block_size], off = t % block_size;
+        size_t vbase = (((size_t)pb * num_kv_heads + g) * block_size + off) * D;
+        double w = exp(x[t] - m);
+        den += w;
+        for (d = 0; d < D; d++) o[d] += w * dec(vc, vbase + d);
+    }
+    for (d = 0; d < D; d++) o[d] /= den;
+    free(x);
+    return 0;
+}
+
+int attn_ref_prefill(double *out, const void *q, const void *k_cache, const void *v_cache,
+                     int dtype, const int32_t *block_tables, const int32_t *seq_lens,
+                     const int32_t *cu_q, int num_seqs, int num_heads, int num_kv_heads,
+                     int head_dim, int block_size, int max_blocks, int num_blocks, double scale,
+                     int n_threads) {
+    dec_fn dec = pick(dtype);
+    long long total, i;
+    int bad = 0;
+    if (!dec || num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
+        num_heads % num_kv_heads || head_dim <= 0 || block_size <= 0 || max_blocks < 0 ||
+        num_blocks <= 0)
+        return -1;
+    total = num_seqs > 0 ? cu_q[num_seqs] : 0;
+    if (n_threads <= 0) n_threads = attn_ref_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads) reduction(| : bad)
+    for (i = 0; i < total * num_heads; i++) {
+        const long long r = i / num_heads;
+        const int h = (int)(i % num_heads);
+        int s = 0, n, L, p;
+        while (s + 1 < num_seqs && cu_q[s + 1] <= r) s++;
+        n = cu_q[s + 1] - cu_q[s];
+        L = seq_lens[s];
+        p = L - n + (int)(r - cu_q[s]);
+        if (n < 0 || n > L || (L + block_size - 1) / block_size > max_blocks) { bad |= 1; continue; }
+        bad |= prefill_row(out + (size_t)i * head_dim, q, ((size_t)r * num_heads + h) * head_dim,
+                           k_cache, v_cache, dec, block_tables + (size_t)s * max_blocks, p + 1,
+                           h / (num_heads / num_kv_heads), num_kv_heads, head_dim, block_size,
+                           num_blocks, scale) != 0;
+    }
+    return bad ? -1 : 0;
+}
