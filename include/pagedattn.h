@@ -150,6 +150,32 @@ int pa_decode_ex(float *out, const void *q, const void *k_cache, const void *v_c
                  int variant, void *stream);
 
 /*
+ * Multi-token (chunked prefill) attention over the paged cache [P1
+ * "Mechanism and details": new positions are appended after the prefix,
+ * whose blocks stay in place; P3 bullet 3: attention reads K/V through the
+ * block table].  For sequence s the query rows are q[cu_q_lens[s] ..
+ * cu_q_lens[s+1]): the last n_s = cu_q_lens[s+1] - cu_q_lens[s] positions of
+ * the sequence, L_s - n_s .. L_s - 1 (their K/V already appended with
+ * pa_reshape_and_cache).  Row r at position p attends causally to the
+ * sequence's tokens 0..p:
+ *   out[r][h][:] = sum_{t<=p} softmax_t(scale * <q[r][h], k_t>) v_t
+ * (the decode is the case n_s = 1).
+ *   out           device, float32 [total][num_heads][head_dim], total = cu_q_lens[B]
+ *   q             device, [total][num_heads][head_dim], `dtype` (bf16/f16)
+ *   cu_q_lens     device, int32 [num_seqs + 1], non-decreasing, cu_q_lens[0] = 0
+ *   seq_lens      device, int32 [num_seqs]: L_s including the chunk
+ *   max_q_len     host bound on n_s; max_seq_len host bound on L_s
+ * block_size >= 8 and a 16-bit dtype; fp32 caches return PA_ERR_UNSUPPORTED.
+ * n_s < 0, n_s > L_s or a bound exceeded leaves the sequence's rows
+ * unwritten and sets PA_DEVERR_SEQLEN.
+ */
+int pa_prefill(float *out, const void *q, const void *k_cache, const void *v_cache,
+               const int32_t *block_tables, const int32_t *seq_lens, const int32_t *cu_q_lens,
+               int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+               int max_blocks_per_seq, int num_blocks, int max_q_len, int max_seq_len,
+               float scale, int dtype, void *stream);
+
+/*
  * pa_decode for callers that cannot allocate device memory.  The paper has no
  * counterpart: this is a deployment variant of pa_decode.
  *

@@ -94,6 +94,14 @@ class OracleRun:
                 if self.keep_cache:
                     cache_ref.copy_between(self.k_cache, self.v_cache, self.k_host, self.v_host,
                                            pairs)
+            elif kind == "prefill":
+                sids = [x for x, _ in op[1]]
+                cu = np.concatenate([[0], np.cumsum([n for _, n in op[1]])]).astype(np.int32)
+                bt, lens = self.tables(sids)
+                res["block_tables"], res["seq_lens"] = bt, lens
+                if decode and self.keep_cache:
+                    res["out"] = attn.paged_prefill(st.q, self.k_cache, self.v_cache, bt, lens,
+                                                    cu, self.shape.scale, n_threads=n_threads)
             elif kind == "decode":
                 sids = list(op[1])
                 bt, lens = self.tables(sids)

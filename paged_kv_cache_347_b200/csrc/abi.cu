@@ -275,6 +275,69 @@ int pa_decode(float *out, const void *q, const void *k_cache, const void *v_cach
                         max_seq_len, scale, dtype, workspace, workspace_bytes, 0, 0, stream);
 }
 
+int pa_prefill(float *out, const void *q, const void *k_cache, const void *v_cache,
+               const int32_t *block_tables, const int32_t *seq_lens, const int32_t *cu_q_lens,
+               int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+               int max_blocks_per_seq, int num_blocks, int max_q_len, int max_seq_len,
+               float scale, int dtype, void *stream) {
+    clear_error();
+    int rc = check_shape(num_kv_heads, head_dim, block_size, dtype);
+    if (rc) return rc;
+    if (dtype == PA_F32 || block_size < 8)
+        return fail(PA_ERR_UNSUPPORTED, "pa_prefill takes bf16/f16 caches with block_size >= 8");
+    if (num_heads <= 0 || num_heads % num_kv_heads != 0)
+        return fail(PA_ERR_INVALID_ARG, "num_heads %d not a multiple of num_kv_heads %d",
+                    num_heads, num_kv_heads);
+    const int G = num_heads / num_kv_heads;
+    if (G > 8) return fail(PA_ERR_UNSUPPORTED, "GQA group %d > 8", G);
+    if (num_seqs < 0 || num_seqs > 65535)
+        return fail(PA_ERR_INVALID_ARG, "num_seqs %d outside [0, 65535]", num_seqs);
+    if (num_blocks <= 0 || max_blocks_per_seq < 0 || max_seq_len < 0 || max_q_len < 0 ||
+        max_q_len > max_seq_len)
+        return fail(PA_ERR_INVALID_ARG, "bad sizes");
+    if ((int64_t)max_seq_len > (int64_t)max_blocks_per_seq * block_size)
+        return fail(PA_ERR_INVALID_ARG, "max_seq_len %d > max_blocks_per_seq * block_size",
+                    max_seq_len);
+    if (!std::isfinite(scale)) return fail(PA_ERR_INVALID_ARG, "scale is not finite");
+    if (num_seqs == 0 || max_q_len == 0) return PA_OK;
+    if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens || !cu_q_lens)
+        return fail(PA_ERR_INVALID_ARG, "NULL pointer");
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) ||
+        (reinterpret_cast<uintptr_t>(block_tables) & 3u) ||
+        (reinterpret_cast<uintptr_t>(seq_lens) & 3u) ||
+        (reinterpret_cast<uintptr_t>(cu_q_lens) & 3u))
+        return fail(PA_ERR_INVALID_ARG, "misaligned pointer");
+    const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
+    if (rows + (int64_t)(num_kv_heads + 1) * block_size >= (int64_t(1) << 31))
+        return fail(PA_ERR_UNSUPPORTED, "cache too large for 32-bit TMA row coordinates");
+    unsigned int *err = device_error_ptr();
+    if (!err) return fail(PA_ERR_CUDA, "no CUDA device");
+    PrefillParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.out = out;
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.cu_q = cu_q_lens;
+    p.err = err;
+    p.num_seqs = num_seqs;
+    p.num_heads = num_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.head_dim = head_dim;
+    p.block_size = block_size;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_blocks = num_blocks;
+    p.max_seq_len = max_seq_len;
+    p.max_q_len = max_q_len;
+    p.tokens_per_cta = 64 / G;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    cudaError_t e = launch_prefill_tc(p, dtype, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+    return PA_OK;
+}
+
 int pa_copy_blocks(void *k_cache, void *v_cache, const int64_t *src_dst_pairs, int num_pairs,
                    size_t block_bytes, int num_blocks, void *stream) {
     clear_error();

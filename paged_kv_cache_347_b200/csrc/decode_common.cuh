@@ -36,6 +36,17 @@ __device__ __forceinline__ int checked_block(const DecodeParams &p, int s, int j
     return b;
 }
 
+// The same check on a raw table: entry j of row s, or -1 (PA_DEVERR_TABLE).
+__device__ __forceinline__ int checked_block_row(const int32_t *tables, int max_blocks,
+                                                 int num_blocks, unsigned int *err, int s, int j) {
+    const int b = __ldg(tables + (int64_t)s * max_blocks + j);
+    if (b < 0 || b >= num_blocks) {
+        raise_device_error(err, PA_DEVERR_TABLE);
+        return -1;
+    }
+    return b;
+}
+
 // Writes the result of one (sequence, head, split) unit: the normalised
 // output when the sequence has a single split, else the partial triple.
 // m is in log2 units; m == -inf with l == 0 means "no tokens".

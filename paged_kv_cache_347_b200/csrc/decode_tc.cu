@@ -376,10 +376,14 @@ static EncodeTiledFn encode_fn() {
     return fn;
 }
 
+}  // namespace tc
+
 // Rows of 128 bytes (64 elements), `box_rows` rows per box, over the cache
-// viewed as a [NB*Hkv*bs][D] matrix.
-static bool make_map(CUtensorMap *m, const void *base, int dtype, int D, int64_t rows,
-                     int box_rows) {
+// viewed as a [NB*Hkv*bs][D] matrix, 128B swizzle.
+bool make_cache_tensor_map(CUtensorMap *m, const void *base, int dtype, int D, int64_t rows,
+                           int box_rows) {
+    using tc::EncodeTiledFn;
+    using tc::encode_fn;
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
@@ -393,6 +397,8 @@ static bool make_map(CUtensorMap *m, const void *base, int dtype, int D, int64_t
                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
+
+namespace tc {
 
 template <typename T, int D, int BS, int W, int NS>
 static cudaError_t launch_tc_inst(const DecodeParams &p, const CUtensorMap &mk,
@@ -454,8 +460,8 @@ cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, cudaStream_t stre
     if (p.num_seqs == 0) return cudaSuccess;
     const int64_t rows = (int64_t)p.num_blocks * p.num_kv_heads * p.block_size;
     CUtensorMap mk, mv;
-    if (!tc::make_map(&mk, p.k_cache, dtype, p.head_dim, rows, p.block_size) ||
-        !tc::make_map(&mv, p.v_cache, dtype, p.head_dim, rows, p.block_size))
+    if (!make_cache_tensor_map(&mk, p.k_cache, dtype, p.head_dim, rows, p.block_size) ||
+        !make_cache_tensor_map(&mv, p.v_cache, dtype, p.head_dim, rows, p.block_size))
         return cudaErrorInvalidValue;
     if (dtype == PA_BF16)
         return p.head_dim == 128 ? tc::launch_tc_d<__nv_bfloat16, 128>(p, mk, mv, stream)

@@ -1,6 +1,7 @@
 // Host-side declarations shared by the library's translation units.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -45,6 +46,27 @@ cudaError_t launch_decode_simt(const DecodeParams &p, int dtype, cudaStream_t st
 // Tensor-core decode (bf16/f16, block_size >= 8): TMA-staged K/V, mma.sync.
 // Returns cudaErrorNotSupported for shapes it does not cover.
 cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, cudaStream_t stream);
+
+// TMA map of a cache viewed as [rows][D] 16-bit elements: 128-byte boxes of
+// box_rows rows, 128B swizzle.  False if the driver refuses it.
+bool make_cache_tensor_map(CUtensorMap *m, const void *base, int dtype, int D, int64_t rows,
+                           int box_rows);
+
+// Causal multi-token attention over the paged cache (bf16/f16, bs >= 8).
+struct PrefillParams {
+    float *out;                     // [total][Hq][D]
+    const void *q;                  // [total][Hq][D]
+    const void *k_cache, *v_cache;  // [NB][Hkv][bs][D]
+    const int32_t *block_tables;    // [B][max_blocks_per_seq]
+    const int32_t *seq_lens;        // [B], context length including the chunk
+    const int32_t *cu_q;            // [B + 1], chunk row offsets
+    unsigned int *err;
+    int num_seqs, num_heads, num_kv_heads, head_dim, block_size;
+    int max_blocks_per_seq, num_blocks, max_seq_len, max_q_len;
+    int tokens_per_cta;             // query tokens per CTA: 64 / G
+    float scale_log2;
+};
+cudaError_t launch_prefill_tc(const PrefillParams &p, int dtype, cudaStream_t stream);
 
 // Merge of split partials into out; a no-op when max_splits == 1.
 cudaError_t launch_decode_reduce(const DecodeParams &p, cudaStream_t stream);

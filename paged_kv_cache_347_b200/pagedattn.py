@@ -82,6 +82,8 @@ _sig("pa_alloc_set_host_pool", _i, _vp, _i)
 _sig("pa_seq_swap_out", _i, _vp, _i64, _vp, _i, _vp)
 _sig("pa_seq_swap_in", _i, _vp, _i64, _vp, _i, _vp)
 _sig("pa_swap_blocks", _i, _vp, _vp, _vp, _vp, _vp, _i, _sz, _i, _i, _vp)
+_sig("pa_prefill", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i,
+     _f, _i, _vp)
 
 
 class PagedAttnError(RuntimeError):
@@ -207,6 +209,30 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
         _dev(seq_lens, "seq_lens", torch.int32), B, Hq, Hkv, D, bs, W, NB, int(max_seq_len),
         float(scale), DTYPE_CODE[k_cache.dtype], ws_ptr, ws_bytes, int(partition_size),
         int(variant), _stream(q)), "pa_decode")
+    return out
+
+
+def pa_prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+               block_tables: torch.Tensor, seq_lens: torch.Tensor, cu_q_lens: torch.Tensor,
+               scale: float, max_q_len: int, max_seq_len: Optional[int] = None) -> torch.Tensor:
+    """Causal attention of each sequence's last n_s tokens (rows cu_q_lens[s]..
+    cu_q_lens[s+1] of q [total, Hq, D]) over its paged context; out float32."""
+    NB, Hkv, bs, D = k_cache.shape
+    total, Hq, Dq = q.shape
+    if Dq != D or tuple(out.shape) != (total, Hq, D):
+        raise ValueError("q/out shape mismatch")
+    B = seq_lens.numel()
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or cu_q_lens.numel() != B + 1:
+        raise ValueError("block_tables [B, W], seq_lens [B], cu_q_lens [B + 1]")
+    W = block_tables.shape[1]
+    if max_seq_len is None:
+        max_seq_len = W * bs
+    _check(_lib.pa_prefill(
+        _dev(out, "out", torch.float32), _dev(q, "q", k_cache.dtype), _dev(k_cache, "k_cache"),
+        _dev(v_cache, "v_cache", k_cache.dtype), _dev(block_tables, "block_tables", torch.int32),
+        _dev(seq_lens, "seq_lens", torch.int32), _dev(cu_q_lens, "cu_q_lens", torch.int32), B, Hq,
+        Hkv, D, bs, W, NB, int(max_q_len), int(max_seq_len), float(scale),
+        DTYPE_CODE[k_cache.dtype], _stream(q)), "pa_prefill")
     return out
 
 

@@ -34,7 +34,7 @@ from . import pagedattn as pa
 
 @dataclass
 class Action:
-    kind: str                            # "write" | "decode" | "swap_out" | "swap_in"
+    kind: str                            # "write" | "decode" | "prefill" | "swap_out" | "swap_in"
     slots: Optional[np.ndarray] = None   # int64 [n]
     pairs: Optional[np.ndarray] = None   # int64 [k, 2]
     row0: int = 0
@@ -42,6 +42,8 @@ class Action:
     tables: Optional[np.ndarray] = None  # int32 [b, width]
     lens: Optional[np.ndarray] = None    # int32 [b]
     max_len: int = 0
+    cu: Optional[np.ndarray] = None      # prefill: int32 [b + 1] row offsets
+    max_q: int = 0
     dev: dict = field(default_factory=dict)
 
 
@@ -135,6 +137,15 @@ class PagedKVRunner:
                     tables, lens = self.alloc.block_tables(list(op[1]), self.width)
                     acts.append(Action("decode", tables=tables, lens=lens,
                                        max_len=int(lens.max()) if lens.size else 0))
+                elif kind == "prefill":
+                    sids = [x for x, _ in op[1]]
+                    ns = np.array([n for _, n in op[1]], np.int32)
+                    tables, lens = self.alloc.block_tables(sids, self.width)
+                    a = Action("prefill", tables=tables, lens=lens,
+                               max_len=int(lens.max()) if lens.size else 0)
+                    a.cu = np.concatenate([[0], np.cumsum(ns)]).astype(np.int32)
+                    a.max_q = int(ns.max()) if ns.size else 0
+                    acts.append(a)
                 elif kind == "host_pool":
                     self.enable_swap(op[1])
                 elif kind == "swap_out":
@@ -162,9 +173,11 @@ class PagedKVRunner:
                 a.dev["slots"] = put(a.slots)
                 if len(a.pairs):
                     a.dev["pairs"] = put(a.pairs)
-            elif a.kind == "decode":
+            elif a.kind in ("decode", "prefill"):
                 a.dev["tables"] = put(a.tables)
                 a.dev["lens"] = put(a.lens)
+                if a.kind == "prefill":
+                    a.dev["cu"] = put(a.cu)
             elif len(a.pairs):
                 a.dev["pairs"] = put(a.pairs)
 
@@ -180,6 +193,13 @@ class PagedKVRunner:
                     pa.pa_reshape_and_cache(k_new[a.row0:a.row0 + a.nrows],
                                             v_new[a.row0:a.row0 + a.nrows], self.k_cache,
                                             self.v_cache, a.dev["slots"])
+            elif a.kind == "prefill":
+                o = torch.empty((int(a.cu[-1]), self.num_heads, self.head_dim),
+                                dtype=torch.float32, device=self.device)
+                pa.pa_prefill(o, q, self.k_cache, self.v_cache, a.dev["tables"], a.dev["lens"],
+                              a.dev["cu"], self.scale, max_q_len=a.max_q,
+                              max_seq_len=a.max_len)
+                res = o
             elif a.kind == "swap_out":
                 if "pairs" in a.dev:
                     pa.pa_swap_blocks(self.k_host, self.v_host, self.k_cache, self.v_cache,
@@ -235,9 +255,11 @@ class PagedKVRunner:
                 arrays.append((a, "slots", a.slots))
                 if len(a.pairs):
                     arrays.append((a, "pairs", a.pairs))
-            elif a.kind == "decode":
+            elif a.kind in ("decode", "prefill"):
                 arrays.append((a, "tables", a.tables))
                 arrays.append((a, "lens", a.lens))
+                if a.kind == "prefill":
+                    arrays.append((a, "cu", a.cu))
             elif len(a.pairs):
                 arrays.append((a, "pairs", a.pairs))
         offs, total = [], 0

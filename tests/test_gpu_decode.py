@@ -256,3 +256,22 @@ def test_preempted_sequence_swaps_out_and_back_and_decodes_on():
     assert len(errs) == 6 and max(errs) <= TOL["bf16"], errs
     # the victim's rows came back from host blocks into fresh device blocks
     assert gpu.alloc.stats()["swapped_seqs"] == 0 and gpu.alloc.stats()["host_free_blocks"] == 64
+
+
+# ---------------------------------------------------------------- chunked prefill
+@pytest.mark.parametrize("dtype,Hq,Hkv,D,bs", [("bf16", 32, 8, 128, 16), ("f16", 8, 8, 64, 8),
+                                               ("bf16", 16, 2, 128, 32), ("bf16", 6, 2, 64, 64),
+                                               ("f16", 12, 2, 128, 16)])
+def test_chunked_prefill_matches_oracle(dtype, Hq, Hkv, D, bs):
+    wl = workloads.chunked_prefill(batch=5, ctx_lo=0, ctx_hi=400, chunk_lo=1, chunk_hi=200,
+                                   num_heads=Hq, num_kv_heads=Hkv, head_dim=D, dtype=dtype,
+                                   block_size=bs, num_blocks=4096 // bs * 2, chunks=2)
+    errs, _, _ = run_parity(wl, table_width=1000 // bs + 2)
+    assert len(errs) == 2 and max(errs) <= TOL[dtype], errs
+
+
+def test_chunk_covering_the_whole_sequence_and_single_tokens():
+    wl = workloads.chunked_prefill(batch=6, ctx_lo=0, ctx_hi=0, chunk_lo=1, chunk_hi=130,
+                                   num_blocks=512, chunks=3)
+    errs, _, _ = run_parity(wl, table_width=32)
+    assert max(errs) <= TOL["bf16"], errs

@@ -102,6 +102,8 @@ class Shape:
 #   ("admit", sid, token_ids)        new sequence with token ids (prefix cache)
 #   ("append_tokens", sid, token_ids)
 #   ("host_pool", n_blocks) ("swap_out", sid) ("swap_in", sid)
+#   ("prefill", [(sid, n), ...])     causal attention of each sid's last n
+#                                    tokens; the step's q holds their rows
 Op = Tuple
 
 
@@ -391,6 +393,33 @@ def preempt(seed: int = 6, batch: int = 8, lo: int = 200, hi: int = 3000, steps:
             yield st
 
     return Workload(sh, gen(), "preemption by swap", {"lens": lens, "victim": victim})
+
+
+def chunked_prefill(seed: int = 7, batch: int = 4, ctx_lo: int = 0, ctx_hi: int = 600,
+                    chunk_lo: int = 1, chunk_hi: int = 300, num_heads: int = 32,
+                    num_kv_heads: int = 8, head_dim: int = 128, dtype: str = "bf16",
+                    block_size: int = 16, num_blocks: int = 1024, chunks: int = 1) -> Workload:
+    """Multi-token attention over the paged cache: each sequence has a
+    context of U[ctx_lo, ctx_hi] tokens, then ``chunks`` times appends a chunk
+    of U[chunk_lo, chunk_hi] tokens and attends them causally ("prefill",
+    [(sid, n), ...]); the chunk's queries are packed in op order."""
+    sh = Shape("chunked", num_heads, num_kv_heads, head_dim, dtype, block_size, num_blocks, seed)
+    sh.free_order = permutation(seed, num_blocks)
+    r = rng_for(seed, (6,))
+    ctx = r.integers(ctx_lo, ctx_hi, size=batch, endpoint=True).tolist()
+    sids = list(range(batch))
+
+    def gen():
+        yield _prefill_step(sh, ctx, sids, (10,), decode=False)
+        for c in range(chunks):
+            n = r.integers(chunk_lo, chunk_hi, size=batch, endpoint=True).tolist()
+            ops: List[Op] = [("append", s, int(x)) for s, x in zip(sids, n)]
+            ops.append(("prefill", [(s, int(x)) for s, x in zip(sids, n)]))
+            k, v = _kv(sh, (60, c), int(sum(n)))
+            q = normal(sh.seed, (60, c, 2), (int(sum(n)), sh.num_heads, sh.head_dim), sh.dtype)
+            yield Step(ops, k, v, q, tag="chunk")
+
+    return Workload(sh, gen(), "chunked prefill", {"ctx": ctx})
 
 
 WORKLOADS = {
