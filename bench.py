@@ -596,6 +596,47 @@ def study_blocksize(args):
     return out
 
 
+def study_prefill(args):
+    """Chunked prefill: causal attention of a 1024-token chunk per sequence
+    over a 4096-token context (8 sequences, 32/8 heads, D 128, bf16, bs 16).
+    FLOPs = sum over query rows of 4 * D * Hq * (keys attended)."""
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    from paged_kv_cache_347_b200.runner import PagedKVRunner
+    res = {"study": "prefill", "rows": []}
+    for ctx, chunk in ((4096, 1024), (0, 4096), (16384, 512)):
+        wl = workloads.chunked_prefill(batch=8, ctx_lo=ctx, ctx_hi=ctx, chunk_lo=chunk,
+                                       chunk_hi=chunk, num_blocks=8 * (ctx + chunk) // 16 + 64)
+        steps = list(wl.steps)
+        r = PagedKVRunner.for_shape(wl.shape, (ctx + chunk) // 16 + 2)
+        r.run(steps[0])
+        st = steps[1]
+        acts = r.plan(st.ops)
+        r.upload(acts)
+        dev = [t.cuda() for t in (st.k_new, st.v_new, st.q)]
+        r.execute(acts, *dev)
+        a = [x for x in acts if x.kind == "prefill"][0]
+        o = torch.empty((int(a.cu[-1]), 32, 128), dtype=torch.float32, device="cuda")
+        ms = _events_ms(lambda: pa.pa_prefill(o, dev[2], r.k_cache, r.v_cache, a.dev["tables"],
+                                              a.dev["lens"], a.dev["cu"], r.scale,
+                                              max_q_len=a.max_q, max_seq_len=a.max_len), reps=20)
+        keys = sum(ctx + i + 1 for i in range(chunk)) * 8
+        flops = 4.0 * 128 * 32 * keys
+        peak, _ = (1656.9, "measured cuBLAS bf16 burst")
+        try:
+            with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+                peak = float(json.load(f)["bf16_tflops"])
+        except (OSError, KeyError, ValueError):
+            peak = 1590.0
+        tf = flops / (ms * 1e-3) / 1e12
+        res["rows"].append({"context": ctx, "chunk": chunk, "batch": 8, "ms": round(ms, 3),
+                            "tflops": round(tf, 1), "frac_of_bf16_peak": round(tf / peak, 4),
+                            "peak_tflops": peak})
+        del r
+        torch.cuda.empty_cache()
+    res["device_errors"] = pa.device_errors()
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -606,7 +647,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--study", default="", choices=["", "prefix", "swap", "blocksize"],
+    ap.add_argument("--study", default="", choices=["", "prefix", "swap", "blocksize", "prefill"],
                     help="print one of the side studies instead of the bench line")
     ap.add_argument("--partition", type=int, default=0,
                     help="split length in tokens (0: the library default, 512)")
@@ -616,7 +657,8 @@ def main():
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.study:
-        fn = {"prefix": study_prefix, "swap": study_swap, "blocksize": study_blocksize}[args.study]
+        fn = {"prefix": study_prefix, "swap": study_swap, "blocksize": study_blocksize,
+              "prefill": study_prefill}[args.study]
         print(json.dumps(fn(args)), flush=True)
         return
     ws, rank, local, _ = dist_setup()
