@@ -616,21 +616,28 @@ def study_prefill(args):
         r.execute(acts, *dev)
         a = [x for x in acts if x.kind == "prefill"][0]
         o = torch.empty((int(a.cu[-1]), 32, 128), dtype=torch.float32, device="cuda")
-        ms = _events_ms(lambda: pa.pa_prefill(o, dev[2], r.k_cache, r.v_cache, a.dev["tables"],
-                                              a.dev["lens"], a.dev["cu"], r.scale,
-                                              max_q_len=a.max_q, max_seq_len=a.max_len), reps=20)
         keys = sum(ctx + i + 1 for i in range(chunk)) * 8
         flops = 4.0 * 128 * 32 * keys
-        peak, _ = (1656.9, "measured cuBLAS bf16 burst")
         try:
             with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
                 peak = float(json.load(f)["bf16_tflops"])
         except (OSError, KeyError, ValueError):
             peak = 1590.0
-        tf = flops / (ms * 1e-3) / 1e12
-        res["rows"].append({"context": ctx, "chunk": chunk, "batch": 8, "ms": round(ms, 3),
-                            "tflops": round(tf, 1), "frac_of_bf16_peak": round(tf / peak, 4),
-                            "peak_tflops": peak})
+        for variant, kernel in ((1, "mma.sync"), (2, "tcgen05")):
+            ms = _events_ms(lambda: pa.pa_prefill(o, dev[2], r.k_cache, r.v_cache,
+                                                  a.dev["tables"], a.dev["lens"], a.dev["cu"],
+                                                  r.scale, max_q_len=a.max_q,
+                                                  max_seq_len=a.max_len, variant=variant),
+                            reps=20)
+            tf = flops / (ms * 1e-3) / 1e12
+            row = {"kernel": kernel, "context": ctx, "chunk": chunk, "batch": 8,
+                   "ms": round(ms, 3), "tflops": round(tf, 1),
+                   "frac_of_bf16_peak": round(tf / peak, 4), "peak_tflops": peak}
+            if variant == 1:
+                first = o.clone()
+            else:  # both kernels compute the same rows at full size
+                row["max_abs_diff_vs_mma_sync"] = float((o - first).abs().max())
+            res["rows"].append(row)
         del r
         torch.cuda.empty_cache()
     res["device_errors"] = pa.device_errors()

@@ -176,6 +176,20 @@ int pa_prefill(float *out, const void *q, const void *k_cache, const void *v_cac
                float scale, int dtype, void *stream);
 
 /*
+ * pa_prefill with a choice of kernel: variant 0 = automatic, 1 = the
+ * mma.sync kernel (64 (token, head) rows per CTA, accumulators in
+ * registers), 2 = the tcgen05 kernel (128 rows per CTA, S = Q K^T and
+ * O = P V accumulated in tensor memory).  Same arguments, results (within
+ * fp32 rounding) and errors as pa_prefill; another variant returns
+ * PA_ERR_INVALID_ARG.
+ */
+int pa_prefill_ex(float *out, const void *q, const void *k_cache, const void *v_cache,
+                  const int32_t *block_tables, const int32_t *seq_lens, const int32_t *cu_q_lens,
+                  int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                  int max_blocks_per_seq, int num_blocks, int max_q_len, int max_seq_len,
+                  float scale, int dtype, int variant, void *stream);
+
+/*
  * pa_decode for callers that cannot allocate device memory.  The paper has no
  * counterpart: this is a deployment variant of pa_decode.
  *

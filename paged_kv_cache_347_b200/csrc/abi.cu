@@ -86,6 +86,8 @@ static int check_shape(int num_kv_heads, int head_dim, int block_size, int dtype
 }
 
 constexpr int kDefaultPartition = 512;
+// pa_prefill's kernel: 1 = mma.sync (registers), 2 = tcgen05 (TMEM).
+constexpr int kPrefillDefault = 1;
 
 static int partition_or_default(int partition_size) {
     return partition_size == 0 ? kDefaultPartition : partition_size;
@@ -280,7 +282,20 @@ int pa_prefill(float *out, const void *q, const void *k_cache, const void *v_cac
                int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
                int max_blocks_per_seq, int num_blocks, int max_q_len, int max_seq_len,
                float scale, int dtype, void *stream) {
+    return pa_prefill_ex(out, q, k_cache, v_cache, block_tables, seq_lens, cu_q_lens, num_seqs,
+                         num_heads, num_kv_heads, head_dim, block_size, max_blocks_per_seq,
+                         num_blocks, max_q_len, max_seq_len, scale, dtype, 0, stream);
+}
+
+int pa_prefill_ex(float *out, const void *q, const void *k_cache, const void *v_cache,
+                  const int32_t *block_tables, const int32_t *seq_lens, const int32_t *cu_q_lens,
+                  int num_seqs, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                  int max_blocks_per_seq, int num_blocks, int max_q_len, int max_seq_len,
+                  float scale, int dtype, int variant, void *stream) {
     clear_error();
+    if (variant < 0 || variant > 2)
+        return fail(PA_ERR_INVALID_ARG, "prefill variant %d not in {0, 1, 2}", variant);
+    if (variant == 0) variant = kPrefillDefault;
     int rc = check_shape(num_kv_heads, head_dim, block_size, dtype);
     if (rc) return rc;
     if (dtype == PA_F32 || block_size < 8)
@@ -331,9 +346,10 @@ int pa_prefill(float *out, const void *q, const void *k_cache, const void *v_cac
     p.num_blocks = num_blocks;
     p.max_seq_len = max_seq_len;
     p.max_q_len = max_q_len;
-    p.tokens_per_cta = 64 / G;
+    p.tokens_per_cta = (variant == 2 ? 128 : 64) / G;
     p.scale_log2 = scale * 1.4426950408889634f;
-    cudaError_t e = launch_prefill_tc(p, dtype, static_cast<cudaStream_t>(stream));
+    cudaError_t e = variant == 2 ? launch_prefill_umma(p, dtype, static_cast<cudaStream_t>(stream))
+                                 : launch_prefill_tc(p, dtype, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
     return PA_OK;
 }

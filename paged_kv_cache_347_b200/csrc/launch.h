@@ -63,10 +63,13 @@ struct PrefillParams {
     unsigned int *err;
     int num_seqs, num_heads, num_kv_heads, head_dim, block_size;
     int max_blocks_per_seq, num_blocks, max_seq_len, max_q_len;
-    int tokens_per_cta;             // query tokens per CTA: 64 / G
+    int tokens_per_cta;             // query tokens per CTA: 64 / G (mma.sync), 128 / G (tcgen05)
     float scale_log2;
 };
+// mma.sync kernel: 64 (token, head) rows per CTA, accumulators in registers.
 cudaError_t launch_prefill_tc(const PrefillParams &p, int dtype, cudaStream_t stream);
+// tcgen05 kernel: 128 rows per CTA, S and O accumulated in TMEM.
+cudaError_t launch_prefill_umma(const PrefillParams &p, int dtype, cudaStream_t stream);
 
 // Merge of split partials into out; a no-op when max_splits == 1.
 cudaError_t launch_decode_reduce(const DecodeParams &p, cudaStream_t stream);

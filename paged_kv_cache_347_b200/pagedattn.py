@@ -84,6 +84,8 @@ _sig("pa_seq_swap_in", _i, _vp, _i64, _vp, _i, _vp)
 _sig("pa_swap_blocks", _i, _vp, _vp, _vp, _vp, _vp, _i, _sz, _i, _i, _vp)
 _sig("pa_prefill", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i,
      _f, _i, _vp)
+_sig("pa_prefill_ex", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
+     _i, _f, _i, _i, _vp)
 
 
 class PagedAttnError(RuntimeError):
@@ -214,9 +216,11 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
 
 def pa_prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                block_tables: torch.Tensor, seq_lens: torch.Tensor, cu_q_lens: torch.Tensor,
-               scale: float, max_q_len: int, max_seq_len: Optional[int] = None) -> torch.Tensor:
+               scale: float, max_q_len: int, max_seq_len: Optional[int] = None,
+               variant: int = 0) -> torch.Tensor:
     """Causal attention of each sequence's last n_s tokens (rows cu_q_lens[s]..
-    cu_q_lens[s+1] of q [total, Hq, D]) over its paged context; out float32."""
+    cu_q_lens[s+1] of q [total, Hq, D]) over its paged context; out float32.
+    variant: 0 automatic, 1 the mma.sync kernel, 2 the tcgen05 kernel."""
     NB, Hkv, bs, D = k_cache.shape
     total, Hq, Dq = q.shape
     if Dq != D or tuple(out.shape) != (total, Hq, D):
@@ -227,12 +231,12 @@ def pa_prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cach
     W = block_tables.shape[1]
     if max_seq_len is None:
         max_seq_len = W * bs
-    _check(_lib.pa_prefill(
+    _check(_lib.pa_prefill_ex(
         _dev(out, "out", torch.float32), _dev(q, "q", k_cache.dtype), _dev(k_cache, "k_cache"),
         _dev(v_cache, "v_cache", k_cache.dtype), _dev(block_tables, "block_tables", torch.int32),
         _dev(seq_lens, "seq_lens", torch.int32), _dev(cu_q_lens, "cu_q_lens", torch.int32), B, Hq,
         Hkv, D, bs, W, NB, int(max_q_len), int(max_seq_len), float(scale),
-        DTYPE_CODE[k_cache.dtype], _stream(q)), "pa_prefill")
+        DTYPE_CODE[k_cache.dtype], int(variant), _stream(q)), "pa_prefill")
     return out
 
 

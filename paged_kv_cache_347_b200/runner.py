@@ -51,7 +51,8 @@ class PagedKVRunner:
     def __init__(self, num_blocks: int, block_size: int, num_heads: int, num_kv_heads: int,
                  head_dim: int, dtype: torch.dtype, scale: float, table_width: int,
                  free_order: Optional[Sequence[int]] = None, max_blocks_per_seq: int = 0,
-                 device: str = "cuda", partition_size: int = 0, variant: int = 0):
+                 device: str = "cuda", partition_size: int = 0, variant: int = 0,
+                 prefill_variant: int = 0):
         self.alloc = pa.BlockAllocator(num_blocks, block_size, free_order, max_blocks_per_seq)
         self.device = torch.device(device)
         dims = (num_blocks, num_kv_heads, block_size, head_dim)
@@ -61,6 +62,7 @@ class PagedKVRunner:
         self.block_size, self.num_blocks = block_size, num_blocks
         self.dtype, self.scale, self.width = dtype, scale, table_width
         self.partition_size, self.variant = partition_size, variant
+        self.prefill_variant = prefill_variant
 
     @classmethod
     def for_shape(cls, shape, table_width: int, **kw) -> "PagedKVRunner":
@@ -198,7 +200,7 @@ class PagedKVRunner:
                                 dtype=torch.float32, device=self.device)
                 pa.pa_prefill(o, q, self.k_cache, self.v_cache, a.dev["tables"], a.dev["lens"],
                               a.dev["cu"], self.scale, max_q_len=a.max_q,
-                              max_seq_len=a.max_len)
+                              max_seq_len=a.max_len, variant=self.prefill_variant)
                 res = o
             elif a.kind == "swap_out":
                 if "pairs" in a.dev:

@@ -23,14 +23,14 @@ def sample_pairs(b: int, hq: int, n: int, seed: int) -> List[Tuple[int, int]]:
 
 def run_parity(wl, table_width: int, sample: Optional[int] = None, max_steps: Optional[int] = None,
                partition_size: int = 0, variant: int = 0, compare_cache: bool = False,
-               check_slots: bool = True):
+               check_slots: bool = True, prefill_variant: int = 0):
     """Returns a list of per-decode max-abs errors; asserts slots and pairs
     are bit-exact (and the caches too, when ``compare_cache``)."""
     from paged_kv_cache_347_b200.runner import PagedKVRunner
     sh = wl.shape
     orc = OracleRun(sh)
     gpu = PagedKVRunner.for_shape(sh, table_width, partition_size=partition_size,
-                                  variant=variant)
+                                  variant=variant, prefill_variant=prefill_variant)
     errs = []
     for i, st in enumerate(wl.steps):
         if max_steps is not None and i >= max_steps:

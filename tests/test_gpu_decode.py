@@ -259,19 +259,33 @@ def test_preempted_sequence_swaps_out_and_back_and_decodes_on():
 
 
 # ---------------------------------------------------------------- chunked prefill
+# prefill_variant 1 = mma.sync kernel, 2 = tcgen05 kernel (TMEM accumulators)
+@pytest.mark.parametrize("pv", [1, 2])
 @pytest.mark.parametrize("dtype,Hq,Hkv,D,bs", [("bf16", 32, 8, 128, 16), ("f16", 8, 8, 64, 8),
                                                ("bf16", 16, 2, 128, 32), ("bf16", 6, 2, 64, 64),
-                                               ("f16", 12, 2, 128, 16)])
-def test_chunked_prefill_matches_oracle(dtype, Hq, Hkv, D, bs):
+                                               ("f16", 12, 2, 128, 16), ("bf16", 7, 7, 128, 8)])
+def test_chunked_prefill_matches_oracle(dtype, Hq, Hkv, D, bs, pv):
     wl = workloads.chunked_prefill(batch=5, ctx_lo=0, ctx_hi=400, chunk_lo=1, chunk_hi=200,
                                    num_heads=Hq, num_kv_heads=Hkv, head_dim=D, dtype=dtype,
                                    block_size=bs, num_blocks=4096 // bs * 2, chunks=2)
-    errs, _, _ = run_parity(wl, table_width=1000 // bs + 2)
+    errs, _, _ = run_parity(wl, table_width=1000 // bs + 2, prefill_variant=pv)
     assert len(errs) == 2 and max(errs) <= TOL[dtype], errs
 
 
-def test_chunk_covering_the_whole_sequence_and_single_tokens():
+@pytest.mark.parametrize("pv", [1, 2])
+def test_chunk_covering_the_whole_sequence_and_single_tokens(pv):
     wl = workloads.chunked_prefill(batch=6, ctx_lo=0, ctx_hi=0, chunk_lo=1, chunk_hi=130,
                                    num_blocks=512, chunks=3)
-    errs, _, _ = run_parity(wl, table_width=32)
+    errs, _, _ = run_parity(wl, table_width=32, prefill_variant=pv)
+    assert max(errs) <= TOL["bf16"], errs
+
+
+@pytest.mark.parametrize("pv", [1, 2])
+def test_prefill_long_context(pv):
+    """Chunks of 512-1024 rows after 2k-6k tokens of context: many 64-key
+    stages per CTA, several CTAs per sequence, ragged last CTA and stage."""
+    wl = workloads.chunked_prefill(batch=2, ctx_lo=2000, ctx_hi=4000, chunk_lo=512,
+                                   chunk_hi=1024, num_heads=16, num_kv_heads=4, head_dim=128,
+                                   dtype="bf16", block_size=16, num_blocks=1024, chunks=1)
+    errs, _, _ = run_parity(wl, table_width=5100 // 16 + 2, prefill_variant=pv)
     assert max(errs) <= TOL["bf16"], errs
