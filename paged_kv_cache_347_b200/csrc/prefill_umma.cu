@@ -1,5 +1,5 @@
 // Causal multi-token attention over the paged cache on the 5th-generation
-// tensor cores (tcgen05, accumulators in TMEM), sm_100a.
+// tensor cores (tcgen05, accumulators in tensor memory), sm_100a.
 //
 // Same quantity as prefill_tc.cu (mbrenndoerfer.com "Paged Attention >
 // Summary", bullet 3; paweldubiel.com "PagedAttention", "Mechanism and
@@ -7,24 +7,28 @@
 // positions 0..L-n+r through the block table.
 //
 // CTA = 128 (token, query head) rows: 128/G chunk tokens of one KV head g of
-// one sequence.  Six warps:
-//   * warps 0-3 (one thread per row, thread i <-> TMEM lane i): load the Q rows
-//     into a 128B-swizzled shared tile; per stage read the S tile from TMEM,
-//     apply the causal mask, keep the row's running max and sum in fp32, write
-//     P (bf16/f16 high part and remainder) into a swizzled shared tile,
-//     rescale the O accumulator in TMEM when the row max grows by more than
-//     2^8; at the end read O from TMEM, divide by the sum and store;
-//   * warp 4: TMA producer of 64-key K/V stages (the decode's ring);
-//   * warp 5, one thread: issues the UMMAs --
-//       S[128 x 64]  = Q[128 x D] . K_stage^T            (both K-major)
-//       O[128 x D]  += P[128 x 64] . V_stage[64 x D]     (P K-major, V N-major)
-//     and commits them to mbarriers.  S is double-buffered in TMEM, so S of
-//     stage i+1 is computed while the softmax works on stage i.
-// TMEM: S0 (64 cols), S1 (64), O (D): 256 columns allocated.
+// one sequence; the context is walked in stages of 128 keys.  Ten warps:
+//   * warps 0-7, softmax: two threads per row -- warp w serves TMEM lanes
+//     32 (w % 4) .. +31 (the rows) and keys 64 (w / 4) .. +63 of each stage.
+//     Per stage a thread reads its 64 S values from TMEM, applies the causal
+//     mask, agrees the row maximum with its partner thread (through shared
+//     memory and an mbarrier), writes P = 2^(x - m) into TMEM as 16-bit
+//     high part + remainder, and rescales its half of the O row when the
+//     maximum has grown by more than 2^8; at the end it divides by the summed
+//     weights and stores its half of the row;
+//   * warp 8: TMA producer of K/V stages gathered block by block through the
+//     table (the decode's ring);
+//   * warp 9, one thread: issues the UMMAs --
+//       S[128 x 128]  = Q[128 x D] . K_stage^T       (Q, K from shared memory)
+//       O[128 x D]   += P[128 x 128] . V_stage       (P from TMEM, V N-major)
+//     and commits them to mbarriers.  S is double-buffered, so S of stage
+//     i+1 runs on the tensor core while the softmax works on stage i.
+// TMEM (512 columns): S0 [0,128), S1 [128,256), O [256,256+D),
+// P high part [384,448), P remainder [448,512).
 //
 // Every wait is bounded (~2 s); on a timeout the CTA records
-// PA_DEVERR_TIMEOUT, waits (bounded) for its own copies and MMAs, frees its
-// TMEM and exits.
+// PA_DEVERR_TIMEOUT, the other warps stop waiting, the producer waits
+// (bounded) for its copies, warp 0 waits for the MMAs and frees the TMEM.
 #include <math.h>
 
 #include <mutex>
@@ -35,48 +39,64 @@
 namespace pa {
 namespace pu {
 
-constexpr int kM = 128;          // rows per CTA
-constexpr int kKeys = 64;        // keys per stage
-constexpr int kThreads = 6 * 32;
-constexpr int kSoftmaxThreads = 128;
-constexpr int kTmemCols = 256;
-constexpr int kRowBytes = 128;
+constexpr int kM = 128;              // rows per CTA
+constexpr int kKeys = 128;           // keys per stage
+constexpr int kSoftmaxThreads = 256; // 8 warps, two threads per row
+constexpr int kThreads = kSoftmaxThreads + 64;
+constexpr int kTmemCols = 512;
+constexpr int kColO = 256, kColPHi = 384, kColPLo = 448;
+constexpr int kRowBytes = 128;       // one 64-element piece of a 16-bit row
 
 template <int D, int BS, int NS>
 struct Cfg {
     static constexpr int kPieces = D / 64;
-    static constexpr int kQPiece = kM * kRowBytes;              // 16 KB
+    static constexpr int kQPiece = kM * kRowBytes;        // 16 KB
     static constexpr int kQBytes = kPieces * kQPiece;
-    static constexpr int kKVPiece = kKeys * kRowBytes;          // 8 KB
+    static constexpr int kKVPiece = kKeys * kRowBytes;    // 16 KB
     static constexpr int kKBytes = kPieces * kKVPiece;
-    static constexpr int kStageBytes = 2 * kKBytes;             // K + V
-    static constexpr int kPTile = kM * kRowBytes;               // 128 rows x 64 keys x 2 B
-    static constexpr int kPBytes = 2 * kPTile;                  // high part + remainder
+    static constexpr int kStageBytes = 2 * kKBytes;       // K + V
     static constexpr int kQOffset = 0;
     static constexpr int kKVOffset = kQBytes;
-    static constexpr int kPOffset = kKVOffset + NS * kStageBytes;
-    static constexpr int kBarOffset = kPOffset + 2 * kPBytes;
-    // barriers: kv_full[NS] kv_empty[NS] s_full[2] s_empty[2] p_full[2] pv_done[2] q_full mma_done
-    static constexpr int kNumBars = 2 * NS + 8 + 2;
+    static constexpr int kXchOffset = kKVOffset + NS * kStageBytes;  // float [2][2][128]
+    static constexpr int kBarOffset = kXchOffset + 2 * 2 * kM * 4;
+    // kv_full[NS] kv_empty[NS] s_full[2] s_empty[2] p_full pv_done q_full mma_done xchg[4]
+    static constexpr int kNumBars = 2 * NS + 4 + 4 + 4;
     static constexpr int kTmemSlot = kBarOffset + kNumBars * 8;
     static constexpr int kAbortOffset = kTmemSlot + 16;
     static constexpr int kSmemBytes = kAbortOffset + 16;
     static constexpr int kDynSmem = kSmemBytes + 1024;
     static constexpr int kBlocksPerStage = kKeys / BS;
     static_assert(kDynSmem <= 227 * 1024, "shared memory");
-    static_assert(kKeys % BS == 0, "block size divides a stage");
+    static_assert(kKeys % BS == 0 && kBlocksPerStage <= 32, "block size");
+    static_assert(D == 64 || D == 128, "head size");
 };
 
-__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
-    return mbar_wait_bounded(bar, parity, abort_flag);
-}
-
-// The same wait taken by a whole warp, with one outcome for all its lanes
-// (the tcgen05 loads and stores that follow are warp-collective).
-__device__ __forceinline__ bool warp_wait_bar(uint32_t bar, uint32_t parity,
-                                              volatile int *abort_flag) {
+// A bounded mbarrier wait taken by a whole warp, with one outcome for all
+// its lanes (the tcgen05 loads and stores that follow are warp-collective).
+__device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag) {
     return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort_flag));
 }
+
+// Two weights -> their 16-bit high parts and remainders, one 32-bit word each
+// (lower key in the low half).  bf16: round the fp32 bit pattern to its upper
+// 16 bits (half up in magnitude); the remainder x - hi is exact in fp32 and
+// is rounded the same way.  f16 uses the hardware conversions.
+template <typename T> struct PSplit;
+template <> struct PSplit<__nv_bfloat16> {
+    __device__ __forceinline__ static void run(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+        const uint32_t a = __float_as_uint(x0) + 0x8000u, b = __float_as_uint(x1) + 0x8000u;
+        hi = __byte_perm(a, b, 0x7632);
+        const float r0 = x0 - __uint_as_float(a & 0xffff0000u);
+        const float r1 = x1 - __uint_as_float(b & 0xffff0000u);
+        lo = __byte_perm(__float_as_uint(r0) + 0x8000u, __float_as_uint(r1) + 0x8000u, 0x7632);
+    }
+};
+template <> struct PSplit<__half> {
+    __device__ __forceinline__ static void run(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+        hi = Mma<__half>::pack(x0, x1);
+        lo = Mma<__half>::pack(x0 - Mma<__half>::lo(hi), x1 - Mma<__half>::hi(hi));
+    }
+};
 
 template <typename T, int D, int BS, int NS>
 __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
@@ -110,11 +130,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t q_s = sbase + C::kQOffset, kv_s = sbase + C::kKVOffset, p_s = sbase + C::kPOffset;
+    const uint32_t q_s = sbase + C::kQOffset, kv_s = sbase + C::kKVOffset;
     const uint32_t bar0 = sbase + C::kBarOffset;
     const uint32_t kv_full = bar0, kv_empty = bar0 + 8 * NS, s_full = bar0 + 16 * NS,
-                   s_empty = s_full + 16, p_full = s_empty + 16, pv_done = p_full + 16,
-                   q_full = pv_done + 16, mma_done = q_full + 8;
+                   s_empty = s_full + 16, p_full = s_empty + 16, pv_done = p_full + 8,
+                   q_full = pv_done + 8, mma_done = q_full + 8, xchg = mma_done + 8;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kAbortOffset);
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + C::kTmemSlot);
 
@@ -126,11 +146,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         for (int i = 0; i < 2; ++i) {
             mbar_init(s_full + 8 * i, 1);
             mbar_init(s_empty + 8 * i, kSoftmaxThreads);
-            mbar_init(p_full + 8 * i, kSoftmaxThreads);
-            mbar_init(pv_done + 8 * i, 1);
         }
+        mbar_init(p_full, kSoftmaxThreads);
+        mbar_init(pv_done, 1);
         mbar_init(q_full, kSoftmaxThreads);
         mbar_init(mma_done, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(xchg + 8 * i, 64);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -144,7 +165,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     const uint32_t tmem = *tmem_slot;
 
     // ------------------------------------------------------------ producer
-    if (warp == 4) {
+    if (warp == 8) {
         if (lane == 0) {
             prefetch_tensormap(&tmap_k);
             prefetch_tensormap(&tmap_v);
@@ -158,39 +179,32 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
             if (lane < jn) {
                 const int b = checked_block_row(p.block_tables, p.max_blocks_per_seq, p.num_blocks,
                                                 p.err, s, jb + lane);
-                mine = b < 0 ? p.num_blocks : b;
+                mine = b < 0 ? p.num_blocks : b;  // out of range: the copy reads the fill value
             }
-            int ent[C::kBlocksPerStage];
-#pragma unroll
-            for (int j = 0; j < C::kBlocksPerStage; ++j) ent[j] = __shfl_sync(0xffffffffu, mine, j);
             int stop = 0;
-            if (lane == 0) {
-                const int buf = i % NS;
-                if (i >= NS && !wait_bar(kv_empty + 8 * buf, ((i / NS) - 1) & 1, abort_flag)) {
-                    raise_device_error(p.err, PA_DEVERR_TIMEOUT);
-                    *abort_flag = 1;
-                    stop = 1;
-                } else {
-                    const uint32_t full = kv_full + 8 * buf;
-                    mbar_arrive_expect_tx(full, (uint32_t)(jn * 4 * BS * D));
-                    const uint32_t kdst = kv_s + buf * C::kStageBytes;
-                    const uint32_t vdst = kdst + C::kKBytes;
-#pragma unroll
-                    for (int j = 0; j < C::kBlocksPerStage; ++j) {
-                        if (j < jn) {
-                            const int y = (ent[j] * p.num_kv_heads + g) * BS;
-#pragma unroll
-                            for (int pc = 0; pc < C::kPieces; ++pc) {
-                                const uint32_t off = pc * C::kKVPiece + j * BS * kRowBytes;
-                                tma_load_2d(kdst + off, &tmap_k, pc * 64, y, full, policy);
-                                tma_load_2d(vdst + off, &tmap_v, pc * 64, y, full, policy);
-                            }
-                        }
-                    }
-                    issued = i + 1;
-                }
+            const int buf = i % NS;
+            if (lane == 0 && i >= NS &&
+                !mbar_wait_bounded(kv_empty + 8 * buf, ((i / NS) - 1) & 1, abort_flag)) {
+                raise_device_error(p.err, PA_DEVERR_TIMEOUT);
+                *abort_flag = 1;
+                stop = 1;
             }
             if (__shfl_sync(0xffffffffu, stop, 0)) break;
+            const uint32_t full = kv_full + 8 * buf;
+            if (lane == 0) mbar_arrive_expect_tx(full, (uint32_t)(jn * 4 * BS * D));
+            __syncwarp();
+            // lane j < jn copies block j of the stage: its K and V rows, every piece
+            if (lane < jn) {
+                const uint32_t kdst = kv_s + buf * C::kStageBytes;
+                const int y = (mine * p.num_kv_heads + g) * BS;
+#pragma unroll
+                for (int pc = 0; pc < C::kPieces; ++pc) {
+                    const uint32_t off = pc * C::kKVPiece + lane * BS * kRowBytes;
+                    tma_load_2d(kdst + off, &tmap_k, pc * 64, y, full, policy);
+                    tma_load_2d(kdst + C::kKBytes + off, &tmap_v, pc * 64, y, full, policy);
+                }
+            }
+            issued = i + 1;
         }
         if (lane == 0)
             for (int i = max(0, issued - NS); i < issued; ++i)
@@ -199,17 +213,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     }
 
     // ------------------------------------------------------------ MMA issuer
-    if (warp == 5) {
+    if (warp == 9) {
         if (lane == 0) {
             constexpr uint32_t fmt = StoreT<T>::kCode == PA_BF16 ? 1u : 0u;
             constexpr uint32_t idesc_s = umma::idesc_f16(fmt, kM, kKeys, 0);
             constexpr uint32_t idesc_o = umma::idesc_f16(fmt, kM, D, 1);
-            bool ok = wait_bar(q_full, 0, abort_flag);
-            // S_i = Q . K_i^T into TMEM columns 64 * (i % 2)
+            bool ok = mbar_wait_bounded(q_full, 0, abort_flag);
+            // S_i = Q . K_i^T into TMEM columns 128 * (i % 2)
             auto issue_s = [&](int i) -> bool {
                 const int buf = i % NS;
-                if (!wait_bar(kv_full + 8 * buf, (i / NS) & 1, abort_flag)) return false;
-                if (i >= 2 && !wait_bar(s_empty + 8 * (i % 2), ((i / 2) - 1) & 1, abort_flag))
+                if (!mbar_wait_bounded(kv_full + 8 * buf, (i / NS) & 1, abort_flag)) return false;
+                if (i >= 2 && !mbar_wait_bounded(s_empty + 8 * (i % 2), ((i / 2) - 1) & 1,
+                                                 abort_flag))
                     return false;
                 umma::fence_after_sync();
                 const uint32_t kst = kv_s + buf * C::kStageBytes;
@@ -231,23 +246,22 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
                     break;
                 }
                 // O += P_i . V_i once the softmax has written P_i
-                if (!wait_bar(p_full + 8 * (i % 2), (i / 2) & 1, abort_flag)) {
+                if (!mbar_wait_bounded(p_full, i & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 umma::fence_after_sync();
                 const uint32_t vst = kv_s + (i % NS) * C::kStageBytes + C::kKBytes;
-                const uint32_t pst = p_s + (i % 2) * C::kPBytes;
 #pragma unroll
                 for (int j = 0; j < kKeys / 16; ++j) {
+                    // keys 16j..16j+15: V rows (8-row groups 1 KB apart), 64-column pieces 16 KB apart
                     const uint64_t b = umma::smem_desc_sw128(vst + j * 16 * kRowBytes,
                                                              C::kKVPiece, 1024);
-                    const uint64_t a_hi = umma::smem_desc_sw128(pst + j * 32, 16, 1024);
-                    const uint64_t a_lo = umma::smem_desc_sw128(pst + C::kPTile + j * 32, 16, 1024);
-                    umma::mma_f16(tmem + 2 * kKeys, a_hi, b, idesc_o, (i > 0 || j > 0) ? 1u : 0u);
-                    umma::mma_f16(tmem + 2 * kKeys, a_lo, b, idesc_o, 1u);
+                    umma::mma_f16_ts(tmem + kColO, tmem + kColPHi + 8 * j, b, idesc_o,
+                                     (i > 0 || j > 0) ? 1u : 0u);
+                    umma::mma_f16_ts(tmem + kColO, tmem + kColPLo + 8 * j, b, idesc_o, 1u);
                 }
-                umma::commit(pv_done + 8 * (i % 2));
+                umma::commit(pv_done);
                 umma::commit(kv_empty + 8 * (i % NS));
             }
             if (!ok) {
@@ -260,138 +274,148 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     }
 
     // ------------------------------------------------------------ softmax warps
-    const int r = threadIdx.x;  // row == TMEM lane
-    const int t = r / G, hh = r - (r / G) * G;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;  // row == TMEM lane
+    const int t = r / G, hh = r - t * G;
     const bool valid = t < ntok && r < TQ * G;
     const int qp = valid ? pos0 + t : nkeys - 1;
     const int64_t qrow = ((int64_t)(q0 + tok0 + t) * p.num_heads + g * G + hh) * D;
     {
-        // Q row -> swizzled K-major tile (row r, 16-byte chunk c at c ^ (r & 7))
+        // this thread's half of the Q row -> swizzled K-major tile
+        // (row r, 16-byte chunk c at c ^ (r & 7) within its 128-byte piece row)
         const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.q) + qrow);
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
+        for (int k = 0; k < D / 16; ++k) {
+            const int c = half * (D / 16) + k;
             const uint4 v = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-            const int pc = c >> 3, cc = c & 7;
-            *reinterpret_cast<uint4 *>(smem + C::kQOffset + pc * C::kQPiece + r * kRowBytes +
-                                       ((cc ^ (r & 7)) << 4)) = v;
+            *reinterpret_cast<uint4 *>(smem + C::kQOffset + (c >> 3) * C::kQPiece +
+                                       r * kRowBytes + (((c & 7) ^ (r & 7)) << 4)) = v;
         }
         umma::fence_proxy_async_smem();
         mbar_arrive(q_full);
     }
-    const uint32_t lane_base = tmem + ((uint32_t)(warp * 32) << 16);
+    float *xch = reinterpret_cast<float *>(smem + C::kXchOffset);  // [parity][half][row]
+    const uint32_t my_xchg = xchg + 8 * quarter;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int i = 0; i < nstages; ++i) {
-        const int sb = i % 2;
-        if (!warp_wait_bar(s_full + 8 * sb, (i / 2) & 1, abort_flag)) {
+        const int sb = i & 1;
+        if (!warp_wait(s_full + 8 * sb, (i >> 1) & 1, abort_flag)) {
             ok = false;
             break;
         }
         umma::fence_after_sync();
         uint32_t sr[2][32];
-        umma::ld32(lane_base + sb * kKeys, sr[0]);
-        umma::ld32(lane_base + sb * kKeys + 32, sr[1]);
+        umma::ld32(lane_base + sb * kKeys + half * 64, sr[0]);
+        umma::ld32(lane_base + sb * kKeys + half * 64 + 32, sr[1]);
         umma::wait_ld();
         umma::fence_before_sync();
         mbar_arrive(s_empty + 8 * sb);
-        const int kb = i * kKeys;
-        float x[kKeys];
+        const int kb = i * kKeys + half * 64;
+        float x[64];
         float mx = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < kKeys; ++c) {
+        for (int c = 0; c < 64; ++c) {
             const float v = __uint_as_float(sr[c >> 5][c & 31]) * sl2;
             x[c] = kb + c > qp ? -INFINITY : v;
             mx = fmaxf(mx, x[c]);
         }
+        // the row maximum of this stage over both halves
+        xch[(sb * 2 + half) * kM + r] = mx;
+        mbar_arrive(my_xchg);
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(my_xchg, i & 1, abort_flag))) {
+            ok = false;
+            break;
+        }
+        mx = fmaxf(mx, xch[(sb * 2 + (half ^ 1)) * kM + r]);
         // the running max moves only when it grows by more than 8 (log2 units):
         // weights then stay below 2^8 and O is rescaled rarely
         float alpha = 1.f;
         bool rescale = false;
         if (mx > m + 8.f) {
-            alpha = exp2f(m - mx);  // 0 on the first stage (m = -inf)
+            alpha = umma::ex2(m - mx);  // 0 on the first stage (m = -inf)
             rescale = m != -INFINITY;
             m = mx;
         }
         float sum = 0.f;
 #pragma unroll
-        for (int c = 0; c < kKeys; ++c) {
-            x[c] = exp2f(x[c] - m);
+        for (int c = 0; c < 64; ++c) {
+            x[c] = umma::ex2(x[c] - m);
             sum += x[c];
         }
         l = l * alpha + sum;
-        // PV of stage i-1 (and of i-2, which used this P buffer) must be done
-        if (i > 0 && !warp_wait_bar(pv_done + 8 * ((i - 1) % 2), ((i - 1) / 2) & 1, abort_flag)) {
+        uint32_t ph[32], pl[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) PSplit<T>::run(x[2 * e], x[2 * e + 1], ph[e], pl[e]);
+        // PV of stage i-1 must be done before O is rescaled and P overwritten
+        if (i > 0 && !warp_wait(pv_done, (i - 1) & 1, abort_flag)) {
             ok = false;
             break;
         }
+        umma::fence_after_sync();
+        umma::st32(lane_base + kColPHi + half * 32, ph);
+        umma::st32(lane_base + kColPLo + half * 32, pl);
         if (__any_sync(0xffffffffu, rescale)) {  // warp-collective TMEM access
-            umma::fence_after_sync();
 #pragma unroll
-            for (int cb = 0; cb < D / 32; ++cb) {
-                uint32_t orr[32];
-                umma::ld32(lane_base + 2 * kKeys + cb * 32, orr);
+            for (int cb = 0; cb < D / 64; ++cb) {
+                uint32_t o[32];
+                const uint32_t col = lane_base + kColO + half * (D / 2) + cb * 32;
+                umma::ld32(col, o);
                 umma::wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
-                umma::st32(lane_base + 2 * kKeys + cb * 32, orr);
+                for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                umma::st32(col, o);
             }
-            umma::wait_st();
         }
-        // stale K/V rows past the last key of the tile: zero V so 0 * x stays 0
-        if (kb + kKeys > nkeys) {
-            // the stage's copies have landed (the S MMA waited for them); this
-            // wait only orders the zero stores after them
-            if (!warp_wait_bar(kv_full + 8 * (i % NS), (i / NS) & 1, abort_flag)) {
+        if (i * kKeys + kKeys > nkeys) {
+            // last stage: rows past the last key hold stale or unwritten data;
+            // zero them in V so that their zero weights give exact zeros.  The
+            // wait only orders these stores after the stage's copies.
+            if (!warp_wait(kv_full + 8 * (i % NS), (i / NS) & 1, abort_flag)) {
                 ok = false;
                 break;
             }
-            const int first = nkeys - kb;  // rows [first, 64) of this stage
+            const int first = nkeys - i * kKeys;  // rows [first, 128)
             uint8_t *vst = smem + C::kKVOffset + (i % NS) * C::kStageBytes + C::kKBytes;
-            for (int idx = r; idx < (kKeys - first) * C::kPieces * 8; idx += kSoftmaxThreads) {
+            for (int idx = threadIdx.x; idx < (kKeys - first) * C::kPieces * 8;
+                 idx += kSoftmaxThreads) {
                 const int row = first + idx / (C::kPieces * 8);
                 const int rem = idx % (C::kPieces * 8);
                 *reinterpret_cast<uint4 *>(vst + (rem >> 3) * C::kKVPiece + row * kRowBytes +
                                            ((rem & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
             }
+            umma::fence_proxy_async_smem();
         }
-        // P (high part, remainder) -> swizzled K-major tiles, row r
-        uint8_t *ph = smem + C::kPOffset + sb * C::kPBytes;
-#pragma unroll
-        for (int c = 0; c < kKeys / 8; ++c) {
-            uint32_t hi[4], lo[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                hi[e] = Mma<T>::pack(x[8 * c + 2 * e], x[8 * c + 2 * e + 1]);
-                lo[e] = Mma<T>::pack(x[8 * c + 2 * e] - Mma<T>::lo(hi[e]),
-                                     x[8 * c + 2 * e + 1] - Mma<T>::hi(hi[e]));
-            }
-            const int off = r * kRowBytes + ((c ^ (r & 7)) << 4);
-            *reinterpret_cast<uint4 *>(ph + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-            *reinterpret_cast<uint4 *>(ph + C::kPTile + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-        }
-        umma::fence_proxy_async_smem();
+        umma::wait_st();
         umma::fence_before_sync();
-        mbar_arrive(p_full + 8 * sb);
+        mbar_arrive(p_full);
     }
-    if (ok && !warp_wait_bar(pv_done + 8 * ((nstages - 1) % 2), ((nstages - 1) / 2) & 1, abort_flag))
-        ok = false;
+    if (ok && !warp_wait(pv_done, (nstages - 1) & 1, abort_flag)) ok = false;
     if (ok) {
+        // the two halves' weight sums
+        xch[((nstages & 1) * 2 + half) * kM + r] = l;
+        mbar_arrive(my_xchg);
+        ok = __all_sync(0xffffffffu, mbar_wait_bounded(my_xchg, nstages & 1, abort_flag));
+    }
+    if (ok) {
+        l += xch[((nstages & 1) * 2 + (half ^ 1)) * kM + r];
         umma::fence_after_sync();
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        float *dst = p.out + qrow;
+        float *dst = p.out + qrow + half * (D / 2);
 #pragma unroll
-        for (int cb = 0; cb < D / 32; ++cb) {
-            uint32_t orr[32];
-            umma::ld32(lane_base + 2 * kKeys + cb * 32, orr);
+        for (int cb = 0; cb < D / 64; ++cb) {
+            uint32_t o[32];
+            umma::ld32(lane_base + kColO + half * (D / 2) + cb * 32, o);
             umma::wait_ld();
             if (valid) {
 #pragma unroll
                 for (int e = 0; e < 32; e += 4)
                     *reinterpret_cast<float4 *>(dst + cb * 32 + e) =
-                        make_float4(__uint_as_float(orr[e]) * inv, __uint_as_float(orr[e + 1]) * inv,
-                                    __uint_as_float(orr[e + 2]) * inv,
-                                    __uint_as_float(orr[e + 3]) * inv);
+                        make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
+                                    __uint_as_float(o[e + 2]) * inv,
+                                    __uint_as_float(o[e + 3]) * inv);
             }
         }
     } else if (lane == 0) {
@@ -399,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         *abort_flag = 1;  // the other warps stop waiting
     }
     // TMEM is freed once every MMA of this CTA has completed and every
-    // softmax warp is done reading it
+    // softmax warp is done with it
     umma::fence_before_sync();
     named_barrier_sync(1, kSoftmaxThreads);
     if (warp == 0) {
