@@ -16,8 +16,9 @@
 //     high part + remainder, and rescales its half of the O row when the
 //     maximum has grown by more than 2^8; at the end it divides by the summed
 //     weights and stores its half of the row;
-//   * warp 8: TMA producer of K/V stages gathered block by block through the
-//     table (the decode's ring);
+//   * warp 8: TMA producer of K and V stages gathered block by block through
+//     the table, in two rings: a K slot is free again as soon as its S MMA
+//     has run, a V slot once its PV MMA has;
 //   * warp 9, one thread: issues the UMMAs --
 //       S[128 x 128]  = Q[128 x D] . K_stage^T       (Q, K from shared memory)
 //       O[128 x D]   += P[128 x 128] . V_stage       (P from TMEM, V N-major)
@@ -47,20 +48,21 @@ constexpr int kTmemCols = 512;
 constexpr int kColO = 256, kColPHi = 384, kColPLo = 448;
 constexpr int kRowBytes = 128;       // one 64-element piece of a 16-bit row
 
-template <int D, int BS, int NS>
+template <int D, int BS, int NK, int NV>
 struct Cfg {
     static constexpr int kPieces = D / 64;
     static constexpr int kQPiece = kM * kRowBytes;        // 16 KB
     static constexpr int kQBytes = kPieces * kQPiece;
     static constexpr int kKVPiece = kKeys * kRowBytes;    // 16 KB
-    static constexpr int kKBytes = kPieces * kKVPiece;
-    static constexpr int kStageBytes = 2 * kKBytes;       // K + V
+    static constexpr int kStageBytes = kPieces * kKVPiece;  // one K or V stage
     static constexpr int kQOffset = 0;
-    static constexpr int kKVOffset = kQBytes;
-    static constexpr int kXchOffset = kKVOffset + NS * kStageBytes;  // float [2][2][128]
+    static constexpr int kKOffset = kQBytes;                        // K ring [NK]
+    static constexpr int kVOffset = kKOffset + NK * kStageBytes;    // V ring [NV]
+    static constexpr int kXchOffset = kVOffset + NV * kStageBytes;  // float [2][2][128]
     static constexpr int kBarOffset = kXchOffset + 2 * 2 * kM * 4;
-    // kv_full[NS] kv_empty[NS] s_full[2] s_empty[2] p_full pv_done q_full mma_done xchg[4]
-    static constexpr int kNumBars = 2 * NS + 4 + 4 + 4;
+    // k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] s_full[2] s_empty[2]
+    // p_full pv_done q_full mma_done xchg[4]
+    static constexpr int kNumBars = 2 * NK + 2 * NV + 4 + 4 + 4;
     static constexpr int kTmemSlot = kBarOffset + kNumBars * 8;
     static constexpr int kAbortOffset = kTmemSlot + 16;
     static constexpr int kSmemBytes = kAbortOffset + 16;
@@ -98,11 +100,11 @@ template <> struct PSplit<__half> {
     }
 };
 
-template <typename T, int D, int BS, int NS>
+template <typename T, int D, int BS, int NK, int NV>
 __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
     const PrefillParams p) {
-    using C = Cfg<D, BS, NS>;
+    using C = Cfg<D, BS, NK, NV>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -130,18 +132,24 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t q_s = sbase + C::kQOffset, kv_s = sbase + C::kKVOffset;
+    const uint32_t q_s = sbase + C::kQOffset, k_s = sbase + C::kKOffset,
+                   v_s = sbase + C::kVOffset;
     const uint32_t bar0 = sbase + C::kBarOffset;
-    const uint32_t kv_full = bar0, kv_empty = bar0 + 8 * NS, s_full = bar0 + 16 * NS,
-                   s_empty = s_full + 16, p_full = s_empty + 16, pv_done = p_full + 8,
-                   q_full = pv_done + 8, mma_done = q_full + 8, xchg = mma_done + 8;
+    const uint32_t k_full = bar0, k_empty = k_full + 8 * NK, v_full = k_empty + 8 * NK,
+                   v_empty = v_full + 8 * NV, s_full = v_empty + 8 * NV, s_empty = s_full + 16,
+                   p_full = s_empty + 16, pv_done = p_full + 8, q_full = pv_done + 8,
+                   mma_done = q_full + 8, xchg = mma_done + 8;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kAbortOffset);
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + C::kTmemSlot);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < NS; ++i) {
-            mbar_init(kv_full + 8 * i, 1);
-            mbar_init(kv_empty + 8 * i, 1);
+        for (int i = 0; i < NK; ++i) {
+            mbar_init(k_full + 8 * i, 1);
+            mbar_init(k_empty + 8 * i, 1);
+        }
+        for (int i = 0; i < NV; ++i) {
+            mbar_init(v_full + 8 * i, 1);
+            mbar_init(v_empty + 8 * i, 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(s_full + 8 * i, 1);
@@ -165,50 +173,68 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     const uint32_t tmem = *tmem_slot;
 
     // ------------------------------------------------------------ producer
+    // K runs one stage ahead of V: K(0), then K(i+1), V(i) for each stage i.
     if (warp == 8) {
         if (lane == 0) {
             prefetch_tensormap(&tmap_k);
             prefetch_tensormap(&tmap_v);
         }
         const uint64_t policy = l2_policy_evict_first();
-        int issued = 0;
-        for (int i = 0; i < nstages; ++i) {
+        // lane j < jn(i) holds the physical block of the stage's j-th table entry
+        auto lookup = [&](int i) -> int {
             const int jb = i * C::kBlocksPerStage;
             const int jn = min(C::kBlocksPerStage, nblk - jb);
-            int mine = 0;
-            if (lane < jn) {
-                const int b = checked_block_row(p.block_tables, p.max_blocks_per_seq, p.num_blocks,
-                                                p.err, s, jb + lane);
-                mine = b < 0 ? p.num_blocks : b;  // out of range: the copy reads the fill value
-            }
+            if (lane >= jn) return -1;
+            const int b = checked_block_row(p.block_tables, p.max_blocks_per_seq, p.num_blocks,
+                                            p.err, s, jb + lane);
+            return b < 0 ? p.num_blocks : b;  // out of range: the copy reads the fill value
+        };
+        // one K or V stage: wait for the slot, announce the bytes, lane j copies block j
+        auto load = [&](int i, int blk, const CUtensorMap *map, uint32_t ring, uint32_t full,
+                        uint32_t empty, int nslots) -> bool {
+            const int slot = i % nslots;
             int stop = 0;
-            const int buf = i % NS;
-            if (lane == 0 && i >= NS &&
-                !mbar_wait_bounded(kv_empty + 8 * buf, ((i / NS) - 1) & 1, abort_flag)) {
+            if (lane == 0 && i >= nslots &&
+                !mbar_wait_bounded(empty + 8 * slot, ((i / nslots) - 1) & 1, abort_flag))
+                stop = 1;
+            if (__shfl_sync(0xffffffffu, stop, 0)) return false;
+            const int jn = min(C::kBlocksPerStage, nblk - i * C::kBlocksPerStage);
+            if (lane == 0) mbar_arrive_expect_tx(full + 8 * slot, (uint32_t)(jn * 2 * BS * D));
+            __syncwarp();
+            if (blk >= 0) {
+                const uint32_t dst = ring + slot * C::kStageBytes + lane * BS * kRowBytes;
+                const int y = (blk * p.num_kv_heads + g) * BS;
+#pragma unroll
+                for (int pc = 0; pc < C::kPieces; ++pc)
+                    tma_load_2d(dst + pc * C::kKVPiece, map, pc * 64, y, full + 8 * slot, policy);
+            }
+            return true;
+        };
+        int k_issued = 0, v_issued = 0;
+        bool ok = true;
+        int blk_next = lookup(0);
+        if (load(0, blk_next, &tmap_k, k_s, k_full, k_empty, NK)) k_issued = 1; else ok = false;
+        for (int i = 0; ok && i < nstages; ++i) {
+            const int blk = blk_next;
+            if (i + 1 < nstages) {
+                blk_next = lookup(i + 1);
+                if (!load(i + 1, blk_next, &tmap_k, k_s, k_full, k_empty, NK)) { ok = false; break; }
+                k_issued = i + 2;
+            }
+            if (!load(i, blk, &tmap_v, v_s, v_full, v_empty, NV)) { ok = false; break; }
+            v_issued = i + 1;
+        }
+        if (lane == 0) {
+            if (!ok) {
                 raise_device_error(p.err, PA_DEVERR_TIMEOUT);
                 *abort_flag = 1;
-                stop = 1;
             }
-            if (__shfl_sync(0xffffffffu, stop, 0)) break;
-            const uint32_t full = kv_full + 8 * buf;
-            if (lane == 0) mbar_arrive_expect_tx(full, (uint32_t)(jn * 4 * BS * D));
-            __syncwarp();
-            // lane j < jn copies block j of the stage: its K and V rows, every piece
-            if (lane < jn) {
-                const uint32_t kdst = kv_s + buf * C::kStageBytes;
-                const int y = (mine * p.num_kv_heads + g) * BS;
-#pragma unroll
-                for (int pc = 0; pc < C::kPieces; ++pc) {
-                    const uint32_t off = pc * C::kKVPiece + lane * BS * kRowBytes;
-                    tma_load_2d(kdst + off, &tmap_k, pc * 64, y, full, policy);
-                    tma_load_2d(kdst + C::kKBytes + off, &tmap_v, pc * 64, y, full, policy);
-                }
-            }
-            issued = i + 1;
+            // wait (bounded) for the copies still in flight
+            for (int i = max(0, k_issued - NK); i < k_issued; ++i)
+                mbar_wait_bounded(k_full + 8 * (i % NK), (i / NK) & 1, nullptr);
+            for (int i = max(0, v_issued - NV); i < v_issued; ++i)
+                mbar_wait_bounded(v_full + 8 * (i % NV), (i / NV) & 1, nullptr);
         }
-        if (lane == 0)
-            for (int i = max(0, issued - NS); i < issued; ++i)
-                mbar_wait_bounded(kv_full + 8 * (i % NS), (i / NS) & 1, nullptr);
         return;
     }
 
@@ -221,13 +247,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
             bool ok = mbar_wait_bounded(q_full, 0, abort_flag);
             // S_i = Q . K_i^T into TMEM columns 128 * (i % 2)
             auto issue_s = [&](int i) -> bool {
-                const int buf = i % NS;
-                if (!mbar_wait_bounded(kv_full + 8 * buf, (i / NS) & 1, abort_flag)) return false;
+                const int buf = i % NK;
+                if (!mbar_wait_bounded(k_full + 8 * buf, (i / NK) & 1, abort_flag)) return false;
                 if (i >= 2 && !mbar_wait_bounded(s_empty + 8 * (i % 2), ((i / 2) - 1) & 1,
                                                  abort_flag))
                     return false;
                 umma::fence_after_sync();
-                const uint32_t kst = kv_s + buf * C::kStageBytes;
+                const uint32_t kst = k_s + buf * C::kStageBytes;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     const uint64_t a = umma::smem_desc_sw128(
@@ -237,6 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
                     umma::mma_f16(tmem + (i % 2) * kKeys, a, b, idesc_s, kk > 0);
                 }
                 umma::commit(s_full + 8 * (i % 2));
+                umma::commit(k_empty + 8 * buf);
                 return true;
             };
             if (ok) ok = issue_s(0);
@@ -246,12 +273,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
                     break;
                 }
                 // O += P_i . V_i once the softmax has written P_i
-                if (!mbar_wait_bounded(p_full, i & 1, abort_flag)) {
+                if (!mbar_wait_bounded(p_full, i & 1, abort_flag) ||
+                    !mbar_wait_bounded(v_full + 8 * (i % NV), (i / NV) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
                 umma::fence_after_sync();
-                const uint32_t vst = kv_s + (i % NS) * C::kStageBytes + C::kKBytes;
+                const uint32_t vst = v_s + (i % NV) * C::kStageBytes;
 #pragma unroll
                 for (int j = 0; j < kKeys / 16; ++j) {
                     // keys 16j..16j+15: V rows (8-row groups 1 KB apart), 64-column pieces 16 KB apart
@@ -262,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
                     umma::mma_f16_ts(tmem + kColO, tmem + kColPLo + 8 * j, b, idesc_o, 1u);
                 }
                 umma::commit(pv_done);
-                umma::commit(kv_empty + 8 * (i % NS));
+                umma::commit(v_empty + 8 * (i % NV));
             }
             if (!ok) {
                 raise_device_error(p.err, PA_DEVERR_TIMEOUT);
@@ -373,12 +401,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
             // last stage: rows past the last key hold stale or unwritten data;
             // zero them in V so that their zero weights give exact zeros.  The
             // wait only orders these stores after the stage's copies.
-            if (!warp_wait(kv_full + 8 * (i % NS), (i / NS) & 1, abort_flag)) {
+            if (!warp_wait(v_full + 8 * (i % NV), (i / NV) & 1, abort_flag)) {
                 ok = false;
                 break;
             }
             const int first = nkeys - i * kKeys;  // rows [first, 128)
-            uint8_t *vst = smem + C::kKVOffset + (i % NS) * C::kStageBytes + C::kKBytes;
+            uint8_t *vst = smem + C::kVOffset + (i % NV) * C::kStageBytes;
             for (int idx = threadIdx.x; idx < (kKeys - first) * C::kPieces * 8;
                  idx += kSoftmaxThreads) {
                 const int row = first + idx / (C::kPieces * 8);
@@ -437,15 +465,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
 template <typename T, int D, int BS>
 static cudaError_t launch_inst(const PrefillParams &p, const CUtensorMap &mk,
                                const CUtensorMap &mv, cudaStream_t stream) {
-    constexpr int NS = 2;
-    using C = Cfg<D, BS, NS>;
+    constexpr int NK = D == 128 ? 3 : 4, NV = D == 128 ? 2 : 4;
+    using C = Cfg<D, BS, NK, NV>;
     static std::once_flag once[64];
     static cudaError_t attr_err[64];
     int dev = 0;
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[dev], [&] {
-        attr_err[dev] = cudaFuncSetAttribute(prefill_umma_kernel<T, D, BS, NS>,
+        attr_err[dev] = cudaFuncSetAttribute(prefill_umma_kernel<T, D, BS, NK, NV>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kDynSmem);
     });
@@ -461,7 +489,7 @@ static cudaError_t launch_inst(const PrefillParams &p, const CUtensorMap &mk,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_umma_kernel<T, D, BS, NS>, mk, mv, p);
+    return cudaLaunchKernelEx(&cfg, prefill_umma_kernel<T, D, BS, NK, NV>, mk, mv, p);
 }
 
 template <typename T, int D>
