@@ -80,16 +80,18 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 // Two weights -> their 16-bit high parts and remainders, one 32-bit word each
-// (lower key in the low half).  bf16: round the fp32 bit pattern to its upper
-// 16 bits (half up in magnitude); the remainder x - hi is exact in fp32 and
-// is rounded the same way.  f16 uses the hardware conversions.
+// (lower key in the low half).  bf16: the high part is the upper 16 bits of
+// the fp32 pattern, the remainder x - hi is exact in fp32 and is rounded to
+// its upper 16 bits; integer and permute instructions only.  f16 uses the
+// hardware conversions.
 template <typename T> struct PSplit;
 template <> struct PSplit<__nv_bfloat16> {
     __device__ __forceinline__ static void run(float x0, float x1, uint32_t &hi, uint32_t &lo) {
-        const uint32_t a = __float_as_uint(x0) + 0x8000u, b = __float_as_uint(x1) + 0x8000u;
-        hi = __byte_perm(a, b, 0x7632);
+        const uint32_t a = __float_as_uint(x0), b = __float_as_uint(x1);
+        hi = __byte_perm(a, b, 0x7632);  // truncated: 0 <= x - hi < 2^-7 x
         const float r0 = x0 - __uint_as_float(a & 0xffff0000u);
         const float r1 = x1 - __uint_as_float(b & 0xffff0000u);
+        // remainder rounded half up in magnitude: |x - hi - lo| <= 2^-16 x
         lo = __byte_perm(__float_as_uint(r0) + 0x8000u, __float_as_uint(r1) + 0x8000u, 0x7632);
     }
 };
@@ -308,6 +310,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     const bool valid = t < ntok && r < TQ * G;
     const int qp = valid ? pos0 + t : nkeys - 1;
     const int64_t qrow = ((int64_t)(q0 + tok0 + t) * p.num_heads + g * G + hh) * D;
+    // S is computed with sign(scale) folded into Q (a sign-bit flip, exact),
+    // so that the logit scale applied below is non-negative
+    const uint32_t qflip = p.scale_log2 < 0.f ? 0x80008000u : 0u;
+    const float sl2 = fabsf(p.scale_log2);
     {
         // this thread's half of the Q row -> swizzled K-major tile
         // (row r, 16-byte chunk c at c ^ (r & 7) within its 128-byte piece row)
@@ -315,7 +321,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
             const int c = half * (D / 16) + k;
-            const uint4 v = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            uint4 v = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            v.x ^= qflip; v.y ^= qflip; v.z ^= qflip; v.w ^= qflip;
             *reinterpret_cast<uint4 *>(smem + C::kQOffset + (c >> 3) * C::kQPiece +
                                        r * kRowBytes + (((c & 7) ^ (r & 7)) << 4)) = v;
         }
@@ -325,7 +332,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     float *xch = reinterpret_cast<float *>(smem + C::kXchOffset);  // [parity][half][row]
     const uint32_t my_xchg = xchg + 8 * quarter;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
-    const float sl2 = p.scale_log2;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int i = 0; i < nstages; ++i) {
@@ -342,13 +348,29 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         umma::fence_before_sync();
         mbar_arrive(s_empty + 8 * sb);
         const int kb = i * kKeys + half * 64;
-        float x[64];
-        float mx = -INFINITY;
+        float sv[64];
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-            const float v = __uint_as_float(sr[c >> 5][c & 31]) * sl2;
-            x[c] = kb + c > qp ? -INFINITY : v;
-            mx = fmaxf(mx, x[c]);
+        for (int c = 0; c < 64; ++c) sv[c] = __uint_as_float(sr[c >> 5][c & 31]);
+        // Keys past a row's position exist only on stages reaching beyond the
+        // first chunk token's position (the test is uniform over the CTA);
+        // there the logits are scaled and masked here, elsewhere the scale is
+        // applied inside the exponent's FMA.
+        const bool masked = i * kKeys + kKeys - 1 > pos0;
+        float mx;
+        {
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            if (masked) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) {
+                    sv[c] = kb + c > qp ? -INFINITY : sv[c] * sl2;
+                    m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
+            }
+            mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            if (!masked) mx *= sl2;  // sl2 >= 0
         }
         // the row maximum of this stage over both halves
         xch[(sb * 2 + half) * kM + r] = mx;
@@ -367,16 +389,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
             rescale = m != -INFINITY;
             m = mx;
         }
-        float sum = 0.f;
-#pragma unroll
-        for (int c = 0; c < 64; ++c) {
-            x[c] = umma::ex2(x[c] - m);
-            sum += x[c];
-        }
-        l = l * alpha + sum;
+        // weights 2^(x - m), summed and split into TMEM words as they are made
+        const float fm = masked ? 1.f : sl2;
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
         uint32_t ph[32], pl[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) PSplit<T>::run(x[2 * e], x[2 * e + 1], ph[e], pl[e]);
+        for (int e = 0; e < 32; ++e) {
+            const float p0 = umma::ex2(fmaf(sv[2 * e], fm, -m));
+            const float p1 = umma::ex2(fmaf(sv[2 * e + 1], fm, -m));
+            s4[e & 3] += p0 + p1;
+            PSplit<T>::run(p0, p1, ph[e], pl[e]);
+        }
+        l = l * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
         // PV of stage i-1 must be done before O is rescaled and P overwritten
         if (i > 0 && !warp_wait(pv_done, (i - 1) & 1, abort_flag)) {
             ok = false;

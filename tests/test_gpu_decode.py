@@ -289,3 +289,36 @@ def test_prefill_long_context(pv):
                                    dtype="bf16", block_size=16, num_blocks=1024, chunks=1)
     errs, _, _ = run_parity(wl, table_width=5100 // 16 + 2, prefill_variant=pv)
     assert max(errs) <= TOL["bf16"], errs
+
+
+@pytest.mark.parametrize("pv", [1, 2])
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+@pytest.mark.parametrize("scale", [-0.2, 0.0, 0.5])
+def test_prefill_any_finite_scale(pv, dtype, scale):
+    """The logit scale is any finite number: negative scales reverse the
+    softmax order, 0 gives the plain mean of the attended values."""
+    from oracle import attn
+    from oracle.run import OracleRun
+    from paged_kv_cache_347_b200.runner import PagedKVRunner
+    pa = _pa()
+    wl = workloads.chunked_prefill(batch=3, ctx_lo=100, ctx_hi=300, chunk_lo=1, chunk_hi=160,
+                                   num_heads=8, num_kv_heads=2, head_dim=128, dtype=dtype,
+                                   block_size=16, num_blocks=256, chunks=1)
+    sh = wl.shape
+    orc, gpu = OracleRun(sh), PagedKVRunner.for_shape(sh, 32)
+    for st in wl.steps:
+        ref = orc.step(st, decode=False)
+        acts = gpu.plan(st.ops)
+        gpu.upload(acts)
+        gpu.execute(acts, st.k_new.cuda(), st.v_new.cuda(),
+                    None if st.q is None else st.q.cuda())
+    a = [x for x in acts if x.kind == "prefill"][0]
+    q = st.q
+    out = torch.empty((q.shape[0], sh.num_heads, sh.head_dim), dtype=torch.float32,
+                      device="cuda")
+    pa.pa_prefill(out, q.cuda(), gpu.k_cache, gpu.v_cache, a.dev["tables"], a.dev["lens"],
+                  a.dev["cu"], scale, max_q_len=a.max_q, max_seq_len=a.max_len, variant=pv)
+    exp = attn.paged_prefill(q, orc.k_cache, orc.v_cache, ref["block_tables"],
+                             ref["seq_lens"], a.cu, scale)
+    err = float(np.abs(out.double().cpu().numpy() - exp).max())
+    assert err <= TOL[dtype], err
