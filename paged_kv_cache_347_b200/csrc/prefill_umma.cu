@@ -7,7 +7,7 @@
 // positions 0..L-n+r through the block table.
 //
 // CTA = 128 (token, query head) rows: 128/G chunk tokens of one KV head g of
-// one sequence; the context is walked in stages of 128 keys.  Ten warps:
+// one sequence; the context is walked in stages of 128 keys.  Eleven warps:
 //   * warps 0-7, softmax: two threads per row -- warp w serves TMEM lanes
 //     32 (w % 4) .. +31 (the rows) and keys 64 (w / 4) .. +63 of each stage.
 //     Per stage a thread reads its 64 S values from TMEM, applies the causal
@@ -16,10 +16,10 @@
 //     high part + remainder, and rescales its half of the O row when the
 //     maximum has grown by more than 2^8; at the end it divides by the summed
 //     weights and stores its half of the row;
-//   * warp 8: TMA producer of K and V stages gathered block by block through
-//     the table, in two rings: a K slot is free again as soon as its S MMA
-//     has run, a V slot once its PV MMA has;
-//   * warp 9, one thread: issues the UMMAs --
+//   * warps 8 and 9: TMA producers of the K and the V stages, gathered block
+//     by block through the table into two rings: a K slot is free again as
+//     soon as its S MMA has run, a V slot once its PV MMA has;
+//   * warp 10, one thread: issues the UMMAs --
 //       S[128 x 128]  = Q[128 x D] . K_stage^T       (Q, K from shared memory)
 //       O[128 x D]   += P[128 x 128] . V_stage       (P from TMEM, V N-major)
 //     and commits them to mbarriers.  S is double-buffered, so S of stage
@@ -43,7 +43,7 @@ namespace pu {
 constexpr int kM = 128;              // rows per CTA
 constexpr int kKeys = 128;           // keys per stage
 constexpr int kSoftmaxThreads = 256; // 8 warps, two threads per row
-constexpr int kThreads = kSoftmaxThreads + 64;
+constexpr int kThreads = kSoftmaxThreads + 96;  // + K producer, V producer, MMA issuer
 constexpr int kTmemCols = 512;
 constexpr int kColO = 256, kColPHi = 384, kColPLo = 448;
 constexpr int kRowBytes = 128;       // one 64-element piece of a 16-bit row
@@ -175,8 +175,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     const uint32_t tmem = *tmem_slot;
 
     // ------------------------------------------------------------ producer
-    // K runs one stage ahead of V: K(0), then K(i+1), V(i) for each stage i.
-    if (warp == 8) {
+    // warp 8 loads the K stages, warp 9 the V stages, each at its own pace
+    if (warp == 8 || warp == 9) {
         if (lane == 0) {
             prefetch_tensormap(&tmap_k);
             prefetch_tensormap(&tmap_v);
@@ -212,36 +212,30 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
             }
             return true;
         };
-        int k_issued = 0, v_issued = 0;
-        bool ok = true;
-        int blk_next = lookup(0);
-        if (load(0, blk_next, &tmap_k, k_s, k_full, k_empty, NK)) k_issued = 1; else ok = false;
-        for (int i = 0; ok && i < nstages; ++i) {
-            const int blk = blk_next;
-            if (i + 1 < nstages) {
-                blk_next = lookup(i + 1);
-                if (!load(i + 1, blk_next, &tmap_k, k_s, k_full, k_empty, NK)) { ok = false; break; }
-                k_issued = i + 2;
-            }
-            if (!load(i, blk, &tmap_v, v_s, v_full, v_empty, NV)) { ok = false; break; }
-            v_issued = i + 1;
+        const bool is_k = warp == 8;
+        const CUtensorMap *map = is_k ? &tmap_k : &tmap_v;
+        const uint32_t ring = is_k ? k_s : v_s, full = is_k ? k_full : v_full,
+                       empty = is_k ? k_empty : v_empty;
+        const int nslots = is_k ? NK : NV;
+        int issued = 0;
+        for (int i = 0; i < nstages; ++i) {
+            if (!load(i, lookup(i), map, ring, full, empty, nslots)) break;
+            issued = i + 1;
         }
         if (lane == 0) {
-            if (!ok) {
+            if (issued < nstages) {
                 raise_device_error(p.err, PA_DEVERR_TIMEOUT);
                 *abort_flag = 1;
             }
             // wait (bounded) for the copies still in flight
-            for (int i = max(0, k_issued - NK); i < k_issued; ++i)
-                mbar_wait_bounded(k_full + 8 * (i % NK), (i / NK) & 1, nullptr);
-            for (int i = max(0, v_issued - NV); i < v_issued; ++i)
-                mbar_wait_bounded(v_full + 8 * (i % NV), (i / NV) & 1, nullptr);
+            for (int i = max(0, issued - nslots); i < issued; ++i)
+                mbar_wait_bounded(full + 8 * (i % nslots), (i / nslots) & 1, nullptr);
         }
         return;
     }
 
     // ------------------------------------------------------------ MMA issuer
-    if (warp == 9) {
+    if (warp == 10) {
         if (lane == 0) {
             constexpr uint32_t fmt = StoreT<T>::kCode == PA_BF16 ? 1u : 0u;
             constexpr uint32_t idesc_s = umma::idesc_f16(fmt, kM, kKeys, 0);
