@@ -176,7 +176,8 @@ int pa_prefill(float *out, const void *q, const void *k_cache, const void *v_cac
                float scale, int dtype, void *stream);
 
 /*
- * pa_prefill with a choice of kernel: variant 0 = automatic, 1 = the
+ * pa_prefill with a choice of kernel: variant 0 = automatic (the tcgen05
+ * kernel; pa_prefill uses it), 1 = the
  * mma.sync kernel (64 (token, head) rows per CTA, accumulators in
  * registers), 2 = the tcgen05 kernel (128 rows per CTA, S = Q K^T and
  * O = P V accumulated in tensor memory).  Same arguments, results (within

@@ -87,7 +87,7 @@ static int check_shape(int num_kv_heads, int head_dim, int block_size, int dtype
 
 constexpr int kDefaultPartition = 512;
 // pa_prefill's kernel: 1 = mma.sync (registers), 2 = tcgen05 (TMEM).
-constexpr int kPrefillDefault = 1;
+constexpr int kPrefillDefault = 2;
 
 static int partition_or_default(int partition_size) {
     return partition_size == 0 ? kDefaultPartition : partition_size;
