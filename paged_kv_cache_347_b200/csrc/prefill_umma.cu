@@ -6,33 +6,38 @@
 // details"): row r of a sequence's chunk, at position L - n + r, attends to
 // positions 0..L-n+r through the block table.
 //
-// CTA = 128 (token, query head) rows: 128/G chunk tokens of one KV head g of
-// one sequence; the context is walked in stages of 128 keys.  Eleven warps:
-//   * warps 0-7, softmax: two threads per row -- warp w serves TMEM lanes
-//     32 (w % 4) .. +31 (the rows) and keys 64 (w / 4) .. +63 of each stage.
-//     Per stage a thread reads its 64 S values from TMEM, applies the causal
-//     mask, agrees the row maximum with its partner thread (through shared
-//     memory and an mbarrier), writes P = 2^(x - m) into TMEM as 16-bit
-//     high part + remainder, and rescales its half of the O row when the
-//     maximum has grown by more than 2^8; at the end it divides by the summed
-//     weights and stores its half of the row;
+// CTA = two tiles of 128 (token, query head) rows -- 2 x 128/G chunk tokens
+// of one KV head g of one sequence -- walking the context in stages of 128
+// keys.  Twelve warps:
+//   * warps 0-3 (tile 0) and 4-7 (tile 1), softmax: one thread per row
+//     (thread i of a tile <-> TMEM lane i).  Per stage a thread reads its
+//     128 S values from TMEM (the row maximum first), writes
+//     P = 2^(x - m) as 16-bit high part + remainder into the same TMEM
+//     columns, and rescales its O row when the maximum has grown by
+//     more than 2^8; at the end it divides by the summed weights and stores
+//     the row;
 //   * warps 8 and 9: TMA producers of the K and the V stages, gathered block
-//     by block through the table into two rings: a K slot is free again as
-//     soon as its S MMA has run, a V slot once its PV MMA has;
-//   * warp 10, one thread: issues the UMMAs --
-//       S[128 x 128]  = Q[128 x D] . K_stage^T       (Q, K from shared memory)
-//       O[128 x D]   += P[128 x 128] . V_stage       (P from TMEM, V N-major)
-//     and commits them to mbarriers.  S is double-buffered, so S of stage
-//     i+1 runs on the tensor core while the softmax works on stage i.
-// TMEM (512 columns): S0 [0,128), S1 [128,256), O [256,256+D),
-// P high part [384,448), P remainder [448,512).
+//     by block through the table into two rings;
+//   * warp 10, one thread: issues the UMMAs in the order
+//       PV(0,i), S(0,i+1), PV(1,i), S(1,i+1), ...   with
+//       S(t,i)  [128 x 128] = Q_t . K_i^T        (Q, K from shared memory)
+//       PV(t,i) O_t [128 x D] += P_t . V_i        (P from TMEM, V N-major)
+//     so that the tensor core works on one tile while the other tile's
+//     softmax runs.  S(t,i+1) overwrites the columns PV(t,i) reads; the two
+//     are issued by the same thread and tcgen05 MMAs of one thread execute
+//     in issue order;
+//   * warp 11 has no work after set-up.
+// TMEM (512 columns): tile t at 256 t: S / P [0,128), O [128,128+D).  In P,
+// key block j (keys 16j..16j+15) holds its high parts in columns 16j..16j+7
+// and its remainders in 16j+8..16j+15, two keys per column.
 //
 // Every wait is bounded (~2 s); on a timeout the CTA records
-// PA_DEVERR_TIMEOUT, the other warps stop waiting, the producer waits
-// (bounded) for its copies, warp 0 waits for the MMAs and frees the TMEM.
+// PA_DEVERR_TIMEOUT, the other warps stop waiting, the producers wait
+// (bounded) for their copies, warp 0 waits for the MMAs and frees the TMEM.
 #include <math.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "decode_common.cuh"
 #include "umma.cuh"
@@ -40,29 +45,28 @@
 namespace pa {
 namespace pu {
 
-constexpr int kM = 128;              // rows per CTA
-constexpr int kKeys = 128;           // keys per stage
-constexpr int kSoftmaxThreads = 256; // 8 warps, two threads per row
-constexpr int kThreads = kSoftmaxThreads + 96;  // + K producer, V producer, MMA issuer
+constexpr int kM = 128;               // rows per tile
+constexpr int kKeys = 128;            // keys per stage
+constexpr int kSoftmaxThreads = 256;  // two tiles x 4 warps
+constexpr int kThreads = kSoftmaxThreads + 128;
 constexpr int kTmemCols = 512;
-constexpr int kColO = 256, kColPHi = 384, kColPLo = 448;
-constexpr int kRowBytes = 128;       // one 64-element piece of a 16-bit row
+constexpr int kTileCols = 256;        // per tile: S / P, then O
+constexpr int kColO = 128;
+constexpr int kRowBytes = 128;        // one 64-element piece of a 16-bit row
 
 template <int D, int BS, int NK, int NV>
 struct Cfg {
     static constexpr int kPieces = D / 64;
-    static constexpr int kQPiece = kM * kRowBytes;        // 16 KB
-    static constexpr int kQBytes = kPieces * kQPiece;
-    static constexpr int kKVPiece = kKeys * kRowBytes;    // 16 KB
+    static constexpr int kQPiece = kM * kRowBytes;          // 16 KB
+    static constexpr int kQTile = kPieces * kQPiece;
+    static constexpr int kKVPiece = kKeys * kRowBytes;      // 16 KB
     static constexpr int kStageBytes = kPieces * kKVPiece;  // one K or V stage
-    static constexpr int kQOffset = 0;
-    static constexpr int kKOffset = kQBytes;                        // K ring [NK]
-    static constexpr int kVOffset = kKOffset + NK * kStageBytes;    // V ring [NV]
-    static constexpr int kXchOffset = kVOffset + NV * kStageBytes;  // float [2][2][128]
-    static constexpr int kBarOffset = kXchOffset + 2 * 2 * kM * 4;
-    // k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] s_full[2] s_empty[2]
-    // p_full pv_done q_full mma_done xchg[4]
-    static constexpr int kNumBars = 2 * NK + 2 * NV + 4 + 4 + 4;
+    static constexpr int kQOffset = 0;                      // Q tiles [2]
+    static constexpr int kKOffset = 2 * kQTile;             // K ring [NK]
+    static constexpr int kVOffset = kKOffset + NK * kStageBytes;  // V ring [NV]
+    static constexpr int kBarOffset = kVOffset + NV * kStageBytes;
+    // k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] s_full[2] p_full[2] o_full[2] q_full mma_done
+    static constexpr int kNumBars = 2 * NK + 2 * NV + 8;
     static constexpr int kTmemSlot = kBarOffset + kNumBars * 8;
     static constexpr int kAbortOffset = kTmemSlot + 16;
     static constexpr int kSmemBytes = kAbortOffset + 16;
@@ -81,9 +85,9 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
 
 // Two weights -> their 16-bit high parts and remainders, one 32-bit word each
 // (lower key in the low half).  bf16: the high part is the upper 16 bits of
-// the fp32 pattern, the remainder x - hi is exact in fp32 and is rounded to
-// its upper 16 bits; integer and permute instructions only.  f16 uses the
-// hardware conversions.
+// the fp32 pattern, the remainder x - hi is exact in fp32 and is cut to its
+// upper 16 bits as well (one logic op, one add and one permute per weight);
+// f16 uses the hardware conversions.
 template <typename T> struct PSplit;
 template <> struct PSplit<__nv_bfloat16> {
     __device__ __forceinline__ static void run(float x0, float x1, uint32_t &hi, uint32_t &lo) {
@@ -91,8 +95,8 @@ template <> struct PSplit<__nv_bfloat16> {
         hi = __byte_perm(a, b, 0x7632);  // truncated: 0 <= x - hi < 2^-7 x
         const float r0 = x0 - __uint_as_float(a & 0xffff0000u);
         const float r1 = x1 - __uint_as_float(b & 0xffff0000u);
-        // remainder rounded half up in magnitude: |x - hi - lo| <= 2^-16 x
-        lo = __byte_perm(__float_as_uint(r0) + 0x8000u, __float_as_uint(r1) + 0x8000u, 0x7632);
+        // remainder truncated too: 0 <= x - hi - lo < 2^-14 x
+        lo = __byte_perm(__float_as_uint(r0), __float_as_uint(r1), 0x7632);
     }
 };
 template <> struct PSplit<__half> {
@@ -115,7 +119,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
 
     const int qt = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
     const int G = p.num_heads / p.num_kv_heads;
-    const int TQ = p.tokens_per_cta;  // 128 / G
+    const int TQ = p.tokens_per_cta / 2;  // tokens per tile: 128 / G
     const int q0 = __ldg(p.cu_q + s);
     const int n = __ldg(p.cu_q + s + 1) - q0;
     const int L = __ldg(p.seq_lens + s);
@@ -124,9 +128,10 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         if (qt == 0 && g == 0 && threadIdx.x == 0) raise_device_error(p.err, PA_DEVERR_SEQLEN);
         return;
     }
-    const int tok0 = qt * TQ;
+    const int tok0 = qt * 2 * TQ;
     if (tok0 >= n) return;  // uniform, before any barrier or TMEM use
-    const int ntok = min(TQ, n - tok0);
+    const int ntok = min(2 * TQ, n - tok0);
+    const bool two = ntok > TQ;  // tile 1 has rows
     const int pos0 = L - n + tok0;
     const int nkeys = pos0 + ntok;
     const int nstages = (nkeys + kKeys - 1) / kKeys;
@@ -138,9 +143,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
                    v_s = sbase + C::kVOffset;
     const uint32_t bar0 = sbase + C::kBarOffset;
     const uint32_t k_full = bar0, k_empty = k_full + 8 * NK, v_full = k_empty + 8 * NK,
-                   v_empty = v_full + 8 * NV, s_full = v_empty + 8 * NV, s_empty = s_full + 16,
-                   p_full = s_empty + 16, pv_done = p_full + 8, q_full = pv_done + 8,
-                   mma_done = q_full + 8, xchg = mma_done + 8;
+                   v_empty = v_full + 8 * NV, s_full = v_empty + 8 * NV, p_full = s_full + 16,
+                   o_full = p_full + 16, q_full = o_full + 16, mma_done = q_full + 8;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kAbortOffset);
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + C::kTmemSlot);
 
@@ -153,15 +157,13 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
             mbar_init(v_full + 8 * i, 1);
             mbar_init(v_empty + 8 * i, 1);
         }
-        for (int i = 0; i < 2; ++i) {
-            mbar_init(s_full + 8 * i, 1);
-            mbar_init(s_empty + 8 * i, kSoftmaxThreads);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(s_full + 8 * t, 1);
+            mbar_init(p_full + 8 * t, kM);
+            mbar_init(o_full + 8 * t, 1);
         }
-        mbar_init(p_full, kSoftmaxThreads);
-        mbar_init(pv_done, 1);
         mbar_init(q_full, kSoftmaxThreads);
         mbar_init(mma_done, 1);
-        for (int i = 0; i < 4; ++i) mbar_init(xchg + 8 * i, 64);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -174,33 +176,35 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     umma::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
 
-    // ------------------------------------------------------------ producer
+    if (warp == 11) return;
+
+    // ------------------------------------------------------------ producers
     // warp 8 loads the K stages, warp 9 the V stages, each at its own pace
     if (warp == 8 || warp == 9) {
-        if (lane == 0) {
-            prefetch_tensormap(&tmap_k);
-            prefetch_tensormap(&tmap_v);
-        }
+        const bool is_k = warp == 8;
+        const CUtensorMap *map = is_k ? &tmap_k : &tmap_v;
+        if (lane == 0) prefetch_tensormap(map);
         const uint64_t policy = l2_policy_evict_first();
-        // lane j < jn(i) holds the physical block of the stage's j-th table entry
-        auto lookup = [&](int i) -> int {
+        const uint32_t ring = is_k ? k_s : v_s, full = is_k ? k_full : v_full,
+                       empty = is_k ? k_empty : v_empty;
+        const int nslots = is_k ? NK : NV;
+        int issued = 0;
+        for (int i = 0; i < nstages; ++i) {
+            const int slot = i % nslots;
             const int jb = i * C::kBlocksPerStage;
             const int jn = min(C::kBlocksPerStage, nblk - jb);
-            if (lane >= jn) return -1;
-            const int b = checked_block_row(p.block_tables, p.max_blocks_per_seq, p.num_blocks,
-                                            p.err, s, jb + lane);
-            return b < 0 ? p.num_blocks : b;  // out of range: the copy reads the fill value
-        };
-        // one K or V stage: wait for the slot, announce the bytes, lane j copies block j
-        auto load = [&](int i, int blk, const CUtensorMap *map, uint32_t ring, uint32_t full,
-                        uint32_t empty, int nslots) -> bool {
-            const int slot = i % nslots;
+            // lane j < jn holds the physical block of the stage's j-th table entry
+            int blk = -1;
+            if (lane < jn) {
+                const int b = checked_block_row(p.block_tables, p.max_blocks_per_seq, p.num_blocks,
+                                                p.err, s, jb + lane);
+                blk = b < 0 ? p.num_blocks : b;  // out of range: the copy reads the fill value
+            }
             int stop = 0;
             if (lane == 0 && i >= nslots &&
                 !mbar_wait_bounded(empty + 8 * slot, ((i / nslots) - 1) & 1, abort_flag))
                 stop = 1;
-            if (__shfl_sync(0xffffffffu, stop, 0)) return false;
-            const int jn = min(C::kBlocksPerStage, nblk - i * C::kBlocksPerStage);
+            if (__shfl_sync(0xffffffffu, stop, 0)) break;
             if (lane == 0) mbar_arrive_expect_tx(full + 8 * slot, (uint32_t)(jn * 2 * BS * D));
             __syncwarp();
             if (blk >= 0) {
@@ -210,16 +214,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
                 for (int pc = 0; pc < C::kPieces; ++pc)
                     tma_load_2d(dst + pc * C::kKVPiece, map, pc * 64, y, full + 8 * slot, policy);
             }
-            return true;
-        };
-        const bool is_k = warp == 8;
-        const CUtensorMap *map = is_k ? &tmap_k : &tmap_v;
-        const uint32_t ring = is_k ? k_s : v_s, full = is_k ? k_full : v_full,
-                       empty = is_k ? k_empty : v_empty;
-        const int nslots = is_k ? NK : NV;
-        int issued = 0;
-        for (int i = 0; i < nstages; ++i) {
-            if (!load(i, lookup(i), map, ring, full, empty, nslots)) break;
             issued = i + 1;
         }
         if (lane == 0) {
@@ -240,53 +234,56 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
             constexpr uint32_t fmt = StoreT<T>::kCode == PA_BF16 ? 1u : 0u;
             constexpr uint32_t idesc_s = umma::idesc_f16(fmt, kM, kKeys, 0);
             constexpr uint32_t idesc_o = umma::idesc_f16(fmt, kM, D, 1);
-            bool ok = mbar_wait_bounded(q_full, 0, abort_flag);
-            // S_i = Q . K_i^T into TMEM columns 128 * (i % 2)
-            auto issue_s = [&](int i) -> bool {
-                const int buf = i % NK;
-                if (!mbar_wait_bounded(k_full + 8 * buf, (i / NK) & 1, abort_flag)) return false;
-                if (i >= 2 && !mbar_wait_bounded(s_empty + 8 * (i % 2), ((i / 2) - 1) & 1,
-                                                 abort_flag))
+            const int last_tile = two ? 1 : 0;  // the tile whose MMAs free a K / V slot
+            // S(t,i) = Q_t . K_i^T into tile t's S columns
+            auto issue_s = [&](int t, int i) -> bool {
+                const int slot = i % NK;
+                if (t == 0 && !mbar_wait_bounded(k_full + 8 * slot, (i / NK) & 1, abort_flag))
                     return false;
                 umma::fence_after_sync();
-                const uint32_t kst = k_s + buf * C::kStageBytes;
+                // descriptors advance by (bytes >> 4) in their start-address field
+                const uint64_t a0 = umma::smem_desc_sw128(q_s + t * C::kQTile, 16, 1024);
+                const uint64_t b0 = umma::smem_desc_sw128(k_s + slot * C::kStageBytes, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint64_t a = umma::smem_desc_sw128(
-                        q_s + (kk >> 2) * C::kQPiece + (kk & 3) * 32, 16, 1024);
-                    const uint64_t b = umma::smem_desc_sw128(
-                        kst + (kk >> 2) * C::kKVPiece + (kk & 3) * 32, 16, 1024);
-                    umma::mma_f16(tmem + (i % 2) * kKeys, a, b, idesc_s, kk > 0);
+                    const uint32_t qa = ((kk >> 2) * C::kQPiece + (kk & 3) * 32) >> 4;
+                    const uint32_t ka = ((kk >> 2) * C::kKVPiece + (kk & 3) * 32) >> 4;
+                    umma::mma_f16(tmem + t * kTileCols, a0 + qa, b0 + ka, idesc_s, kk > 0);
                 }
-                umma::commit(s_full + 8 * (i % 2));
-                umma::commit(k_empty + 8 * buf);
+                umma::commit(s_full + 8 * t);
+                if (t == last_tile) umma::commit(k_empty + 8 * slot);
                 return true;
             };
-            if (ok) ok = issue_s(0);
-            for (int i = 0; ok && i < nstages; ++i) {
-                if (i + 1 < nstages && !issue_s(i + 1)) {
-                    ok = false;
-                    break;
-                }
-                // O += P_i . V_i once the softmax has written P_i
-                if (!mbar_wait_bounded(p_full, i & 1, abort_flag) ||
-                    !mbar_wait_bounded(v_full + 8 * (i % NV), (i / NV) & 1, abort_flag)) {
-                    ok = false;
-                    break;
-                }
+            // O_t += P_t . V_i once tile t's softmax has written P_t
+            auto issue_pv = [&](int t, int i) -> bool {
+                const int slot = i % NV;
+                if (!mbar_wait_bounded(p_full + 8 * t, i & 1, abort_flag)) return false;
+                if (t == 0 && !mbar_wait_bounded(v_full + 8 * slot, (i / NV) & 1, abort_flag))
+                    return false;
                 umma::fence_after_sync();
-                const uint32_t vst = v_s + (i % NV) * C::kStageBytes;
+                // V rows: 8-row groups 1 KB apart, 64-column pieces 16 KB apart
+                const uint64_t b0 = umma::smem_desc_sw128(v_s + slot * C::kStageBytes,
+                                                          C::kKVPiece, 1024);
+                const uint32_t tb = tmem + t * kTileCols;
 #pragma unroll
-                for (int j = 0; j < kKeys / 16; ++j) {
-                    // keys 16j..16j+15: V rows (8-row groups 1 KB apart), 64-column pieces 16 KB apart
-                    const uint64_t b = umma::smem_desc_sw128(vst + j * 16 * kRowBytes,
-                                                             C::kKVPiece, 1024);
-                    umma::mma_f16_ts(tmem + kColO, tmem + kColPHi + 8 * j, b, idesc_o,
-                                     (i > 0 || j > 0) ? 1u : 0u);
-                    umma::mma_f16_ts(tmem + kColO, tmem + kColPLo + 8 * j, b, idesc_o, 1u);
+                for (int j = 0; j < kKeys / 16; ++j) {  // keys 16j..16j+15
+                    const uint64_t b = b0 + ((j * 16 * kRowBytes) >> 4);
+                    umma::mma_f16_ts(tb + kColO, tb + 16 * j, b, idesc_o, (i > 0 || j > 0) ? 1u : 0u);
+                    umma::mma_f16_ts(tb + kColO, tb + 16 * j + 8, b, idesc_o, 1u);
                 }
-                umma::commit(pv_done);
-                umma::commit(v_empty + 8 * (i % NV));
+                if (t == last_tile) umma::commit(v_empty + 8 * slot);
+                if (i == nstages - 1) umma::commit(o_full + 8 * t);
+                return true;
+            };
+            bool ok = mbar_wait_bounded(q_full, 0, abort_flag);
+            if (ok) ok = issue_s(0, 0);
+            if (ok && two) ok = issue_s(1, 0);
+#pragma unroll 1
+            for (int i = 0; ok && i < nstages; ++i) {
+                ok = issue_pv(0, i);
+                if (ok && i + 1 < nstages) ok = issue_s(0, i + 1);
+                if (ok && two) ok = issue_pv(1, i);
+                if (ok && two && i + 1 < nstages) ok = issue_s(1, i + 1);
             }
             if (!ok) {
                 raise_device_error(p.err, PA_DEVERR_TIMEOUT);
@@ -298,82 +295,77 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     }
 
     // ------------------------------------------------------------ softmax warps
-    const int quarter = warp & 3, half = warp >> 2;
-    const int r = quarter * 32 + lane;  // row == TMEM lane
-    const int t = r / G, hh = r - t * G;
-    const bool valid = t < ntok && r < TQ * G;
-    const int qp = valid ? pos0 + t : nkeys - 1;
-    const int64_t qrow = ((int64_t)(q0 + tok0 + t) * p.num_heads + g * G + hh) * D;
+    const int tile = warp >> 2, quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // row of the tile == TMEM lane
+    const int tl = r / G, hh = r - tl * G;
+    const int ttok = tile * TQ + tl;  // chunk token of this row, relative to tok0
+    const bool valid = r < TQ * G && ttok < ntok;
+    const int qp = valid ? pos0 + ttok : nkeys - 1;
+    const int tile_pos0 = pos0 + tile * TQ;  // position of the tile's first token
+    const int64_t qrow = ((int64_t)(q0 + tok0 + ttok) * p.num_heads + g * G + hh) * D;
     // S is computed with sign(scale) folded into Q (a sign-bit flip, exact),
     // so that the logit scale applied below is non-negative
     const uint32_t qflip = p.scale_log2 < 0.f ? 0x80008000u : 0u;
     const float sl2 = fabsf(p.scale_log2);
     {
-        // this thread's half of the Q row -> swizzled K-major tile
-        // (row r, 16-byte chunk c at c ^ (r & 7) within its 128-byte piece row)
+        // the Q row -> tile's swizzled K-major Q (row r, 16-byte chunk c at
+        // c ^ (r & 7) within its 128-byte piece row)
         const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.q) + qrow);
+        uint8_t *qt_s = smem + C::kQOffset + tile * C::kQTile;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-            const int c = half * (D / 16) + k;
+        for (int c = 0; c < D / 8; ++c) {
             uint4 v = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
             v.x ^= qflip; v.y ^= qflip; v.z ^= qflip; v.w ^= qflip;
-            *reinterpret_cast<uint4 *>(smem + C::kQOffset + (c >> 3) * C::kQPiece +
-                                       r * kRowBytes + (((c & 7) ^ (r & 7)) << 4)) = v;
+            *reinterpret_cast<uint4 *>(qt_s + (c >> 3) * C::kQPiece + r * kRowBytes +
+                                       (((c & 7) ^ (r & 7)) << 4)) = v;
         }
         umma::fence_proxy_async_smem();
         mbar_arrive(q_full);
     }
-    float *xch = reinterpret_cast<float *>(smem + C::kXchOffset);  // [parity][half][row]
-    const uint32_t my_xchg = xchg + 8 * quarter;
-    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + tile * kTileCols;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int i = 0; i < nstages; ++i) {
-        const int sb = i & 1;
-        if (!warp_wait(s_full + 8 * sb, (i >> 1) & 1, abort_flag)) {
-            ok = false;
-            break;
-        }
+    const bool active = tile == 0 || two;
+    // One stage of the softmax.  Keys past a row's position exist only on
+    // stages reaching beyond the tile's first token; those run the masked
+    // body, every earlier stage the unmasked one (the split also keeps the
+    // hot loop's code small).
+    auto stage = [&](int i, auto masked_c) __attribute__((always_inline)) -> bool {
+        constexpr bool kMasked = decltype(masked_c)::value;
+        if (!warp_wait(s_full + 8 * tile, i & 1, abort_flag)) return false;
         umma::fence_after_sync();
-        uint32_t sr[2][32];
-        umma::ld32(lane_base + sb * kKeys + half * 64, sr[0]);
-        umma::ld32(lane_base + sb * kKeys + half * 64 + 32, sr[1]);
-        umma::wait_ld();
-        umma::fence_before_sync();
-        mbar_arrive(s_empty + 8 * sb);
-        const int kb = i * kKeys + half * 64;
-        float sv[64];
+        const int kb = i * kKeys;
+        // the row maximum over the stage's 128 logits, read as chunks 0-1 then
+        // 2-3 (two loads in flight each time); chunks 2-3 stay in registers
+        const int last = qp - kb;  // the row's last key within the stage (masked body)
+        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+        auto fold_max = [&](int c, const uint32_t (&w)[32]) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) sv[c] = __uint_as_float(sr[c >> 5][c & 31]);
-        // Keys past a row's position exist only on stages reaching beyond the
-        // first chunk token's position (the test is uniform over the CTA);
-        // there the logits are scaled and masked here, elsewhere the scale is
-        // applied inside the exponent's FMA.
-        const bool masked = i * kKeys + kKeys - 1 > pos0;
-        float mx;
-        {
-            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-            if (masked) {
-#pragma unroll
-                for (int c = 0; c < 64; ++c) {
-                    sv[c] = kb + c > qp ? -INFINITY : sv[c] * sl2;
-                    m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
+            for (int e = 0; e < 32; ++e) {
+                if constexpr (kMasked) {
+                    const float v = 32 * c + e > last ? -INFINITY : __uint_as_float(w[e]) * sl2;
+                    m4[e & 3] = fmaxf(m4[e & 3], v);
+                } else {
+                    m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(w[e]));
                 }
-            } else {
-#pragma unroll
-                for (int c = 0; c < 64; ++c) m4[c & 3] = fmaxf(m4[c & 3], sv[c]);
             }
-            mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-            if (!masked) mx *= sl2;  // sl2 >= 0
+        };
+        uint32_t sr[2][32];
+        {
+            uint32_t t0[32], t1[32];
+            umma::ld32(lane_base, t0);
+            umma::ld32(lane_base + 32, t1);
+            umma::wait_ld();
+            fold_max(0, t0);
+            fold_max(1, t1);
         }
-        // the row maximum of this stage over both halves
-        xch[(sb * 2 + half) * kM + r] = mx;
-        mbar_arrive(my_xchg);
-        if (!__all_sync(0xffffffffu, mbar_wait_bounded(my_xchg, i & 1, abort_flag))) {
-            ok = false;
-            break;
-        }
-        mx = fmaxf(mx, xch[(sb * 2 + (half ^ 1)) * kM + r]);
+        umma::ld32(lane_base + 64, sr[0]);
+        umma::ld32(lane_base + 96, sr[1]);
+        umma::wait_ld();
+        fold_max(2, sr[0]);
+        fold_max(3, sr[1]);
+        float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+        if constexpr (!kMasked) mx *= sl2;  // sl2 >= 0
         // the running max moves only when it grows by more than 8 (log2 units):
         // weights then stay below 2^8 and O is rescaled rarely
         float alpha = 1.f;
@@ -383,77 +375,89 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
             rescale = m != -INFINITY;
             m = mx;
         }
-        // weights 2^(x - m), summed and split into TMEM words as they are made
-        const float fm = masked ? 1.f : sl2;
+        // weights 2^(x - m), summed and split in place: the pair of keys
+        // (2e, 2e+1) of a chunk leaves its high-part word in word 2e and its
+        // remainder word in word 2e+1; TMEM column 32c + q then takes key
+        // block q / 16 of the chunk, high parts in its first 8 columns,
+        // remainders in the next 8.  Chunks 3 and 2 come from the registers;
+        // chunks 0 and 1 are read again (issued while chunk 2 is worked on).
         float s4[4] = {0.f, 0.f, 0.f, 0.f};
-        uint32_t ph[32], pl[32];
+        auto emit = [&](int c, uint32_t (&w)[32]) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-            const float p0 = umma::ex2(fmaf(sv[2 * e], fm, -m));
-            const float p1 = umma::ex2(fmaf(sv[2 * e + 1], fm, -m));
-            s4[e & 3] += p0 + p1;
-            PSplit<T>::run(p0, p1, ph[e], pl[e]);
-        }
+            for (int e = 0; e < 16; ++e) {
+                float y0 = fmaf(__uint_as_float(w[2 * e]), sl2, -m);
+                float y1 = fmaf(__uint_as_float(w[2 * e + 1]), sl2, -m);
+                if constexpr (kMasked) {
+                    if (32 * c + 2 * e > last) y0 = -INFINITY;
+                    if (32 * c + 2 * e + 1 > last) y1 = -INFINITY;
+                }
+                const float p0 = umma::ex2(y0), p1 = umma::ex2(y1);
+                s4[e & 3] += p0 + p1;
+                PSplit<T>::run(p0, p1, w[2 * e], w[2 * e + 1]);
+            }
+            uint32_t pw[32];
+#pragma unroll
+            for (int q = 0; q < 32; ++q) pw[q] = w[2 * ((q >> 4) * 8 + (q & 7)) + ((q >> 3) & 1)];
+            umma::st32(lane_base + 32 * c, pw);
+        };
+        emit(3, sr[1]);
+        uint32_t rr[2][32];
+        umma::ld32(lane_base, rr[0]);
+        umma::ld32(lane_base + 32, rr[1]);
+        emit(2, sr[0]);
+        umma::wait_ld();
+        emit(0, rr[0]);
+        emit(1, rr[1]);
         l = l * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
-        // PV of stage i-1 must be done before O is rescaled and P overwritten
-        if (i > 0 && !warp_wait(pv_done, (i - 1) & 1, abort_flag)) {
-            ok = false;
-            break;
-        }
-        umma::fence_after_sync();
-        umma::st32(lane_base + kColPHi + half * 32, ph);
-        umma::st32(lane_base + kColPLo + half * 32, pl);
+        // O holds PV up to stage i-1 (complete: S(tile,i) was issued after it)
         if (__any_sync(0xffffffffu, rescale)) {  // warp-collective TMEM access
 #pragma unroll
-            for (int cb = 0; cb < D / 64; ++cb) {
+            for (int cb = 0; cb < D / 32; ++cb) {
                 uint32_t o[32];
-                const uint32_t col = lane_base + kColO + half * (D / 2) + cb * 32;
-                umma::ld32(col, o);
+                umma::ld32(lane_base + kColO + 32 * cb, o);
                 umma::wait_ld();
 #pragma unroll
                 for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                umma::st32(col, o);
+                umma::st32(lane_base + kColO + 32 * cb, o);
             }
         }
-        if (i * kKeys + kKeys > nkeys) {
-            // last stage: rows past the last key hold stale or unwritten data;
-            // zero them in V so that their zero weights give exact zeros.  The
-            // wait only orders these stores after the stage's copies.
-            if (!warp_wait(v_full + 8 * (i % NV), (i / NV) & 1, abort_flag)) {
-                ok = false;
-                break;
+        if constexpr (kMasked) {
+            if (tile == 0 && kb + kKeys > nkeys) {
+                // last stage: V rows past the last key hold stale or unwritten
+                // data; zero them so that their zero weights give exact zeros
+                // (tile 1's PV of this stage is issued after tile 0's).  The
+                // wait only orders these stores after the stage's copies.
+                if (!warp_wait(v_full + 8 * (i % NV), (i / NV) & 1, abort_flag)) return false;
+                const int first = nkeys - kb;  // rows [first, 128)
+                uint8_t *vst = smem + C::kVOffset + (i % NV) * C::kStageBytes;
+                for (int idx = r; idx < (kKeys - first) * C::kPieces * 8; idx += kM) {
+                    const int row = first + idx / (C::kPieces * 8);
+                    const int rem = idx % (C::kPieces * 8);
+                    *reinterpret_cast<uint4 *>(vst + (rem >> 3) * C::kKVPiece + row * kRowBytes +
+                                               ((rem & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
+                }
+                umma::fence_proxy_async_smem();
             }
-            const int first = nkeys - i * kKeys;  // rows [first, 128)
-            uint8_t *vst = smem + C::kVOffset + (i % NV) * C::kStageBytes;
-            for (int idx = threadIdx.x; idx < (kKeys - first) * C::kPieces * 8;
-                 idx += kSoftmaxThreads) {
-                const int row = first + idx / (C::kPieces * 8);
-                const int rem = idx % (C::kPieces * 8);
-                *reinterpret_cast<uint4 *>(vst + (rem >> 3) * C::kKVPiece + row * kRowBytes +
-                                           ((rem & 7) << 4)) = make_uint4(0u, 0u, 0u, 0u);
-            }
-            umma::fence_proxy_async_smem();
         }
         umma::wait_st();
         umma::fence_before_sync();
-        mbar_arrive(p_full);
-    }
-    if (ok && !warp_wait(pv_done, (nstages - 1) & 1, abort_flag)) ok = false;
-    if (ok) {
-        // the two halves' weight sums
-        xch[((nstages & 1) * 2 + half) * kM + r] = l;
-        mbar_arrive(my_xchg);
-        ok = __all_sync(0xffffffffu, mbar_wait_bounded(my_xchg, nstages & 1, abort_flag));
-    }
-    if (ok) {
-        l += xch[((nstages & 1) * 2 + (half ^ 1)) * kM + r];
+        mbar_arrive(p_full + 8 * tile);
+        return true;
+    };
+    // stages i < n_fast end at or before the tile's first token: no mask
+    const int n_fast = active ? min(nstages, (tile_pos0 + 1) / kKeys) : 0;
+    int i = 0;
+    for (; ok && i < n_fast; ++i) ok = stage(i, std::false_type{});
+    for (; ok && active && i < nstages; ++i) ok = stage(i, std::true_type{});
+    if (active && ok && !warp_wait(o_full + 8 * tile, 0, abort_flag)) ok = false;
+    if (active && ok) {
         umma::fence_after_sync();
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        float *dst = p.out + qrow + half * (D / 2);
+        float *dst = p.out + qrow;
 #pragma unroll
-        for (int cb = 0; cb < D / 64; ++cb) {
+        for (int cb = 0; cb < D / 32; ++cb) {
             uint32_t o[32];
-            umma::ld32(lane_base + kColO + half * (D / 2) + cb * 32, o);
+            umma::ld32(lane_base + kColO + 32 * cb, o);
             umma::wait_ld();
             if (valid) {
 #pragma unroll
@@ -464,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
                                     __uint_as_float(o[e + 3]) * inv);
             }
         }
-    } else if (lane == 0) {
+    } else if (!ok && lane == 0) {
         raise_device_error(p.err, PA_DEVERR_TIMEOUT);
         *abort_flag = 1;  // the other warps stop waiting
     }
@@ -483,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
 template <typename T, int D, int BS>
 static cudaError_t launch_inst(const PrefillParams &p, const CUtensorMap &mk,
                                const CUtensorMap &mv, cudaStream_t stream) {
-    constexpr int NK = D == 128 ? 3 : 4, NV = D == 128 ? 2 : 4;
+    constexpr int NK = D == 128 ? 2 : 4, NV = D == 128 ? 2 : 4;
     using C = Cfg<D, BS, NK, NV>;
     static std::once_flag once[64];
     static cudaError_t attr_err[64];
