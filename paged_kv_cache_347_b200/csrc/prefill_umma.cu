@@ -83,6 +83,27 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatil
     return __all_sync(0xffffffffu, mbar_wait_bounded(bar, parity, abort_flag));
 }
 
+// Paired fp32 arithmetic (sm_100 f32x2 instructions): two lanes per instruction.
+__device__ __forceinline__ uint64_t pk(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ void upk(uint64_t r, float &a, float &b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+// max of three (sm_100 three-input max)
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // Two weights -> their 16-bit high parts and remainders, one 32-bit word each
 // (lower key in the low half).  bf16: the high part is the upper 16 bits of
 // the fp32 pattern, the remainder x - hi is exact in fp32 and is cut to its
@@ -117,7 +138,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
 
     pdl_wait_prior_grid();
 
-    const int qt = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+    // later token tiles attend to more keys: hand them out first
+    const int qt = gridDim.x - 1 - blockIdx.x, g = blockIdx.y, s = blockIdx.z;
     const int G = p.num_heads / p.num_kv_heads;
     const int TQ = p.tokens_per_cta / 2;  // tokens per tile: 128 / G
     const int q0 = __ldg(p.cu_q + s);
@@ -345,8 +367,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
                 if constexpr (kMasked) {
                     const float v = 32 * c + e > last ? -INFINITY : __uint_as_float(w[e]) * sl2;
                     m4[e & 3] = fmaxf(m4[e & 3], v);
-                } else {
-                    m4[e & 3] = fmaxf(m4[e & 3], __uint_as_float(w[e]));
+                } else if (e % 2 == 0) {
+                    m4[(e >> 1) & 3] =
+                        max3(m4[(e >> 1) & 3], __uint_as_float(w[e]), __uint_as_float(w[e + 1]));
                 }
             }
         };
@@ -381,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         // block q / 16 of the chunk, high parts in its first 8 columns,
         // remainders in the next 8.  Chunks 3 and 2 come from the registers;
         // chunks 0 and 1 are read again (issued while chunk 2 is worked on).
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+        uint64_t acc[2] = {pk(0.f, 0.f), pk(0.f, 0.f)};
         auto emit = [&](int c, uint32_t (&w)[32]) {
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
@@ -392,7 +415,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
                     if (32 * c + 2 * e + 1 > last) y1 = -INFINITY;
                 }
                 const float p0 = umma::ex2(y0), p1 = umma::ex2(y1);
-                s4[e & 3] += p0 + p1;
+                acc[e & 1] = add2(acc[e & 1], pk(p0, p1));
                 PSplit<T>::run(p0, p1, w[2 * e], w[2 * e + 1]);
             }
             uint32_t pw[32];
@@ -408,7 +431,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         umma::wait_ld();
         emit(0, rr[0]);
         emit(1, rr[1]);
-        l = l * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+        {
+            float a0, a1, b0, b1;
+            upk(acc[0], a0, a1);
+            upk(acc[1], b0, b1);
+            l = l * alpha + ((a0 + a1) + (b0 + b1));
+        }
         // O holds PV up to stage i-1 (complete: S(tile,i) was issued after it)
         if (__any_sync(0xffffffffu, rescale)) {  // warp-collective TMEM access
 #pragma unroll
