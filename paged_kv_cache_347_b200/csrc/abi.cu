@@ -346,7 +346,7 @@ int pa_prefill_ex(float *out, const void *q, const void *k_cache, const void *v_
     p.num_blocks = num_blocks;
     p.max_seq_len = max_seq_len;
     p.max_q_len = max_q_len;
-    p.tokens_per_cta = variant == 2 ? 2 * (128 / G) : 64 / G;
+    p.tokens_per_cta = (variant == 2 ? 128 : 64) / G;
     p.scale_log2 = scale * 1.4426950408889634f;
     cudaError_t e = variant == 2 ? launch_prefill_umma(p, dtype, static_cast<cudaStream_t>(stream))
                                  : launch_prefill_tc(p, dtype, static_cast<cudaStream_t>(stream));

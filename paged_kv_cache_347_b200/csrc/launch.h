@@ -63,7 +63,7 @@ struct PrefillParams {
     unsigned int *err;
     int num_seqs, num_heads, num_kv_heads, head_dim, block_size;
     int max_blocks_per_seq, num_blocks, max_seq_len, max_q_len;
-    int tokens_per_cta;             // query tokens per CTA: 64 / G (mma.sync), 2 x 128 / G (tcgen05)
+    int tokens_per_cta;             // query tokens per CTA: 64 / G (mma.sync), 128 / G (tcgen05)
     float scale_log2;
 };
 // mma.sync kernel: 64 (token, head) rows per CTA, accumulators in registers.

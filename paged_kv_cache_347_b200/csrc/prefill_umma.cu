@@ -1,35 +1,34 @@
 // Causal multi-token attention over the paged cache on the 5th-generation
-// tensor cores (tcgen05, accumulators in tensor memory), sm_100a.
+// tensor cores (tcgen05, operands and accumulators in tensor memory), sm_100a.
 //
 // Same quantity as prefill_tc.cu (mbrenndoerfer.com "Paged Attention >
 // Summary", bullet 3; paweldubiel.com "PagedAttention", "Mechanism and
 // details"): row r of a sequence's chunk, at position L - n + r, attends to
 // positions 0..L-n+r through the block table.
 //
-// CTA = two tiles of 128 (token, query head) rows -- 2 x 128/G chunk tokens
-// of one KV head g of one sequence -- walking the context in stages of 128
-// keys.  Twelve warps:
-//   * warps 0-3 (tile 0) and 4-7 (tile 1), softmax: one thread per row
-//     (thread i of a tile <-> TMEM lane i).  Per stage a thread reads its
-//     128 S values from TMEM (the row maximum first), writes
-//     P = 2^(x - m) as 16-bit high part + remainder into the same TMEM
-//     columns, and rescales its O row when the maximum has grown by
-//     more than 2^8; at the end it divides by the summed weights and stores
-//     the row;
+// CTA = 128 (token, query head) rows: 128/G chunk tokens of one KV head g of
+// one sequence, walking the context in stages of 128 keys.  Eleven warps:
+//   * warps 0-7, softmax: warp w serves TMEM lanes 32 (w % 4) .. +31 (the
+//     rows) and keys 64 (w / 4) .. +63 of each stage, so each row has two
+//     threads, which agree its maximum through shared memory.  A thread reads
+//     its 64 S values from TMEM, writes P = 2^(x - m) as 16-bit high part +
+//     remainder into the same TMEM columns, and rescales its half of the O
+//     row when the maximum has grown by more than 2^8; at the end the halves'
+//     weight sums are added and each thread divides and stores its half row;
 //   * warps 8 and 9: TMA producers of the K and the V stages, gathered block
 //     by block through the table into two rings;
-//   * warp 10, one thread: issues the UMMAs in the order
-//       PV(0,i), S(0,i+1), PV(1,i), S(1,i+1), ...   with
-//       S(t,i)  [128 x 128] = Q_t . K_i^T        (Q, K from shared memory)
-//       PV(t,i) O_t [128 x D] += P_t . V_i        (P from TMEM, V N-major)
-//     so that the tensor core works on one tile while the other tile's
-//     softmax runs.  S(t,i+1) overwrites the columns PV(t,i) reads; the two
-//     are issued by the same thread and tcgen05 MMAs of one thread execute
-//     in issue order;
-//   * warp 11 has no work after set-up.
-// TMEM (512 columns): tile t at 256 t: S / P [0,128), O [128,128+D).  In P,
-// key block j (keys 16j..16j+15) holds its high parts in columns 16j..16j+7
-// and its remainders in 16j+8..16j+15, two keys per column.
+//   * warp 10, one thread, issues the UMMAs:
+//       S(i)  [128 x 128] = Q . K_i^T      (Q from TMEM, K from shared memory)
+//       PV(i) O [128 x D] += P_i . V_i      (P from TMEM, V N-major, twice:
+//                                            high part and remainder)
+//     in the order S(0), S(1), PV(0), S(2), PV(1), S(3), ...: S is double-
+//     buffered, so the softmax of stage i+1 can start as soon as it ends
+//     stage i.  S(i+2) overwrites the columns PV(i) reads; the two are issued
+//     by the same thread and tcgen05 MMAs of one thread execute in order.
+// TMEM (512 columns): S/P buffers [0,128) and [128,256), O [256,256+D),
+// Q [384,384+D/2).  In P, key block j (keys 16j..16j+15) holds its high parts
+// in columns 16j..16j+7 and its remainders in 16j+8..16j+15, two keys per
+// column; Q holds two elements of a row per column.
 //
 // Every wait is bounded (~2 s); on a timeout the CTA records
 // PA_DEVERR_TIMEOUT, the other warps stop waiting, the producers wait
@@ -45,28 +44,26 @@
 namespace pa {
 namespace pu {
 
-constexpr int kM = 128;               // rows per tile
+constexpr int kM = 128;               // rows per CTA
 constexpr int kKeys = 128;            // keys per stage
-constexpr int kSoftmaxThreads = 256;  // two tiles x 4 warps
-constexpr int kThreads = kSoftmaxThreads + 128;
+constexpr int kSoftmaxThreads = 256;  // 8 warps, two threads per row
+constexpr int kThreads = kSoftmaxThreads + 96;
 constexpr int kTmemCols = 512;
-constexpr int kTileCols = 256;        // per tile: S / P, then O
-constexpr int kColO = 128;
+constexpr int kColO = 256, kColQ = 384;
 constexpr int kRowBytes = 128;        // one 64-element piece of a 16-bit row
 
 template <int D, int BS, int NK, int NV>
 struct Cfg {
     static constexpr int kPieces = D / 64;
-    static constexpr int kQPiece = kM * kRowBytes;          // 16 KB
-    static constexpr int kQTile = kPieces * kQPiece;
     static constexpr int kKVPiece = kKeys * kRowBytes;      // 16 KB
     static constexpr int kStageBytes = kPieces * kKVPiece;  // one K or V stage
-    static constexpr int kQOffset = 0;                      // Q tiles [2]
-    static constexpr int kKOffset = 2 * kQTile;             // K ring [NK]
-    static constexpr int kVOffset = kKOffset + NK * kStageBytes;  // V ring [NV]
-    static constexpr int kBarOffset = kVOffset + NV * kStageBytes;
-    // k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] s_full[2] p_full[2] o_full[2] q_full mma_done
-    static constexpr int kNumBars = 2 * NK + 2 * NV + 8;
+    static constexpr int kKOffset = 0;                              // K ring [NK]
+    static constexpr int kVOffset = kKOffset + NK * kStageBytes;    // V ring [NV]
+    static constexpr int kXchOffset = kVOffset + NV * kStageBytes;  // float [2][2][128]
+    static constexpr int kBarOffset = kXchOffset + 2 * 2 * kM * 4;
+    // k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] s_full[2] p_full[2] pv_done q_full
+    // mma_done xchg[4]
+    static constexpr int kNumBars = 2 * NK + 2 * NV + 4 + 3 + 4;
     static constexpr int kTmemSlot = kBarOffset + kNumBars * 8;
     static constexpr int kAbortOffset = kTmemSlot + 16;
     static constexpr int kSmemBytes = kAbortOffset + 16;
@@ -75,6 +72,7 @@ struct Cfg {
     static_assert(kDynSmem <= 227 * 1024, "shared memory");
     static_assert(kKeys % BS == 0 && kBlocksPerStage <= 32, "block size");
     static_assert(D == 64 || D == 128, "head size");
+    static_assert(kColO + D <= kColQ && kColQ + D / 2 <= kTmemCols, "tensor memory");
 };
 
 // A bounded mbarrier wait taken by a whole warp, with one outcome for all
@@ -141,7 +139,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     // later token tiles attend to more keys: hand them out first
     const int qt = gridDim.x - 1 - blockIdx.x, g = blockIdx.y, s = blockIdx.z;
     const int G = p.num_heads / p.num_kv_heads;
-    const int TQ = p.tokens_per_cta / 2;  // tokens per tile: 128 / G
+    const int TQ = p.tokens_per_cta;  // 128 / G
     const int q0 = __ldg(p.cu_q + s);
     const int n = __ldg(p.cu_q + s + 1) - q0;
     const int L = __ldg(p.seq_lens + s);
@@ -150,10 +148,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         if (qt == 0 && g == 0 && threadIdx.x == 0) raise_device_error(p.err, PA_DEVERR_SEQLEN);
         return;
     }
-    const int tok0 = qt * 2 * TQ;
+    const int tok0 = qt * TQ;
     if (tok0 >= n) return;  // uniform, before any barrier or TMEM use
-    const int ntok = min(2 * TQ, n - tok0);
-    const bool two = ntok > TQ;  // tile 1 has rows
+    const int ntok = min(TQ, n - tok0);
     const int pos0 = L - n + tok0;
     const int nkeys = pos0 + ntok;
     const int nstages = (nkeys + kKeys - 1) / kKeys;
@@ -161,12 +158,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const uint32_t sbase = smem_u32(smem);
-    const uint32_t q_s = sbase + C::kQOffset, k_s = sbase + C::kKOffset,
-                   v_s = sbase + C::kVOffset;
+    const uint32_t k_s = sbase + C::kKOffset, v_s = sbase + C::kVOffset;
     const uint32_t bar0 = sbase + C::kBarOffset;
     const uint32_t k_full = bar0, k_empty = k_full + 8 * NK, v_full = k_empty + 8 * NK,
                    v_empty = v_full + 8 * NV, s_full = v_empty + 8 * NV, p_full = s_full + 16,
-                   o_full = p_full + 16, q_full = o_full + 16, mma_done = q_full + 8;
+                   pv_done = p_full + 16, q_full = pv_done + 8, mma_done = q_full + 8,
+                   xchg = mma_done + 8;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kAbortOffset);
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + C::kTmemSlot);
 
@@ -179,13 +176,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
             mbar_init(v_full + 8 * i, 1);
             mbar_init(v_empty + 8 * i, 1);
         }
-        for (int t = 0; t < 2; ++t) {
-            mbar_init(s_full + 8 * t, 1);
-            mbar_init(p_full + 8 * t, kM);
-            mbar_init(o_full + 8 * t, 1);
+        // one s_full and one p_full per S buffer: the softmax may finish stage
+        // i+1 before the MMA thread has seen stage i, never stage i+2
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(s_full + 8 * b, 1);
+            mbar_init(p_full + 8 * b, kSoftmaxThreads);
         }
+        mbar_init(pv_done, 1);
         mbar_init(q_full, kSoftmaxThreads);
         mbar_init(mma_done, 1);
+        for (int q = 0; q < 4; ++q) mbar_init(xchg + 8 * q, 64);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -197,8 +197,6 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     __syncthreads();
     umma::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-
-    if (warp == 11) return;
 
     // ------------------------------------------------------------ producers
     // warp 8 loads the K stages, warp 9 the V stages, each at its own pace
@@ -256,56 +254,64 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
             constexpr uint32_t fmt = StoreT<T>::kCode == PA_BF16 ? 1u : 0u;
             constexpr uint32_t idesc_s = umma::idesc_f16(fmt, kM, kKeys, 0);
             constexpr uint32_t idesc_o = umma::idesc_f16(fmt, kM, D, 1);
-            const int last_tile = two ? 1 : 0;  // the tile whose MMAs free a K / V slot
-            // S(t,i) = Q_t . K_i^T into tile t's S columns
-            auto issue_s = [&](int t, int i) -> bool {
+            // S(i) = Q . K_i^T into S buffer i % 2
+            auto issue_s = [&](int i) -> bool {
                 const int slot = i % NK;
-                if (t == 0 && !mbar_wait_bounded(k_full + 8 * slot, (i / NK) & 1, abort_flag))
-                    return false;
+                if (!mbar_wait_bounded(k_full + 8 * slot, (i / NK) & 1, abort_flag)) return false;
                 umma::fence_after_sync();
-                // descriptors advance by (bytes >> 4) in their start-address field
-                const uint64_t a0 = umma::smem_desc_sw128(q_s + t * C::kQTile, 16, 1024);
+                // K rows: 8-row groups 1 KB apart; descriptors advance by (bytes >> 4)
                 const uint64_t b0 = umma::smem_desc_sw128(k_s + slot * C::kStageBytes, 16, 1024);
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t qa = ((kk >> 2) * C::kQPiece + (kk & 3) * 32) >> 4;
                     const uint32_t ka = ((kk >> 2) * C::kKVPiece + (kk & 3) * 32) >> 4;
-                    umma::mma_f16(tmem + t * kTileCols, a0 + qa, b0 + ka, idesc_s, kk > 0);
+                    umma::mma_f16_ts(tmem + (i & 1) * kKeys, tmem + kColQ + 8 * kk, b0 + ka,
+                                     idesc_s, kk > 0);
                 }
-                umma::commit(s_full + 8 * t);
-                if (t == last_tile) umma::commit(k_empty + 8 * slot);
                 return true;
             };
-            // O_t += P_t . V_i once tile t's softmax has written P_t
-            auto issue_pv = [&](int t, int i) -> bool {
+            auto commit_s = [&](int i) {
+                umma::commit(s_full + 8 * (i & 1));
+                umma::commit(k_empty + 8 * (i % NK));
+            };
+            // O += P_i . V_i once the softmax has written P_i
+            auto issue_pv = [&](int i) -> bool {
                 const int slot = i % NV;
-                if (!mbar_wait_bounded(p_full + 8 * t, i & 1, abort_flag)) return false;
-                if (t == 0 && !mbar_wait_bounded(v_full + 8 * slot, (i / NV) & 1, abort_flag))
+                if (!mbar_wait_bounded(p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag) ||
+                    !mbar_wait_bounded(v_full + 8 * slot, (i / NV) & 1, abort_flag))
                     return false;
                 umma::fence_after_sync();
                 // V rows: 8-row groups 1 KB apart, 64-column pieces 16 KB apart
                 const uint64_t b0 = umma::smem_desc_sw128(v_s + slot * C::kStageBytes,
                                                           C::kKVPiece, 1024);
-                const uint32_t tb = tmem + t * kTileCols;
+                const uint32_t pb = tmem + (i & 1) * kKeys;
 #pragma unroll
                 for (int j = 0; j < kKeys / 16; ++j) {  // keys 16j..16j+15
                     const uint64_t b = b0 + ((j * 16 * kRowBytes) >> 4);
-                    umma::mma_f16_ts(tb + kColO, tb + 16 * j, b, idesc_o, (i > 0 || j > 0) ? 1u : 0u);
-                    umma::mma_f16_ts(tb + kColO, tb + 16 * j + 8, b, idesc_o, 1u);
+                    umma::mma_f16_ts(tmem + kColO, pb + 16 * j, b, idesc_o, (i > 0 || j > 0) ? 1u : 0u);
+                    umma::mma_f16_ts(tmem + kColO, pb + 16 * j + 8, b, idesc_o, 1u);
                 }
-                if (t == last_tile) umma::commit(v_empty + 8 * slot);
-                if (i == nstages - 1) umma::commit(o_full + 8 * t);
                 return true;
             };
+            auto commit_pv = [&](int i) {
+                umma::commit(pv_done);
+                umma::commit(v_empty + 8 * (i % NV));
+            };
             bool ok = mbar_wait_bounded(q_full, 0, abort_flag);
-            if (ok) ok = issue_s(0, 0);
-            if (ok && two) ok = issue_s(1, 0);
+            umma::fence_after_sync();
+            if (ok) ok = issue_s(0);
+            if (ok) commit_s(0);
+            if (ok && nstages > 1) ok = issue_s(1);
+            if (ok && nstages > 1) commit_s(1);
+            // The commits of PV(i) and S(i+2) follow both groups of MMAs, so they
+            // are issued while the tensor core still has queued work (a commit
+            // arrives once every MMA issued before it has completed).
 #pragma unroll 1
             for (int i = 0; ok && i < nstages; ++i) {
-                ok = issue_pv(0, i);
-                if (ok && i + 1 < nstages) ok = issue_s(0, i + 1);
-                if (ok && two) ok = issue_pv(1, i);
-                if (ok && two && i + 1 < nstages) ok = issue_s(1, i + 1);
+                ok = issue_pv(i);
+                const bool s_next = ok && i + 2 < nstages;
+                if (s_next) ok = issue_s(i + 2);
+                if (s_next && ok) commit_s(i + 2);
+                commit_pv(i);
             }
             if (!ok) {
                 raise_device_error(p.err, PA_DEVERR_TIMEOUT);
@@ -317,78 +323,86 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     }
 
     // ------------------------------------------------------------ softmax warps
-    const int tile = warp >> 2, quarter = warp & 3;
-    const int r = quarter * 32 + lane;  // row of the tile == TMEM lane
+    const int quarter = warp & 3, half = warp >> 2;
+    const int r = quarter * 32 + lane;  // row == TMEM lane
     const int tl = r / G, hh = r - tl * G;
-    const int ttok = tile * TQ + tl;  // chunk token of this row, relative to tok0
-    const bool valid = r < TQ * G && ttok < ntok;
-    const int qp = valid ? pos0 + ttok : nkeys - 1;
-    const int tile_pos0 = pos0 + tile * TQ;  // position of the tile's first token
-    const int64_t qrow = ((int64_t)(q0 + tok0 + ttok) * p.num_heads + g * G + hh) * D;
+    const bool valid = r < TQ * G && tl < ntok;
+    const int qp = valid ? pos0 + tl : nkeys - 1;
+    // stages i < n_fast end at or before the first chunk token: no mask there
+    const int n_fast = min(nstages, (pos0 + 1) / kKeys);
+    const int64_t qrow = ((int64_t)(q0 + tok0 + tl) * p.num_heads + g * G + hh) * D;
+    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     // S is computed with sign(scale) folded into Q (a sign-bit flip, exact),
     // so that the logit scale applied below is non-negative
     const uint32_t qflip = p.scale_log2 < 0.f ? 0x80008000u : 0u;
     const float sl2 = fabsf(p.scale_log2);
     {
-        // the Q row -> tile's swizzled K-major Q (row r, 16-byte chunk c at
-        // c ^ (r & 7) within its 128-byte piece row)
-        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.q) + qrow);
-        uint8_t *qt_s = smem + C::kQOffset + tile * C::kQTile;
+        // the Q row into TMEM, two elements per column: for D 128 each half
+        // of the row's threads writes 32 columns, for D 64 the first writes all
+        if (D == 128 || half == 0) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.q) + qrow) +
+                               half * (D == 128 ? 8 : 0);
+            uint32_t w[32];
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-            uint4 v = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-            v.x ^= qflip; v.y ^= qflip; v.z ^= qflip; v.w ^= qflip;
-            *reinterpret_cast<uint4 *>(qt_s + (c >> 3) * C::kQPiece + r * kRowBytes +
-                                       (((c & 7) ^ (r & 7)) << 4)) = v;
+            for (int c = 0; c < 8; ++c) {
+                uint4 v = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+                w[4 * c] = v.x ^ qflip;
+                w[4 * c + 1] = v.y ^ qflip;
+                w[4 * c + 2] = v.z ^ qflip;
+                w[4 * c + 3] = v.w ^ qflip;
+            }
+            umma::st32(lane_base + kColQ + half * 32, w);
+            umma::wait_st();
         }
-        umma::fence_proxy_async_smem();
+        umma::fence_before_sync();
         mbar_arrive(q_full);
     }
-    const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16) + tile * kTileCols;
+    float *xch = reinterpret_cast<float *>(smem + C::kXchOffset);  // [parity][half][row]
+    const uint32_t my_xchg = xchg + 8 * quarter;
+    int xp = 0;  // exchanges so far (the same sequence for both threads of a row)
+    // the partner thread's value of x (same row, other half of the keys)
+    auto exchange = [&](float x, float &other) -> bool {
+        xch[((xp & 1) * 2 + half) * kM + r] = x;
+        mbar_arrive(my_xchg);
+        const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(my_xchg, xp & 1, abort_flag));
+        other = xch[((xp & 1) * 2 + (half ^ 1)) * kM + r];
+        ++xp;
+        return got;
+    };
     float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    const bool active = tile == 0 || two;
-    // One stage of the softmax.  Keys past a row's position exist only on
-    // stages reaching beyond the tile's first token; those run the masked
-    // body, every earlier stage the unmasked one (the split also keeps the
-    // hot loop's code small).
+    // One stage.  Stages reaching beyond the first chunk token run the
+    // masked body, every earlier stage the unmasked one.
     auto stage = [&](int i, auto masked_c) __attribute__((always_inline)) -> bool {
         constexpr bool kMasked = decltype(masked_c)::value;
-        if (!warp_wait(s_full + 8 * tile, i & 1, abort_flag)) return false;
+        if (!warp_wait(s_full + 8 * (i & 1), (i >> 1) & 1, abort_flag)) return false;
         umma::fence_after_sync();
-        const int kb = i * kKeys;
-        // the row maximum over the stage's 128 logits, read as chunks 0-1 then
-        // 2-3 (two loads in flight each time); chunks 2-3 stay in registers
-        const int last = qp - kb;  // the row's last key within the stage (masked body)
-        float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-        auto fold_max = [&](int c, const uint32_t (&w)[32]) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                if constexpr (kMasked) {
-                    const float v = 32 * c + e > last ? -INFINITY : __uint_as_float(w[e]) * sl2;
-                    m4[e & 3] = fmaxf(m4[e & 3], v);
-                } else if (e % 2 == 0) {
-                    m4[(e >> 1) & 3] =
-                        max3(m4[(e >> 1) & 3], __uint_as_float(w[e]), __uint_as_float(w[e + 1]));
-                }
-            }
-        };
+        const uint32_t hcol = lane_base + (i & 1) * kKeys + half * 64;  // this thread's S / P
+        const int last = qp - (i * kKeys + half * 64);  // the row's last key in the half
         uint32_t sr[2][32];
-        {
-            uint32_t t0[32], t1[32];
-            umma::ld32(lane_base, t0);
-            umma::ld32(lane_base + 32, t1);
-            umma::wait_ld();
-            fold_max(0, t0);
-            fold_max(1, t1);
-        }
-        umma::ld32(lane_base + 64, sr[0]);
-        umma::ld32(lane_base + 96, sr[1]);
+        umma::ld32(hcol, sr[0]);
+        umma::ld32(hcol + 32, sr[1]);
         umma::wait_ld();
-        fold_max(2, sr[0]);
-        fold_max(3, sr[1]);
-        float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-        if constexpr (!kMasked) mx *= sl2;  // sl2 >= 0
+        float mx;
+        {
+            float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    if constexpr (kMasked) {
+                        const float v = 32 * c + e > last ? -INFINITY : __uint_as_float(sr[c][e]) * sl2;
+                        m4[e & 3] = fmaxf(m4[e & 3], v);
+                    } else if (e % 2 == 0) {
+                        m4[(e >> 1) & 3] = max3(m4[(e >> 1) & 3], __uint_as_float(sr[c][e]),
+                                                __uint_as_float(sr[c][e + 1]));
+                    }
+                }
+            mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+            if constexpr (!kMasked) mx *= sl2;  // sl2 >= 0
+        }
+        float other;
+        if (!exchange(mx, other)) return false;
+        mx = fmaxf(mx, other);
         // the running max moves only when it grows by more than 8 (log2 units):
         // weights then stay below 2^8 and O is rescaled rarely
         float alpha = 1.f;
@@ -399,13 +413,14 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
             m = mx;
         }
         // weights 2^(x - m), summed and split in place: the pair of keys
-        // (2e, 2e+1) of a chunk leaves its high-part word in word 2e and its
-        // remainder word in word 2e+1; TMEM column 32c + q then takes key
-        // block q / 16 of the chunk, high parts in its first 8 columns,
-        // remainders in the next 8.  Chunks 3 and 2 come from the registers;
-        // chunks 0 and 1 are read again (issued while chunk 2 is worked on).
+        // (2e, 2e+1) of a 32-key chunk leaves its high-part word in word 2e
+        // and its remainder word in word 2e+1; the chunk's TMEM column q then
+        // takes key block q / 16 of the chunk, high parts in its first 8
+        // columns, remainders in the next 8 (over the chunk's own S columns)
         uint64_t acc[2] = {pk(0.f, 0.f), pk(0.f, 0.f)};
-        auto emit = [&](int c, uint32_t (&w)[32]) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            uint32_t(&w)[32] = sr[c];
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
                 float y0 = fmaf(__uint_as_float(w[2 * e]), sl2, -m);
@@ -421,44 +436,39 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
             uint32_t pw[32];
 #pragma unroll
             for (int q = 0; q < 32; ++q) pw[q] = w[2 * ((q >> 4) * 8 + (q & 7)) + ((q >> 3) & 1)];
-            umma::st32(lane_base + 32 * c, pw);
-        };
-        emit(3, sr[1]);
-        uint32_t rr[2][32];
-        umma::ld32(lane_base, rr[0]);
-        umma::ld32(lane_base + 32, rr[1]);
-        emit(2, sr[0]);
-        umma::wait_ld();
-        emit(0, rr[0]);
-        emit(1, rr[1]);
+            umma::st32(hcol + 32 * c, pw);
+        }
         {
             float a0, a1, b0, b1;
             upk(acc[0], a0, a1);
             upk(acc[1], b0, b1);
             l = l * alpha + ((a0 + a1) + (b0 + b1));
         }
-        // O holds PV up to stage i-1 (complete: S(tile,i) was issued after it)
         if (__any_sync(0xffffffffu, rescale)) {  // warp-collective TMEM access
+            // O must hold PV up to stage i-1 before it is rescaled
+            if (i > 0 && !warp_wait(pv_done, (i - 1) & 1, abort_flag)) return false;
+            umma::fence_after_sync();
 #pragma unroll
-            for (int cb = 0; cb < D / 32; ++cb) {
+            for (int cb = 0; cb < D / 64; ++cb) {
                 uint32_t o[32];
-                umma::ld32(lane_base + kColO + 32 * cb, o);
+                const uint32_t col = lane_base + kColO + half * (D / 2) + 32 * cb;
+                umma::ld32(col, o);
                 umma::wait_ld();
 #pragma unroll
                 for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                umma::st32(lane_base + kColO + 32 * cb, o);
+                umma::st32(col, o);
             }
         }
         if constexpr (kMasked) {
-            if (tile == 0 && kb + kKeys > nkeys) {
+            if (i * kKeys + kKeys > nkeys) {
                 // last stage: V rows past the last key hold stale or unwritten
-                // data; zero them so that their zero weights give exact zeros
-                // (tile 1's PV of this stage is issued after tile 0's).  The
-                // wait only orders these stores after the stage's copies.
+                // data; zero them so that their zero weights give exact zeros.
+                // The wait only orders these stores after the stage's copies.
                 if (!warp_wait(v_full + 8 * (i % NV), (i / NV) & 1, abort_flag)) return false;
-                const int first = nkeys - kb;  // rows [first, 128)
+                const int first = nkeys - i * kKeys;  // rows [first, 128)
                 uint8_t *vst = smem + C::kVOffset + (i % NV) * C::kStageBytes;
-                for (int idx = r; idx < (kKeys - first) * C::kPieces * 8; idx += kM) {
+                for (int idx = threadIdx.x; idx < (kKeys - first) * C::kPieces * 8;
+                     idx += kSoftmaxThreads) {
                     const int row = first + idx / (C::kPieces * 8);
                     const int rem = idx % (C::kPieces * 8);
                     *reinterpret_cast<uint4 *>(vst + (rem >> 3) * C::kKVPiece + row * kRowBytes +
@@ -469,23 +479,24 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         }
         umma::wait_st();
         umma::fence_before_sync();
-        mbar_arrive(p_full + 8 * tile);
+        mbar_arrive(p_full + 8 * (i & 1));
         return true;
     };
-    // stages i < n_fast end at or before the tile's first token: no mask
-    const int n_fast = active ? min(nstages, (tile_pos0 + 1) / kKeys) : 0;
+    bool ok = true;
     int i = 0;
     for (; ok && i < n_fast; ++i) ok = stage(i, std::false_type{});
-    for (; ok && active && i < nstages; ++i) ok = stage(i, std::true_type{});
-    if (active && ok && !warp_wait(o_full + 8 * tile, 0, abort_flag)) ok = false;
-    if (active && ok) {
+    for (; ok && i < nstages; ++i) ok = stage(i, std::true_type{});
+    float other = 0.f;
+    if (ok) ok = warp_wait(pv_done, (nstages - 1) & 1, abort_flag) && exchange(l, other);
+    if (ok) {
         umma::fence_after_sync();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-        float *dst = p.out + qrow;
+        const float lt = l + other;
+        const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        float *dst = p.out + qrow + half * (D / 2);
 #pragma unroll
-        for (int cb = 0; cb < D / 32; ++cb) {
+        for (int cb = 0; cb < D / 64; ++cb) {
             uint32_t o[32];
-            umma::ld32(lane_base + kColO + 32 * cb, o);
+            umma::ld32(lane_base + kColO + half * (D / 2) + 32 * cb, o);
             umma::wait_ld();
             if (valid) {
 #pragma unroll
@@ -496,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
                                     __uint_as_float(o[e + 3]) * inv);
             }
         }
-    } else if (!ok && lane == 0) {
+    } else if (lane == 0) {
         raise_device_error(p.err, PA_DEVERR_TIMEOUT);
         *abort_flag = 1;  // the other warps stop waiting
     }
@@ -515,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
 template <typename T, int D, int BS>
 static cudaError_t launch_inst(const PrefillParams &p, const CUtensorMap &mk,
                                const CUtensorMap &mv, cudaStream_t stream) {
-    constexpr int NK = D == 128 ? 2 : 4, NV = D == 128 ? 2 : 4;
+    constexpr int NK = D == 128 ? 3 : 6, NV = D == 128 ? 3 : 6;
     using C = Cfg<D, BS, NK, NV>;
     static std::once_flag once[64];
     static cudaError_t attr_err[64];
