@@ -408,9 +408,10 @@ def run_ours(args, ws, rank, local):
 
 
 def run_e2e(args, sh, width, seed, prefill, dev, ws):
-    """Live steps through the public API (PagedKVRunner.run_pinned): host
-    allocator, inputs copied from pinned host memory, output read back,
-    every step synchronised."""
+    """Live steps through the public API (PagedKVRunner prepare / stage_graph
+    / replay_graph, or launch when a step has no graph form): host allocator,
+    inputs copied from pinned host memory, output read back, every step
+    synchronised."""
     from paged_kv_cache_347_b200.runner import PagedKVRunner
     n = max(1, min(args.steps, args.e2e_steps))
     w = min(args.warmup, 3)
@@ -425,18 +426,28 @@ def run_e2e(args, sh, width, seed, prefill, dev, ws):
     out_host = torch.empty((b, sh.num_heads, sh.head_dim), dtype=torch.float32).pin_memory()
     h2d = d2h = 0
     total = 0
+    replays = 0
+    graphs = not args.no_graph
 
-    # the allocator work of step i+1 runs on the host while the GPU runs step
-    # i; every step still copies its inputs in and its output back before the
-    # next step's inputs go out
+    # the allocator work of step i+1 (and the copy of its inputs into the
+    # page-locked buffers of its CUDA graph) runs on the host while the GPU
+    # runs step i; every step still copies its inputs in and its output back
+    # before the next step's inputs go out
     def loop(first, count):
-        nonlocal h2d, d2h, total
+        nonlocal h2d, d2h, total, replays
         if count <= 0:
             return
         prep = r.prepare(host[first][0])
+        gr = r.stage_graph(prep, *host[first][1:]) if graphs else None
         for i in range(first, first + count):
-            res = r.launch(prep, *host[i][1:], out_host)
-            prep = r.prepare(host[i + 1][0]) if i + 1 < first + count else None
+            if gr is not None:
+                res = r.replay_graph(gr, prep)
+                replays += first >= w
+            else:
+                res = r.launch(prep, *host[i][1:], out_host)
+            if i + 1 < first + count:
+                prep = r.prepare(host[i + 1][0])
+                gr = r.stage_graph(prep, *host[i + 1][1:]) if graphs else None
             r.wait()
             if first >= w:
                 d = [a for a in res["acts"] if a.kind == "decode"][0]
@@ -452,7 +463,8 @@ def run_e2e(args, sh, width, seed, prefill, dev, ws):
     el, total = aggregate(el, float(total), ws, dev)
     return {"value": round(total / el / 1e9, 1), "unit": "GB/s",
             "h2d_bytes_per_step": int(h2d / n), "d2h_bytes_per_step": int(d2h / n),
-            "steps": n, "us_per_step": round(el / n * 1e6, 2)}
+            "steps": n, "us_per_step": round(el / n * 1e6, 2),
+            "graph_replayed_steps": replays}
 
 
 def run_reference(args, ws, rank):
@@ -652,6 +664,8 @@ def main():
     ap.add_argument("--workload", default="long32k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--no-graph", action="store_true",
+                    help="e2e: launch every step eagerly instead of replaying CUDA graphs")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--study", default="", choices=["", "prefix", "swap", "blocksize", "prefill"],

@@ -298,6 +298,107 @@ class PagedKVRunner:
     def wait(self) -> None:
         torch.cuda.current_stream(self.device).synchronize()
 
+    # ------------------------------------------------------------ graph replay
+    # Steps of the same layout (the same action kinds and sizes, no copy-on-
+    # write pairs, prepared in the same staging slot) repeat the same device
+    # work on different bytes.  launch_graph() captures that work once per
+    # layout -- the copy of the packed arrays, the copies of the new K/V rows
+    # and queries from page-locked buffers owned by the graph, the kernels and
+    # the copy of the output back -- and replays it; a decode inside a graph
+    # takes the table capacity as its length bound, so that its grid is fixed.
+    def _graph_key(self, prep: dict, k_new: torch.Tensor, q: torch.Tensor):
+        acts = prep["acts"]
+        if not acts or any(a.kind not in ("write", "decode") for a in acts):
+            return None
+        if any(a.kind == "write" and len(a.pairs) for a in acts):
+            return None
+        if sum(a.kind == "decode" for a in acts) != 1:
+            return None
+        layout = tuple((a.kind, a.nrows, None if a.tables is None else a.tables.shape)
+                       for a in acts)
+        return (layout, prep["bytes"], prep["slot"], prep["host"].data_ptr(),
+                tuple(k_new.shape), tuple(q.shape), k_new.dtype)
+
+    def _capture(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
+                 q: torch.Tensor) -> dict:
+        dec = [a for a in prep["acts"] if a.kind == "decode"][0]
+        g = {"k": torch.empty_like(k_new, device="cpu").pin_memory(),
+             "v": torch.empty_like(v_new, device="cpu").pin_memory(),
+             "q": torch.empty_like(q, device="cpu").pin_memory(),
+             "out": torch.empty((dec.tables.shape[0], self.num_heads, self.head_dim),
+                                dtype=torch.float32).pin_memory()}
+        g["dk"], g["dv"], g["dq"] = (torch.empty_like(t, device=self.device)
+                                     for t in (k_new, v_new, q))
+        for t, src in ((g["k"], k_new), (g["v"], v_new), (g["q"], q)):
+            t.copy_(src)
+        total, host, devb = prep["bytes"], prep["host"], prep["dev"]
+        for a in prep["acts"]:
+            if a.kind == "decode":
+                a.max_len = self.width * self.block_size
+
+        def body():
+            if total:
+                devb[:total].copy_(host[:total], non_blocking=True)
+            for (a, name, arr), off in zip(prep["arrays"], prep["offs"]):
+                dt = torch.int64 if arr.dtype == np.int64 else torch.int32
+                a.dev[name] = devb[off:off + arr.nbytes].view(dt).view(arr.shape)
+            for d, h in (("dk", "k"), ("dv", "v"), ("dq", "q")):
+                g[d].copy_(g[h], non_blocking=True)
+            g["o"] = self.execute(prep["acts"], g["dk"], g["dv"], g["dq"])
+            g["out"].copy_(g["o"], non_blocking=True)
+
+        # one eager run first (workspace, per-device set-up); it applies this
+        # step, and the replay below applies it again to the same bytes
+        side = torch.cuda.Stream(self.device)
+        side.wait_stream(torch.cuda.current_stream(self.device))
+        with torch.cuda.stream(side):
+            body()
+        side.synchronize()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side, capture_error_mode="thread_local"):
+            body()
+        g["graph"] = graph
+        return g
+
+    def stage_graph(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
+                    q: torch.Tensor) -> Optional[dict]:
+        """Host half of a graph step: copy the new K/V rows and queries into
+        the page-locked buffers of the graph for this step's layout (capturing
+        it the first time, which runs the step once eagerly).  Safe while the
+        GPU still works on the previous step, whose graph is the other
+        staging slot's.  None when the step's layout has no graph form."""
+        key = self._graph_key(prep, k_new, q)
+        if key is None:
+            return None
+        if not hasattr(self, "_graphs"):
+            self._graphs = {}
+        g = self._graphs.get(key)
+        if g is None:
+            g = self._graphs[key] = self._capture(prep, k_new, v_new, q)
+        else:
+            for t, src in ((g["k"], k_new), (g["v"], v_new), (g["q"], q)):
+                t.copy_(src)
+        return g
+
+    def replay_graph(self, g: dict, prep: dict) -> dict:
+        """Device half of a graph step: replay it on the current stream.  The
+        output lands in a page-locked tensor owned by the graph, readable after
+        wait() until the next replay of the same layout."""
+        g["graph"].replay()
+        if prep["bytes"]:
+            ev = torch.cuda.Event()
+            ev.record()
+            self._stage_ev[prep["slot"]] = ev
+        h2d = prep["bytes"] + sum(g[t].nbytes for t in ("k", "v", "q"))
+        return {"h2d": h2d, "d2h": g["out"].nbytes, "acts": prep["acts"], "out": g["out"]}
+
+    def launch_graph(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
+                     q: torch.Tensor) -> Optional[dict]:
+        """stage_graph + replay_graph; None (nothing launched) when the step's
+        layout has no graph form."""
+        g = self.stage_graph(prep, k_new, v_new, q)
+        return None if g is None else self.replay_graph(g, prep)
+
     def run_pinned(self, ops, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,
                    out_host: torch.Tensor) -> dict:
         """prepare + launch + wait for one step fed from pinned host memory."""

@@ -322,3 +322,37 @@ def test_prefill_any_finite_scale(pv, dtype, scale):
                              ref["seq_lens"], a.cu, scale)
     err = float(np.abs(out.double().cpu().numpy() - exp).max())
     assert err <= TOL[dtype], err
+
+
+# ---------------------------------------------------------------- graph replay
+def test_graph_replayed_steps_match_the_oracle():
+    """Decode steps fed from page-locked host memory and replayed from CUDA
+    graphs (PagedKVRunner.launch_graph: one capture per staging slot, then
+    replays with new allocator output, K/V rows and queries) give the oracle's
+    output at every step; the lengths cross block and 512-token split edges."""
+    from oracle.run import OracleRun
+    from paged_kv_cache_347_b200.runner import PagedKVRunner
+    wl = workloads.custom("graph", [700, 33, 1, 510], 16, 4, 128, "bf16", 16, 256, seed=5,
+                          steps=7)
+    steps = list(wl.steps)
+    orc, gpu = OracleRun(wl.shape), PagedKVRunner.for_shape(wl.shape, 48)
+    orc.step(steps[0])
+    gpu.run(steps[0])
+    replays = 0
+    for st in steps[1:]:
+        ref = orc.step(st)
+        prep = gpu.prepare(st.ops)
+        res = gpu.launch_graph(prep, st.k_new.pin_memory(), st.v_new.pin_memory(),
+                               st.q.pin_memory())
+        assert res is not None, "a plain append + decode step has a graph form"
+        gpu.wait()
+        err = float(np.abs(res["out"].double().numpy() - ref["out"]).max())
+        assert err <= TOL["bf16"], err
+        replays += 1
+    assert replays == 7
+    # a copy-on-write step has no graph form: nothing is launched
+    gpu.alloc.seq_fork(0, 99)
+    prep = gpu.prepare([("append", 0, 1), ("decode", [0, 99])])
+    assert gpu.launch_graph(prep, torch.zeros(1, 4, 128, dtype=torch.bfloat16).pin_memory(),
+                            torch.zeros(1, 4, 128, dtype=torch.bfloat16).pin_memory(),
+                            torch.zeros(2, 16, 128, dtype=torch.bfloat16).pin_memory()) is None
