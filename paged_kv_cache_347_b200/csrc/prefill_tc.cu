@@ -37,6 +37,7 @@ namespace pf {
 constexpr int kWarps = 4;
 constexpr int kThreads = (kWarps + 1) * 32;
 constexpr int kRows = 16 * kWarps;  // (token, head) rows per CTA
+static_assert(kRows == 64, "the ABI sizes this kernel's grid with 64 / G tokens per CTA");
 constexpr int kStageKeys = 64;
 constexpr int kRowBytes = 128;
 

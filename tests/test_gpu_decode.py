@@ -356,3 +356,18 @@ def test_graph_replayed_steps_match_the_oracle():
     assert gpu.launch_graph(prep, torch.zeros(1, 4, 128, dtype=torch.bfloat16).pin_memory(),
                             torch.zeros(1, 4, 128, dtype=torch.bfloat16).pin_memory(),
                             torch.zeros(2, 16, 128, dtype=torch.bfloat16).pin_memory()) is None
+
+
+@pytest.mark.parametrize("pv", [1, 2])
+@pytest.mark.parametrize("dtype,Hq,Hkv,D,bs,ctx,chunk_lo,chunk_hi", [
+    ("bf16", 16, 4, 128, 16, 300, 0, 3),     # empty chunks next to 1-3-token ones (seed 11)
+    ("bf16", 10, 2, 128, 16, 500, 1, 300),   # G = 5: 25 tokens x 5 heads + 3 idle rows per tile
+    ("f16", 8, 2, 64, 64, 3000, 200, 700),   # 64-token blocks, D 64, 3000-token context
+])
+def test_prefill_edge_shapes(pv, dtype, Hq, Hkv, D, bs, ctx, chunk_lo, chunk_hi):
+    wl = workloads.chunked_prefill(seed=11, batch=6, ctx_lo=ctx // 2, ctx_hi=ctx,
+                                   chunk_lo=chunk_lo, chunk_hi=chunk_hi, num_heads=Hq,
+                                   num_kv_heads=Hkv, head_dim=D, dtype=dtype, block_size=bs,
+                                   num_blocks=6 * (ctx + 2 * chunk_hi) // bs + 64, chunks=2)
+    errs, _, _ = run_parity(wl, table_width=(ctx + 2 * chunk_hi) // bs + 2, prefill_variant=pv)
+    assert len(errs) == 2 and max(errs) <= TOL[dtype], errs
