@@ -7,7 +7,7 @@
 // positions 0..L-n+r through the block table.
 //
 // CTA = 128 (token, query head) rows: 128/G chunk tokens of one KV head g of
-// one sequence, walking the context in stages of 128 keys.  Eleven warps:
+// one sequence, walking the context in stages of 128 keys.  Twelve warps:
 //   * warps 0-7, softmax: warp w serves TMEM lanes 32 (w % 4) .. +31 (the
 //     rows) and keys 64 (w / 4) .. +63 of each stage, so each row has two
 //     threads, which agree its maximum through shared memory.  A thread reads
@@ -17,14 +17,13 @@
 //     weight sums are added and each thread divides and stores its half row;
 //   * warps 8 and 9: TMA producers of the K and the V stages, gathered block
 //     by block through the table into two rings;
-//   * warp 10, one thread, issues the UMMAs:
+//   * warps 10 and 11, one thread each, issue the UMMAs:
 //       S(i)  [128 x 128] = Q . K_i^T      (Q from TMEM, K from shared memory)
 //       PV(i) O [128 x D] += P_i . V_i      (P from TMEM, V N-major, twice:
 //                                            high part and remainder)
-//     in the order S(0), S(1), PV(0), S(2), PV(1), S(3), ...: S is double-
-//     buffered, so the softmax of stage i+1 can start as soon as it ends
-//     stage i.  S(i+2) overwrites the columns PV(i) reads; the two are issued
-//     by the same thread and tcgen05 MMAs of one thread execute in order.
+//     S is double-buffered, so the softmax of stage i+1 can start as soon as
+//     it ends stage i; S(i+2), which overwrites the columns PV(i) reads, is
+//     issued once PV(i) has completed.
 // TMEM (512 columns): S/P buffers [0,128) and [128,256), O [256,256+D),
 // Q [384,384+D/2).  In P, key block j (keys 16j..16j+15) holds its high parts
 // in columns 16j..16j+7 and its remainders in 16j+8..16j+15, two keys per
@@ -47,7 +46,7 @@ namespace pu {
 constexpr int kM = 128;               // rows per CTA
 constexpr int kKeys = 128;            // keys per stage
 constexpr int kSoftmaxThreads = 256;  // 8 warps, two threads per row
-constexpr int kThreads = kSoftmaxThreads + 96;
+constexpr int kThreads = kSoftmaxThreads + 128;  // + K, V producers, S, PV issuers
 constexpr int kTmemCols = 512;
 constexpr int kColO = 256, kColQ = 384;
 constexpr int kRowBytes = 128;        // one 64-element piece of a 16-bit row
@@ -61,9 +60,9 @@ struct Cfg {
     static constexpr int kVOffset = kKOffset + NK * kStageBytes;    // V ring [NV]
     static constexpr int kXchOffset = kVOffset + NV * kStageBytes;  // float [2][2][128]
     static constexpr int kBarOffset = kXchOffset + 2 * 2 * kM * 4;
-    // k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] s_full[2] p_full[2] pv_done q_full
-    // mma_done xchg[4]
-    static constexpr int kNumBars = 2 * NK + 2 * NV + 4 + 3 + 4;
+    // k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] s_full[2] p_full[2] pv_done[2]
+    // q_full mma_done xchg[4]
+    static constexpr int kNumBars = 2 * NK + 2 * NV + 6 + 2 + 4;
     static constexpr int kTmemSlot = kBarOffset + kNumBars * 8;
     static constexpr int kAbortOffset = kTmemSlot + 16;
     static constexpr int kSmemBytes = kAbortOffset + 16;
@@ -162,7 +161,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     const uint32_t bar0 = sbase + C::kBarOffset;
     const uint32_t k_full = bar0, k_empty = k_full + 8 * NK, v_full = k_empty + 8 * NK,
                    v_empty = v_full + 8 * NV, s_full = v_empty + 8 * NV, p_full = s_full + 16,
-                   pv_done = p_full + 16, q_full = pv_done + 8, mma_done = q_full + 8,
+                   pv_done = p_full + 16, q_full = pv_done + 16, mma_done = q_full + 8,
                    xchg = mma_done + 8;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kAbortOffset);
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + C::kTmemSlot);
@@ -176,15 +175,15 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
             mbar_init(v_full + 8 * i, 1);
             mbar_init(v_empty + 8 * i, 1);
         }
-        // one s_full and one p_full per S buffer: the softmax may finish stage
-        // i+1 before the MMA thread has seen stage i, never stage i+2
+        // s_full, p_full and pv_done once per S buffer: stage i+1 can run ahead
+        // of a waiter on stage i, stage i+2 never can
         for (int b = 0; b < 2; ++b) {
             mbar_init(s_full + 8 * b, 1);
             mbar_init(p_full + 8 * b, kSoftmaxThreads);
+            mbar_init(pv_done + 8 * b, 1);
         }
-        mbar_init(pv_done, 1);
         mbar_init(q_full, kSoftmaxThreads);
-        mbar_init(mma_done, 1);
+        mbar_init(mma_done, 2);  // both issuing threads
         for (int q = 0; q < 4; ++q) mbar_init(xchg + 8 * q, 64);
         *abort_flag = 0;
         fence_mbarrier_init();
@@ -248,76 +247,75 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         return;
     }
 
-    // ------------------------------------------------------------ MMA issuer
-    if (warp == 10) {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp 10 issues the S MMAs, warp 11 the PV MMAs, each from one thread, so
+    // that neither waits behind the other's barrier checks.  MMAs of two
+    // threads are not ordered against each other: S(i+2) overwrites the TMEM
+    // columns PV(i) reads, so the S thread waits for PV(i) to complete.
+    if (warp == 10 || warp == 11) {
         if (lane == 0) {
             constexpr uint32_t fmt = StoreT<T>::kCode == PA_BF16 ? 1u : 0u;
-            constexpr uint32_t idesc_s = umma::idesc_f16(fmt, kM, kKeys, 0);
-            constexpr uint32_t idesc_o = umma::idesc_f16(fmt, kM, D, 1);
-            // S(i) = Q . K_i^T into S buffer i % 2
-            auto issue_s = [&](int i) -> bool {
-                const int slot = i % NK;
-                if (!mbar_wait_bounded(k_full + 8 * slot, (i / NK) & 1, abort_flag)) return false;
-                umma::fence_after_sync();
-                // K rows: 8-row groups 1 KB apart; descriptors advance by (bytes >> 4)
-                const uint64_t b0 = umma::smem_desc_sw128(k_s + slot * C::kStageBytes, 16, 1024);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t ka = ((kk >> 2) * C::kKVPiece + (kk & 3) * 32) >> 4;
-                    umma::mma_f16_ts(tmem + (i & 1) * kKeys, tmem + kColQ + 8 * kk, b0 + ka,
-                                     idesc_s, kk > 0);
-                }
-                return true;
-            };
-            auto commit_s = [&](int i) {
-                umma::commit(s_full + 8 * (i & 1));
-                umma::commit(k_empty + 8 * (i % NK));
-            };
-            // O += P_i . V_i once the softmax has written P_i
-            auto issue_pv = [&](int i) -> bool {
-                const int slot = i % NV;
-                if (!mbar_wait_bounded(p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag) ||
-                    !mbar_wait_bounded(v_full + 8 * slot, (i / NV) & 1, abort_flag))
-                    return false;
-                umma::fence_after_sync();
-                // V rows: 8-row groups 1 KB apart, 64-column pieces 16 KB apart
-                const uint64_t b0 = umma::smem_desc_sw128(v_s + slot * C::kStageBytes,
-                                                          C::kKVPiece, 1024);
-                const uint32_t pb = tmem + (i & 1) * kKeys;
-#pragma unroll
-                for (int j = 0; j < kKeys / 16; ++j) {  // keys 16j..16j+15
-                    const uint64_t b = b0 + ((j * 16 * kRowBytes) >> 4);
-                    umma::mma_f16_ts(tmem + kColO, pb + 16 * j, b, idesc_o, (i > 0 || j > 0) ? 1u : 0u);
-                    umma::mma_f16_ts(tmem + kColO, pb + 16 * j + 8, b, idesc_o, 1u);
-                }
-                return true;
-            };
-            auto commit_pv = [&](int i) {
-                umma::commit(pv_done);
-                umma::commit(v_empty + 8 * (i % NV));
-            };
             bool ok = mbar_wait_bounded(q_full, 0, abort_flag);
             umma::fence_after_sync();
-            if (ok) ok = issue_s(0);
-            if (ok) commit_s(0);
-            if (ok && nstages > 1) ok = issue_s(1);
-            if (ok && nstages > 1) commit_s(1);
-            // The commits of PV(i) and S(i+2) follow both groups of MMAs, so they
-            // are issued while the tensor core still has queued work (a commit
-            // arrives once every MMA issued before it has completed).
+            if (warp == 10) {
+                constexpr uint32_t idesc_s = umma::idesc_f16(fmt, kM, kKeys, 0);
 #pragma unroll 1
-            for (int i = 0; ok && i < nstages; ++i) {
-                ok = issue_pv(i);
-                const bool s_next = ok && i + 2 < nstages;
-                if (s_next) ok = issue_s(i + 2);
-                if (s_next && ok) commit_s(i + 2);
-                commit_pv(i);
+                for (int i = 0; ok && i < nstages; ++i) {
+                    // S(i) = Q . K_i^T into S buffer i % 2, once PV(i-2) has read it
+                    const int slot = i % NK;
+                    if (i >= 2 && !mbar_wait_bounded(pv_done + 8 * (i & 1), ((i >> 1) - 1) & 1,
+                                                     abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (!mbar_wait_bounded(k_full + 8 * slot, (i / NK) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    umma::fence_after_sync();
+                    // K rows: 8-row groups 1 KB apart; descriptors advance by (bytes >> 4)
+                    const uint64_t b0 = umma::smem_desc_sw128(k_s + slot * C::kStageBytes, 16, 1024);
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t ka = ((kk >> 2) * C::kKVPiece + (kk & 3) * 32) >> 4;
+                        umma::mma_f16_ts(tmem + (i & 1) * kKeys, tmem + kColQ + 8 * kk, b0 + ka,
+                                         idesc_s, kk > 0);
+                    }
+                    umma::commit(s_full + 8 * (i & 1));
+                    umma::commit(k_empty + 8 * slot);
+                }
+            } else {
+                constexpr uint32_t idesc_o = umma::idesc_f16(fmt, kM, D, 1);
+#pragma unroll 1
+                for (int i = 0; ok && i < nstages; ++i) {
+                    // O += P_i . V_i once the softmax has written P_i
+                    const int slot = i % NV;
+                    if (!mbar_wait_bounded(p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag) ||
+                        !mbar_wait_bounded(v_full + 8 * slot, (i / NV) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    umma::fence_after_sync();
+                    // V rows: 8-row groups 1 KB apart, 64-column pieces 16 KB apart
+                    const uint64_t b0 = umma::smem_desc_sw128(v_s + slot * C::kStageBytes,
+                                                              C::kKVPiece, 1024);
+                    const uint32_t pb = tmem + (i & 1) * kKeys;
+#pragma unroll
+                    for (int j = 0; j < kKeys / 16; ++j) {  // keys 16j..16j+15
+                        const uint64_t b = b0 + ((j * 16 * kRowBytes) >> 4);
+                        umma::mma_f16_ts(tmem + kColO, pb + 16 * j, b, idesc_o,
+                                         (i > 0 || j > 0) ? 1u : 0u);
+                        umma::mma_f16_ts(tmem + kColO, pb + 16 * j + 8, b, idesc_o, 1u);
+                    }
+                    umma::commit(pv_done + 8 * (i & 1));
+                    umma::commit(v_empty + 8 * slot);
+                }
             }
             if (!ok) {
                 raise_device_error(p.err, PA_DEVERR_TIMEOUT);
                 *abort_flag = 1;
             }
-            umma::commit(mma_done);  // arrives when every MMA issued above is done
+            umma::commit(mma_done);  // arrives when every MMA this thread issued is done
         }
         return;
     }
@@ -446,7 +444,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         }
         if (__any_sync(0xffffffffu, rescale)) {  // warp-collective TMEM access
             // O must hold PV up to stage i-1 before it is rescaled
-            if (i > 0 && !warp_wait(pv_done, (i - 1) & 1, abort_flag)) return false;
+            if (i > 0 && !warp_wait(pv_done + 8 * ((i - 1) & 1), ((i - 1) >> 1) & 1, abort_flag))
+                return false;
             umma::fence_after_sync();
 #pragma unroll
             for (int cb = 0; cb < D / 64; ++cb) {
@@ -487,7 +486,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     for (; ok && i < n_fast; ++i) ok = stage(i, std::false_type{});
     for (; ok && i < nstages; ++i) ok = stage(i, std::true_type{});
     float other = 0.f;
-    if (ok) ok = warp_wait(pv_done, (nstages - 1) & 1, abort_flag) && exchange(l, other);
+    if (ok)
+        ok = warp_wait(pv_done + 8 * ((nstages - 1) & 1), ((nstages - 1) >> 1) & 1, abort_flag) &&
+             exchange(l, other);
     if (ok) {
         umma::fence_after_sync();
         const float lt = l + other;
