@@ -325,11 +325,13 @@ class BlockAllocator:
         self.num_blocks = num_blocks
         self.block_size = block_size
 
-    def __del__(self, _destroy=_lib.pa_alloc_destroy):
+    def __del__(self, _destroy=_lib.pa_alloc_destroy, _null=ctypes.c_void_p):
+        # bound at definition time: at interpreter shutdown the module globals
+        # (ctypes among them) may already be None
         h = getattr(self, "_h", None)
         if h is not None and h.value:
             _destroy(h)
-            self._h = ctypes.c_void_p()
+            self._h = _null()
 
     def seq_add(self, seq_id: int) -> None:
         _check(_lib.pa_seq_add(self._h, seq_id), "pa_seq_add")
