@@ -136,7 +136,8 @@ def decode_storage(t: torch.Tensor) -> np.ndarray:
         return t.view(torch.int16).numpy().view(np.float16).astype(np.float64)
     if t.dtype == torch.bfloat16:
         bits = t.view(torch.int16).numpy().view(np.uint16).astype(np.uint32) << 16
-        return bits.view(np.float32).astype(np.float64)
+        with np.errstate(invalid="ignore"):  # NaN patterns stay NaN
+            return bits.view(np.float32).astype(np.float64)
     raise TypeError(t.dtype)
 
 
