@@ -255,6 +255,21 @@ int pa_swap_blocks(void *dst_k, void *dst_v, const void *src_k, const void *src_
  */
 int pa_set_profile_events(void *ev_begin, void *ev_end);
 
+/*
+ * Self-test of the bounded pipeline wait that every TMA / tensor-core kernel
+ * of this library uses (no counterpart on the pages: failure detection).
+ * One CTA waits on an mbarrier phase that nothing completes.  The wait must
+ * give up after limit_ns, or as soon as a second warp of the CTA sets the
+ * abort flag (after abort_after_ns; 0 = never), then set PA_DEVERR_TIMEOUT in
+ * the device error word and return; the CUDA context stays usable.
+ *   limit_ns        (0, 10^10]
+ *   elapsed_ns      device, one uint64: nanoseconds the wait took
+ * Returns PA_ERR_INVALID_ARG for a limit out of range or a NULL elapsed_ns,
+ * PA_ERR_CUDA if the launch fails.  Asynchronous on `stream`.
+ */
+int pa_selftest_wait(uint64_t limit_ns, uint64_t abort_after_ns, unsigned long long *elapsed_ns,
+                     void *stream);
+
 /* ------------------------------------------------------------------------
  * Host block allocator [P1 "Mechanism and details"; P2 "Separate logical
  * order from physical location", "Sharing needs ownership rules", "Exercise

@@ -433,4 +433,18 @@ int pa_set_profile_events(void *ev_begin, void *ev_end) {
     return PA_OK;
 }
 
+int pa_selftest_wait(uint64_t limit_ns, uint64_t abort_after_ns, unsigned long long *elapsed_ns,
+                     void *stream) {
+    clear_error();
+    if (limit_ns == 0 || limit_ns > 10000000000ull || abort_after_ns > 10000000000ull)
+        return fail(PA_ERR_INVALID_ARG, "limit_ns must be in (0, 1e10], abort_after_ns <= 1e10");
+    if (!elapsed_ns) return fail(PA_ERR_INVALID_ARG, "NULL elapsed_ns");
+    unsigned int *err = device_error_ptr();
+    if (!err) return fail(PA_ERR_CUDA, "no CUDA device");
+    cudaError_t e = launch_wait_selftest(err, limit_ns, abort_after_ns, elapsed_ns,
+                                         static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "wait self-test launch");
+    return PA_OK;
+}
+
 }  // extern "C"

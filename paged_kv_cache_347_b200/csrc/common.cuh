@@ -111,17 +111,19 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Gives up after
-// about two seconds, or as soon as *abort is set by another warp, and returns
-// false; the caller then records PA_DEVERR_TIMEOUT and winds down.
+// limit_ns (about two seconds by default), or as soon as *abort is set by
+// another warp, and returns false; the caller then records
+// PA_DEVERR_TIMEOUT and winds down.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
-                                                  volatile int *abort) {
+                                                  volatile int *abort,
+                                                  uint64_t limit_ns = 2000000000ull) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t i = 1;; ++i) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((i & 255u) == 0) {
             if (abort && *abort) return false;
-            if (global_timer_ns() - t0 > 2000000000ull) return false;
+            if (global_timer_ns() - t0 > limit_ns) return false;
         }
     }
 }

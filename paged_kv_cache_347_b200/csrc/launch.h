@@ -71,6 +71,10 @@ cudaError_t launch_prefill_tc(const PrefillParams &p, int dtype, cudaStream_t st
 // tcgen05 kernel: 128 rows per CTA, S and O accumulated in TMEM.
 cudaError_t launch_prefill_umma(const PrefillParams &p, int dtype, cudaStream_t stream);
 
+// One CTA waiting, bounded, on an mbarrier phase nothing completes (selftest.cu).
+cudaError_t launch_wait_selftest(unsigned int *err, uint64_t limit_ns, uint64_t abort_after_ns,
+                                 unsigned long long *elapsed_ns, cudaStream_t stream);
+
 // Merge of split partials into out; a no-op when max_splits == 1.
 cudaError_t launch_decode_reduce(const DecodeParams &p, cudaStream_t stream);
 

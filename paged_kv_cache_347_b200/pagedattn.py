@@ -84,6 +84,7 @@ _sig("pa_seq_swap_in", _i, _vp, _i64, _vp, _i, _vp)
 _sig("pa_swap_blocks", _i, _vp, _vp, _vp, _vp, _vp, _i, _sz, _i, _i, _vp)
 _sig("pa_prefill", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _i,
      _f, _i, _vp)
+_sig("pa_selftest_wait", _i, _c.c_uint64, _c.c_uint64, _vp, _vp)
 _sig("pa_prefill_ex", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i,
      _i, _f, _i, _i, _vp)
 
@@ -238,6 +239,16 @@ def pa_prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cach
         Hkv, D, bs, W, NB, int(max_q_len), int(max_seq_len), float(scale),
         DTYPE_CODE[k_cache.dtype], int(variant), _stream(q)), "pa_prefill")
     return out
+
+
+def selftest_wait(limit_s: float, abort_after_s: float = 0.0) -> float:
+    """Run the bounded-wait self-test on the current device and stream;
+    returns the seconds the wait took (it sets the "timeout" device error)."""
+    el = torch.zeros(1, dtype=torch.int64, device="cuda")
+    _check(_lib.pa_selftest_wait(int(limit_s * 1e9), int(abort_after_s * 1e9), el.data_ptr(),
+                                 torch.cuda.current_stream().cuda_stream), "pa_selftest_wait")
+    torch.cuda.synchronize()
+    return int(el.item()) / 1e9
 
 
 def pa_decode_static(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor,

@@ -87,3 +87,11 @@ def test_python_binding_rejects_cpu_tensors():
         pa.pa_reshape_and_cache(torch.zeros(1, 1, 128, dtype=torch.bfloat16),
                                 torch.zeros(1, 1, 128, dtype=torch.bfloat16), kc, kc.clone(),
                                 torch.zeros(1, dtype=torch.int64))
+
+
+def test_selftest_wait_rejects_bad_arguments_before_any_cuda_call():
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    invalid = -1  # PA_ERR_INVALID_ARG
+    assert pa._lib.pa_selftest_wait(0, 0, None, None) == invalid
+    assert pa._lib.pa_selftest_wait(10**11, 0, None, None) == invalid
+    assert pa._lib.pa_selftest_wait(10**6, 0, None, None) == invalid  # NULL elapsed
