@@ -23,6 +23,7 @@ memory before timing it.
 """
 from __future__ import annotations
 
+import warnings
 from dataclasses import dataclass, field
 from typing import List, Optional, Sequence
 
@@ -372,9 +373,18 @@ class PagedKVRunner:
             return None
         if not hasattr(self, "_graphs"):
             self._graphs = {}
+        if key in self._graphs and self._graphs[key] is None:
+            return None  # this layout failed to capture before: launch eagerly
         g = self._graphs.get(key)
         if g is None:
-            g = self._graphs[key] = self._capture(prep, k_new, v_new, q)
+            try:
+                g = self._capture(prep, k_new, v_new, q)
+            except RuntimeError as e:  # capture refused: this layout runs eagerly
+                warnings.warn(f"CUDA graph capture failed, launching eagerly: {e}")
+                self._graphs[key] = None
+                torch.cuda.synchronize(self.device)
+                return None
+            self._graphs[key] = g
         else:
             for t, src in ((g["k"], k_new), (g["v"], v_new), (g["q"], q)):
                 t.copy_(src)
