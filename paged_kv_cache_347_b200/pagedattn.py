@@ -169,6 +169,14 @@ def decode_workspace_size(num_seqs: int, num_heads: int, head_dim: int, max_seq_
                                          partition_size)
 
 
+def cached_workspace(device: torch.device) -> Optional[torch.Tensor]:
+    """The split-partial workspace pa_decode currently uses on ``device``
+    (None before the first call).  A CUDA graph that captured a decode keeps
+    a reference to it, so that a later, larger request, which replaces the
+    cached buffer, cannot free the memory the graph writes to."""
+    return _ws_cache.get((device.index or 0, 0))
+
+
 def _workspace(device: torch.device, nbytes: int) -> torch.Tensor:
     key = (device.index or 0, 0)
     ws = _ws_cache.get(key)

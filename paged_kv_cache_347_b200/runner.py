@@ -355,6 +355,9 @@ class PagedKVRunner:
         with torch.cuda.stream(side):
             body()
         side.synchronize()
+        # the graph writes split partials into the binding's cached workspace:
+        # keep that buffer alive for as long as the graph
+        g["ws"] = pa.cached_workspace(self.device)
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph, stream=side, capture_error_mode="thread_local"):
             body()
