@@ -50,6 +50,12 @@ def lib() -> ctypes.CDLL:
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
             ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
             ctypes.c_double, ctypes.c_int]
+        L.attn_ref_prefill_sel.restype = ctypes.c_int
+        L.attn_ref_prefill_sel.argtypes = [
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_double, ctypes.c_void_p, ctypes.c_int, ctypes.c_int]
         _lib = L
     return _lib
 
@@ -102,12 +108,14 @@ def paged_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
 
 def paged_prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
                   block_tables: np.ndarray, seq_lens: np.ndarray, cu_q: np.ndarray,
-                  scale: float, n_threads: int = 0) -> np.ndarray:
+                  scale: float, n_threads: int = 0,
+                  sel: Optional[Sequence[Tuple[int, int]]] = None) -> np.ndarray:
     """fp64 causal attention of chunk rows over the paged cache.
 
     q [total, Hq, D] holds, for sequence s, rows cu_q[s]..cu_q[s+1]-1 at
     positions L_s - n_s .. L_s - 1 (n_s = cu_q[s+1] - cu_q[s]); each attends to
-    tokens 0..its position.  Returns float64 [total, Hq, D]."""
+    tokens 0..its position.  Returns float64 [total, Hq, D], or [len(sel), D]
+    for a list of (row, head) pairs."""
     q = q.contiguous(); k_cache = k_cache.contiguous(); v_cache = v_cache.contiguous()
     total, Hq, D = q.shape
     NB, Hkv, bs, _ = k_cache.shape
@@ -116,6 +124,17 @@ def paged_prefill(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
     cu = np.ascontiguousarray(cu_q, dtype=np.int32)
     B = sl.shape[0]
     assert cu.shape == (B + 1,) and int(cu[-1]) == total and bt.shape[0] == B
+    if sel is not None:
+        sa = np.ascontiguousarray(np.asarray(sel, dtype=np.int32).reshape(-1, 2))
+        out = np.zeros((sa.shape[0], D), np.float64)
+        rc = lib().attn_ref_prefill_sel(out.ctypes.data, q.data_ptr(), k_cache.data_ptr(),
+                                        v_cache.data_ptr(), _DT[_dtype_name(q)], bt.ctypes.data,
+                                        sl.ctypes.data, cu.ctypes.data, B, Hq, Hkv, D, bs,
+                                        bt.shape[1], NB, float(scale), sa.ctypes.data,
+                                        sa.shape[0], int(n_threads))
+        if rc != 0:
+            raise ValueError("oracle: bad prefill argument or table entry out of range")
+        return out
     out = np.zeros((total, Hq, D), np.float64)
     rc = lib().attn_ref_prefill(out.ctypes.data, q.data_ptr(), k_cache.data_ptr(),
                                 v_cache.data_ptr(), _DT[_dtype_name(q)], bt.ctypes.data,

@@ -236,3 +236,38 @@ int attn_ref_prefill(double *out, const void *q, const void *k_cache, const void
     }
     return bad ? -1 : 0;
 }
+
+/* The same rows as attn_ref_prefill, only the (row, head) pairs listed in
+ * sel[2 * j], sel[2 * j + 1]; out[j][D] for pair j. */
+int attn_ref_prefill_sel(double *out, const void *q, const void *k_cache, const void *v_cache,
+                         int dtype, const int32_t *block_tables, const int32_t *seq_lens,
+                         const int32_t *cu_q, int num_seqs, int num_heads, int num_kv_heads,
+                         int head_dim, int block_size, int max_blocks, int num_blocks,
+                         double scale, const int32_t *sel, int n_sel, int n_threads) {
+    dec_fn dec = pick(dtype);
+    long long total;
+    int j, bad = 0;
+    if (!dec || num_seqs < 0 || num_heads <= 0 || num_kv_heads <= 0 ||
+        num_heads % num_kv_heads || head_dim <= 0 || block_size <= 0 || max_blocks < 0 ||
+        num_blocks <= 0 || n_sel < 0)
+        return -1;
+    total = num_seqs > 0 ? cu_q[num_seqs] : 0;
+    if (n_threads <= 0) n_threads = attn_ref_max_threads();
+#pragma omp parallel for schedule(dynamic, 1) num_threads(n_threads) reduction(| : bad)
+    for (j = 0; j < n_sel; j++) {
+        const long long r = sel[2 * j];
+        const int h = sel[2 * j + 1];
+        int s = 0, n, L, p;
+        if (r < 0 || r >= total || h < 0 || h >= num_heads) { bad |= 1; continue; }
+        while (s + 1 < num_seqs && cu_q[s + 1] <= r) s++;
+        n = cu_q[s + 1] - cu_q[s];
+        L = seq_lens[s];
+        p = L - n + (int)(r - cu_q[s]);
+        if (n < 0 || n > L || (L + block_size - 1) / block_size > max_blocks) { bad |= 1; continue; }
+        bad |= prefill_row(out + (size_t)j * head_dim, q, ((size_t)r * num_heads + h) * head_dim,
+                           k_cache, v_cache, dec, block_tables + (size_t)s * max_blocks, p + 1,
+                           h / (num_heads / num_kv_heads), num_kv_heads, head_dim, block_size,
+                           num_blocks, scale) != 0;
+    }
+    return bad ? -1 : 0;
+}

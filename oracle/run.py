@@ -43,7 +43,9 @@ class OracleRun:
              decode: bool = True, n_threads: int = 0) -> Dict:
         """Apply one step.  Returns the slots and copy-on-write pairs of its
         appends (in op order) and, when ``decode``, the fp64 outputs of its
-        decode op ([b, Hq, D], or [len(sel), D] for (batch index, head) pairs)."""
+        decode op ([b, Hq, D], or [len(sel), D] for (batch index, head) pairs)
+        or of its prefill op ([rows, Hq, D], or [len(sel), D] for (row, head)
+        pairs)."""
         res: Dict = {"slots": [], "pairs": [], "out": None}
         row = 0
         for op in st.ops:
@@ -101,7 +103,8 @@ class OracleRun:
                 res["block_tables"], res["seq_lens"] = bt, lens
                 if decode and self.keep_cache:
                     res["out"] = attn.paged_prefill(st.q, self.k_cache, self.v_cache, bt, lens,
-                                                    cu, self.shape.scale, n_threads=n_threads)
+                                                    cu, self.shape.scale, n_threads=n_threads,
+                                                    sel=sel)
             elif kind == "decode":
                 sids = list(op[1])
                 bt, lens = self.tables(sids)

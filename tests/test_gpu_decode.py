@@ -382,3 +382,16 @@ def test_prefill_edge_shapes(pv, dtype, Hq, Hkv, D, bs, ctx, chunk_lo, chunk_hi)
                                    num_blocks=6 * (ctx + 2 * chunk_hi) // bs + 64, chunks=2)
     errs, _, _ = run_parity(wl, table_width=(ctx + 2 * chunk_hi) // bs + 2, prefill_variant=pv)
     assert len(errs) == 2 and max(errs) <= TOL[dtype], errs
+
+
+@pytest.mark.parametrize("pv", [1, 2])
+def test_prefill_full_study_size_sampled(pv):
+    """The prefill study's first workload at full size (8 sequences, 4096
+    tokens of context + a 1024-token chunk, 32/8 heads, D 128, bf16, bs 16),
+    in the launch configuration the study times; 64 sampled (row, head) pairs,
+    the first and the last row among them, against the fp64 oracle."""
+    wl = workloads.chunked_prefill(batch=8, ctx_lo=4096, ctx_hi=4096, chunk_lo=1024,
+                                   chunk_hi=1024, num_blocks=8 * (4096 + 1024) // 16 + 64)
+    errs, _, _ = run_parity(wl, table_width=(4096 + 1024) // 16 + 2, sample=64,
+                            prefill_variant=pv)
+    assert len(errs) == 1 and max(errs) <= TOL["bf16"], errs

@@ -102,3 +102,28 @@ def test_bad_chunk_is_an_error():
     q, kc, vc, bt, sl, cu, _ = _case(1, "f32", [5], [5], 2, 1, 16, 4)
     with pytest.raises(ValueError):
         attn.paged_prefill(q[:5], kc, vc, bt, np.array([4], np.int32), cu, 1.0)
+
+
+def test_selected_rows_equal_the_full_computation():
+    """attn_ref_prefill_sel computes exactly the listed (row, head) pairs of
+    attn_ref_prefill (same per-row loop); an out-of-range pair is an error."""
+    import workloads
+    from oracle.run import OracleRun
+    wl = workloads.chunked_prefill(batch=3, ctx_lo=20, ctx_hi=90, chunk_lo=1, chunk_hi=40,
+                                   num_heads=8, num_kv_heads=2, head_dim=64, dtype="bf16",
+                                   block_size=8, num_blocks=128)
+    o = OracleRun(wl.shape)
+    steps = list(wl.steps)
+    o.step(steps[0])
+    st = steps[1]
+    ref = o.step(st)
+    ns = [n for op in st.ops if op[0] == "prefill" for _, n in op[1]]
+    cu = np.concatenate([[0], np.cumsum(ns)]).astype(np.int32)
+    sel = [(0, 0), (5, 3), (int(cu[-1]) - 1, 7), (int(cu[1]), 2)]
+    part = attn.paged_prefill(st.q, o.k_cache, o.v_cache, ref["block_tables"], ref["seq_lens"],
+                              cu, wl.shape.scale, sel=sel)
+    for j, (r, h) in enumerate(sel):
+        assert np.array_equal(part[j], ref["out"][r, h])
+    with pytest.raises(ValueError):
+        attn.paged_prefill(st.q, o.k_cache, o.v_cache, ref["block_tables"], ref["seq_lens"],
+                           cu, wl.shape.scale, sel=[(int(cu[-1]), 0)])
