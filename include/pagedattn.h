@@ -176,13 +176,16 @@ int pa_prefill(float *out, const void *q, const void *k_cache, const void *v_cac
                float scale, int dtype, void *stream);
 
 /*
- * pa_prefill with a choice of kernel: variant 0 = automatic (the tcgen05
- * kernel; pa_prefill uses it), 1 = the
- * mma.sync kernel (64 (token, head) rows per CTA, accumulators in
- * registers), 2 = the tcgen05 kernel (128 rows per CTA, S = Q K^T and
- * O = P V accumulated in tensor memory).  Same arguments, results (within
- * fp32 rounding) and errors as pa_prefill; another variant returns
- * PA_ERR_INVALID_ARG.
+ * pa_prefill with a choice of kernel:
+ *   0  automatic: the tcgen05 kernel (pa_prefill uses it);
+ *   1  the mma.sync kernel: 64 (token, head) rows per CTA, accumulators in
+ *      registers;
+ *   2  the tcgen05 kernel: 128 rows per CTA; Q, S = Q K^T, P and O = P V held
+ *      in tensor memory, the MMAs issued by two threads.
+ * Same arguments, results (within fp32 rounding) and errors as pa_prefill;
+ * another variant returns PA_ERR_INVALID_ARG.  Both kernels need all of a
+ * sequence's table entries for positions < L_s to be valid blocks (an entry
+ * outside [0, num_blocks) reads as zeros and sets PA_DEVERR_TABLE).
  */
 int pa_prefill_ex(float *out, const void *q, const void *k_cache, const void *v_cache,
                   const int32_t *block_tables, const int32_t *seq_lens, const int32_t *cu_q_lens,
