@@ -395,3 +395,38 @@ def test_prefill_full_study_size_sampled(pv):
     errs, _, _ = run_parity(wl, table_width=(4096 + 1024) // 16 + 2, sample=64,
                             prefill_variant=pv)
     assert len(errs) == 1 and max(errs) <= TOL["bf16"], errs
+
+
+@pytest.mark.parametrize("pv", [1, 2])
+def test_prefill_bad_table_entry_is_reported(pv):
+    """A table entry outside [0, num_blocks) is read as zeros and sets the
+    "table" device error bit; the other sequences still match the oracle."""
+    from oracle import attn
+    from oracle.run import OracleRun
+    from paged_kv_cache_347_b200.runner import PagedKVRunner
+    pa = _pa()
+    wl = workloads.chunked_prefill(batch=3, ctx_lo=100, ctx_hi=200, chunk_lo=20, chunk_hi=80,
+                                   num_heads=8, num_kv_heads=2, head_dim=128, dtype="bf16",
+                                   block_size=16, num_blocks=128, chunks=1)
+    sh = wl.shape
+    orc, gpu = OracleRun(sh), PagedKVRunner.for_shape(sh, 24)
+    for st in wl.steps:
+        ref = orc.step(st)
+        acts = gpu.plan(st.ops)
+        gpu.upload(acts)
+        gpu.execute(acts, st.k_new.cuda(), st.v_new.cuda(),
+                    None if st.q is None else st.q.cuda())
+    a = [x for x in acts if x.kind == "prefill"][0]
+    tables = a.dev["tables"].clone()
+    tables[0, 1] = sh.num_blocks + 5  # sequence 0's second block
+    out = torch.empty((st.q.shape[0], sh.num_heads, sh.head_dim), dtype=torch.float32,
+                      device="cuda")
+    pa.device_errors(clear=True)
+    pa.pa_prefill(out, st.q.cuda(), gpu.k_cache, gpu.v_cache, tables, a.dev["lens"],
+                  a.dev["cu"], sh.scale, max_q_len=a.max_q, max_seq_len=a.max_len, variant=pv)
+    torch.cuda.synchronize()
+    assert pa.device_errors(clear=True) == ["table"]
+    got = out.double().cpu().numpy()
+    assert np.isfinite(got).all()
+    rows = slice(int(a.cu[1]), int(a.cu[-1]))  # sequences 1 and 2 are untouched
+    assert float(np.abs(got[rows] - ref["out"][rows]).max()) <= TOL["bf16"]
