@@ -71,40 +71,52 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
         for (int e = 0; e < E; ++e) o[h][e] = 0.f;
     }
 
-    for (int base = t0 + warp * TPW; base < t1; base += NW * TPW) {
-        const int t = base + slot;
-        const bool valid = t < t1;
-        float kf[E], vf[E];
+    // U steps of a warp have their loads in flight together (table entry,
+    // then the K and V words), then their math runs step by step
+    constexpr int U = GM >= 8 ? 2 : 4;
+    for (int base = t0 + warp * TPW; base < t1; base += NW * TPW * U) {
+        uint4 ku[U], vu[U];
 #pragma unroll
-        for (int e = 0; e < E; ++e) kf[e] = vf[e] = 0.f;
-        if (valid) {
-            const int pb = checked_block(p, s, t / bs);
-            if (pb >= 0) {
-                const int64_t row = ((int64_t)pb * Hkv + g) * bs + t % bs;
-                const uint4 ku = __ldg(reinterpret_cast<const uint4 *>(kc + row * D + li * E));
-                const uint4 vu = __ldg(reinterpret_cast<const uint4 *>(vc + row * D + li * E));
-                Vec16<T>::unpack(ku, kf);
-                Vec16<T>::unpack(vu, vf);
+        for (int u = 0; u < U; ++u) {
+            const int t = base + u * NW * TPW + slot;
+            ku[u] = vu[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (t < t1) {
+                const int pb = checked_block(p, s, t / bs);
+                if (pb >= 0) {
+                    const int64_t row = ((int64_t)pb * Hkv + g) * bs + t % bs;
+                    ku[u] = __ldg(reinterpret_cast<const uint4 *>(kc + row * D + li * E));
+                    vu[u] = __ldg(reinterpret_cast<const uint4 *>(vc + row * D + li * E));
+                }
             }
         }
 #pragma unroll
-        for (int h = 0; h < GM; ++h) {
-            float acc = 0.f;
+        for (int u = 0; u < U; ++u) {
+            // a step wholly past the split's end does nothing (uniform over the warp)
+            if (base + u * NW * TPW >= t1) break;
+            const int t = base + u * NW * TPW + slot;
+            const bool valid = t < t1;
+            float kf[E], vf[E];
+            Vec16<T>::unpack(ku[u], kf);
+            Vec16<T>::unpack(vu[u], vf);
 #pragma unroll
-            for (int e = 0; e < E; ++e) acc = fmaf(qf[h][e], kf[e], acc);
+            for (int h = 0; h < GM; ++h) {
+                float acc = 0.f;
 #pragma unroll
-            for (int off = TG / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-            const float x = valid ? acc * p.scale_log2 : -INFINITY;
-            float cm = x;
+                for (int e = 0; e < E; ++e) acc = fmaf(qf[h][e], kf[e], acc);
 #pragma unroll
-            for (int off = TG; off < 32; off <<= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
-            const float mn = fmaxf(m[h], cm);  // finite: slot 0 of every step is valid
-            const float al = exp2f(m[h] - mn);
-            const float pr = exp2f(x - mn);
-            l[h] = l[h] * al + pr;
+                for (int off = TG / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+                const float x = valid ? acc * p.scale_log2 : -INFINITY;
+                float cm = x;
 #pragma unroll
-            for (int e = 0; e < E; ++e) o[h][e] = fmaf(pr, vf[e], o[h][e] * al);
-            m[h] = mn;
+                for (int off = TG; off < 32; off <<= 1) cm = fmaxf(cm, __shfl_xor_sync(0xffffffffu, cm, off));
+                const float mn = fmaxf(m[h], cm);  // finite: slot 0 of every step is valid
+                const float al = exp2f(m[h] - mn);
+                const float pr = exp2f(x - mn);
+                l[h] = l[h] * al + pr;
+#pragma unroll
+                for (int e = 0; e < E; ++e) o[h][e] = fmaf(pr, vf[e], o[h][e] * al);
+                m[h] = mn;
+            }
         }
     }
 
