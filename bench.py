@@ -21,12 +21,18 @@ sequence and decodes; the last planned step decodes exactly 32768 tokens.
   L2, so no flush is needed between steps.
 * ``e2e``: the same metric through the public API with host buffers: the
   allocator runs live, inputs are copied from pinned host memory, the output
-  is read back, each step synchronised.
+  is read back, each step synchronised (steps of a repeated layout replayed
+  from CUDA graphs).
 * ``roofline``: the main decode kernel's algorithmic bytes per launch over
   its own CUDA-event time (events recorded by the library around that launch
   on the launching stream), against the measured HBM copy bandwidth.
 * ``cpu_baseline``: the fp64 oracle on the host cores on a bounded sample of
   the same workload.
+* ``prefill`` (N = 1): the chunked-prefill kernel on 8 x (4096 context +
+  1024-token chunk), its TFLOP/s against the measured bf16 tensor peak, timed
+  apart from the decode steps.
+
+``--study prefix|swap|blocksize|prefill`` prints one side study instead.
 
 ``--impl reference`` times the oracle alone (the CPU arm).  With N > 1 GPUs
 (torchrun) every rank runs its own batch (a different seed) with no
@@ -396,6 +402,20 @@ def run_ours(args, ws, rank, local):
                    "partition_tokens": args.partition or 512, "allocator_after_prefill": alloc_info},
         "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
     }
+    if rank == 0 and ws == 1 and not args.no_prefill:
+        # the chunked-prefill kernel (tensor-core bound), timed apart from the
+        # decode steps above
+        mma_sync, tc = prefill_rows(4096, 1024)
+        peak_tf, peak_tf_src = _bf16_peak_tflops()
+        res["prefill"] = {
+            "workload": "chunked prefill: 8 x (4096 context + 1024-token chunk), 32/8 heads, "
+                        "D 128, bf16 KV, block 16",
+            "kernel": "pa_prefill (prefill_umma_kernel, tcgen05)", "ms": tc["ms"],
+            "roofline": {"bound": "tensor", "achieved": tc["tflops"], "peak": peak_tf,
+                         "unit": "TFLOP/s", "frac": tc["frac_of_bf16_peak"],
+                         "flops_per_launch": tc["flops_per_launch"], "peak_source": peak_tf_src},
+            "mma_sync_kernel_ms": mma_sync["ms"],
+            "max_abs_diff_vs_mma_sync": tc["max_abs_diff_vs_mma_sync"]}
     if rank == 0 and ws == 1 and not args.no_cpu:
         smp = OracleSampler(args.workload, seed)
         nb, secs, pairs = smp.run(args.cpu_budget)
@@ -608,50 +628,62 @@ def study_blocksize(args):
     return out
 
 
-def study_prefill(args):
-    """Chunked prefill: causal attention of a 1024-token chunk per sequence
-    over a 4096-token context (8 sequences, 32/8 heads, D 128, bf16, bs 16).
-    FLOPs = sum over query rows of 4 * D * Hq * (keys attended)."""
+def _bf16_peak_tflops():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, cuBLAS burst)"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback 1.59 PFLOP/s"
+
+
+def prefill_rows(ctx: int, chunk: int, batch: int = 8):
+    """Both prefill kernels on one chunked-prefill workload (32/8 heads, D 128,
+    bf16, bs 16): CUDA-event ms over 20 launches each, the definition's FLOPs
+    (4 * D * Hq per (row, attended key)) and the kernels' full-size agreement."""
     from paged_kv_cache_347_b200 import pagedattn as pa
     from paged_kv_cache_347_b200.runner import PagedKVRunner
+    wl = workloads.chunked_prefill(batch=batch, ctx_lo=ctx, ctx_hi=ctx, chunk_lo=chunk,
+                                   chunk_hi=chunk, num_blocks=batch * (ctx + chunk) // 16 + 64)
+    steps = list(wl.steps)
+    r = PagedKVRunner.for_shape(wl.shape, (ctx + chunk) // 16 + 2)
+    r.run(steps[0])
+    st = steps[1]
+    acts = r.plan(st.ops)
+    r.upload(acts)
+    dev = [t.cuda() for t in (st.k_new, st.v_new, st.q)]
+    r.execute(acts, *dev)
+    a = [x for x in acts if x.kind == "prefill"][0]
+    o = torch.empty((int(a.cu[-1]), 32, 128), dtype=torch.float32, device="cuda")
+    flops = 4.0 * 128 * 32 * sum(ctx + i + 1 for i in range(chunk)) * batch
+    peak, _ = _bf16_peak_tflops()
+    rows = []
+    for variant, kernel in ((1, "mma.sync"), (2, "tcgen05")):
+        ms = _events_ms(lambda: pa.pa_prefill(o, dev[2], r.k_cache, r.v_cache, a.dev["tables"],
+                                              a.dev["lens"], a.dev["cu"], r.scale,
+                                              max_q_len=a.max_q, max_seq_len=a.max_len,
+                                              variant=variant), reps=20)
+        tf = flops / (ms * 1e-3) / 1e12
+        row = {"kernel": kernel, "context": ctx, "chunk": chunk, "batch": batch,
+               "ms": round(ms, 3), "tflops": round(tf, 1),
+               "frac_of_bf16_peak": round(tf / peak, 4), "peak_tflops": peak,
+               "flops_per_launch": flops}
+        if variant == 1:
+            first = o.clone()
+        else:  # both kernels compute the same rows at full size
+            row["max_abs_diff_vs_mma_sync"] = float((o - first).abs().max())
+        rows.append(row)
+    del r
+    torch.cuda.empty_cache()
+    return rows
+
+
+def study_prefill(args):
+    """Chunked prefill, both kernels: 8 sequences x (4096 context + 1024
+    chunk), (0 + 4096), (16384 + 512); 32/8 heads, D 128, bf16, bs 16."""
+    from paged_kv_cache_347_b200 import pagedattn as pa
     res = {"study": "prefill", "rows": []}
     for ctx, chunk in ((4096, 1024), (0, 4096), (16384, 512)):
-        wl = workloads.chunked_prefill(batch=8, ctx_lo=ctx, ctx_hi=ctx, chunk_lo=chunk,
-                                       chunk_hi=chunk, num_blocks=8 * (ctx + chunk) // 16 + 64)
-        steps = list(wl.steps)
-        r = PagedKVRunner.for_shape(wl.shape, (ctx + chunk) // 16 + 2)
-        r.run(steps[0])
-        st = steps[1]
-        acts = r.plan(st.ops)
-        r.upload(acts)
-        dev = [t.cuda() for t in (st.k_new, st.v_new, st.q)]
-        r.execute(acts, *dev)
-        a = [x for x in acts if x.kind == "prefill"][0]
-        o = torch.empty((int(a.cu[-1]), 32, 128), dtype=torch.float32, device="cuda")
-        keys = sum(ctx + i + 1 for i in range(chunk)) * 8
-        flops = 4.0 * 128 * 32 * keys
-        try:
-            with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
-                peak = float(json.load(f)["bf16_tflops"])
-        except (OSError, KeyError, ValueError):
-            peak = 1590.0
-        for variant, kernel in ((1, "mma.sync"), (2, "tcgen05")):
-            ms = _events_ms(lambda: pa.pa_prefill(o, dev[2], r.k_cache, r.v_cache,
-                                                  a.dev["tables"], a.dev["lens"], a.dev["cu"],
-                                                  r.scale, max_q_len=a.max_q,
-                                                  max_seq_len=a.max_len, variant=variant),
-                            reps=20)
-            tf = flops / (ms * 1e-3) / 1e12
-            row = {"kernel": kernel, "context": ctx, "chunk": chunk, "batch": 8,
-                   "ms": round(ms, 3), "tflops": round(tf, 1),
-                   "frac_of_bf16_peak": round(tf / peak, 4), "peak_tflops": peak}
-            if variant == 1:
-                first = o.clone()
-            else:  # both kernels compute the same rows at full size
-                row["max_abs_diff_vs_mma_sync"] = float((o - first).abs().max())
-            res["rows"].append(row)
-        del r
-        torch.cuda.empty_cache()
+        res["rows"] += prefill_rows(ctx, chunk)
     res["device_errors"] = pa.device_errors()
     return res
 
@@ -664,6 +696,8 @@ def main():
     ap.add_argument("--workload", default="long32k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--no-prefill", action="store_true",
+                    help="skip the chunked-prefill line added to the N = 1 bench output")
     ap.add_argument("--no-graph", action="store_true",
                     help="e2e: launch every step eagerly instead of replaying CUDA graphs")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
