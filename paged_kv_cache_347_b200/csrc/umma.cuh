@@ -53,15 +53,6 @@ __device__ __forceinline__ float ex2(float x) {
 }
 
 // --------------------------------------------------------------- MMA
-// D[tmem] (+)= A[smem desc] . B[smem desc], kind::f16, one CTA.
-__device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                        uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
 // D[tmem] (+)= A[tmem] . B[smem desc]: A (M rows on M lanes, K-major, two 16-bit
 // elements per 32-bit column, the lower k in the low half) read from tensor memory.
 __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc,
