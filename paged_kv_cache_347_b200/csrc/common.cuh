@@ -21,19 +21,11 @@ __device__ __forceinline__ void raise_device_error(unsigned int *err, unsigned i
 }
 
 // ----------------------------------------------------------------- types
+// the pa_dtype code of a storage type
 template <typename T> struct StoreT;
-template <> struct StoreT<float> {
-    static constexpr int kCode = PA_F32;
-    __device__ __forceinline__ static float to_float(float x) { return x; }
-};
-template <> struct StoreT<__nv_bfloat16> {
-    static constexpr int kCode = PA_BF16;
-    __device__ __forceinline__ static float to_float(__nv_bfloat16 x) { return __bfloat162float(x); }
-};
-template <> struct StoreT<__half> {
-    static constexpr int kCode = PA_F16;
-    __device__ __forceinline__ static float to_float(__half x) { return __half2float(x); }
-};
+template <> struct StoreT<float> { static constexpr int kCode = PA_F32; };
+template <> struct StoreT<__nv_bfloat16> { static constexpr int kCode = PA_BF16; };
+template <> struct StoreT<__half> { static constexpr int kCode = PA_F16; };
 
 // 16 bytes of storage elements -> floats
 template <typename T> struct Vec16;
@@ -137,16 +129,6 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar), "l"(policy)
-        : "memory");
-}
-
-// 1-D bulk copy global -> this CTA's shared memory (no multicast); both
-// addresses 16-byte aligned, size a multiple of 16.
-__device__ __forceinline__ void bulk_load_1d(uint32_t dst, const void *src, uint32_t bytes,
-                                             uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        ::"r"(dst), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
         : "memory");
 }
 
