@@ -378,6 +378,8 @@ def run_ours(args, ws, rank, local):
             "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
             "main_us_per_launch": round(mean_main_s * 1e6, 2),
             "timed_launches": len(main_ms),
+            "main_us_p10_median_p90": [round(float(np.percentile(main_ms, q)) * 1e3, 2)
+                                       for q in (10, 50, 90)],
             "algorithmic_bytes_per_launch": int(alg_per_launch)}
 
     # end to end through the public API with host buffers
