@@ -20,9 +20,11 @@ sequence and decodes; the last planned step decodes exactly 32768 tokens.
   every pass does identical work).  The KV cache (1.07 GB) is larger than
   L2, so no flush is needed between steps.
 * ``e2e``: the same metric through the public API with host buffers: the
-  allocator runs live, inputs are copied from pinned host memory, the output
-  is read back, each step synchronised (steps of a repeated layout replayed
-  from CUDA graphs).
+  allocator runs live, inputs are copied from pinned host memory and every
+  step's output is copied back to pinned host memory (steps of a repeated
+  layout replayed from CUDA graphs).  The host reads step i's output while
+  the GPU runs step i+1 (two output buffers), so the GPU always has the next
+  step queued; ``--sync-e2e`` waits for each step before launching the next.
 * ``roofline``: the main decode kernel's algorithmic bytes per launch over
   its own CUDA-event time (events recorded by the library around that launch
   on the launching stream), against the measured HBM copy bandwidth.
@@ -432,8 +434,9 @@ def run_ours(args, ws, rank, local):
 def run_e2e(args, sh, width, seed, prefill, dev, ws):
     """Live steps through the public API (PagedKVRunner prepare / stage_graph
     / replay_graph, or launch when a step has no graph form): host allocator,
-    inputs copied from pinned host memory, output read back, every step
-    synchronised."""
+    inputs copied from pinned host memory, every output copied back to pinned
+    host memory and waited for, one step behind the launches unless
+    ``--sync-e2e``."""
     from paged_kv_cache_347_b200.runner import PagedKVRunner
     n = max(1, min(args.steps, args.e2e_steps))
     w = min(args.warmup, 3)
@@ -445,48 +448,61 @@ def run_e2e(args, sh, width, seed, prefill, dev, ws):
     host = [(st.ops, st.k_new.pin_memory(), st.v_new.pin_memory(), st.q.pin_memory())
             for st in steps[1:]]
     b = steps[1].q.shape[0]
-    out_host = torch.empty((b, sh.num_heads, sh.head_dim), dtype=torch.float32).pin_memory()
-    h2d = d2h = 0
-    total = 0
-    replays = 0
+    # eager steps alternate between two output buffers, as the graphs of the
+    # two staging slots do, so that step i+1 never overwrites the output of
+    # step i before the host has it
+    out_host = [torch.empty((b, sh.num_heads, sh.head_dim), dtype=torch.float32).pin_memory()
+                for _ in range(2)]
+    acc = {"h2d": 0, "d2h": 0, "kv": 0, "replays": 0}
     graphs = not args.no_graph
+    lag = 0 if args.sync_e2e else 1
 
-    # the allocator work of step i+1 (and the copy of its inputs into the
-    # page-locked buffers of its CUDA graph) runs on the host while the GPU
-    # runs step i; every step still copies its inputs in and its output back
-    # before the next step's inputs go out
+    def done(ev, res, counted):
+        ev.synchronize()  # this step's output is in host memory
+        if counted:
+            d = [a for a in res["acts"] if a.kind == "decode"][0]
+            acc["h2d"] += res["h2d"]
+            acc["d2h"] += res["d2h"]
+            acc["kv"] += kv_bytes(d.lens, sh.num_kv_heads, sh.head_dim, sh.elem_bytes)
+
+    # Step i+1's allocator work and the copy of its inputs into page-locked
+    # staging buffers run on the host while the GPU runs step i.  Staging
+    # slot and output buffer of step i+1 are those of step i-1, whose output
+    # is waited for first.
     def loop(first, count):
-        nonlocal h2d, d2h, total, replays
         if count <= 0:
             return
+        pending = []
         prep = r.prepare(host[first][0])
         gr = r.stage_graph(prep, *host[first][1:]) if graphs else None
         for i in range(first, first + count):
             if gr is not None:
                 res = r.replay_graph(gr, prep)
-                replays += first >= w
+                acc["replays"] += first >= w
             else:
-                res = r.launch(prep, *host[i][1:], out_host)
+                res = r.launch(prep, *host[i][1:], out_host[i & 1])
+            ev = torch.cuda.Event()
+            ev.record()
+            pending.append((ev, res, first >= w))
+            while len(pending) > lag:
+                done(*pending.pop(0))
             if i + 1 < first + count:
                 prep = r.prepare(host[i + 1][0])
                 gr = r.stage_graph(prep, *host[i + 1][1:]) if graphs else None
-            r.wait()
-            if first >= w:
-                d = [a for a in res["acts"] if a.kind == "decode"][0]
-                h2d += res["h2d"]
-                d2h += res["d2h"]
-                total += kv_bytes(d.lens, sh.num_kv_heads, sh.head_dim, sh.elem_bytes)
+        while pending:
+            done(*pending.pop(0))
 
     loop(0, w)
     barrier(ws)
     t = time.perf_counter()
     loop(w, n)
     el = time.perf_counter() - t
-    el, total = aggregate(el, float(total), ws, dev)
+    el, total = aggregate(el, float(acc["kv"]), ws, dev)
     return {"value": round(total / el / 1e9, 1), "unit": "GB/s",
-            "h2d_bytes_per_step": int(h2d / n), "d2h_bytes_per_step": int(d2h / n),
+            "h2d_bytes_per_step": int(acc["h2d"] / n), "d2h_bytes_per_step": int(acc["d2h"] / n),
             "steps": n, "us_per_step": round(el / n * 1e6, 2),
-            "graph_replayed_steps": replays}
+            "graph_replayed_steps": acc["replays"],
+            "outputs_read": "one step behind the launches" if lag else "each step before the next"}
 
 
 def run_reference(args, ws, rank):
@@ -698,6 +714,8 @@ def main():
     ap.add_argument("--workload", default="long32k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--sync-e2e", action="store_true",
+                    help="e2e: wait for each step's output before launching the next")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the chunked-prefill line added to the N = 1 bench output")
     ap.add_argument("--no-graph", action="store_true",

@@ -369,6 +369,54 @@ def test_graph_replayed_steps_match_the_oracle():
                             torch.zeros(2, 16, 128, dtype=torch.bfloat16).pin_memory()) is None
 
 
+def test_steps_read_one_step_behind_match_the_oracle():
+    """The benchmark's pipelined loop: step i+1 is prepared, staged and
+    launched before the host waits for step i's output, graph steps and eager
+    (copy-on-write) steps mixed; every output, read one step late, is the
+    oracle's for its own step."""
+    from oracle.run import OracleRun
+    from paged_kv_cache_347_b200.runner import PagedKVRunner
+    wl = workloads.custom("pipe", [700, 33, 1, 510], 16, 4, 128, "bf16", 16, 256, seed=6,
+                          steps=8)
+    steps = list(wl.steps)
+    orc, gpu = OracleRun(wl.shape), PagedKVRunner.for_shape(wl.shape, 48)
+    orc.step(steps[0])
+    gpu.run(steps[0])
+    refs = [orc.step(st)["out"] for st in steps[1:]]
+    host = [(st.ops, st.k_new.pin_memory(), st.v_new.pin_memory(), st.q.pin_memory())
+            for st in steps[1:]]
+    outs = [torch.empty(tuple(refs[0].shape), dtype=torch.float32).pin_memory() for _ in range(2)]
+    got, pending, kinds = [], [], []
+    prep = gpu.prepare(host[0][0])
+    gr = gpu.stage_graph(prep, *host[0][1:]) if 0 % 3 else None
+    for i in range(len(host)):
+        if gr is not None:
+            res = gpu.replay_graph(gr, prep)
+            kinds.append("graph")
+        else:
+            res = gpu.launch(prep, *host[i][1:], outs[i & 1])
+            res["out"] = outs[i & 1]
+            kinds.append("eager")
+        ev = torch.cuda.Event()
+        ev.record()
+        pending.append((ev, res))
+        if len(pending) > 1:
+            e, r = pending.pop(0)
+            e.synchronize()
+            got.append(r["out"].double().numpy().copy())
+        if i + 1 < len(host):
+            prep = gpu.prepare(host[i + 1][0])
+            # every third step launches eagerly, the rest replay graphs
+            gr = gpu.stage_graph(prep, *host[i + 1][1:]) if (i + 1) % 3 else None
+    e, r = pending.pop(0)
+    e.synchronize()
+    got.append(r["out"].double().numpy().copy())
+    assert "graph" in kinds and "eager" in kinds
+    for i, (g, ref) in enumerate(zip(got, refs)):
+        err = float(np.abs(g - ref).max())
+        assert err <= TOL["bf16"], (i, kinds[i], err)
+
+
 @pytest.mark.parametrize("pv", [1, 2])
 @pytest.mark.parametrize("dtype,Hq,Hkv,D,bs,ctx,chunk_lo,chunk_hi", [
     ("bf16", 16, 4, 128, 16, 300, 0, 3),     # empty chunks next to 1-3-token ones (seed 11)
