@@ -559,7 +559,11 @@ def _events_ms(fn, reps=20):
 
 def study_prefix(args):
     """Prefix caching on vs off for requests sharing a system prompt: K/V rows
-    written at admission, admission time (allocator + append kernel), hits."""
+    written at admission, admission time (allocator + append kernel), hits,
+    and the causal attention the admission's prefill then needs (pa_prefill
+    over the tokens each request must compute: its own suffix after the
+    cached prompt, or every token without the cache)."""
+    from paged_kv_cache_347_b200 import pagedattn as pa
     from paged_kv_cache_347_b200.runner import PagedKVRunner
     res = {"study": "prefix_cache", "requests": 64, "prompt_tokens": 2048}
     for mode in ("on", "off"):
@@ -581,12 +585,35 @@ def study_prefix(args):
         rows = int(sum(int((a.slots >= 0).sum()) for a in acts if a.kind == "write"))
         ms = _events_ms(lambda: r.execute(acts, k, v, None), reps=10)
         st = r.alloc.stats()
+        # tokens each request computes: those whose rows were written (a
+        # cached token's row is skipped, slot -1, and its attention is done)
+        ids = [op[1] for op in steps[0].ops]
+        lens_all = [len(op[2]) for op in steps[0].ops]
+        slots = np.concatenate([a.slots for a in acts if a.kind == "write"])
+        own, o = [], 0
+        for n in lens_all:
+            own.append(int((slots[o:o + n] >= 0).sum()))
+            o += n
+        tables, lens = r.alloc.block_tables(ids, 160)
+        cu = np.concatenate([[0], np.cumsum(own)]).astype(np.int32)
+        g = torch.Generator(device="cuda").manual_seed(3)
+        q = torch.randn(int(cu[-1]), 32, 128, generator=g, device="cuda").to(torch.bfloat16)
+        out = torch.empty(int(cu[-1]), 32, 128, dtype=torch.float32, device="cuda")
+        tab_d, len_d, cu_d = (torch.from_numpy(x).cuda() for x in (tables, lens, cu))
+        pms = _events_ms(lambda: pa.pa_prefill(out, q, r.k_cache, r.v_cache, tab_d, len_d, cu_d,
+                                                 r.scale, max_q_len=max(own),
+                                                 max_seq_len=160 * 16), reps=10)
+        flops = 4.0 * 128 * 32 * sum(sum(L - n + i + 1 for i in range(n))
+                                      for L, n in zip(lens_all, own))
         res[mode] = {"rows_written": rows, "kv_bytes_written": rows * 8 * 128 * 2 * 2,
                      "append_kernel_us": round(ms * 1e3, 2), "allocator_us": round(host_us, 1),
                      "used_blocks": st["used_blocks"], "prefix_hit_blocks": st["prefix_hit_blocks"],
-                     "prefix_query_blocks": st["prefix_query_blocks"]}
+                     "prefix_query_blocks": st["prefix_query_blocks"],
+                     "prefill_tokens": int(cu[-1]), "prefill_ms": round(pms, 3),
+                     "prefill_tflops": round(flops / pms / 1e9, 1), "prefill_flops": flops}
         del r
         torch.cuda.empty_cache()
+    res["device_errors"] = pa.device_errors()
     return res
 
 
