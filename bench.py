@@ -305,7 +305,7 @@ def run_ours(args, ws, rank, local):
             if a.kind == "write":
                 n += (1 if len(a.pairs) else 0) + (1 if a.nrows else 0)
             else:
-                n += 1 + (1 if math.ceil(a.max_len / (args.partition or 512)) > 1 else 0)
+                n += 1 + (1 if math.ceil(a.max_len / (a.partition or 512)) > 1 else 0)
         launches_per.append(n)
 
     def step(i):
@@ -403,7 +403,11 @@ def run_ours(args, ws, rank, local):
                    "parallelism": f"dp{ws} (independent batches, no collective)",
                    "l2": "inputs larger than L2 (KV cache 1.07 GB per step), no flush",
                    "planned_steps": len(plans), "host_alloc_us_per_step": round(alloc_us, 2),
-                   "partition_tokens": args.partition or 512, "allocator_after_prefill": alloc_info},
+                   "partition_tokens": sorted({a.partition or 512 for acts in plans
+                                               for a in acts if a.kind == "decode"}),
+                   "partition_policy": {-1: "per step, pa_decode_partition_for",
+                                        0: "library default"}.get(args.partition, "fixed"),
+                   "allocator_after_prefill": alloc_info},
         "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
     }
     if rank == 0 and ws == 1 and not args.no_prefill:
@@ -751,8 +755,10 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--study", default="", choices=["", "prefix", "swap", "blocksize", "prefill"],
                     help="print one of the side studies instead of the bench line")
-    ap.add_argument("--partition", type=int, default=0,
-                    help="split length in tokens (0: the library default, 512)")
+    ap.add_argument("--partition", type=int, default=-1,
+                    help="split length in tokens: -1 chosen per step from the lengths "
+                         "(pa_decode_partition_for), 0 the library default (512), or a "
+                         "multiple of 64 in [64, 1024]")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (small cases for profiling)")
     args = ap.parse_args()

@@ -150,6 +150,27 @@ int pa_decode_ex(float *out, const void *q, const void *k_cache, const void *v_c
                  int variant, void *stream);
 
 /*
+ * A partition_size for pa_decode_ex, from the sequence lengths as the caller
+ * knows them on the host (a runtime does: it owns the block tables).  The
+ * decode launches one CTA per (sequence, KV head, partition); when the 512-
+ * token default gives between one and two waves of the CTAs the device holds
+ * at once, the second wave runs part-empty and the kernel's tail grows.  In
+ * that case the result is 1024 if its CTAs fit one wave; otherwise it is 512.
+ * (One alternative only: a runtime that keys CUDA graphs on the split length
+ * then sees it change rarely as its sequences grow.)
+ *   seq_lens_host   host, int32 [num_seqs], each >= 0 (a 0 counts as one CTA)
+ *   slots           CTAs resident at once; 0 = ask the device for the
+ *                   tensor-core kernel's occupancy of this shape times the
+ *                   SM count (the CUDA-core kernel, fp32 or block_size 4,
+ *                   always gets 512)
+ * Returns the partition size (> 0), or a negative pa_status on bad arguments
+ * or, with slots == 0, when the device cannot be queried.  Host only; it
+ * launches nothing.
+ */
+int pa_decode_partition_for(const int32_t *seq_lens_host, int num_seqs, int num_kv_heads,
+                            int head_dim, int block_size, int dtype, int slots);
+
+/*
  * Multi-token (chunked prefill) attention over the paged cache [P1
  * "Mechanism and details": new positions are appended after the prefix,
  * whose blocks stay in place; P3 bullet 3: attention reads K/V through the

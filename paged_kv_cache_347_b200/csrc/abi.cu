@@ -267,6 +267,48 @@ int pa_decode_ex(float *out, const void *q, const void *k_cache, const void *v_c
     return PA_OK;
 }
 
+int pa_decode_partition_for(const int32_t *seq_lens_host, int num_seqs, int num_kv_heads,
+                            int head_dim, int block_size, int dtype, int slots) {
+    clear_error();
+    int rc = check_shape(num_kv_heads, head_dim, block_size, dtype);
+    if (rc) return rc;
+    if (num_seqs < 0 || num_seqs > 65535)
+        return fail(PA_ERR_INVALID_ARG, "num_seqs %d outside [0, 65535]", num_seqs);
+    if (num_seqs > 0 && !seq_lens_host) return fail(PA_ERR_INVALID_ARG, "NULL seq_lens_host");
+    if (slots < 0) return fail(PA_ERR_INVALID_ARG, "slots %d", slots);
+    for (int s = 0; s < num_seqs; ++s)
+        if (seq_lens_host[s] < 0)
+            return fail(PA_ERR_INVALID_ARG, "seq_lens_host[%d] = %d", s, seq_lens_host[s]);
+    if (dtype == PA_F32 || block_size < 8) return kDefaultPartition;  // CUDA-core kernel
+    if (slots == 0) {
+        // per device and shape, asked once: [device][bf16|f16][D 64|128][bs 8..64]
+        static std::atomic<int> cache[kMaxDevices][2][2][4];
+        const int dev = current_device();
+        if (dev < 0 || dev >= kMaxDevices) return fail(PA_ERR_CUDA, "no CUDA device");
+        const int bsi = block_size == 8 ? 0 : block_size == 16 ? 1 : block_size == 32 ? 2 : 3;
+        std::atomic<int> &c = cache[dev][dtype == PA_F16][head_dim == 128][bsi];
+        int per_sm = c.load(std::memory_order_relaxed);
+        if (per_sm <= 0) {
+            per_sm = decode_tc_resident_per_sm(dtype, head_dim, block_size);
+            if (per_sm <= 0) return fail(PA_ERR_CUDA, "occupancy query failed");
+            c.store(per_sm, std::memory_order_relaxed);
+        }
+        slots = per_sm * num_sms();
+    }
+    // CTAs of a partition length: one per (sequence, KV head, partition)
+    auto ctas = [&](int part) {
+        int64_t n = 0;
+        for (int s = 0; s < num_seqs; ++s)
+            n += seq_lens_host[s] == 0 ? 1 : (seq_lens_host[s] + part - 1) / part;
+        return n * num_kv_heads;
+    };
+    // one alternative only, so that a runtime replaying CUDA graphs keyed on
+    // the split length sees it change rarely as its sequences grow
+    const int64_t n0 = ctas(kDefaultPartition);
+    if (n0 > slots && n0 <= 2 * (int64_t)slots && ctas(1024) <= slots) return 1024;
+    return kDefaultPartition;
+}
+
 int pa_decode(float *out, const void *q, const void *k_cache, const void *v_cache,
               const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
               int num_heads, int num_kv_heads, int head_dim, int block_size,

@@ -448,7 +448,46 @@ static cudaError_t launch_tc_d(const DecodeParams &p, const CUtensorMap &mk,
     }
 }
 
+// CTAs of one instance resident per SM (the launch's shared-memory attribute
+// set first, as launch_tc_inst does), or -1.
+template <typename T, int D, int BS, int W, int NS>
+static int resident_inst() {
+    using C = Cfg<T, D, BS, W, NS>;
+    if (cudaFuncSetAttribute(decode_tc_kernel<T, D, BS, W, NS>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             C::kDynSmem) != cudaSuccess)
+        return -1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_tc_kernel<T, D, BS, W, NS>,
+                                                      C::kThreads, C::kDynSmem) != cudaSuccess)
+        return -1;
+    return n;
+}
+
+// the instances launch_tc_d picks
+template <typename T, int D>
+static int resident_d(int block_size) {
+    constexpr int NS = D == 128 ? 2 : 4;
+    switch (block_size) {
+    case 8: return resident_inst<T, D, 8, 2, NS>();
+    case 16: return resident_inst<T, D, 16, 2, NS>();
+    case 32: return resident_inst<T, D, 32, 2, NS>();
+    case 64: return resident_inst<T, D, 64, 4, D == 128 ? 2 : 4>();
+    default: return -1;
+    }
+}
+
 }  // namespace tc
+
+int decode_tc_resident_per_sm(int dtype, int head_dim, int block_size) {
+    if (dtype != PA_BF16 && dtype != PA_F16) return -1;
+    if (head_dim != 64 && head_dim != 128) return -1;
+    if (dtype == PA_BF16)
+        return head_dim == 128 ? tc::resident_d<__nv_bfloat16, 128>(block_size)
+                               : tc::resident_d<__nv_bfloat16, 64>(block_size);
+    return head_dim == 128 ? tc::resident_d<__half, 128>(block_size)
+                           : tc::resident_d<__half, 64>(block_size);
+}
 
 cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, cudaStream_t stream) {
     if (dtype != PA_BF16 && dtype != PA_F16) return cudaErrorNotSupported;

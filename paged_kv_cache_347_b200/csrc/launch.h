@@ -46,6 +46,8 @@ cudaError_t launch_decode_simt(const DecodeParams &p, int dtype, cudaStream_t st
 // Tensor-core decode (bf16/f16, block_size >= 8): TMA-staged K/V, mma.sync.
 // Returns cudaErrorNotSupported for shapes it does not cover.
 cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, cudaStream_t stream);
+// CTAs of the tensor-core decode kernel for this shape resident per SM, or -1
+int decode_tc_resident_per_sm(int dtype, int head_dim, int block_size);
 
 // TMA map of a cache viewed as [rows][D] 16-bit elements: 128-byte boxes of
 // box_rows rows, 128B swizzle.  False if the driver refuses it.

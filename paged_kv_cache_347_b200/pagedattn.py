@@ -60,6 +60,7 @@ _sig("pa_decode", _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, 
      _vp, _sz, _vp)
 _sig("pa_decode_ex", _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i,
      _vp, _sz, _i, _i, _vp)
+_sig("pa_decode_partition_for", _i, _vp, _i, _i, _i, _i, _i, _i)
 _sig("pa_copy_blocks", _i, _vp, _vp, _vp, _i, _sz, _i, _vp)
 _sig("pa_decode_static", _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
      _i, _vp)
@@ -167,6 +168,21 @@ def decode_workspace_size(num_seqs: int, num_heads: int, head_dim: int, max_seq_
                           partition_size: int = 0) -> int:
     return _lib.pa_decode_workspace_size(num_seqs, num_heads, head_dim, max_seq_len,
                                          partition_size)
+
+
+def decode_partition_for(seq_lens, num_kv_heads: int, head_dim: int, block_size: int,
+                         dtype, slots: int = 0) -> int:
+    """pa_decode_partition_for: a partition_size for pa_decode from the host
+    copy of the sequence lengths (512 unless that leaves a part-empty second
+    wave of CTAs).  dtype: a torch dtype or a PA_* code; slots 0 asks the
+    device how many decode CTAs it holds at once."""
+    lens = np.ascontiguousarray(np.asarray(seq_lens), dtype=np.int32).reshape(-1)
+    code = DTYPE_CODE[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    rc = _lib.pa_decode_partition_for(lens.ctypes.data if lens.size else None, lens.size,
+                                      num_kv_heads, head_dim, block_size, code, slots)
+    if rc < 0:
+        raise PagedAttnError(rc, "pa_decode_partition_for")
+    return rc
 
 
 def cached_workspace(device: torch.device) -> Optional[torch.Tensor]:

@@ -17,6 +17,10 @@ runner turns a step into device actions in two phases:
   ``pa_reshape_and_cache``, and for a decode ``pa_decode``; all on the
   current stream, nothing synchronised.
 
+``partition_size`` 0 keeps pa_decode's 512-token splits; -1 picks, for each
+decode, pa_decode_partition_for's length from the batch's lengths (longer
+splits when 512 would leave a part-empty second wave of CTAs).
+
 ``run`` does both for one step, moving the host arrays to the device on the
 way.  Planning ahead lets a caller stage a whole run of steps in device
 memory before timing it.
@@ -45,6 +49,7 @@ class Action:
     max_len: int = 0
     cu: Optional[np.ndarray] = None      # prefill: int32 [b + 1] row offsets
     max_q: int = 0
+    partition: int = 0                   # decode: split length passed to pa_decode
     dev: dict = field(default_factory=dict)
 
 
@@ -138,8 +143,13 @@ class PagedKVRunner:
                     self.alloc.seq_free(op[1])
                 elif kind == "decode":
                     tables, lens = self.alloc.block_tables(list(op[1]), self.width)
+                    part = self.partition_size
+                    if part < 0:
+                        part = pa.decode_partition_for(lens, self.num_kv_heads, self.head_dim,
+                                                       self.block_size, self.dtype)
                     acts.append(Action("decode", tables=tables, lens=lens,
-                                       max_len=int(lens.max()) if lens.size else 0))
+                                       max_len=int(lens.max()) if lens.size else 0,
+                                       partition=part))
                 elif kind == "prefill":
                     sids = [x for x, _ in op[1]]
                     ns = np.array([n for _, n in op[1]], np.int32)
@@ -217,7 +227,7 @@ class PagedKVRunner:
                     (b, self.num_heads, self.head_dim), dtype=torch.float32, device=self.device)
                 pa.pa_decode(o, q, self.k_cache, self.v_cache, a.dev["tables"], a.dev["lens"],
                              self.scale, max_seq_len=a.max_len,
-                             partition_size=self.partition_size, variant=self.variant)
+                             partition_size=a.partition, variant=self.variant)
                 res = o
         return res
 
@@ -315,8 +325,8 @@ class PagedKVRunner:
             return None
         if sum(a.kind == "decode" for a in acts) != 1:
             return None
-        layout = tuple((a.kind, a.nrows, None if a.tables is None else a.tables.shape)
-                       for a in acts)
+        layout = tuple((a.kind, a.nrows, None if a.tables is None else a.tables.shape,
+                        a.partition) for a in acts)
         return (layout, prep["bytes"], prep["slot"], prep["host"].data_ptr(),
                 tuple(k_new.shape), tuple(q.shape), k_new.dtype)
 

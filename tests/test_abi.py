@@ -95,3 +95,45 @@ def test_selftest_wait_rejects_bad_arguments_before_any_cuda_call():
     assert pa._lib.pa_selftest_wait(0, 0, None, None) == invalid
     assert pa._lib.pa_selftest_wait(10**11, 0, None, None) == invalid
     assert pa._lib.pa_selftest_wait(10**6, 0, None, None) == invalid  # NULL elapsed
+
+
+def _ctas(lens, part, hkv):
+    return hkv * sum(1 if L == 0 else -(-int(L) // part) for L in lens)
+
+
+@pytest.mark.parametrize("lens,slots", [
+    ([3000] * 32, 888),                       # 6 splits x 32 x 8 = 1536 CTAs at 512: 1.7 waves
+    ([3000] * 50, 888),                       # 2400 CTAs: 2.7 waves, keeps 512
+    ([4000] * 20, 700),                       # 1280 at 512, 640 at 1024
+    ([2048] * 32, 888),                       # 1024 CTAs at 512: one CTA past a full wave
+    ([32768] * 2, 888),
+    ([32768] * 8, 888),                       # 4096 CTAs: many waves, keeps 512
+    ([1024] * 32, 888),                       # 512 CTAs: one wave, keeps 512
+    ([0, 1, 511, 512, 513, 4096, 4097] * 20, 700),
+    (list(range(0, 9000, 37)), 1000),
+])
+def test_partition_choice_follows_its_rule(lens, slots):
+    """pa_decode_partition_for against its stated rule, evaluated here by
+    brute force: 512 unless 512-token CTAs fill more than one wave and at most
+    two, then 1024 if that fits one wave."""
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    hkv = 8
+    got = pa.decode_partition_for(lens, hkv, 128, 16, torch.bfloat16, slots=slots)
+    n0 = _ctas(lens, 512, hkv)
+    want = 1024 if slots < n0 <= 2 * slots and _ctas(lens, 1024, hkv) <= slots else 512
+    assert got == want
+
+
+def test_partition_choice_edge_cases():
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    # the CUDA-core kernel (fp32, or 4-row blocks) keeps 512
+    assert pa.decode_partition_for([2048] * 32, 8, 128, 16, torch.float32, slots=888) == 512
+    assert pa.decode_partition_for([2048] * 32, 8, 128, 4, torch.bfloat16, slots=888) == 512
+    assert pa.decode_partition_for([], 8, 128, 16, torch.bfloat16, slots=888) == 512
+    with pytest.raises(pa.PagedAttnError):
+        pa.decode_partition_for([5, -1], 8, 128, 16, torch.bfloat16, slots=888)
+    with pytest.raises(pa.PagedAttnError):
+        pa.decode_partition_for([5], 8, 100, 16, torch.bfloat16, slots=888)
+    with pytest.raises(pa.PagedAttnError):
+        pa.decode_partition_for([5], 8, 128, 16, torch.bfloat16, slots=-1)
+    assert pa._lib.pa_decode_partition_for(None, 2, 8, 128, 16, 1, 888) == -1

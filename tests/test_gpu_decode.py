@@ -82,6 +82,22 @@ def test_llama_shaped_full_sampled():
     assert max(errs) <= TOL["bf16"], errs
 
 
+def test_llama_shaped_with_chosen_partition():
+    """The runner's per-step split length (pa_decode_partition_for, asking the
+    device for its slot count): the Llama-8B-shaped batch leaves 512-token
+    CTAs part-way into a second wave on a B200, so a longer split is chosen;
+    sampled outputs still match the oracle."""
+    pa = _pa()
+    wl = workloads.llama(steps=2)
+    errs, gpu, _ = run_parity(wl, table_width=257, sample=48, partition_size=-1)
+    assert max(errs) <= TOL["bf16"], errs
+    lens = np.random.default_rng(1).integers(512, 4096, size=32, endpoint=True)
+    p = pa.decode_partition_for(lens, 8, 128, 16, torch.bfloat16)
+    assert p in (512, 1024)
+    # the long-context batch is many waves deep at 512 and keeps it
+    assert pa.decode_partition_for([32768] * 8, 8, 128, 16, torch.bfloat16) == 512
+
+
 @pytest.mark.parametrize("partition", [64, 512, 1024])
 def test_long_context_reduced(partition):
     wl = workloads.long_context(batch=2, seq_len=4096 + 37, steps=2, num_blocks=1024)
