@@ -313,49 +313,67 @@ class PagedKVRunner:
     # Steps of the same layout (the same action kinds and sizes, no copy-on-
     # write pairs, prepared in the same staging slot) repeat the same device
     # work on different bytes.  launch_graph() captures that work once per
-    # layout -- the copy of the packed arrays, the copies of the new K/V rows
-    # and queries from page-locked buffers owned by the graph, the kernels and
-    # the copy of the output back -- and replays it; a decode inside a graph
-    # takes the table capacity as its length bound, so that its grid is fixed.
+    # layout -- one copy of the slot's staging buffer (the packed arrays and,
+    # behind them, the new K/V rows and queries), the kernels and the copy of
+    # the output back -- and replays it; a decode inside a graph takes the
+    # table capacity as its length bound, so that its grid is fixed.
+    @staticmethod
+    def _graphable(acts) -> bool:
+        return (bool(acts) and all(a.kind in ("write", "decode") for a in acts)
+                and not any(a.kind == "write" and len(a.pairs) for a in acts)
+                and sum(a.kind == "decode" for a in acts) == 1)
+
     def _graph_key(self, prep: dict, k_new: torch.Tensor, q: torch.Tensor):
         acts = prep["acts"]
-        if not acts or any(a.kind not in ("write", "decode") for a in acts):
-            return None
-        if any(a.kind == "write" and len(a.pairs) for a in acts):
-            return None
-        if sum(a.kind == "decode" for a in acts) != 1:
+        if not self._graphable(acts):
             return None
         layout = tuple((a.kind, a.nrows, None if a.tables is None else a.tables.shape,
                         a.partition) for a in acts)
         return (layout, prep["bytes"], prep["slot"], prep["host"].data_ptr(),
                 tuple(k_new.shape), tuple(q.shape), k_new.dtype)
 
+    def _place_inputs(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
+                      q: torch.Tensor) -> None:
+        """Room for the step's new K/V rows and queries in the slot's staging
+        buffer behind its packed arrays (256-byte aligned; the buffers grow,
+        keeping the arrays, when too small), so that a graph step moves all of
+        its inputs with one host-to-device copy."""
+        total = prep["bytes"]
+        offs, end = [], (total + 255) & ~255
+        for t in (k_new, v_new, q):
+            offs.append(end)
+            end = (end + t.nbytes + 255) & ~255
+        if prep["host"].numel() < end:
+            old = prep["host"]
+            prep["host"], prep["dev"] = self._staging(prep["slot"], end)
+            prep["host"][:total].copy_(old[:total])
+        prep["in_offs"], prep["in_end"] = offs, end
+
     def _capture(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
                  q: torch.Tensor) -> dict:
         dec = [a for a in prep["acts"] if a.kind == "decode"][0]
-        g = {"k": torch.empty_like(k_new, device="cpu").pin_memory(),
-             "v": torch.empty_like(v_new, device="cpu").pin_memory(),
-             "q": torch.empty_like(q, device="cpu").pin_memory(),
-             "out": torch.empty((dec.tables.shape[0], self.num_heads, self.head_dim),
-                                dtype=torch.float32).pin_memory()}
-        g["dk"], g["dv"], g["dq"] = (torch.empty_like(t, device=self.device)
-                                     for t in (k_new, v_new, q))
-        for t, src in ((g["k"], k_new), (g["v"], v_new), (g["q"], q)):
-            t.copy_(src)
-        total, host, devb = prep["bytes"], prep["host"], prep["dev"]
+        g = {"out": torch.empty((dec.tables.shape[0], self.num_heads, self.head_dim),
+                                dtype=torch.float32).pin_memory(),
+             "in_bytes": sum(t.nbytes for t in (k_new, v_new, q))}
+        end, host, devb = prep["in_end"], prep["host"], prep["dev"]
+        # typed host views the later steps of this layout copy their inputs into
+        g["in"] = [host[off:off + t.nbytes].view(t.dtype).view(t.shape)
+                   for off, t in zip(prep["in_offs"], (k_new, v_new, q))]
+        for v, t in zip(g["in"], (k_new, v_new, q)):
+            v.copy_(t)
+        ins = [devb[off:off + t.nbytes].view(t.dtype).view(t.shape)
+               for off, t in zip(prep["in_offs"], (k_new, v_new, q))]
         for a in prep["acts"]:
             if a.kind == "decode":
                 a.max_len = self.width * self.block_size
 
         def body():
-            if total:
-                devb[:total].copy_(host[:total], non_blocking=True)
+            # one copy brings the packed arrays and the new rows and queries
+            devb[:end].copy_(host[:end], non_blocking=True)
             for (a, name, arr), off in zip(prep["arrays"], prep["offs"]):
                 dt = torch.int64 if arr.dtype == np.int64 else torch.int32
                 a.dev[name] = devb[off:off + arr.nbytes].view(dt).view(arr.shape)
-            for d, h in (("dk", "k"), ("dv", "v"), ("dq", "q")):
-                g[d].copy_(g[h], non_blocking=True)
-            g["o"] = self.execute(prep["acts"], g["dk"], g["dv"], g["dq"])
+            g["o"] = self.execute(prep["acts"], *ins)
             g["out"].copy_(g["o"], non_blocking=True)
 
         # one eager run first (workspace, per-device set-up); it applies this
@@ -377,13 +395,15 @@ class PagedKVRunner:
     def stage_graph(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
                     q: torch.Tensor) -> Optional[dict]:
         """Host half of a graph step: copy the new K/V rows and queries into
-        the page-locked buffers of the graph for this step's layout (capturing
-        it the first time, which runs the step once eagerly).  Safe while the
-        GPU still works on the previous step, whose graph is the other
-        staging slot's.  None when the step's layout has no graph form."""
-        key = self._graph_key(prep, k_new, q)
-        if key is None:
+        the slot's page-locked staging buffer behind the packed arrays
+        (capturing the graph for this step's layout the first time, which runs
+        the step once eagerly).  Safe while the GPU still works on the previous
+        step, whose graph is the other staging slot's.  None when the step's
+        layout has no graph form."""
+        if not self._graphable(prep["acts"]):
             return None
+        self._place_inputs(prep, k_new, v_new, q)
+        key = self._graph_key(prep, k_new, q)
         if not hasattr(self, "_graphs"):
             self._graphs = {}
         if key in self._graphs and self._graphs[key] is None:
@@ -399,8 +419,8 @@ class PagedKVRunner:
                 return None
             self._graphs[key] = g
         else:
-            for t, src in ((g["k"], k_new), (g["v"], v_new), (g["q"], q)):
-                t.copy_(src)
+            for v, t in zip(g["in"], (k_new, v_new, q)):
+                v.copy_(t)
         return g
 
     def replay_graph(self, g: dict, prep: dict) -> dict:
@@ -408,11 +428,10 @@ class PagedKVRunner:
         output lands in a page-locked tensor owned by the graph, readable after
         wait() until the next replay of the same layout."""
         g["graph"].replay()
-        if prep["bytes"]:
-            ev = torch.cuda.Event()
-            ev.record()
-            self._stage_ev[prep["slot"]] = ev
-        h2d = prep["bytes"] + sum(g[t].nbytes for t in ("k", "v", "q"))
+        ev = torch.cuda.Event()
+        ev.record()
+        self._stage_ev[prep["slot"]] = ev  # the staging buffer is free again after this
+        h2d = prep["bytes"] + g["in_bytes"]
         return {"h2d": h2d, "d2h": g["out"].nbytes, "acts": prep["acts"], "out": g["out"]}
 
     def launch_graph(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
