@@ -485,8 +485,10 @@ def run_e2e(args, sh, width, seed, prefill, dev, ws):
                 acc["replays"] += first >= w
             else:
                 res = r.launch(prep, *host[i][1:], out_host[i & 1])
-            ev = torch.cuda.Event()
-            ev.record()
+            ev = res.get("ready")  # a graph step's output copy runs on its own stream
+            if ev is None:
+                ev = torch.cuda.Event()
+                ev.record()
             pending.append((ev, res, first >= w))
             while len(pending) > lag:
                 done(*pending.pop(0))

@@ -302,21 +302,31 @@ class PagedKVRunner:
             a.dev[name] = devb[off:off + arr.nbytes].view(dt).view(arr.shape)
         dev = [t.to(self.device, non_blocking=True) for t in (k_new, v_new, q)]
         o = self.execute(prep["acts"], *dev)
+        if not hasattr(self, "_run_ev"):
+            self._run_ev = [None, None]
+        ev_run = torch.cuda.Event()
+        ev_run.record()
+        self._run_ev[prep["slot"]] = ev_run  # a graph step's copy in waits for it
         out_host.copy_(o, non_blocking=True)
         h2d = total + sum(t.nbytes for t in (k_new, v_new, q))
         return {"h2d": h2d, "d2h": out_host.nbytes, "acts": prep["acts"]}
 
     def wait(self) -> None:
+        """Synchronise the current stream and the graph steps' copy streams."""
         torch.cuda.current_stream(self.device).synchronize()
+        if hasattr(self, "_s_out"):
+            self._s_in.synchronize()
+            self._s_out.synchronize()
 
     # ------------------------------------------------------------ graph replay
     # Steps of the same layout (the same action kinds and sizes, no copy-on-
     # write pairs, prepared in the same staging slot) repeat the same device
     # work on different bytes.  launch_graph() captures that work once per
-    # layout -- one copy of the slot's staging buffer (the packed arrays and,
-    # behind them, the new K/V rows and queries), the kernels and the copy of
-    # the output back -- and replays it; a decode inside a graph takes the
-    # table capacity as its length bound, so that its grid is fixed.
+    # layout, as three graphs -- one copy of the slot's staging buffer (the
+    # packed arrays and, behind them, the new K/V rows and queries), the
+    # kernels, and the copy of the output back -- and replays them on two copy
+    # streams and the current stream; a decode inside a graph takes the table
+    # capacity as its length bound, so that its grid is fixed.
     @staticmethod
     def _graphable(acts) -> bool:
         return (bool(acts) and all(a.kind in ("write", "decode") for a in acts)
@@ -367,13 +377,19 @@ class PagedKVRunner:
             if a.kind == "decode":
                 a.max_len = self.width * self.block_size
 
-        def body():
-            # one copy brings the packed arrays and the new rows and queries
+        # three graphs, replayed on three streams so that a step's copies
+        # overlap its neighbours' kernels: copy in (one copy brings the packed
+        # arrays and the new rows and queries), run, copy the output out
+        def body_in():
             devb[:end].copy_(host[:end], non_blocking=True)
+
+        def body_run():
             for (a, name, arr), off in zip(prep["arrays"], prep["offs"]):
                 dt = torch.int64 if arr.dtype == np.int64 else torch.int32
                 a.dev[name] = devb[off:off + arr.nbytes].view(dt).view(arr.shape)
             g["o"] = self.execute(prep["acts"], *ins)
+
+        def body_out():
             g["out"].copy_(g["o"], non_blocking=True)
 
         # one eager run first (workspace, per-device set-up); it applies this
@@ -381,15 +397,22 @@ class PagedKVRunner:
         side = torch.cuda.Stream(self.device)
         side.wait_stream(torch.cuda.current_stream(self.device))
         with torch.cuda.stream(side):
-            body()
+            body_in()
+            body_run()
+            body_out()
         side.synchronize()
         # the graph writes split partials into the binding's cached workspace:
         # keep that buffer alive for as long as the graph
         g["ws"] = pa.cached_workspace(self.device)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=side, capture_error_mode="thread_local"):
-            body()
-        g["graph"] = graph
+        for name, body in (("g_in", body_in), ("g_run", body_run), ("g_out", body_out)):
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=side, capture_error_mode="thread_local"):
+                body()
+            g[name] = graph
+        # events re-recorded at every replay of this layout (made once: the
+        # host side of a replay stays short)
+        g["ev_in"], g["ev_run"], g["ev_out"] = (torch.cuda.Event() for _ in range(3))
+        g["replayed"] = False
         return g
 
     def stage_graph(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
@@ -423,16 +446,48 @@ class PagedKVRunner:
                 v.copy_(t)
         return g
 
+    def _copy_streams(self):
+        if not hasattr(self, "_s_in"):
+            self._s_in = torch.cuda.Stream(self.device)
+            self._s_out = torch.cuda.Stream(self.device)
+        return self._s_in, self._s_out
+
     def replay_graph(self, g: dict, prep: dict) -> dict:
-        """Device half of a graph step: replay it on the current stream.  The
-        output lands in a page-locked tensor owned by the graph, readable after
-        wait() until the next replay of the same layout."""
-        g["graph"].replay()
-        ev = torch.cuda.Event()
-        ev.record()
-        self._stage_ev[prep["slot"]] = ev  # the staging buffer is free again after this
+        """Device half of a graph step.  The copy in runs on a copy stream
+        once the previous step of this staging slot has finished with the
+        slot's device buffer; the kernels run on the current stream after the
+        copy in (and after this layout's previous output has been copied
+        out); the output's copy back runs on a second copy stream.  The
+        output lands in a page-locked tensor owned by the graph, readable once
+        the returned "ready" event has completed (or after wait()) until the
+        next replay of the same layout, which also re-records that event."""
+        cur = torch.cuda.current_stream(self.device)
+        s_in, s_out = self._copy_streams()
+        slot = prep["slot"]
+        if not hasattr(self, "_run_ev"):
+            self._run_ev = [None, None]
+        if self._run_ev[slot] is not None:
+            s_in.wait_event(self._run_ev[slot])
+        torch.cuda.set_stream(s_in)
+        g["g_in"].replay()
+        g["ev_in"].record(s_in)
+        torch.cuda.set_stream(cur)
+        self._stage_ev[slot] = g["ev_in"]  # the host staging buffer is free again after this
+        cur.wait_event(g["ev_in"])
+        if g["replayed"]:
+            cur.wait_event(g["ev_out"])  # the previous output of this layout has left
+        g["g_run"].replay()
+        g["ev_run"].record(cur)
+        self._run_ev[slot] = g["ev_run"]
+        s_out.wait_event(g["ev_run"])
+        torch.cuda.set_stream(s_out)
+        g["g_out"].replay()
+        g["ev_out"].record(s_out)
+        torch.cuda.set_stream(cur)
+        g["replayed"] = True
         h2d = prep["bytes"] + g["in_bytes"]
-        return {"h2d": h2d, "d2h": g["out"].nbytes, "acts": prep["acts"], "out": g["out"]}
+        return {"h2d": h2d, "d2h": g["out"].nbytes, "acts": prep["acts"], "out": g["out"],
+                "ready": g["ev_out"]}
 
     def launch_graph(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
                      q: torch.Tensor) -> Optional[dict]:
