@@ -22,9 +22,10 @@ sequence and decodes; the last planned step decodes exactly 32768 tokens.
 * ``e2e``: the same metric through the public API with host buffers: the
   allocator runs live, inputs are copied from pinned host memory and every
   step's output is copied back to pinned host memory (steps of a repeated
-  layout replayed from CUDA graphs).  The host reads step i's output while
-  the GPU runs step i+1 (two output buffers), so the GPU always has the next
-  step queued; ``--sync-e2e`` waits for each step before launching the next.
+  layout replayed from CUDA graphs, their copies on copy streams of their
+  own).  The host reads step i's output while the GPU runs step i+1 (two
+  output buffers), so the GPU always has the next step queued;
+  ``--sync-e2e`` waits for each step before launching the next.
 * ``roofline``: the main decode kernel's algorithmic bytes per launch over
   its own CUDA-event time (events recorded by the library around that launch
   on the launching stream), against the measured HBM copy bandwidth.
