@@ -69,6 +69,16 @@ class PagedKVRunner:
         self.dtype, self.scale, self.width = dtype, scale, table_width
         self.partition_size, self.variant = partition_size, variant
         self.prefill_variant = prefill_variant
+        # host-fed steps: two staging slots (page-locked host / device buffer
+        # pairs), the event after which each slot's host buffer is free, the
+        # event after which each slot's device buffer is free, and the graphs
+        # of the layouts seen so far with their two copy streams
+        self._stage = [None, None]
+        self._stage_ev = [None, None]
+        self._run_ev = [None, None]
+        self._next_slot = 0
+        self._graphs = {}
+        self._s_in = self._s_out = None
 
     @classmethod
     def for_shape(cls, shape, table_width: int, **kw) -> "PagedKVRunner":
@@ -242,9 +252,6 @@ class PagedKVRunner:
     #   wait()        -> synchronise the stream (the output is then readable).
     def _staging(self, slot: int, nbytes: int):
         """Pinned host / device buffer pair number ``slot`` (of 2), grown on demand."""
-        if not hasattr(self, "_stage"):
-            self._stage = [None, None]
-            self._stage_ev = [None, None]
         cur = self._stage[slot]
         if cur is None or cur[0].numel() < nbytes:
             n = max(nbytes, 1 << 20)
@@ -279,7 +286,7 @@ class PagedKVRunner:
         for _, _, arr in arrays:
             offs.append(total)
             total += (arr.nbytes + 15) & ~15
-        slot = getattr(self, "_next_slot", 0)
+        slot = self._next_slot
         self._next_slot = 1 - slot
         host, devb = self._staging(slot, total)
         hb = host.numpy()
@@ -302,8 +309,6 @@ class PagedKVRunner:
             a.dev[name] = devb[off:off + arr.nbytes].view(dt).view(arr.shape)
         dev = [t.to(self.device, non_blocking=True) for t in (k_new, v_new, q)]
         o = self.execute(prep["acts"], *dev)
-        if not hasattr(self, "_run_ev"):
-            self._run_ev = [None, None]
         ev_run = torch.cuda.Event()
         ev_run.record()
         self._run_ev[prep["slot"]] = ev_run  # a graph step's copy in waits for it
@@ -314,7 +319,7 @@ class PagedKVRunner:
     def wait(self) -> None:
         """Synchronise the current stream and the graph steps' copy streams."""
         torch.cuda.current_stream(self.device).synchronize()
-        if hasattr(self, "_s_out"):
+        if self._s_out is not None:
             self._s_in.synchronize()
             self._s_out.synchronize()
 
@@ -427,8 +432,6 @@ class PagedKVRunner:
             return None
         self._place_inputs(prep, k_new, v_new, q)
         key = self._graph_key(prep, k_new, q)
-        if not hasattr(self, "_graphs"):
-            self._graphs = {}
         if key in self._graphs and self._graphs[key] is None:
             return None  # this layout failed to capture before: launch eagerly
         g = self._graphs.get(key)
@@ -447,7 +450,7 @@ class PagedKVRunner:
         return g
 
     def _copy_streams(self):
-        if not hasattr(self, "_s_in"):
+        if self._s_in is None:
             self._s_in = torch.cuda.Stream(self.device)
             self._s_out = torch.cuda.Stream(self.device)
         return self._s_in, self._s_out
@@ -464,8 +467,6 @@ class PagedKVRunner:
         cur = torch.cuda.current_stream(self.device)
         s_in, s_out = self._copy_streams()
         slot = prep["slot"]
-        if not hasattr(self, "_run_ev"):
-            self._run_ev = [None, None]
         if self._run_ev[slot] is not None:
             s_in.wait_event(self._run_ev[slot])
         torch.cuda.set_stream(s_in)
