@@ -62,7 +62,6 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 NOMINAL_HBM_GBS = 8000.0
-PROFILE_EVERY = 8
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -119,11 +118,17 @@ def make_workload(name: str, n_steps: int, seed: int, batch: int = 0):
     raise SystemExit(f"unknown workload {name}")
 
 
+SEEDS = {"long32k": 2, "llama8b": 1, "beam": 3}
+
 DESCR = {
     "long32k": "long context: B 8, Hq 64 / Hkv 8, D 128, bf16 KV, block 16, seq_len 32768, "
                "split 512 + reduce, 32768-block pool in a seeded permutation",
     "llama8b": "Llama-8B-shaped decode: B 32, Hq 32 / Hkv 8, D 128, bf16 KV, block 16, "
                "seq_len U[512, 4096], 16384-block pool in a seeded permutation",
+    "beam": "prefix sharing / beam search: 4 prompts x 4 beams, 2050-token shared prefix, "
+            "32/8 heads, D 128, fp16 KV, block 16",
+    "mix_bs16": "continuous-batching mix: 256 sequences, seq_len log-U[16, 8192], 32/8 heads, "
+                "D 128, bf16 KV, block 16, 10% finish and 128-token admissions per step",
 }
 
 
@@ -203,20 +208,38 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback 6.65 TB/s"
 
 
-def traffic_from_profile(kernel_src: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the kernel source as it is now; else None."""
+DECODE_SOURCES = ("decode_tc.cu", "decode_common.cuh", "common.cuh", "launch.h")
+
+
+def decode_source_hash() -> str:
+    """First 16 hex digits of the sha256 of the main decode kernel's sources."""
+    h = hashlib.sha256()
+    for name in DECODE_SOURCES:
+        with open(os.path.join(ROOT, "paged_kv_cache_347_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_from_profile(workload: str, alg_bytes_per_launch: float):
+    """DRAM bytes (read + write) per launch of the main decode kernel, from
+    the committed ncu summary, if it was taken on the kernel's sources as they
+    are now (else None).  A summary taken on a smaller case of the workload
+    is scaled to a full launch by the ratio of algorithmic bytes, which
+    holds while traffic grows in proportion to the tokens read."""
     path = os.path.join(ROOT, "profiles", f"decode_tc_{workload}.json")
     try:
         with open(path) as f:
             prof = json.load(f)
-        with open(kernel_src, "rb") as f:
-            h = hashlib.sha256(f.read()).hexdigest()[:16]
+        h = decode_source_hash()
     except (OSError, ValueError):
         return None
     if prof.get("kernel_src_sha256_16") != h:
         return None
-    return prof.get("dram_bytes_per_launch")
+    dram = float(prof["dram_bytes_per_launch"])
+    alg = float(prof.get("algorithmic_bytes_per_launch") or 0)
+    if alg > 0:
+        dram *= alg_bytes_per_launch / alg
+    return int(round(dram))
 
 
 # ----------------------------------------------------------------- CPU oracle
@@ -263,65 +286,144 @@ class OracleSampler:
 
 
 # ----------------------------------------------------------------- main arm
+class Planned:
+    """One workload made ready for timing: its runner with the prefill
+    applied, every decode step planned by the host allocator (timed apart)
+    and its inputs staged in HBM."""
+
+    def __init__(self, name: str, n_plan: int, seed: int, dev, batch: int = 0,
+                 partition: int = -1):
+        from paged_kv_cache_347_b200.runner import PagedKVRunner
+        self.name = name
+        wl, self.width = make_workload(name, n_plan, seed, batch)
+        self.sh = sh = wl.shape
+        self.runner = PagedKVRunner.for_shape(sh, self.width, device=str(dev),
+                                              partition_size=partition)
+        steps = list(wl.steps)
+        self.prefill, dec = steps[0], steps[1:]
+        self.runner.run(self.prefill)                      # untimed prefill
+        torch.cuda.synchronize()
+        ast = self.runner.alloc.stats()
+        self.alloc_info = {"block_size": sh.block_size, "used_blocks": ast["used_blocks"],
+                           "reserved_slots": ast["reserved_slots"],
+                           "logical_tokens": ast["logical_tokens"],
+                           "tail_waste_frac": round(1 - ast["logical_tokens"]
+                                                    / max(1, ast["reserved_slots"]), 5)}
+        t = time.perf_counter()
+        self.plans = [self.runner.plan(st.ops) for st in dec]
+        self.alloc_us = (time.perf_counter() - t) / len(dec) * 1e6
+        for acts in self.plans:
+            self.runner.upload(acts)
+        self.dev_in = [(st.k_new.to(dev), st.v_new.to(dev), st.q.to(dev)) for st in dec]
+        self.b = dec[0].q.shape[0]
+        self.out = torch.empty((self.b, sh.num_heads, sh.head_dim), dtype=torch.float32,
+                               device=dev)
+        self.decodes = [[a for a in acts if a.kind == "decode"][0] for acts in self.plans]
+        self.step_bytes = [kv_bytes(d.lens, sh.num_kv_heads, sh.head_dim, sh.elem_bytes)
+                           for d in self.decodes]
+        # kernels each step launches: the copy-on-write copy, the append, the
+        # main decode and, when some sequence has more than one split, the reduce
+        self.launches_per = []
+        for acts in self.plans:
+            n = 0
+            for a in acts:
+                if a.kind == "write":
+                    n += (1 if len(a.pairs) else 0) + (1 if a.nrows else 0)
+                else:
+                    n += 1 + (1 if math.ceil(a.max_len / (a.partition or 512)) > 1 else 0)
+            self.launches_per.append(n)
+
+    def step(self, i: int) -> None:
+        j = i % len(self.plans)
+        k, v, q = self.dev_in[j]
+        self.runner.execute(self.plans[j], k, v, q, out=self.out)
+
+    def alg_bytes(self, j: int) -> int:
+        """Algorithmic bytes of step j's main decode launch: K/V of every
+        token, the queries, the table entries and the lengths."""
+        sh, d = self.sh, self.decodes[j]
+        nb = int(sum(-(-int(x) // sh.block_size) for x in d.lens))
+        return (self.step_bytes[j] + self.b * sh.num_heads * sh.head_dim * sh.elem_bytes
+                + nb * 4 + self.b * 4)
+
+    def partitions(self):
+        return sorted({d.partition or 512 for d in self.decodes})
+
+    def close(self):
+        self.runner = self.plans = self.dev_in = None
+        torch.cuda.empty_cache()
+
+
+_FLUSH = {}
+
+
+def flush_l2(dev) -> None:
+    """Writes 256 MB (twice the 126 MB L2) so that the next kernel starts cold."""
+    buf = _FLUSH.get(dev)
+    if buf is None:
+        buf = _FLUSH[dev] = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    buf.fill_(1)
+
+
+def time_main_kernel(pl: Planned, n: int, dev) -> dict:
+    """The main decode kernel alone, over n launches (cycling through the
+    planned steps' decodes), each between CUDA events that the library
+    records on the launching stream around that kernel, with L2 flushed
+    before every launch (outside the events)."""
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    r, sh = pl.runner, pl.sh
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    alg = []
+    for i in range(n + 2):
+        j = i % len(pl.plans)
+        d, q = pl.decodes[j], pl.dev_in[j][2]
+        flush_l2(dev)
+        if i >= 2:
+            pa.set_profile_events(*evs[i - 2])
+        pa.pa_decode(pl.out, q, r.k_cache, r.v_cache, d.dev["tables"], d.dev["lens"], r.scale,
+                     max_seq_len=d.max_len, partition_size=d.partition, variant=r.variant)
+        if i >= 2:
+            pa.set_profile_events(None, None)
+            alg.append(pl.alg_bytes(j))
+    torch.cuda.synchronize()
+    us = [b.elapsed_time(e) * 1e3 for b, e in evs]
+    return {"us": us, "alg": alg}
+
+
+def roofline_of(main: dict, peak: float, peak_src: str, traffic) -> dict:
+    us = np.asarray(main["us"])
+    per_launch = float(np.mean(main["alg"]))
+    # bytes over time launch by launch, averaged: the launches differ in size
+    achieved = float(np.sum(main["alg"]) / np.sum(us) / 1e3)
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "kernel": "pa_decode main (decode_tc_kernel)", "peak_source": peak_src,
+            "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+            "main_us_per_launch": round(float(us.mean()), 2),
+            "main_us_median": round(float(np.median(us)), 2),
+            "timed_launches": int(us.size),
+            "main_us_p10_median_p90": [round(float(np.percentile(us, q)), 2)
+                                       for q in (10, 50, 90)],
+            "l2": "flushed before every timed launch",
+            "algorithmic_bytes_per_launch": int(per_launch)}
+
+
 def run_ours(args, ws, rank, local):
     from paged_kv_cache_347_b200 import pagedattn as pa
-    from paged_kv_cache_347_b200.runner import PagedKVRunner
 
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    seed = rank_seed({"long32k": 2, "llama8b": 1}.get(args.workload, 4), rank)
+    seed = rank_seed(SEEDS.get(args.workload, 4), rank)
     n_plan = min(args.steps + args.warmup, 64)
-    wl, width = make_workload(args.workload, n_plan, seed, args.batch)
-    sh = wl.shape
-    runner = PagedKVRunner.for_shape(sh, width, device=str(dev), partition_size=args.partition)
-    steps = list(wl.steps)
-    prefill, dec = steps[0], steps[1:]
-    runner.run(prefill)                                   # untimed prefill
-    torch.cuda.synchronize()
-    ast = runner.alloc.stats()
-    alloc_info = {"block_size": sh.block_size, "used_blocks": ast["used_blocks"],
-                  "reserved_slots": ast["reserved_slots"], "logical_tokens": ast["logical_tokens"],
-                  "tail_waste_frac": round(1 - ast["logical_tokens"] / max(1, ast["reserved_slots"]),
-                                           5)}
-
-    # plan every decode step (host allocator) and stage its inputs in HBM
-    plans = []
-    alloc_t = time.perf_counter()
-    for st in dec:
-        plans.append(runner.plan(st.ops))
-    alloc_us = (time.perf_counter() - alloc_t) / len(dec) * 1e6
-    for acts, st in zip(plans, dec):
-        runner.upload(acts)
-    dev_in = [(st.k_new.to(dev), st.v_new.to(dev), st.q.to(dev)) for st in dec]
-    b = dec[0].q.shape[0]
-    out = torch.empty((b, sh.num_heads, sh.head_dim), dtype=torch.float32, device=dev)
-    step_bytes = []
-    for acts in plans:
-        d = [a for a in acts if a.kind == "decode"][0]
-        step_bytes.append(kv_bytes(d.lens, sh.num_kv_heads, sh.head_dim, sh.elem_bytes))
-    launches_per = []
-    for acts in plans:
-        n = 0
-        for a in acts:
-            if a.kind == "write":
-                n += (1 if len(a.pairs) else 0) + (1 if a.nrows else 0)
-            else:
-                n += 1 + (1 if math.ceil(a.max_len / (a.partition or 512)) > 1 else 0)
-        launches_per.append(n)
-
-    def step(i):
-        j = i % len(plans)
-        k, v, q = dev_in[j]
-        runner.execute(plans[j], k, v, q, out=out)
+    pl = Planned(args.workload, n_plan, seed, dev, args.batch, args.partition)
+    sh, plans, b = pl.sh, pl.plans, pl.b
 
     # warm-up (the first W planned steps, then cycling)
     for i in range(args.warmup):
-        step(i)
+        pl.step(i)
     torch.cuda.synchronize()
 
-    n_ev = args.steps
-    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
-    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[0])
                           if os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")[0].isdigit()
@@ -333,25 +435,21 @@ def run_ours(args, ws, rank, local):
     t_start.record()
     total_bytes = 0
     launches = 0
-    sampled = []
+    # nothing but the steps between the two events: an event between two
+    # kernels would stop the second launching as a programmatic dependent
     for i in range(args.steps):
-        # events between kernels cost the step its programmatic-dependent-launch
-        # overlap, so the main kernel is timed on every PROFILE_EVERY-th step
-        if i % PROFILE_EVERY == 0:
-            pa.set_profile_events(ev_b[i], ev_e[i])
-            sampled.append(i)
-        step(args.warmup + i)
-        if i % PROFILE_EVERY == 0:
-            pa.set_profile_events(None, None)
-        total_bytes += step_bytes[(args.warmup + i) % len(plans)]
-        launches += launches_per[(args.warmup + i) % len(plans)]
+        pl.step(args.warmup + i)
+        total_bytes += pl.step_bytes[(args.warmup + i) % len(plans)]
+        launches += pl.launches_per[(args.warmup + i) % len(plans)]
     t_end.record()
     torch.cuda.synchronize()
+    # the main kernel alone, after the steps (its own launches, not counted
+    # in gpu_launches); still inside the clock record
+    main = time_main_kernel(pl, max(16, args.main_launches), dev)
     clocks.mark("t1")
     barrier(ws)
     clk = clocks.stop()
     elapsed = t_start.elapsed_time(t_end) / 1e3
-    main_ms = [ev_b[i].elapsed_time(ev_e[i]) for i in sampled]
     errs = pa.device_errors(clear=True)
     if errs:
         raise SystemExit(f"device errors during the bench: {errs}")
@@ -360,34 +458,13 @@ def run_ours(args, ws, rank, local):
     value = bytes_all / elapsed_max / 1e9
     ms_per_step = elapsed_max / args.steps * 1e3
 
-    # roofline of the main decode kernel
     peak, peak_src = hbm_peak()
-    d0 = [a for a in plans[0] if a.kind == "decode"][0]
-    mean_main_s = float(np.mean(main_ms)) / 1e3
-    alg = []
-    for i in sampled:
-        acts = plans[(args.warmup + i) % len(plans)]
-        d = [a for a in acts if a.kind == "decode"][0]
-        nb = int(sum(-(-int(x) // sh.block_size) for x in d.lens))
-        alg.append(kv_bytes(d.lens, sh.num_kv_heads, sh.head_dim, sh.elem_bytes)
-                   + b * sh.num_heads * sh.head_dim * sh.elem_bytes + nb * 4 + b * 4)
-    alg_per_launch = float(np.mean(alg))
-    achieved = alg_per_launch / mean_main_s / 1e9
-    traffic = traffic_from_profile(os.path.join(ROOT, "paged_kv_cache_347_b200", "csrc",
-                                                "decode_tc.cu"), args.workload)
-    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "traffic": traffic,
-            "kernel": "pa_decode main (decode_tc_kernel)", "peak_source": peak_src,
-            "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
-            "main_us_per_launch": round(mean_main_s * 1e6, 2),
-            "timed_launches": len(main_ms),
-            "main_us_p10_median_p90": [round(float(np.percentile(main_ms, q)) * 1e3, 2)
-                                       for q in (10, 50, 90)],
-            "algorithmic_bytes_per_launch": int(alg_per_launch)}
+    traffic = traffic_from_profile(args.workload, float(np.mean(main["alg"])))
+    roof = roofline_of(main, peak, peak_src, traffic)
 
     # end to end through the public API with host buffers
-    e2e = run_e2e(args, sh, width, seed, prefill, dev, ws)
-
+    e2e = run_e2e(args, sh, pl.width, seed, pl.prefill, dev, ws)
+    seq_len = int(max(int(max(d.lens)) for d in pl.decodes))
     res = {
         "metric": "paged decode attention: KV-read GB/s (% of B200 HBM peak), us/step",
         "value": round(value, 1), "unit": "GB/s", "n_gpus": ws, "steps": args.steps,
@@ -398,19 +475,20 @@ def run_ours(args, ws, rank, local):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1), numpy PCG64, rounded to bf16)",
         "config": {"workload": f"{args.workload}: {DESCR.get(args.workload, args.workload)}",
-                   "global_batch": b * ws,
-                   "seq_len": int(max(int(max(a.lens)) for acts in plans for a in acts
-                                      if a.kind == "decode")),
+                   "global_batch": b * ws, "seq_len": seq_len,
                    "parallelism": f"dp{ws} (independent batches, no collective)",
                    "l2": "inputs larger than L2 (KV cache 1.07 GB per step), no flush",
-                   "planned_steps": len(plans), "host_alloc_us_per_step": round(alloc_us, 2),
-                   "partition_tokens": sorted({a.partition or 512 for acts in plans
-                                               for a in acts if a.kind == "decode"}),
+                   "planned_steps": len(plans), "host_alloc_us_per_step": round(pl.alloc_us, 2),
+                   "partition_tokens": pl.partitions(),
                    "partition_policy": {-1: "per step, pa_decode_partition_for",
                                         0: "library default"}.get(args.partition, "fixed"),
-                   "allocator_after_prefill": alloc_info},
+                   "allocator_after_prefill": pl.alloc_info},
         "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
     }
+    pl.close()
+    if rank == 0 and ws == 1 and not args.no_configs:
+        res["configs"] = {name: measure_config(name, args, dev, peak)
+                          for name in CONFIG_LINES}
     if rank == 0 and ws == 1 and not args.no_prefill:
         # the chunked-prefill kernel (tensor-core bound), timed apart from the
         # decode steps above
@@ -434,6 +512,58 @@ def run_ours(args, ws, rank, local):
                                          f"{pairs} (sequence, head) pairs, fp64 C loop, "
                                          f"{secs:.1f} s"}
     return res
+
+
+# The other configurations, measured on the default N = 1 run next to the
+# headline workload: (planned decode steps, timed steps, e2e steps).
+CONFIG_LINES = {"llama8b": (24, 24, 24), "beam": (24, 24, 24), "mix_bs16": (32, 32, 32)}
+
+
+def measure_config(name: str, args, dev, peak: float) -> dict:
+    """One configuration: device step time (each step between CUDA events,
+    L2 flushed before it, outside the events), the main kernel alone over 16+
+    launches, and end to end through the public API."""
+    n_plan, n_steps, n_e2e = CONFIG_LINES[name]
+    seed = SEEDS.get(name, 4)
+    pl = Planned(name, n_plan + 3, seed, dev, 0, args.partition)
+    for i in range(3):
+        pl.step(i)
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_steps)]
+    kv = 0
+    for i in range(n_steps):
+        flush_l2(dev)
+        evs[i][0].record()
+        pl.step(3 + i)
+        evs[i][1].record()
+        kv += pl.step_bytes[(3 + i) % len(pl.plans)]
+    torch.cuda.synchronize()
+    step_us = [b_.elapsed_time(e_) * 1e3 for b_, e_ in evs]
+    main = time_main_kernel(pl, 16, dev)
+    roof = roofline_of(main, peak, "", None)
+    sh = pl.sh
+    e2e_args = argparse.Namespace(**vars(args))
+    e2e_args.workload, e2e_args.steps, e2e_args.e2e_steps, e2e_args.batch = name, n_e2e, n_e2e, 0
+    e2e_args.warmup = 3
+    e2e = run_e2e(e2e_args, sh, pl.width, seed, pl.prefill, dev, 1)
+    mean_step = float(np.mean(step_us))
+    out = {"workload": DESCR.get(name, name), "steps": n_steps,
+           "us_per_step": round(mean_step, 2),
+           "kv_GBs_step": round(kv / (mean_step * 1e-6 * n_steps) / 1e9, 1),
+           "main_us": roof["main_us_per_launch"], "main_GBs": roof["achieved"],
+           "main_frac_of_peak": roof["frac"], "main_timed_launches": roof["timed_launches"],
+           "partition_tokens": pl.partitions(),
+           "tokens_per_s": round(pl.b / (mean_step * 1e-6), 1),
+           "e2e_us_per_step": e2e["us_per_step"], "e2e": e2e,
+           "host_alloc_us_per_step": round(pl.alloc_us, 2),
+           "l2": "flushed before every timed step and launch"}
+    if name == "beam":
+        out["note"] = ("16 beams' unique K/V (51 MB) fits in L2: GB/s are logical bytes "
+                       "(each beam's reads), not HBM traffic; the first decode step, with "
+                       "its 12 copy-on-write copies, is a warm-up step")
+    pl.close()
+    return out
 
 
 def run_e2e(args, sh, width, seed, prefill, dev, ws):
@@ -516,7 +646,7 @@ def run_reference(args, ws, rank):
     """The oracle as it stands on the host cores, on a bounded sample per step."""
     if rank != 0:
         return None
-    seed = {"long32k": 2, "llama8b": 1}.get(args.workload, 4)
+    seed = SEEDS.get(args.workload, 4)
     smp = OracleSampler(args.workload, seed)
     # calibrate, then size each step so the whole run takes about two minutes
     _, secs1, pairs1 = smp.run(0.0)
@@ -762,6 +892,10 @@ def main():
                     help="split length in tokens: -1 chosen per step from the lengths "
                          "(pa_decode_partition_for), 0 the library default (512), or a "
                          "multiple of 64 in [64, 1024]")
+    ap.add_argument("--main-launches", type=int, default=32,
+                    help="launches of the main decode kernel timed alone after the steps")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other configurations' lines (Llama-8B-shaped, beam, mix)")
     ap.add_argument("--batch", type=int, default=0,
                     help="override the workload's batch (small cases for profiling)")
     args = ap.parse_args()

@@ -38,6 +38,12 @@
  *     on.  pa_device_errors() reads that word.
  *   - All device buffers must be 16-byte aligned and contiguous in the
  *     layouts given below.
+ *   - The library's own device variables (the error word, and the array of
+ *     pa_decode_static) are located once per device, on the first call that
+ *     needs them, and their addresses are kept.  Do not go on using the
+ *     library in a process after cudaDeviceReset (or anything else that
+ *     destroys the device's primary context): the kept addresses would
+ *     then point into a context that no longer exists.
  *   - Supported: head_dim D in {64, 128}; block_size bs in {4, 8, 16, 32, 64};
  *     num_heads / num_kv_heads = G in 1..8; dtype f32, bf16, f16.  Anything
  *     else returns PA_ERR_UNSUPPORTED.
@@ -232,7 +238,8 @@ int pa_prefill_ex(float *out, const void *q, const void *k_cache, const void *v_
  *     tokens at head_dim 128 need 17 MB); larger requests return
  *     PA_ERR_INVALID_ARG before anything is launched.
  *   - The first call on a device looks up the array's device address (with
- *     that device current); make that first call before any stream capture.
+ *     that device current) and keeps it; make that first call before any
+ *     stream capture, and do not use the call after cudaDeviceReset.
  *   - Every call shares the one array and it keeps the last call's contents;
  *     nothing in it needs to start at zero.  Calls that overlap on the GPU
  *     (e.g. on two streams at once) race on it: serialise them.

@@ -93,8 +93,10 @@ static int partition_or_default(int partition_size) {
     return partition_size == 0 ? kDefaultPartition : partition_size;
 }
 
+// Splits of `partition` tokens covering max_seq_len (in 64-bit: max_seq_len
+// may be close to INT_MAX).
 static int splits_for(int max_seq_len, int partition) {
-    return max_seq_len <= 0 ? 1 : (max_seq_len + partition - 1) / partition;
+    return max_seq_len <= 0 ? 1 : (int)(((int64_t)max_seq_len + partition - 1) / partition);
 }
 
 static size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }

@@ -78,6 +78,11 @@ def test_workspace_size():
     units = 8 * 64 * 64
     assert n == units * 128 * 4 + units * 2 * 4
     assert pa.decode_workspace_size(8, 64, 128, 32768, 1024) < n
+    # a length bound near INT_MAX: the split count is formed in 64 bits
+    big = 2 ** 31 - 1
+    splits = -(-big // 512)
+    assert pa.decode_workspace_size(1, 1, 128, big) == (
+        -(-splits * 128 * 4 // 256) * 256 + -(-splits * 2 * 4 // 256) * 256)
 
 
 def test_python_binding_rejects_cpu_tensors():

@@ -112,12 +112,17 @@ def test_long_context_full_sampled():
 
 
 def test_beam_cow_and_decode():
-    """Step 1 makes 12 copy-on-write pairs; caches stay bit-exact; outputs match."""
-    wl = workloads.beam(steps=6)
+    """Step 1 makes 12 copy-on-write pairs; step 15 appends position 2064, so
+    every beam opens its second private block; the caches stay bit-exact
+    after every step and every output matches (mbrenndoerfer.com "Paged
+    Attention > Summary", bullet 4: beams share the prompt's blocks)."""
+    wl = workloads.beam(steps=18)
     errs, gpu, orc = run_parity(wl, table_width=152, compare_cache=True)
-    assert max(errs) <= TOL["f16"], errs
+    assert len(errs) == 18 and max(errs) <= TOL["f16"], errs
     st = gpu.alloc.stats()
-    assert st["used_blocks"] == 4 * (128 + 4 * 1) == orc.alloc.stats()["used_blocks"]
+    # 4 prompts x (128 shared blocks + 4 beams x 2 private blocks)
+    assert st["used_blocks"] == 4 * (128 + 4 * 2) == orc.alloc.stats()["used_blocks"]
+    assert st["shared_blocks"] == 4 * 128
 
 
 @pytest.mark.parametrize("bs", [8, 16, 32, 64])

@@ -1,0 +1,211 @@
+"""Decode edge cases against the fp64 oracle (needs a B200).
+
+Paging must not change the attention result (paweldubiel.com
+"PagedAttention", "Text order is not a memory address") on any input the
+method can meet, so these cases feed what the workload tests never do:
+
+* slots past each sequence's length in its last block, blocks no table
+  names, and table entries past a sequence's last block hold NaN, +Inf or
+  -Inf -- the oracle never reads them and neither may the kernels;
+* logits of magnitude ~1e3 (queries scaled up), where the softmax is nearly
+  one-hot and any missing max subtraction overflows;
+* a scale of 0 (the plain mean of the values) and negative scales (the order
+  of the softmax reversed);
+* lengths on both sides of the 16-token MMA tile, the 32-token stage and the
+  512-token split.
+
+Both decode kernels run every case: variant 1 (CUDA cores, every dtype and
+block size) and variant 2 (tensor cores, 16-bit caches, block size >= 8).
+Tolerances: max-abs 1e-5 for fp32 caches, 3e-3 for bf16 / f16; at logits of
+~1e3 the fp32 caches add the bound that fp32 rounding of the logits itself
+puts on the output (``_fp32_logit_tolerance``)."""
+import numpy as np
+import pytest
+import torch
+
+from parity import TOL
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}
+LENS = [0, 1, 15, 16, 17, 31, 32, 33, 511, 512, 513, 1023, 1025, 1537]
+
+
+@pytest.fixture(scope="module")
+def pa():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from paged_kv_cache_347_b200 import pagedattn
+    pagedattn.device_errors(clear=True)
+    yield pagedattn
+    assert pagedattn.device_errors(clear=True) == []
+
+
+def _case(seed, lens, Hq, Hkv, D, bs, dtype, q_scale=1.0, fill=None):
+    """Host caches, tables and queries.  Every sequence's blocks are drawn from
+    a seeded permutation of the pool; with ``fill``, everything the attention
+    must not read is set to that value: the slots past L in each last block,
+    the blocks that no table names, and one spare block that the table
+    entries past each sequence's last block point to."""
+    nblk = [-(-L // bs) for L in lens]
+    W = max(max(nblk), 1) + 2
+    NB = sum(nblk) + 8
+    perm = workloads.permutation(seed, NB)
+    kc = workloads.normal(seed, (1,), (NB, Hkv, bs, D), dtype)
+    vc = workloads.normal(seed, (2,), (NB, Hkv, bs, D), dtype)
+    q = workloads.normal(seed, (3,), (len(lens), Hq, D), "f32") * q_scale
+    q = q.to(TORCH_DT[dtype])
+    spare = int(perm[-1])
+    tables = np.full((len(lens), W), spare, np.int32)
+    used = set()
+    o = 0
+    for s, n in enumerate(nblk):
+        tables[s, :n] = perm[o:o + n]
+        used.update(int(b) for b in perm[o:o + n])
+        o += n
+    if fill is not None:
+        for b in range(NB):
+            if b not in used:
+                kc[b] = fill
+                vc[b] = fill
+        for s, L in enumerate(lens):
+            if L % bs:
+                last = int(tables[s, (L - 1) // bs])
+                kc[last, :, L % bs:, :] = fill
+                vc[last, :, L % bs:, :] = fill
+    return q, kc, vc, tables, np.asarray(lens, np.int32)
+
+
+def _run(pa, q, kc, vc, tables, lens, scale, variant, partition=0):
+    dev = [t.cuda() for t in (q, kc, vc)]
+    tab = torch.from_numpy(tables).cuda()
+    sl = torch.from_numpy(lens).cuda()
+    out = torch.full(tuple(q.shape), float("nan"), dtype=torch.float32, device="cuda")
+    pa.pa_decode(out, dev[0], dev[1], dev[2], tab, sl, scale, partition_size=partition,
+                 variant=variant)
+    torch.cuda.synchronize()
+    return out.double().cpu().numpy()
+
+
+def _check(got, exp, dtype, what):
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    err = float(np.abs(got - exp).max())
+    assert err <= TOL[dtype], f"{what}: max-abs {err}"
+    return err
+
+
+KERNELS = [(1, "f32", 4), (1, "f32", 16), (1, "bf16", 4), (1, "f16", 16),
+           (2, "bf16", 8), (2, "bf16", 16), (2, "f16", 32), (2, "bf16", 64)]
+
+
+@pytest.mark.parametrize("fill", [float("nan"), float("inf"), float("-inf")])
+@pytest.mark.parametrize("variant,dtype,bs", KERNELS)
+def test_poisoned_slots_are_never_read(pa, variant, dtype, bs, fill):
+    from oracle import attn
+    Hq, Hkv, D = 8, 2, 128
+    q, kc, vc, tables, lens = _case(21, LENS, Hq, Hkv, D, bs, dtype, fill=fill)
+    scale = D ** -0.5
+    exp = attn.paged_decode(q, kc, vc, tables, lens, scale)
+    got = _run(pa, q, kc, vc, tables, lens, scale, variant)
+    _check(got, exp, dtype, f"variant {variant} {dtype} bs {bs} fill {fill}")
+    # an empty sequence still gives zeros next to poisoned neighbours
+    assert np.all(got[0] == 0.0)
+
+
+def _fp32_logit_tolerance(q, kc, vc, tables, lens, scale, G):
+    """Per (sequence, head) bound on what rounding the logits to fp32 does to
+    the output, for fp32 caches.  A perturbation d_t of the logits moves the
+    output by sum_t w_t (d_t - sum_u w_u d_u)(v_t - out), so |d_t| <= eps
+    bounds it by 2 eps sum_t w_t |v_t - out|.  The kernels form each logit as
+    a sum of D products with at most 2 log2(D) + 4 roundings on any path (FMA
+    chains and a shuffle tree), then scale it, shift it by the running maximum
+    and exponentiate; eps = 16 u max_t sum_d |scale q_d k_td| with u = 2^-24
+    covers all of it.  At |logits| ~ 1e3 that is ~1e-3, against rounding
+    effects of ~1e-4 in a float32 emulation of these inputs: the 1e-5 bound
+    stated for N(0, 1) data cannot hold there for any fp32 kernel (half an
+    ulp of 1000.0 in fp32 is already 3e-5)."""
+    from oracle import attn
+    qd, kd, vd = (attn.decode_storage(t) for t in (q, kc, vc))
+    B, Hq, D = qd.shape
+    tol = np.zeros((B, Hq))
+    for s, L in enumerate(lens):
+        for h in range(Hq):
+            if L == 0:
+                continue
+            K = attn.gather_logical(kd, tables[s], int(L), h // G)
+            V = attn.gather_logical(vd, tables[s], int(L), h // G)
+            x = scale * (K @ qd[s, h])
+            w = np.exp(x - x.max())
+            w /= w.sum()
+            out = w @ V
+            eps = 16 * 2.0 ** -24 * float((np.abs(K) @ np.abs(qd[s, h])).max()) * abs(scale)
+            tol[s, h] = 2 * eps * float((w @ np.abs(V - out)).max())
+    return tol
+
+
+@pytest.mark.parametrize("variant,dtype,bs", KERNELS)
+@pytest.mark.parametrize("G", [1, 4, 8])
+def test_logits_of_magnitude_one_thousand(pa, variant, dtype, bs, G):
+    """Queries scaled so that scale * q.k reaches about +-1e3: the softmax is
+    close to one-hot, exp of an unshifted logit would overflow fp32, and the
+    online rescale sees running maxima jump by hundreds.  16-bit caches keep
+    the 3e-3 bound; fp32 caches get 1e-5 plus the fp32 logit-rounding bound
+    of ``_fp32_logit_tolerance``."""
+    from oracle import attn
+    Hkv, D = 2, 128
+    lens = [1, 17, 33, 513, 1100]
+    q, kc, vc, tables, lens = _case(22, lens, G * Hkv, Hkv, D, bs, dtype, q_scale=300.0,
+                                    fill=float("nan"))
+    scale = D ** -0.5
+    qd = attn.decode_storage(q)
+    kd = attn.decode_storage(kc)
+    # the logits really are that large
+    big = max(float(np.abs(scale * attn.gather_logical(kd, tables[s], int(L), 0) @ qd[s, 0]).max())
+              for s, L in enumerate(lens))
+    assert big > 500.0, big
+    exp = attn.paged_decode(q, kc, vc, tables, lens, scale)
+    got = _run(pa, q, kc, vc, tables, lens, scale, variant)
+    assert np.isfinite(got).all()
+    err = np.abs(got - exp).max(axis=2)
+    tol = TOL[dtype]
+    if dtype == "f32":
+        tol = tol + _fp32_logit_tolerance(q, kc, vc, tables, lens, scale, G)
+    assert np.all(err <= tol), (float(err.max()), np.argwhere(err > tol)[:4].tolist())
+
+
+@pytest.mark.parametrize("variant,dtype,bs", KERNELS)
+@pytest.mark.parametrize("scale", [0.0, -0.05, -1.0 / 128 ** 0.5])
+def test_zero_and_negative_scale(pa, variant, dtype, bs, scale):
+    from oracle import attn
+    Hq, Hkv, D = 8, 2, 128
+    lens = [1, 16, 33, 600, 1025]
+    q, kc, vc, tables, lens = _case(23, lens, Hq, Hkv, D, bs, dtype, fill=float("nan"))
+    exp = attn.paged_decode(q, kc, vc, tables, lens, scale)
+    got = _run(pa, q, kc, vc, tables, lens, scale, variant)
+    _check(got, exp, dtype, f"variant {variant} {dtype} bs {bs} scale {scale}")
+    if scale == 0.0:
+        # every weight is 1: the output is the mean of the sequence's values
+        vd = attn.decode_storage(vc)
+        for s, L in enumerate(lens):
+            rows = attn.gather_logical(vd, tables[s], int(L), 0)
+            assert np.abs(got[s, 0] - rows.mean(axis=0)).max() <= TOL[dtype]
+
+
+@pytest.mark.parametrize("variant,dtype,bs", [(1, "f32", 16), (1, "bf16", 8), (2, "bf16", 16),
+                                              (2, "f16", 8)])
+@pytest.mark.parametrize("partition", [64, 512, 1024])
+def test_lengths_around_tiles_stages_and_splits(pa, variant, dtype, bs, partition):
+    """Every length from 1 to 70 (tiles of 16, stages of 32 and 64 tokens)
+    and the lengths on both sides of the split edges, one batch per split
+    length."""
+    from oracle import attn
+    Hq, Hkv, D = 16, 4, 64
+    lens = list(range(0, 71)) + [partition + d for d in (-1, 0, 1)] + \
+           [2 * partition + d for d in (-1, 0, 1)] + [3 * partition - 17]
+    q, kc, vc, tables, lens = _case(24 + partition, lens, Hq, Hkv, D, bs, dtype,
+                                    fill=float("inf"))
+    scale = D ** -0.5
+    exp = attn.paged_decode(q, kc, vc, tables, lens, scale)
+    got = _run(pa, q, kc, vc, tables, lens, scale, variant, partition=partition)
+    _check(got, exp, dtype, f"variant {variant} {dtype} bs {bs} split {partition}")

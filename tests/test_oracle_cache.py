@@ -85,3 +85,56 @@ def test_workload_values_are_seeded_and_rounded():
     big = workloads.normal(5, (9,), (1 << 23,), "f32")
     small = workloads.normal(5, (9,), (1000,), "f32")
     assert torch.equal(big[:1000], small)
+
+
+def test_copy_between_moves_each_source_block_onto_its_destination():
+    """The swap copy (sanketn26 "PagedAttention", "What this does not solve":
+    a preempted request's blocks leave for host memory and come back).  Pairs
+    are (source block, destination block); the expected caches are written out
+    value by value, so a swapped orientation, a copy of the wrong cache or a
+    touched bystander block fails."""
+    # source caches: 3 blocks of [Hkv 1][bs 2][D 2]; block b holds 10*b + i
+    src_k = torch.tensor([[[[0., 1.], [2., 3.]]],
+                          [[[10., 11.], [12., 13.]]],
+                          [[[20., 21.], [22., 23.]]]])
+    src_v = -src_k - 100.
+    # destination caches: 4 blocks, every value 7 (K) and 9 (V)
+    dst_k = torch.full((4, 1, 2, 2), 7.)
+    dst_v = torch.full((4, 1, 2, 2), 9.)
+    src_k0, src_v0 = src_k.clone(), src_v.clone()
+    # source 2 -> destination 0, source 0 -> destination 3; source 1 unused
+    cache_ref.copy_between(dst_k, dst_v, src_k, src_v, [(2, 0), (0, 3)])
+    exp_k = torch.tensor([[[[20., 21.], [22., 23.]]],
+                          [[[7., 7.], [7., 7.]]],
+                          [[[7., 7.], [7., 7.]]],
+                          [[[0., 1.], [2., 3.]]]])
+    exp_v = torch.tensor([[[[-120., -121.], [-122., -123.]]],
+                          [[[9., 9.], [9., 9.]]],
+                          [[[9., 9.], [9., 9.]]],
+                          [[[-100., -101.], [-102., -103.]]]])
+    assert torch.equal(dst_k, exp_k)
+    assert torch.equal(dst_v, exp_v)
+    # the source side is read only
+    assert torch.equal(src_k, src_k0) and torch.equal(src_v, src_v0)
+
+
+def test_copy_between_round_trip_restores_the_blocks_in_new_places():
+    """Out to a host pool and back in to different device blocks: the
+    sequence's rows reappear bit for bit at the new places (16-bit storage,
+    so the copy must be bitwise, not a value conversion)."""
+    g = torch.Generator().manual_seed(3)
+    dev_k = torch.randn(6, 2, 4, 8, generator=g).to(torch.bfloat16)
+    dev_v = torch.randn(6, 2, 4, 8, generator=g).to(torch.bfloat16)
+    host_k = torch.zeros(3, 2, 4, 8, dtype=torch.bfloat16)
+    host_v = torch.zeros(3, 2, 4, 8, dtype=torch.bfloat16)
+    orig_k, orig_v = dev_k.clone(), dev_v.clone()
+    cache_ref.copy_between(host_k, host_v, dev_k, dev_v, [(4, 0), (1, 1), (5, 2)])
+    assert torch.equal(host_k[0].view(torch.int16), orig_k[4].view(torch.int16))
+    assert torch.equal(host_v[2].view(torch.int16), orig_v[5].view(torch.int16))
+    cache_ref.copy_between(dev_k, dev_v, host_k, host_v, [(0, 0), (1, 2), (2, 3)])
+    for new, old in ((0, 4), (2, 1), (3, 5)):
+        assert torch.equal(dev_k[new].view(torch.int16), orig_k[old].view(torch.int16))
+        assert torch.equal(dev_v[new].view(torch.int16), orig_v[old].view(torch.int16))
+    # blocks 1, 4 and 5 were not destinations of the way back in
+    for b in (1, 4, 5):
+        assert torch.equal(dev_k[b].view(torch.int16), orig_k[b].view(torch.int16))

@@ -68,6 +68,33 @@ def test_static_scratch_matches_workspace_decode_twice(pa, dtype):
         assert np.isfinite(err) and err <= tol, err
 
 
+def test_static_call_allocates_no_device_memory(pa):
+    """After a first call (which looks up the array's address), further calls
+    leave the device's free memory and the caching allocator's counters
+    exactly as they were: the partials go to the library's own array."""
+    q, kc, vc, tables, sl, max_len = _case(4, 3, 32, 8, 128, 16, [3000, 700, 2049],
+                                           torch.bfloat16)
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    scale = 128 ** -0.5
+    assert _static(pa, out, q, kc, vc, tables, sl, max_len, scale) == 0
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    stats0 = torch.cuda.memory_stats()
+    for _ in range(3):
+        assert _static(pa, out, q, kc, vc, tables, sl, max_len, scale) == 0
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    stats1 = torch.cuda.memory_stats()
+    assert free1 == free0
+    for key in ("allocation.all.allocated", "segment.all.allocated",
+                "allocated_bytes.all.allocated"):
+        assert stats1.get(key, 0) == stats0.get(key, 0), key
+    ref = torch.empty_like(out)
+    pa.pa_decode(ref, q, kc, vc, tables, sl, scale, max_seq_len=max_len)
+    torch.cuda.synchronize()
+    assert (out - ref).abs().max().item() <= TOL["bf16"]
+
+
 def test_static_scratch_rejects_oversize_requests(pa):
     q, kc, vc, tables, sl, _ = _case(3, 2, 32, 8, 128, 16, [64, 64], torch.bfloat16)
     out = torch.zeros(q.shape, dtype=torch.float32, device="cuda")
@@ -76,5 +103,9 @@ def test_static_scratch_rejects_oversize_requests(pa):
     rc = _static(pa, out, q, kc, vc, big_table, sl, 1 << 20, 0.1)
     assert rc == -1
     assert b"static array" in pa._lib.pa_last_error()
+    # a bound near INT_MAX: the split count is formed in 64 bits and the
+    # request is refused before anything is launched
+    rc = _static(pa, out, q, kc, vc, big_table, sl, 2 ** 31 - 1, 0.1)
+    assert rc in (-1, -2), rc
     torch.cuda.synchronize()
     assert torch.all(out == 0)
