@@ -580,8 +580,10 @@ def run_e2e(args, sh, width, seed, prefill, dev, ws):
     r = PagedKVRunner.for_shape(sh, width, device=str(dev), partition_size=args.partition)
     r.run(steps[0])
     torch.cuda.synchronize()
-    host = [(st.ops, st.k_new.pin_memory(), st.v_new.pin_memory(), st.q.pin_memory())
-            for st in steps[1:]]
+    # a step's host inputs: its events as arrays (pa_step_plan's form; ops it
+    # does not take stay a list), new K/V rows and queries in page-locked memory
+    host = [(r.encode_ops(st.ops) or st.ops, st.k_new.pin_memory(), st.v_new.pin_memory(),
+             st.q.pin_memory()) for st in steps[1:]]
     b = steps[1].q.shape[0]
     # eager steps alternate between two output buffers, as the graphs of the
     # two staging slots do, so that step i+1 never overwrites the output of

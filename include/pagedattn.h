@@ -381,6 +381,80 @@ int pa_seq_block_table(const pa_alloc *a, int64_t seq_id, int32_t *out, int cap,
 int pa_block_tables(const pa_alloc *a, const int64_t *seq_ids, int n_seqs, int32_t *tables_out,
                     int width, int32_t *seq_lens_out);
 
+/* ------------------------------------------------------------------------
+ * One decode step planned in one call.  The pages leave the runtime that
+ * owns the block tables to hand the device what a step needs (sanketn26
+ * "PagedAttention", "Use a runtime that owns the blocks": the runtime, not
+ * the client, keeps the tables and the allocation).  pa_step_plan applies a
+ * step's events to the allocator in order and writes everything the device
+ * work of the step reads -- the slots of the appended tokens, the
+ * copy-on-write pairs, and the decode batch's table rows and lengths -- into
+ * one caller-given host buffer (page-locked, typically), so that the step
+ * crosses to the device in one copy.
+ *
+ * Events: n_events triples {code, x, y} of int64, applied in order:
+ *   {PA_EV_ADD, seq_id, 0}      pa_seq_add
+ *   {PA_EV_FREE, seq_id, 0}     pa_seq_free
+ *   {PA_EV_FORK, parent, child} pa_seq_fork
+ *   {PA_EV_APPEND, seq_id, n}   n new tokens (pa_seq_append); a run of
+ *                               consecutive appends is all or nothing, as in
+ *                               pa_batch_append
+ *   {PA_EV_DECODE, 0, 0}        at most one: the decode batch decode_ids
+ *                               [num_seqs] is read here, after the events
+ *                               before it and before those after it
+ * Stage layout (byte offsets in *out, each 16-byte aligned; they depend only
+ * on the events' kinds and token counts and on num_seqs and width, not on
+ * what the allocator decides):
+ *   off_slots   int64 [n_slots]          slots of every appended token, in
+ *                                        event order (n_slots_pre of them
+ *                                        before the decode event)
+ *   off_pairs   int64 [n_pairs][2]       copy-on-write (src, dst) pairs, in
+ *                                        event order (room for one per append
+ *                                        event; n_pairs_pre before the decode)
+ *   off_tables  int32 [num_seqs][width]  table rows (entries past a table's
+ *                                        length 0), as of the decode event
+ *   off_lens    int32 [num_seqs]         lengths, as of the decode event
+ *   bytes       end of the last array
+ * The device work of the step then follows the events' order: for each run
+ * of consecutive appends its copies, then its rows; the decode at its place
+ * -- so that blocks freed and reused after the decode are not written
+ * before the decode reads them.
+ * pairs_before (host int32 [n_events + 1], or NULL) receives, for each
+ * event, the number of pairs the events before it produced, and the total
+ * last: the pairs of events [i, j) are [pairs_before[i], pairs_before[j]).
+ * A caller that keeps the order of the step's events on the device splits
+ * the appends into runs at every other event, like the op-by-op calls would
+ * (a fork or a free between two appends can make a later copy read, or a
+ * later append reuse, a block written by an earlier one).
+ * stage NULL: only the layout is computed (nothing is applied).  Errors: an
+ * unknown code, more than one decode event, a bad count, or a stage smaller
+ * than out->bytes return PA_ERR_INVALID_ARG before anything is applied; an
+ * event that fails stops the call with its error, out->events_applied = the
+ * index of the first event not applied (for a run of appends, the run's
+ * first event), everything before it stays applied.
+ */
+#define PA_EV_ADD 1
+#define PA_EV_FREE 2
+#define PA_EV_FORK 3
+#define PA_EV_APPEND 4
+#define PA_EV_DECODE 5
+
+typedef struct {
+    int32_t n_slots;        /* appended tokens in the step */
+    int32_t n_slots_pre;    /* of which before the decode event */
+    int32_t n_pairs;        /* copy-on-write pairs */
+    int32_t n_pairs_pre;    /* of which before the decode event */
+    int32_t num_seqs;       /* decode batch rows */
+    int32_t width;          /* table entries per row */
+    int32_t max_seq_len;    /* longest length in the decode batch */
+    int32_t events_applied; /* events applied (all of them on success) */
+    int64_t off_slots, off_pairs, off_tables, off_lens, bytes;
+} pa_step_layout;
+
+int pa_step_plan(pa_alloc *a, const int64_t *events, int n_events, const int64_t *decode_ids,
+                 int num_seqs, int width, void *stage, size_t stage_bytes,
+                 int32_t *pairs_before, pa_step_layout *out);
+
 int pa_alloc_stats(const pa_alloc *a, pa_alloc_stats_t *out);
 
 /* Free list from head to tail into out (host int32, up to cap); *n_out =

@@ -26,6 +26,7 @@
 //
 // Pure host code; no CUDA.
 #include <cstdint>
+#include <climits>
 #include <cstring>
 #include <deque>
 #include <new>
@@ -553,6 +554,135 @@ int pa_block_tables(const pa_alloc *a, const int64_t *seq_ids, int n_seqs, int32
         }
         if (seq_lens_out) seq_lens_out[i] = (int32_t)it->second.len;
     }
+    return PA_OK;
+}
+
+// One step's events in a single call, written straight into the caller's
+// staging buffer (see pagedattn.h): a runtime then hands the device one
+// contiguous copy per step, and the host does no per-sequence work outside
+// this loop.
+int pa_step_plan(pa_alloc *a, const int64_t *events, int n_events, const int64_t *decode_ids,
+                 int num_seqs, int width, void *stage, size_t stage_bytes,
+                 int32_t *pairs_before, pa_step_layout *out) {
+    pa::clear_error();
+    if (!a || !out) return pa::fail(PA_ERR_INVALID_ARG, "allocator or layout is NULL");
+    std::memset(out, 0, sizeof(*out));
+    if (n_events < 0 || (n_events > 0 && !events) || num_seqs < 0 || width < 0 ||
+        (num_seqs > 0 && !decode_ids))
+        return pa::fail(PA_ERR_INVALID_ARG, "bad step arguments");
+    // sizes from the events alone, before anything is applied
+    int64_t n_slots = 0, n_appends = 0;
+    int n_decode = 0;
+    for (int i = 0; i < n_events; ++i) {
+        const int64_t code = events[3 * i], n = events[3 * i + 2];
+        if (code == PA_EV_APPEND) {
+            if (n < 0 || n > INT32_MAX)
+                return pa::fail(PA_ERR_INVALID_ARG, "event %d: token count %lld", i,
+                                (long long)n);
+            n_slots += n;
+            n_appends += 1;
+        } else if (code == PA_EV_DECODE) {
+            n_decode += 1;
+        } else if (code != PA_EV_ADD && code != PA_EV_FREE && code != PA_EV_FORK) {
+            return pa::fail(PA_ERR_INVALID_ARG, "event %d: unknown code %lld", i,
+                            (long long)code);
+        }
+    }
+    if (n_decode > 1) return pa::fail(PA_ERR_INVALID_ARG, "more than one decode event");
+    if (n_decode == 0 && num_seqs > 0)
+        return pa::fail(PA_ERR_INVALID_ARG, "decode rows given without a decode event");
+    if (n_slots > INT32_MAX) return pa::fail(PA_ERR_INVALID_ARG, "too many appended tokens");
+    auto a16 = [](int64_t x) { return (x + 15) & ~int64_t(15); };
+    out->n_slots = (int32_t)n_slots;
+    out->num_seqs = num_seqs;
+    out->width = width;
+    out->off_slots = 0;
+    out->off_pairs = a16(8 * n_slots);
+    out->off_tables = out->off_pairs + a16(16 * n_appends);
+    out->off_lens = out->off_tables + a16(4 * (int64_t)num_seqs * width);
+    out->bytes = out->off_lens + 4 * (int64_t)num_seqs;
+    if (!stage) return PA_OK;  // size query: nothing applied
+    if ((reinterpret_cast<uintptr_t>(stage) & 15u) != 0)
+        return pa::fail(PA_ERR_INVALID_ARG, "stage must be 16-byte aligned");
+    if ((int64_t)stage_bytes < out->bytes)
+        return pa::fail(PA_ERR_INVALID_ARG, "stage of %zu bytes, %lld needed", stage_bytes,
+                        (long long)out->bytes);
+    char *base = static_cast<char *>(stage);
+    int64_t *slots = reinterpret_cast<int64_t *>(base + out->off_slots);
+    int64_t *pairs = reinterpret_cast<int64_t *>(base + out->off_pairs);
+    int32_t *tables = reinterpret_cast<int32_t *>(base + out->off_tables);
+    int32_t *lens = reinterpret_cast<int32_t *>(base + out->off_lens);
+
+    int64_t slot_off = 0;
+    int npairs = 0;
+    std::vector<Undo> run;
+    int i = 0;
+    while (i < n_events) {
+        const int64_t code = events[3 * i], x = events[3 * i + 1], y = events[3 * i + 2];
+        int rc = PA_OK;
+        if (code == PA_EV_APPEND) {
+            // a run of consecutive appends is applied all or nothing
+            const int first = i;
+            const int pairs0 = npairs;
+            run.clear();
+            for (; i < n_events && events[3 * i] == PA_EV_APPEND; ++i) {
+                if (pairs_before) pairs_before[i] = npairs;
+                const int64_t sid = events[3 * i + 1];
+                const int n = (int)events[3 * i + 2];
+                auto it = a->seqs.find(sid);
+                if (it == a->seqs.end()) {
+                    rc = pa::fail(PA_ERR_UNKNOWN_SEQ, "event %d: unknown sequence %lld", i,
+                                  (long long)sid);
+                    break;
+                }
+                int got = 0;
+                Undo u;
+                rc = a->append(it->second, n, slots + slot_off, pairs + 2 * npairs, &got, &u);
+                if (rc != PA_OK) break;
+                if (n > 0) it->second.tracked = false;
+                run.push_back(std::move(u));
+                slot_off += n;
+                npairs += got;
+            }
+            if (rc != PA_OK) {
+                for (auto u = run.rbegin(); u != run.rend(); ++u) a->undo(*u);
+                out->events_applied = first;
+                out->n_pairs = pairs0;
+                return rc;
+            }
+            continue;
+        }
+        if (pairs_before) pairs_before[i] = npairs;
+        if (code == PA_EV_ADD) {
+            rc = pa_seq_add(a, x);
+        } else if (code == PA_EV_FREE) {
+            rc = pa_seq_free(a, x);
+        } else if (code == PA_EV_FORK) {
+            rc = pa_seq_fork(a, x, y);
+        } else {  // PA_EV_DECODE: the batch's rows as they stand here
+            out->n_slots_pre = (int32_t)slot_off;
+            out->n_pairs_pre = npairs;
+            rc = pa_block_tables(a, decode_ids, num_seqs, tables, width, lens);
+            if (rc == PA_OK) {
+                int32_t mx = 0;
+                for (int r = 0; r < num_seqs; ++r) mx = lens[r] > mx ? lens[r] : mx;
+                out->max_seq_len = mx;
+            }
+        }
+        if (rc != PA_OK) {
+            out->events_applied = i;
+            out->n_pairs = npairs;
+            return rc;
+        }
+        ++i;
+    }
+    if (n_decode == 0) {
+        out->n_slots_pre = (int32_t)slot_off;
+        out->n_pairs_pre = npairs;
+    }
+    if (pairs_before) pairs_before[n_events] = npairs;
+    out->n_pairs = npairs;
+    out->events_applied = n_events;
     return PA_OK;
 }
 

@@ -75,6 +75,17 @@ _sig("pa_seq_free", _i, _vp, _i64)
 _sig("pa_seq_block_table", _i, _vp, _i64, _vp, _i, _vp, _vp)
 _sig("pa_block_tables", _i, _vp, _vp, _i, _vp, _i, _vp)
 _sig("pa_alloc_stats", _i, _vp, _c.POINTER(pa_alloc_stats_t))
+
+
+class pa_step_layout(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "n_slots", "n_slots_pre", "n_pairs", "n_pairs_pre", "num_seqs", "width",
+        "max_seq_len", "events_applied")] + [(n, ctypes.c_int64) for n in (
+            "off_slots", "off_pairs", "off_tables", "off_lens", "bytes")]
+
+
+_sig("pa_step_plan", _i, _vp, _vp, _i, _vp, _i, _i, _vp, _sz, _vp, _c.POINTER(pa_step_layout))
+EV_ADD, EV_FREE, EV_FORK, EV_APPEND, EV_DECODE = 1, 2, 3, 4, 5
 _sig("pa_alloc_free_list", _i, _vp, _vp, _i, _vp)
 _sig("pa_alloc_refcount", _i, _vp, _i)
 _sig("pa_seq_add_cached", _i, _vp, _i64, _vp, _i, _vp)
@@ -393,6 +404,36 @@ class BlockAllocator:
                                     None if nt is None else _np_ptr(nt), _np_ptr(slots),
                                     _np_ptr(pairs), ctypes.addressof(ncow)), "pa_batch_append")
         return slots[:total], pairs[:ncow.value]
+
+    def step_layout(self, events: np.ndarray, num_seqs: int, width: int) -> pa_step_layout:
+        """pa_step_plan's layout for these events, without applying them."""
+        ev = np.ascontiguousarray(events, dtype=np.int64).reshape(-1, 3)
+        lay = pa_step_layout()
+        ids = np.zeros(max(num_seqs, 1), np.int64)
+        _check(_lib.pa_step_plan(self._h, _np_ptr(ev), ev.shape[0], _np_ptr(ids), num_seqs,
+                                 width, None, 0, None, ctypes.byref(lay)), "pa_step_plan")
+        return lay
+
+    def step_plan(self, events: np.ndarray, decode_ids: np.ndarray, width: int,
+                  stage: np.ndarray, pairs_before: Optional[np.ndarray] = None
+                  ) -> pa_step_layout:
+        """Applies a step's events (int64 [n, 3]) and writes slots, copy pairs,
+        table rows and lengths into ``stage`` (a uint8 array, e.g. a view of
+        page-locked memory) at the returned layout's offsets; ``pairs_before``
+        (int32 [n + 1]) receives the pair count before each event."""
+        ev = np.ascontiguousarray(events, dtype=np.int64).reshape(-1, 3)
+        ids = np.ascontiguousarray(decode_ids, dtype=np.int64)
+        lay = pa_step_layout()
+        rc = _lib.pa_step_plan(self._h, _np_ptr(ev), ev.shape[0],
+                               _np_ptr(ids) if ids.size else None, ids.size, width,
+                               stage.ctypes.data, stage.nbytes,
+                               None if pairs_before is None else _np_ptr(pairs_before),
+                               ctypes.byref(lay))
+        if rc != 0:
+            err = PagedAttnError(rc, "pa_step_plan")
+            err.layout = lay  # events_applied: where the step stopped
+            raise err
+        return lay
 
     def seq_fork(self, parent: int, child: int) -> None:
         _check(_lib.pa_seq_fork(self._h, parent, child), "pa_seq_fork")

@@ -37,6 +37,38 @@ import torch
 from . import pagedattn as pa
 
 
+def _a256(x: int) -> int:
+    return (x + 255) & ~255
+
+
+@dataclass
+class EncodedStep:
+    """A step's events as pa_step_plan takes them: int64 [n, 3] triples
+    {code, x, y} and the decode batch's sequence ids.  ``segments`` lists, in
+    event order, each run of consecutive appends as ("write", first event,
+    end event, first row, end row) and the decode as ("decode", index)."""
+    events: np.ndarray
+    decode_ids: np.ndarray
+    segments: list = field(default_factory=list)
+
+    def __post_init__(self):
+        codes = self.events[:, 0]
+        rows = np.concatenate([[0], np.cumsum(np.where(codes == pa.EV_APPEND,
+                                                       self.events[:, 2], 0))])
+        i, n = 0, codes.shape[0]
+        while i < n:
+            if codes[i] == pa.EV_APPEND:
+                j = i
+                while j < n and codes[j] == pa.EV_APPEND:
+                    j += 1
+                self.segments.append(("write", i, j, int(rows[i]), int(rows[j])))
+                i = j
+                continue
+            if codes[i] == pa.EV_DECODE:
+                self.segments.append(("decode", i))
+            i += 1
+
+
 @dataclass
 class Action:
     kind: str                            # "write" | "decode" | "prefill" | "swap_out" | "swap_in"
@@ -243,13 +275,42 @@ class PagedKVRunner:
 
     # ------------------------------------------------------------ host-fed steps
     # A step fed from host memory is split in two so that the host work of the
-    # next step (allocator, packing) can run while the GPU works on this one:
-    #   prepare(ops)  -> host only: plan, pack the small arrays into one of two
-    #                    pinned staging buffers;
-    #   launch(...)   -> one copy of the packed arrays, one copy each of the new
-    #                    K/V rows and queries, the kernels, the output copied
-    #                    back into pinned memory -- all asynchronous;
-    #   wait()        -> synchronise the stream (the output is then readable).
+    # next step (allocator, table rows) can run while the GPU works on this one:
+    #   prepare(ops)  -> host only: pa_step_plan applies the step's events and
+    #                    writes slots, copy pairs, table rows and lengths
+    #                    straight into one of two page-locked staging buffers
+    #                    (steps with ops it does not take -- prefix-cached
+    #                    admissions, swaps, prefills -- are planned op by op
+    #                    and packed into the same buffer);
+    #   launch(...)   -> one copy of the staging buffer, one copy each of the
+    #                    new K/V rows and queries, the kernels, the output
+    #                    copied back into page-locked memory -- all asynchronous;
+    #   wait()        -> synchronise (the output is then readable).
+    @staticmethod
+    def encode_ops(ops) -> Optional[EncodedStep]:
+        """The step's events as pa_step_plan takes them, or None when the
+        step has an op that it does not take."""
+        if isinstance(ops, EncodedStep):
+            return ops
+        ev, ids = [], None
+        for op in ops:
+            k = op[0]
+            if k == "append":
+                ev.append((pa.EV_APPEND, op[1], op[2]))
+            elif k == "add":
+                ev.append((pa.EV_ADD, op[1], 0))
+            elif k == "free":
+                ev.append((pa.EV_FREE, op[1], 0))
+            elif k == "fork":
+                ev.append((pa.EV_FORK, op[1], op[2]))
+            elif k == "decode" and ids is None:
+                ev.append((pa.EV_DECODE, 0, 0))
+                ids = np.asarray(op[1], dtype=np.int64)
+            else:
+                return None
+        return EncodedStep(np.asarray(ev, dtype=np.int64).reshape(-1, 3),
+                           np.empty(0, np.int64) if ids is None else ids)
+
     def _staging(self, slot: int, nbytes: int):
         """Pinned host / device buffer pair number ``slot`` (of 2), grown on demand."""
         cur = self._stage[slot]
@@ -257,6 +318,8 @@ class PagedKVRunner:
             n = max(nbytes, 1 << 20)
             if self._stage_ev[slot] is not None:
                 self._stage_ev[slot].synchronize()
+            if self._run_ev[slot] is not None:
+                self._run_ev[slot].synchronize()
             cur = (torch.empty(n, dtype=torch.uint8).pin_memory(),
                    torch.empty(n, dtype=torch.uint8, device=self.device))
             self._stage[slot] = cur
@@ -265,9 +328,65 @@ class PagedKVRunner:
             self._stage_ev[slot].synchronize()  # its previous copy has left the host buffer
         return cur
 
+    def _input_bytes(self, n_rows: int, b: int) -> int:
+        e = torch.tensor([], dtype=self.dtype).element_size()
+        kv = n_rows * self.num_kv_heads * self.head_dim * e
+        return 2 * _a256(kv) + _a256(b * self.num_heads * self.head_dim * e)
+
     def prepare(self, ops) -> dict:
-        """Host half of a step: run the allocator and pack every action's
-        arrays (slots, copy pairs, tables, lengths) into a pinned buffer."""
+        """Host half of a step: the allocator's work and every array the
+        step's kernels read, in a page-locked staging buffer."""
+        enc = self.encode_ops(ops)
+        if enc is None:
+            return self._prepare_ops(ops)
+        b = int(enc.decode_ids.size)
+        lay = self.alloc.step_layout(enc.events, b, self.width)
+        slot = self._next_slot
+        self._next_slot = 1 - slot
+        host, devb = self._staging(slot, _a256(lay.bytes) + self._input_bytes(lay.n_slots, b))
+        hb = host.numpy()
+        pb = np.empty(enc.events.shape[0] + 1, np.int32)
+        lay = self.alloc.step_plan(enc.events, enc.decode_ids, self.width, hb, pb)
+        slots = hb[lay.off_slots:lay.off_slots + 8 * lay.n_slots].view(np.int64)
+        pairs = hb[lay.off_pairs:lay.off_pairs + 16 * lay.n_pairs].view(np.int64).reshape(-1, 2)
+        acts, arrays, offs = [], [], []
+        # device actions in event order: each run of appends is its copies,
+        # then its rows (as op-by-op planning makes them); the decode in place
+        for seg in enc.segments:
+            if seg[0] == "write":
+                _, e0, e1, r0, r1 = seg
+                p0, p1 = int(pb[e0]), int(pb[e1])
+                w = Action("write", slots=slots[r0:r1], pairs=pairs[p0:p1], row0=r0,
+                           nrows=r1 - r0)
+                acts.append(w)
+                if r1 > r0:
+                    arrays.append((w, "slots", w.slots))
+                    offs.append(lay.off_slots + 8 * r0)
+                if p1 > p0:
+                    arrays.append((w, "pairs", w.pairs))
+                    offs.append(lay.off_pairs + 16 * p0)
+            else:
+                tables = hb[lay.off_tables:lay.off_tables + 4 * b * self.width].view(np.int32)
+                tables = tables.reshape(b, self.width)
+                lens = hb[lay.off_lens:lay.off_lens + 4 * b].view(np.int32)
+                d = Action("decode", tables=tables, lens=lens.copy(), max_len=lay.max_seq_len,
+                           partition=self._partition(lens))
+                acts.append(d)
+                arrays += [(d, "tables", tables), (d, "lens", lens)]
+                offs += [lay.off_tables, lay.off_lens]
+        return {"acts": acts, "arrays": arrays, "offs": offs, "bytes": lay.bytes, "slot": slot,
+                "host": host, "dev": devb}
+
+    def _partition(self, lens: np.ndarray) -> int:
+        part = self.partition_size
+        if part < 0:
+            part = pa.decode_partition_for(lens, self.num_kv_heads, self.head_dim,
+                                           self.block_size, self.dtype)
+        return part
+
+    def _prepare_ops(self, ops) -> dict:
+        """prepare() for steps pa_step_plan does not take: plan op by op,
+        then pack the arrays into the staging buffer."""
         acts = self.plan(ops)
         arrays = []
         for a in acts:
@@ -295,6 +414,13 @@ class PagedKVRunner:
         return {"acts": acts, "arrays": arrays, "offs": offs, "bytes": total, "slot": slot,
                 "host": host, "dev": devb}
 
+    def _bind(self, prep: dict) -> None:
+        """Point each action's device arrays into the slot's device buffer."""
+        devb = prep["dev"]
+        for (a, name, arr), off in zip(prep["arrays"], prep["offs"]):
+            dt = torch.int64 if arr.dtype == np.int64 else torch.int32
+            a.dev[name] = devb[off:off + arr.nbytes].view(dt).view(arr.shape)
+
     def launch(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor,
                out_host: torch.Tensor) -> dict:
         """Device half of a step, all asynchronous on the current stream."""
@@ -304,9 +430,7 @@ class PagedKVRunner:
             ev = torch.cuda.Event()
             ev.record()
             self._stage_ev[prep["slot"]] = ev
-        for (a, name, arr), off in zip(prep["arrays"], prep["offs"]):
-            dt = torch.int64 if arr.dtype == np.int64 else torch.int32
-            a.dev[name] = devb[off:off + arr.nbytes].view(dt).view(arr.shape)
+        self._bind(prep)
         dev = [t.to(self.device, non_blocking=True) for t in (k_new, v_new, q)]
         o = self.execute(prep["acts"], *dev)
         ev_run = torch.cuda.Event()
@@ -326,90 +450,95 @@ class PagedKVRunner:
     # ------------------------------------------------------------ graph replay
     # Steps of the same layout (the same action kinds and sizes, no copy-on-
     # write pairs, prepared in the same staging slot) repeat the same device
-    # work on different bytes.  launch_graph() captures that work once per
-    # layout, as three graphs -- one copy of the slot's staging buffer (the
-    # packed arrays and, behind them, the new K/V rows and queries), the
-    # kernels, and the copy of the output back -- and replays them on two copy
-    # streams and the current stream; a decode inside a graph takes the table
-    # capacity as its length bound, so that its grid is fixed.
+    # work on different bytes.  The kernels of a layout are captured once, as
+    # a graph, and the output's copy back as another; a replay copies the
+    # slot's staging buffer and the step's new K/V rows and queries to fixed
+    # places in the slot's device buffer on a copy stream, runs the kernels'
+    # graph on the current stream and the copy back on a second copy stream.
+    # A decode inside a graph takes a length bound of the step's longest
+    # sequence rounded up to a power of two (at least 512 tokens, at most the
+    # table's capacity), so that its grid is fixed while steps change little.
     @staticmethod
     def _graphable(acts) -> bool:
         return (bool(acts) and all(a.kind in ("write", "decode") for a in acts)
                 and not any(a.kind == "write" and len(a.pairs) for a in acts)
                 and sum(a.kind == "decode" for a in acts) == 1)
 
+    def _graph_bound(self, max_len: int) -> int:
+        cap = self.width * self.block_size
+        bound = 512
+        while bound < max_len:
+            bound *= 2
+        return min(bound, cap)
+
     def _graph_key(self, prep: dict, k_new: torch.Tensor, q: torch.Tensor):
         acts = prep["acts"]
         if not self._graphable(acts):
             return None
         layout = tuple((a.kind, a.nrows, None if a.tables is None else a.tables.shape,
-                        a.partition) for a in acts)
-        return (layout, prep["bytes"], prep["slot"], prep["host"].data_ptr(),
+                        a.partition, self._graph_bound(a.max_len) if a.kind == "decode" else 0)
+                       for a in acts)
+        return (layout, prep["bytes"], prep["slot"], prep["dev"].data_ptr(),
                 tuple(k_new.shape), tuple(q.shape), k_new.dtype)
 
-    def _place_inputs(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
-                      q: torch.Tensor) -> None:
-        """Room for the step's new K/V rows and queries in the slot's staging
-        buffer behind its packed arrays (256-byte aligned; the buffers grow,
-        keeping the arrays, when too small), so that a graph step moves all of
-        its inputs with one host-to-device copy."""
+    def _input_views(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
+                     q: torch.Tensor):
+        """Fixed places for the step's new K/V rows and queries in the slot's
+        device buffer, behind its arrays (256-byte aligned; the buffers grow,
+        keeping the arrays, when too small)."""
         total = prep["bytes"]
-        offs, end = [], (total + 255) & ~255
+        offs, end = [], _a256(total)
         for t in (k_new, v_new, q):
             offs.append(end)
-            end = (end + t.nbytes + 255) & ~255
-        if prep["host"].numel() < end:
+            end = _a256(end + t.nbytes)
+        if prep["dev"].numel() < end:
             old = prep["host"]
             prep["host"], prep["dev"] = self._staging(prep["slot"], end)
             prep["host"][:total].copy_(old[:total])
-        prep["in_offs"], prep["in_end"] = offs, end
+        devb = prep["dev"]
+        return [devb[off:off + t.nbytes].view(t.dtype).view(t.shape)
+                for off, t in zip(offs, (k_new, v_new, q))]
+
+    def _copy_in(self, prep: dict, ins, k_new, v_new, q) -> None:
+        """The step's inputs to the device, on the current stream: the
+        staging buffer's arrays, then the new rows and queries straight from
+        the caller's (page-locked) tensors."""
+        total = prep["bytes"]
+        if total:
+            prep["dev"][:total].copy_(prep["host"][:total], non_blocking=True)
+        for dst, src in zip(ins, (k_new, v_new, q)):
+            dst.copy_(src, non_blocking=True)
 
     def _capture(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
-                 q: torch.Tensor) -> dict:
+                 q: torch.Tensor, ins) -> dict:
         dec = [a for a in prep["acts"] if a.kind == "decode"][0]
         g = {"out": torch.empty((dec.tables.shape[0], self.num_heads, self.head_dim),
                                 dtype=torch.float32).pin_memory(),
-             "in_bytes": sum(t.nbytes for t in (k_new, v_new, q))}
-        end, host, devb = prep["in_end"], prep["host"], prep["dev"]
-        # typed host views the later steps of this layout copy their inputs into
-        g["in"] = [host[off:off + t.nbytes].view(t.dtype).view(t.shape)
-                   for off, t in zip(prep["in_offs"], (k_new, v_new, q))]
-        for v, t in zip(g["in"], (k_new, v_new, q)):
-            v.copy_(t)
-        ins = [devb[off:off + t.nbytes].view(t.dtype).view(t.shape)
-               for off, t in zip(prep["in_offs"], (k_new, v_new, q))]
+             "in_bytes": sum(t.nbytes for t in (k_new, v_new, q)), "ins": ins}
         for a in prep["acts"]:
             if a.kind == "decode":
-                a.max_len = self.width * self.block_size
-
-        # three graphs, replayed on three streams so that a step's copies
-        # overlap its neighbours' kernels: copy in (one copy brings the packed
-        # arrays and the new rows and queries), run, copy the output out
-        def body_in():
-            devb[:end].copy_(host[:end], non_blocking=True)
+                a.max_len = self._graph_bound(a.max_len)
 
         def body_run():
-            for (a, name, arr), off in zip(prep["arrays"], prep["offs"]):
-                dt = torch.int64 if arr.dtype == np.int64 else torch.int32
-                a.dev[name] = devb[off:off + arr.nbytes].view(dt).view(arr.shape)
+            self._bind(prep)
             g["o"] = self.execute(prep["acts"], *ins)
 
         def body_out():
             g["out"].copy_(g["o"], non_blocking=True)
 
         # one eager run first (workspace, per-device set-up); it applies this
-        # step, and the replay below applies it again to the same bytes
+        # step, and the replay applies it again to the same bytes
         side = torch.cuda.Stream(self.device)
         side.wait_stream(torch.cuda.current_stream(self.device))
         with torch.cuda.stream(side):
-            body_in()
+            self._copy_in(prep, ins, k_new, v_new, q)
             body_run()
             body_out()
         side.synchronize()
         # the graph writes split partials into the binding's cached workspace:
         # keep that buffer alive for as long as the graph
         g["ws"] = pa.cached_workspace(self.device)
-        for name, body in (("g_in", body_in), ("g_run", body_run), ("g_out", body_out)):
+        for name, body in (("g_run", body_run), ("g_out", body_out)):
             graph = torch.cuda.CUDAGraph()
             with torch.cuda.graph(graph, stream=side, capture_error_mode="thread_local"):
                 body()
@@ -422,31 +551,28 @@ class PagedKVRunner:
 
     def stage_graph(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
                     q: torch.Tensor) -> Optional[dict]:
-        """Host half of a graph step: copy the new K/V rows and queries into
-        the slot's page-locked staging buffer behind the packed arrays
-        (capturing the graph for this step's layout the first time, which runs
-        the step once eagerly).  Safe while the GPU still works on the previous
-        step, whose graph is the other staging slot's.  None when the step's
-        layout has no graph form."""
+        """Graph of this step's layout, captured the first time (which runs
+        the step once eagerly); None when the layout has no graph form.  The
+        step's inputs are remembered for replay_graph, which copies them: they
+        must stay unchanged until the step's "ready" event."""
         if not self._graphable(prep["acts"]):
             return None
-        self._place_inputs(prep, k_new, v_new, q)
+        ins = self._input_views(prep, k_new, v_new, q)
         key = self._graph_key(prep, k_new, q)
         if key in self._graphs and self._graphs[key] is None:
             return None  # this layout failed to capture before: launch eagerly
         g = self._graphs.get(key)
         if g is None:
             try:
-                g = self._capture(prep, k_new, v_new, q)
+                g = self._capture(prep, k_new, v_new, q, ins)
             except RuntimeError as e:  # capture refused: this layout runs eagerly
                 warnings.warn(f"CUDA graph capture failed, launching eagerly: {e}")
                 self._graphs[key] = None
                 torch.cuda.synchronize(self.device)
                 return None
             self._graphs[key] = g
-        else:
-            for v, t in zip(g["in"], (k_new, v_new, q)):
-                v.copy_(t)
+            prep["captured"] = True
+        prep["inputs"] = (k_new, v_new, q)
         return g
 
     def _copy_streams(self):
@@ -470,7 +596,7 @@ class PagedKVRunner:
         if self._run_ev[slot] is not None:
             s_in.wait_event(self._run_ev[slot])
         torch.cuda.set_stream(s_in)
-        g["g_in"].replay()
+        self._copy_in(prep, g["ins"], *prep["inputs"])
         g["ev_in"].record(s_in)
         torch.cuda.set_stream(cur)
         self._stage_ev[slot] = g["ev_in"]  # the host staging buffer is free again after this
