@@ -109,8 +109,9 @@ int pa_reshape_and_cache(const void *k, const void *v, void *k_cache, void *v_ca
                          int head_dim, int block_size, int num_blocks, int dtype, void *stream);
 
 /*
- * Bytes of device workspace pa_decode needs for the split-context partials:
- * 0 when max_seq_len fits one partition.  partition_size 0 means 512.
+ * Bytes of device workspace pa_decode needs for the split-context partials
+ * and the tickets of their in-kernel merge: 0 when max_seq_len fits one
+ * partition.  partition_size 0 means 512.  The workspace needs no clearing.
  */
 size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim, int max_seq_len,
                                 int partition_size);
@@ -124,7 +125,9 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim, int m
  *   out[s][h][:] = sum_t softmax(x)_t * v_cache[pb][g][off][:]
  * L_s == 0 gives zeros.  The context is cut into partitions of
  * `partition_size` tokens (512 by default) processed by separate CTAs; their
- * (max, sum, weighted sum) partials are merged by a second kernel.
+ * (max, sum, weighted sum) partials are merged inside the kernel by the last
+ * CTA of each (sequence, KV head), or by a second kernel when the longest
+ * sequence has many partitions (pa_decode_opt).
  *   out           device, float32 [num_seqs][num_heads][head_dim]
  *   q             device, [num_seqs][num_heads][head_dim], `dtype`
  *   k_cache,v_cache device, [num_blocks][num_kv_heads][block_size][head_dim]
@@ -154,6 +157,39 @@ int pa_decode_ex(float *out, const void *q, const void *k_cache, const void *v_c
                  int max_blocks_per_seq, int num_blocks, int max_seq_len, float scale,
                  int dtype, void *workspace, size_t workspace_bytes, int partition_size,
                  int variant, void *stream);
+
+/*
+ * pa_decode with every tuning choice in one struct (pa_decode_ex is this
+ * call with merge 0).  Fields, 0 meaning the library's choice:
+ *   partition_size  tokens per split, as for pa_decode_ex
+ *   variant         0 automatic, 1 CUDA cores, 2 tensor cores (as pa_decode_ex)
+ *   merge           how a sequence's split partials are combined:
+ *                   1 a separate reduce kernel (one CTA per (sequence, head));
+ *                   2 inside the main kernel: the CTA of a (sequence, KV head)
+ *                     to finish last merges that pair's partials, found with
+ *                     a ticket word in the workspace (no further launch);
+ *                   0 the second when the longest sequence has at most 16
+ *                     splits, else the first
+ *   reserved        must be 0
+ * The tickets carry a tag that changes with every call, so the workspace
+ * never needs clearing; a call that replays with the same tag (a CUDA graph)
+ * finds its tickets reset by its own previous run.  Results agree with the
+ * other merge within fp32 rounding.  Calls sharing one workspace must not
+ * overlap on the GPU (as for the partials themselves).
+ */
+typedef struct {
+    int partition_size;
+    int variant;
+    int merge;
+    int reserved[5];
+} pa_decode_opts;
+
+int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_cache,
+                  const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
+                  int num_heads, int num_kv_heads, int head_dim, int block_size,
+                  int max_blocks_per_seq, int num_blocks, int max_seq_len, float scale,
+                  int dtype, void *workspace, size_t workspace_bytes,
+                  const pa_decode_opts *opts, void *stream);
 
 /*
  * A partition_size for pa_decode_ex, from the sequence lengths as the caller

@@ -101,11 +101,33 @@ static int splits_for(int max_seq_len, int partition) {
 
 static size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Workspace: part_o [B][Hq][S][D] float, then part_ml [B][Hq][S][2] float.
+// Workspace: part_o [B][Hq][S][D] float, part_ml [B][Hq][S][2] float, then
+// the in-kernel merge's tickets, one 64-bit word per (sequence, KV head)
+// (room for B * Hq of them: the KV head count is not an argument here).
+static size_t workspace_part_ml_offset(int num_seqs, int num_heads, int head_dim, int splits) {
+    return round256((size_t)num_seqs * num_heads * splits * head_dim * sizeof(float));
+}
+static size_t workspace_tickets_offset(int num_seqs, int num_heads, int head_dim, int splits) {
+    return workspace_part_ml_offset(num_seqs, num_heads, head_dim, splits) +
+           round256((size_t)num_seqs * num_heads * splits * 2 * sizeof(float));
+}
 static size_t workspace_bytes_for(int num_seqs, int num_heads, int head_dim, int splits) {
     if (splits <= 1) return 0;
-    const size_t units = (size_t)num_seqs * num_heads * splits;
-    return round256(units * head_dim * sizeof(float)) + round256(units * 2 * sizeof(float));
+    return workspace_tickets_offset(num_seqs, num_heads, head_dim, splits) +
+           round256((size_t)num_seqs * num_heads * sizeof(unsigned long long));
+}
+
+// Splits up to which pa_decode merges the partials inside the main kernel
+// (the last CTA of each (sequence, KV head) reads them all); beyond it the
+// reduce kernel, whose many CTAs read the partials in parallel, does it.
+constexpr int kFusedMergeMaxSplits = 16;
+
+// A tag per decode call for the in-kernel merge's tickets (never 0).
+static uint32_t next_merge_tag() {
+    static std::atomic<uint32_t> tag{0};
+    uint32_t t = tag.fetch_add(1, std::memory_order_relaxed) + 1;
+    if (t == 0) t = tag.fetch_add(1, std::memory_order_relaxed) + 1;
+    return t;
 }
 
 }  // namespace pa
@@ -172,7 +194,27 @@ int pa_decode_ex(float *out, const void *q, const void *k_cache, const void *v_c
                  int max_blocks_per_seq, int num_blocks, int max_seq_len, float scale,
                  int dtype, void *workspace, size_t workspace_bytes, int partition_size,
                  int variant, void *stream) {
+    pa_decode_opts o;
+    std::memset(&o, 0, sizeof(o));
+    o.partition_size = partition_size;
+    o.variant = variant;
+    return pa_decode_opt(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads,
+                         num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                         max_seq_len, scale, dtype, workspace, workspace_bytes, &o, stream);
+}
+
+int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_cache,
+                  const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
+                  int num_heads, int num_kv_heads, int head_dim, int block_size,
+                  int max_blocks_per_seq, int num_blocks, int max_seq_len, float scale,
+                  int dtype, void *workspace, size_t workspace_bytes,
+                  const pa_decode_opts *opts, void *stream) {
     clear_error();
+    pa_decode_opts o;
+    std::memset(&o, 0, sizeof(o));
+    if (opts) o = *opts;
+    const int partition_size = o.partition_size, variant = o.variant;
+    if (o.merge < 0 || o.merge > 2) return fail(PA_ERR_INVALID_ARG, "merge %d", o.merge);
     int rc = check_shape(num_kv_heads, head_dim, block_size, dtype);
     if (rc) return rc;
     if (num_heads <= 0 || num_heads % num_kv_heads != 0)
@@ -216,11 +258,17 @@ int pa_decode_ex(float *out, const void *q, const void *k_cache, const void *v_c
     DecodeParams p;
     std::memset(&p, 0, sizeof(p));
     p.out = out;
+    const bool fused = need > 0 && (o.merge == 2 || (o.merge == 0 && splits <= kFusedMergeMaxSplits));
     if (need > 0) {
-        const size_t units = (size_t)num_seqs * num_heads * splits;
-        p.part_o = static_cast<float *>(workspace);
-        p.part_ml = reinterpret_cast<float *>(static_cast<char *>(workspace) +
-                                              round256(units * head_dim * sizeof(float)));
+        char *ws = static_cast<char *>(workspace);
+        p.part_o = reinterpret_cast<float *>(ws);
+        p.part_ml = reinterpret_cast<float *>(
+            ws + workspace_part_ml_offset(num_seqs, num_heads, head_dim, splits));
+        if (fused) {
+            p.tickets = reinterpret_cast<unsigned long long *>(
+                ws + workspace_tickets_offset(num_seqs, num_heads, head_dim, splits));
+            p.tag = next_merge_tag();
+        }
     }
     p.q = q;
     p.k_cache = k_cache;
@@ -264,8 +312,10 @@ int pa_decode_ex(float *out, const void *q, const void *k_cache, const void *v_c
         e = cudaEventRecord(prof.end, st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     }
-    e = launch_decode_reduce(p, st);
-    if (e != cudaSuccess) return cuda_fail(e, "reduce launch");
+    if (!fused) {
+        e = launch_decode_reduce(p, st);
+        if (e != cudaSuccess) return cuda_fail(e, "reduce launch");
+    }
     return PA_OK;
 }
 

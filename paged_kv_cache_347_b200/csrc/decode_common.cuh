@@ -64,4 +64,73 @@ __device__ __forceinline__ void store_unit(const DecodeParams &p, int s, int h, 
     }
 }
 
+// ---------------------------------------------------------------- in-kernel merge
+// The split-context partials of a (sequence, KV head) can be merged by the
+// main kernel itself: the CTA of that pair to finish last merges them (the
+// online-softmax rescale of mbrenndoerfer.com "Paged Attention > Summary",
+// bullet 3, applied to whole splits).  Which CTA is last is decided by a
+// ticket word in the workspace.  Its high half carries a tag that changes
+// with every call, so the word never has to be cleared: a word left by an
+// earlier call (or any old bytes) carries another tag and counts as zero.
+// The last CTA leaves the count at zero under its own tag, so a CUDA graph
+// that replays a call with the same tag counts from zero again.
+
+// Counts this CTA's split as done; true for the CTA that completes the
+// count.  One thread per CTA, after every thread's partial stores and a
+// __threadfence() by each of them.
+__device__ __forceinline__ bool ticket_arrive_last(unsigned long long *t, uint32_t tag,
+                                                   int nsplit) {
+    unsigned long long seen = *reinterpret_cast<volatile unsigned long long *>(t);
+    uint32_t done = 0;
+    for (;;) {
+        done = (uint32_t)(seen >> 32) == tag ? (uint32_t)seen : 0u;
+        const unsigned long long want = ((unsigned long long)tag << 32) | (done + 1u);
+        const unsigned long long got = atomicCAS(t, seen, want);
+        if (got == seen) break;
+        seen = got;
+    }
+    if (done + 1u == (uint32_t)nsplit) {
+        // every other split of this call has arrived: reset the count for a
+        // replay of the same call
+        atomicExch(t, (unsigned long long)tag << 32);
+        __threadfence();
+        return true;
+    }
+    return false;
+}
+
+// out[s][h0 .. h0+G-1][:] from the nsplit partials of those heads: threads
+// tid = 0 .. nthreads-1 of the merging CTA each take float4 columns.  The
+// partials were written by other CTAs of this grid: read through L2 (.cg).
+__device__ __forceinline__ void merge_splits(const DecodeParams &p, int s, int h0, int G,
+                                             int nsplit, int tid, int nthreads) {
+    const int D4 = p.head_dim >> 2;
+    for (int c = tid; c < G * D4; c += nthreads) {
+        const int h = h0 + c / D4, d4 = c - (c / D4) * D4;
+        const int64_t u0 = ((int64_t)s * p.num_heads + h) * p.max_splits;
+        const float2 *ml = reinterpret_cast<const float2 *>(p.part_ml) + u0;
+        const float4 *po = reinterpret_cast<const float4 *>(p.part_o + u0 * p.head_dim) + d4;
+        float M = -INFINITY;
+        for (int j = 0; j < nsplit; ++j) M = fmaxf(M, __ldcg(ml + j).x);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float den = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll 8
+            for (int j = 0; j < nsplit; ++j) {
+                const float2 v = __ldcg(ml + j);
+                const float4 o = __ldcg(po + (int64_t)j * D4);
+                const float w = exp2f(v.x - M);
+                den = fmaf(w, v.y, den);
+                acc.x = fmaf(w, o.x, acc.x);
+                acc.y = fmaf(w, o.y, acc.y);
+                acc.z = fmaf(w, o.z, acc.z);
+                acc.w = fmaf(w, o.w, acc.w);
+            }
+        }
+        const float inv = den > 0.f ? 1.f / den : 0.f;
+        reinterpret_cast<float4 *>(p.out + ((int64_t)s * p.num_heads + h) * p.head_dim)[d4] =
+            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    }
+}
+
 }  // namespace pa

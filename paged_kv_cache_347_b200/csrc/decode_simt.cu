@@ -163,6 +163,16 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
         }
         store_unit(p, s, g * G + h, split, nsplit, d, M, den, num);
     }
+    if (p.tickets != nullptr && nsplit > 1) {
+        // the CTA of this (sequence, KV head) to finish last merges the splits
+        __shared__ int last;
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0)
+            last = ticket_arrive_last(p.tickets + (int64_t)s * p.num_kv_heads + g, p.tag, nsplit);
+        __syncthreads();
+        if (last) merge_splits(p, s, g * G, G, nsplit, threadIdx.x, kSimtThreads);
+    }
 }
 
 // Merge of the split partials: one CTA per (query head, sequence) with more

@@ -353,7 +353,17 @@ __global__ void __launch_bounds__(Cfg<T, D, BS, W, NS>::kThreads)
         }
         store_unit(p, s, g * G + h, split, nsplit, d, M, den, num);
     }
-    // this CTA's outputs are written: the reduce may begin launching
+    if (p.tickets != nullptr && nsplit > 1) {
+        // the CTA of this (sequence, KV head) to finish last merges the splits
+        __threadfence();
+        named_barrier_sync(1, W * 32);
+        volatile int *last = abort_flag + 1;
+        if (threadIdx.x == 0)
+            *last = ticket_arrive_last(p.tickets + (int64_t)s * p.num_kv_heads + g, p.tag, nsplit);
+        named_barrier_sync(1, W * 32);
+        if (*last) merge_splits(p, s, g * G, G, nsplit, threadIdx.x, W * 32);
+    }
+    // this CTA's outputs are written: a dependent kernel may begin launching
     pdl_launch_dependents();
 }
 

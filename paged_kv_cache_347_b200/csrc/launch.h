@@ -22,6 +22,11 @@ struct DecodeParams {
     int partition_size;  // tokens per split
     int max_splits;      // S = ceil(max_seq_len / partition_size), >= 1
     float scale_log2;    // softmax scale * log2(e)
+    // In-kernel merge of the split partials (null: the reduce kernel merges):
+    // one ticket per (sequence, KV head), high 32 bits the call's tag, low 32
+    // bits the splits of that call done so far.
+    unsigned long long *tickets;
+    uint32_t tag;
 };
 
 int num_sms();  // SMs of the current device (cached per device)

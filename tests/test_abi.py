@@ -76,13 +76,14 @@ def test_workspace_size():
     assert pa.decode_workspace_size(8, 64, 128, 512) == 0
     n = pa.decode_workspace_size(8, 64, 128, 32768)
     units = 8 * 64 * 64
-    assert n == units * 128 * 4 + units * 2 * 4
+    # partials, then one 8-byte merge ticket per (sequence, head)
+    assert n == units * 128 * 4 + units * 2 * 4 + 8 * 64 * 8
     assert pa.decode_workspace_size(8, 64, 128, 32768, 1024) < n
     # a length bound near INT_MAX: the split count is formed in 64 bits
     big = 2 ** 31 - 1
     splits = -(-big // 512)
     assert pa.decode_workspace_size(1, 1, 128, big) == (
-        -(-splits * 128 * 4 // 256) * 256 + -(-splits * 2 * 4 // 256) * 256)
+        -(-splits * 128 * 4 // 256) * 256 + -(-splits * 2 * 4 // 256) * 256 + 256)
 
 
 def test_python_binding_rejects_cpu_tensors():

@@ -209,3 +209,66 @@ def test_lengths_around_tiles_stages_and_splits(pa, variant, dtype, bs, partitio
     exp = attn.paged_decode(q, kc, vc, tables, lens, scale)
     got = _run(pa, q, kc, vc, tables, lens, scale, variant, partition=partition)
     _check(got, exp, dtype, f"variant {variant} {dtype} bs {bs} split {partition}")
+
+
+# ---------------------------------------------------------------- split merges
+@pytest.mark.parametrize("variant,dtype,bs", [(1, "f32", 16), (1, "bf16", 4), (2, "bf16", 16),
+                                              (2, "f16", 8)])
+@pytest.mark.parametrize("partition", [64, 512])
+def test_in_kernel_merge_and_reduce_kernel_agree_with_the_oracle(pa, variant, dtype, bs,
+                                                                  partition):
+    """Both ways of combining the split partials -- the reduce kernel (merge
+    1) and the last CTA of each (sequence, KV head) inside the main kernel
+    (merge 2) -- on a workspace full of old bytes (the tickets are never
+    cleared), two calls in a row."""
+    from oracle import attn
+    Hq, Hkv, D = 16, 4, 128
+    lens = [0, 1, 63, 64, 65, 700, 1025, 2 * partition + 5, 9 * partition]
+    q, kc, vc, tables, lens = _case(31, lens, Hq, Hkv, D, bs, dtype, fill=float("nan"))
+    scale = D ** -0.5
+    exp = attn.paged_decode(q, kc, vc, tables, lens, scale)
+    dev = [t.cuda() for t in (q, kc, vc)]
+    tab, sl = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+    need = pa.decode_workspace_size(len(lens), Hq, D, tables.shape[1] * bs, partition)
+    ws = torch.randint(0, 256, (need,), dtype=torch.uint8, device="cuda")
+    for merge in (1, 2, 2, 1, 2):
+        out = torch.full(tuple(q.shape), float("nan"), dtype=torch.float32, device="cuda")
+        pa.pa_decode(out, dev[0], dev[1], dev[2], tab, sl, scale, workspace=ws,
+                     partition_size=partition, variant=variant, merge=merge)
+        torch.cuda.synchronize()
+        _check(out.double().cpu().numpy(), exp, dtype, f"merge {merge}")
+
+
+def test_in_kernel_merge_replays_from_a_cuda_graph(pa):
+    """A graph replays the same call (the same ticket tag) with new inputs:
+    each replay finds the tickets its previous run reset, and matches the
+    oracle."""
+    from oracle import attn
+    Hq, Hkv, D, bs = 32, 8, 128, 16
+    lens = [1500, 2049, 33, 4000]
+    q, kc, vc, tables, lens = _case(32, lens, Hq, Hkv, D, bs, "bf16")
+    scale = D ** -0.5
+    dq, dk, dv = (t.cuda() for t in (q, kc, vc))
+    tab, sl = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+    need = pa.decode_workspace_size(len(lens), Hq, D, tables.shape[1] * bs, 512)
+    ws = torch.zeros(need, dtype=torch.uint8, device="cuda")
+    out = torch.empty(tuple(q.shape), dtype=torch.float32, device="cuda")
+    run = lambda: pa.pa_decode(out, dq, dk, dv, tab, sl, scale, workspace=ws, partition_size=512,
+                               merge=2)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        run()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        run()
+    for k in range(3):
+        qk = workloads.normal(40 + k, (3,), tuple(q.shape), "f32").to(q.dtype)
+        dq.copy_(qk)
+        out.fill_(float("nan"))
+        g.replay()
+        torch.cuda.synchronize()
+        exp = attn.paged_decode(qk, kc, vc, tables, lens, scale)
+        _check(out.double().cpu().numpy(), exp, "bf16", f"replay {k}")
+    del g
