@@ -802,7 +802,7 @@ def study_blocksize(args):
         st = r.alloc.stats()
         out["rows"].append({"block_size": bs, "decode_us": round(ms * 1e3, 2),
                             "kv_GBs": round(kvb / ms / 1e6, 1),
-                            "kernel": "tensor-core" if bs >= 8 else "cuda-core",
+                            "kernel": "tensor-core, " + ("cp.async" if bs < 8 else "TMA"),
                             "reserved_slots": st["reserved_slots"],
                             "logical_tokens": st["logical_tokens"],
                             "tail_waste_frac": round(1 - st["logical_tokens"] / st["reserved_slots"], 5),

@@ -149,7 +149,7 @@ int pa_decode(float *out, const void *q, const void *k_cache, const void *v_cach
 /*
  * pa_decode with two tuning knobs: partition_size (0 = 512; else a multiple
  * of 64 in [64, 1024]) and variant (0 = automatic; 1 = the CUDA-core kernel,
- * any dtype; 2 = the tensor-core kernel, bf16/f16 with block_size >= 8).
+ * any dtype; 2 = the tensor-core kernel, bf16/f16 caches).
  */
 int pa_decode_ex(float *out, const void *q, const void *k_cache, const void *v_cache,
                  const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,

@@ -235,8 +235,8 @@ int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_
         return fail(PA_ERR_INVALID_ARG, "partition_size %d: a multiple of 64 in [64, 1024]",
                     partition_size);
     if (variant < 0 || variant > 2) return fail(PA_ERR_INVALID_ARG, "variant %d", variant);
-    if (variant == 2 && (dtype == PA_F32 || block_size < 8))
-        return fail(PA_ERR_UNSUPPORTED, "the tensor-core kernel takes bf16/f16, block_size >= 8");
+    if (variant == 2 && dtype == PA_F32)
+        return fail(PA_ERR_UNSUPPORTED, "the tensor-core kernel takes bf16/f16 caches");
     if (num_seqs == 0) return PA_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens)
         return fail(PA_ERR_INVALID_ARG, "NULL pointer");
@@ -288,11 +288,10 @@ int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_
     p.max_splits = splits;
     p.scale_log2 = scale * 1.4426950408889634f;
 
-    // 16-bit caches with blocks of 8+ rows go to the tensor-core kernel (it
-    // needs the cache to fit 2^31 TMA rows); fp32 and block size 4 to the
-    // CUDA-core kernel.
+    // 16-bit caches go to the tensor-core kernel (it needs the cache to fit
+    // 2^31 TMA rows); fp32 caches to the CUDA-core kernel.
     const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
-    const bool tc_ok = dtype != PA_F32 && block_size >= 8 &&
+    const bool tc_ok = dtype != PA_F32 &&
                        rows + (int64_t)(num_kv_heads + 1) * block_size < (int64_t(1) << 31);
     if (variant == 2 && !tc_ok)
         return fail(PA_ERR_UNSUPPORTED, "cache too large for the tensor-core kernel");
@@ -331,13 +330,17 @@ int pa_decode_partition_for(const int32_t *seq_lens_host, int num_seqs, int num_
     for (int s = 0; s < num_seqs; ++s)
         if (seq_lens_host[s] < 0)
             return fail(PA_ERR_INVALID_ARG, "seq_lens_host[%d] = %d", s, seq_lens_host[s]);
-    if (dtype == PA_F32 || block_size < 8) return kDefaultPartition;  // CUDA-core kernel
+    if (dtype == PA_F32) return kDefaultPartition;  // CUDA-core kernel
     if (slots == 0) {
-        // per device and shape, asked once: [device][bf16|f16][D 64|128][bs 8..64]
-        static std::atomic<int> cache[kMaxDevices][2][2][4];
+        // per device and shape, asked once: [device][bf16|f16][D 64|128][bs 4..64]
+        static std::atomic<int> cache[kMaxDevices][2][2][5];
         const int dev = current_device();
         if (dev < 0 || dev >= kMaxDevices) return fail(PA_ERR_CUDA, "no CUDA device");
-        const int bsi = block_size == 8 ? 0 : block_size == 16 ? 1 : block_size == 32 ? 2 : 3;
+        const int bsi = block_size == 4    ? 4
+                        : block_size == 8  ? 0
+                        : block_size == 16 ? 1
+                        : block_size == 32 ? 2
+                                           : 3;
         std::atomic<int> &c = cache[dev][dtype == PA_F16][head_dim == 128][bsi];
         int per_sm = c.load(std::memory_order_relaxed);
         if (per_sm <= 0) {

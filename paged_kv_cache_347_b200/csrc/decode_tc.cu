@@ -62,6 +62,9 @@ constexpr int kMaxG = 8;
 template <typename T, int D, int BS, int W, int NS>
 struct Cfg {
     static constexpr int kThreads = (W + 1) * 32;
+    // blocks of 4 rows are staged by cp.async from all producer lanes: a TMA
+    // box of 4 rows would start halfway into the 1 KB 128B-swizzle atom
+    static constexpr bool kAsync = BS < 8;
     static constexpr int kStageTokens = 16 * W;
     static constexpr int kPieces = D / 64;                        // 128-byte pieces of a row
     static constexpr int kPieceBytes = kStageTokens * kRowBytes;
@@ -138,7 +141,7 @@ __global__ void __launch_bounds__(Cfg<T, D, BS, W, NS>::kThreads)
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < NS; ++i) {
-            mbar_init(full0 + 8 * i, 1);
+            mbar_init(full0 + 8 * i, C::kAsync ? 32 : 1);
             mbar_init(empty0 + 8 * i, W);
         }
         *abort_flag = 0;
@@ -154,6 +157,50 @@ __global__ void __launch_bounds__(Cfg<T, D, BS, W, NS>::kThreads)
     __syncthreads();
 
     // ------------------------------------------------------------ producer
+    if (C::kAsync && warp == W) {
+        // every lane copies 16-byte chunks of the stage's (block, head) rows
+        // into the layout the TMA boxes give (row r of a 1 KB-aligned piece,
+        // chunk c at c ^ (r mod 8)), then arrives on the stage's barrier once
+        // its copies have landed
+        constexpr int kRowChunks = D / 8;              // 16-byte chunks per row
+        constexpr int kBlockChunks = BS * kRowChunks;  // per cache
+        const uint64_t policy = l2_policy_evict_first();
+        const uint32_t stage0 = smem_u32(smem);
+        const char *kc = static_cast<const char *>(p.k_cache);
+        const char *vc = static_cast<const char *>(p.v_cache);
+        for (int i = 0; i < nstages; ++i) {
+            const int buf = i % NS;
+            if (i >= NS && !warp_wait(empty0 + 8 * buf, ((i / NS) - 1) & 1, abort_flag, lane)) {
+                if (lane == 0) {
+                    raise_device_error(p.err, PA_DEVERR_TIMEOUT);
+                    *abort_flag = 1;
+                }
+                break;
+            }
+            const int jb = i * C::kBlocksPerStage;
+            const int jn = min(C::kBlocksPerStage, nblk - jb);
+            const uint32_t kdst = stage0 + buf * C::kStageBytes;
+            const uint32_t vdst = kdst + C::kKBytes;
+            for (int c = lane; c < jn * kBlockChunks; c += 32) {
+                const int j = c / kBlockChunks, rem = c - j * kBlockChunks;
+                const int r = rem / kRowChunks, ch = rem - r * kRowChunks;
+                const int row = j * BS + r;
+                const uint32_t off = (ch >> 3) * C::kPieceBytes + row * kRowBytes +
+                                     (((ch & 7) ^ (row & 7)) << 4);
+                // an entry out of range (marked num_blocks) reads as zeros
+                const int b = table[jb + j];
+                const bool ok = b < p.num_blocks;
+                const int64_t src = ((((int64_t)(ok ? b : 0) * p.num_kv_heads + g) * BS + r) * D +
+                                     ch * 8) * 2;
+                cp_async_16(kdst + off, kc + src, ok ? 16u : 0u, policy);
+                cp_async_16(vdst + off, vc + src, ok ? 16u : 0u, policy);
+            }
+            cp_async_arrive_noinc(full0 + 8 * buf);
+        }
+        // copies still in flight must land before the CTA may exit
+        cp_async_wait_all();
+        return;
+    }
     if (warp == W) {
         if (lane == 0) {
             prefetch_tensormap(&tmap_k);
@@ -449,6 +496,7 @@ static cudaError_t launch_tc_d(const DecodeParams &p, const CUtensorMap &mk,
     constexpr int W = 2;
     constexpr int NS = D == 128 ? 2 : 4;
     switch (p.block_size) {
+    case 4: return launch_tc_inst<T, D, 4, W, NS>(p, mk, mv, stream);
     case 8: return launch_tc_inst<T, D, 8, W, NS>(p, mk, mv, stream);
     case 16: return launch_tc_inst<T, D, 16, W, NS>(p, mk, mv, stream);
     case 32: return launch_tc_inst<T, D, 32, W, NS>(p, mk, mv, stream);
@@ -479,6 +527,7 @@ template <typename T, int D>
 static int resident_d(int block_size) {
     constexpr int NS = D == 128 ? 2 : 4;
     switch (block_size) {
+    case 4: return resident_inst<T, D, 4, 2, NS>();
     case 8: return resident_inst<T, D, 8, 2, NS>();
     case 16: return resident_inst<T, D, 16, 2, NS>();
     case 32: return resident_inst<T, D, 32, 2, NS>();
@@ -501,7 +550,7 @@ int decode_tc_resident_per_sm(int dtype, int head_dim, int block_size) {
 
 cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, cudaStream_t stream) {
     if (dtype != PA_BF16 && dtype != PA_F16) return cudaErrorNotSupported;
-    if (p.block_size < 8 || p.block_size > 64) return cudaErrorNotSupported;
+    if (p.block_size < 4 || p.block_size > 64) return cudaErrorNotSupported;
     if (p.head_dim != 64 && p.head_dim != 128) return cudaErrorNotSupported;
     if (p.partition_size % 64 != 0 || p.partition_size > tc::kMaxPartition)
         return cudaErrorNotSupported;

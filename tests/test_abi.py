@@ -132,9 +132,11 @@ def test_partition_choice_follows_its_rule(lens, slots):
 
 def test_partition_choice_edge_cases():
     from paged_kv_cache_347_b200 import pagedattn as pa
-    # the CUDA-core kernel (fp32, or 4-row blocks) keeps 512
+    # the CUDA-core kernel (fp32 caches) keeps 512
     assert pa.decode_partition_for([2048] * 32, 8, 128, 16, torch.float32, slots=888) == 512
-    assert pa.decode_partition_for([2048] * 32, 8, 128, 4, torch.bfloat16, slots=888) == 512
+    # 4-row blocks of 16-bit caches take the tensor-core kernel and its rule:
+    # 1024 CTAs of 512 tokens fill 1.15 waves of 888, those of 1024 fit one
+    assert pa.decode_partition_for([2048] * 32, 8, 128, 4, torch.bfloat16, slots=888) == 1024
     assert pa.decode_partition_for([], 8, 128, 16, torch.bfloat16, slots=888) == 512
     with pytest.raises(pa.PagedAttnError):
         pa.decode_partition_for([5, -1], 8, 128, 16, torch.bfloat16, slots=888)

@@ -15,7 +15,8 @@ method can meet, so these cases feed what the workload tests never do:
   512-token split.
 
 Both decode kernels run every case: variant 1 (CUDA cores, every dtype and
-block size) and variant 2 (tensor cores, 16-bit caches, block size >= 8).
+block size) and variant 2 (tensor cores, 16-bit caches; blocks of 4 rows staged
+by cp.async, larger ones by TMA).
 Tolerances: max-abs 1e-5 for fp32 caches, 3e-3 for bf16 / f16; at logits of
 ~1e3 the fp32 caches add the bound that fp32 rounding of the logits itself
 puts on the output (``_fp32_logit_tolerance``)."""
@@ -96,7 +97,8 @@ def _check(got, exp, dtype, what):
 
 
 KERNELS = [(1, "f32", 4), (1, "f32", 16), (1, "bf16", 4), (1, "f16", 16),
-           (2, "bf16", 8), (2, "bf16", 16), (2, "f16", 32), (2, "bf16", 64)]
+           (2, "bf16", 4), (2, "f16", 4), (2, "bf16", 8), (2, "bf16", 16), (2, "f16", 32),
+           (2, "bf16", 64)]
 
 
 @pytest.mark.parametrize("fill", [float("nan"), float("inf"), float("-inf")])
