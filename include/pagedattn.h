@@ -162,7 +162,8 @@ int pa_decode_ex(float *out, const void *q, const void *k_cache, const void *v_c
  * pa_decode with every tuning choice in one struct (pa_decode_ex is this
  * call with merge 0).  Fields, 0 meaning the library's choice:
  *   partition_size  tokens per split, as for pa_decode_ex
- *   variant         0 automatic, 1 CUDA cores, 2 tensor cores (as pa_decode_ex)
+ *   variant         0 automatic, 1 CUDA cores, 2 tensor cores (as pa_decode_ex),
+ *                   3 tensor cores, one KV head per warp (below)
  *   merge           how a sequence's split partials are combined:
  *                   1 a separate reduce kernel (one CTA per (sequence, head));
  *                   2 inside the main kernel: the CTA of a (sequence, KV head)
@@ -170,7 +171,13 @@ int pa_decode_ex(float *out, const void *q, const void *k_cache, const void *v_c
  *                     a ticket word in the workspace (no further launch);
  *                   0 the second when the longest sequence has at most 16
  *                     splits, else the first
+ *   heads_per_cta   variant 3 only: KV heads per CTA (1, 2 or 4; 0 = the
+ *                   library's choice)
  *   reserved        must be 0
+ * Variant 3 is the tensor-core kernel with one KV head per consumer warp: a
+ * CTA takes heads_per_cta adjacent KV heads of one (sequence, partition),
+ * needs num_kv_heads divisible by it and heads_per_cta * max(16,
+ * block_size) <= 64, and has no merge across its warps.
  * The tickets carry a tag that changes with every call, so the workspace
  * never needs clearing; a call that replays with the same tag (a CUDA graph)
  * finds its tickets reset by its own previous run.  Results agree with the
@@ -181,7 +188,8 @@ typedef struct {
     int partition_size;
     int variant;
     int merge;
-    int reserved[5];
+    int heads_per_cta;
+    int reserved[4];
 } pa_decode_opts;
 
 int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_cache,

@@ -234,9 +234,24 @@ int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_
     if (part < 64 || part > 1024 || part % 64 != 0)
         return fail(PA_ERR_INVALID_ARG, "partition_size %d: a multiple of 64 in [64, 1024]",
                     partition_size);
-    if (variant < 0 || variant > 2) return fail(PA_ERR_INVALID_ARG, "variant %d", variant);
-    if (variant == 2 && dtype == PA_F32)
-        return fail(PA_ERR_UNSUPPORTED, "the tensor-core kernel takes bf16/f16 caches");
+    if (variant < 0 || variant > 3) return fail(PA_ERR_INVALID_ARG, "variant %d", variant);
+    if (variant >= 2 && dtype == PA_F32)
+        return fail(PA_ERR_UNSUPPORTED, "the tensor-core kernels take bf16/f16 caches");
+    for (int r : o.reserved)
+        if (r != 0) return fail(PA_ERR_INVALID_ARG, "reserved option fields must be 0");
+    int heads_per_cta = o.heads_per_cta;
+    if (heads_per_cta != 0 && variant != 3)
+        return fail(PA_ERR_INVALID_ARG, "heads_per_cta is an option of variant 3");
+    if (variant == 3) {
+        const int ts = block_size < 16 ? 16 : block_size;  // tokens per stage
+        if (heads_per_cta == 0) heads_per_cta = num_kv_heads % 2 == 0 && 2 * ts <= 64 ? 2 : 1;
+        if ((heads_per_cta != 1 && heads_per_cta != 2 && heads_per_cta != 4) ||
+            num_kv_heads % heads_per_cta != 0 || heads_per_cta * ts > 64)
+            return fail(PA_ERR_UNSUPPORTED,
+                        "heads_per_cta %d: 1, 2 or 4, dividing num_kv_heads %d, with "
+                        "heads_per_cta * max(16, block_size) <= 64",
+                        heads_per_cta, num_kv_heads);
+    }
     if (num_seqs == 0) return PA_OK;
     if (!out || !q || !k_cache || !v_cache || !block_tables || !seq_lens)
         return fail(PA_ERR_INVALID_ARG, "NULL pointer");
@@ -293,8 +308,8 @@ int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_
     const int64_t rows = (int64_t)num_blocks * num_kv_heads * block_size;
     const bool tc_ok = dtype != PA_F32 &&
                        rows + (int64_t)(num_kv_heads + 1) * block_size < (int64_t(1) << 31);
-    if (variant == 2 && !tc_ok)
-        return fail(PA_ERR_UNSUPPORTED, "cache too large for the tensor-core kernel");
+    if (variant >= 2 && !tc_ok)
+        return fail(PA_ERR_UNSUPPORTED, "cache too large for the tensor-core kernels");
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const ProfileEvents prof = t_prof;
     cudaError_t e;
@@ -302,7 +317,9 @@ int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_
         e = cudaEventRecord(prof.begin, st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     }
-    if ((variant == 0 && tc_ok) || variant == 2)
+    if (variant == 3)
+        e = launch_decode_hw(p, dtype, heads_per_cta, st);
+    else if ((variant == 0 && tc_ok) || variant == 2)
         e = launch_decode_tc(p, dtype, st);
     else
         e = launch_decode_simt(p, dtype, st);

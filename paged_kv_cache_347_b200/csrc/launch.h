@@ -51,6 +51,11 @@ cudaError_t launch_decode_simt(const DecodeParams &p, int dtype, cudaStream_t st
 // Tensor-core decode (bf16/f16, block_size >= 8): TMA-staged K/V, mma.sync.
 // Returns cudaErrorNotSupported for shapes it does not cover.
 cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, cudaStream_t stream);
+// Tensor-core decode with one KV head per consumer warp, heads_per_cta (1, 2
+// or 4, dividing num_kv_heads, with heads_per_cta * max(16, block_size) <=
+// 64) heads per CTA.  cudaErrorNotSupported for shapes it does not cover.
+cudaError_t launch_decode_hw(const DecodeParams &p, int dtype, int heads_per_cta,
+                             cudaStream_t stream);
 // CTAs of the tensor-core decode kernel for this shape resident per SM, or -1
 int decode_tc_resident_per_sm(int dtype, int head_dim, int block_size);
 

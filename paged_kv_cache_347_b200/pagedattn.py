@@ -65,7 +65,8 @@ _sig("pa_decode_partition_for", _i, _vp, _i, _i, _i, _i, _i, _i)
 
 class pa_decode_opts(ctypes.Structure):
     _fields_ = [("partition_size", ctypes.c_int), ("variant", ctypes.c_int),
-                ("merge", ctypes.c_int), ("reserved", ctypes.c_int * 5)]
+                ("merge", ctypes.c_int), ("heads_per_cta", ctypes.c_int),
+                ("reserved", ctypes.c_int * 4)]
 
 
 _sig("pa_decode_opt", _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i,
@@ -226,13 +227,16 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
               block_tables: torch.Tensor, seq_lens: torch.Tensor, scale: float,
               block_size: Optional[int] = None, num_kv_heads: Optional[int] = None,
               max_seq_len: Optional[int] = None, workspace: Optional[torch.Tensor] = None,
-              partition_size: int = 0, variant: int = 0, merge: int = 0) -> torch.Tensor:
+              partition_size: int = 0, variant: int = 0, merge: int = 0,
+              heads_per_cta: int = 0) -> torch.Tensor:
     """out float32 [B, Hq, D] <- paged attention of q [B, Hq, D] over the caches.
 
     max_seq_len (a host bound on seq_lens) defaults to the table width times
     the block size.  The workspace for split partials is taken from a cached
-    device buffer unless one is given.  merge: 0 the library's choice, 1 the
-    reduce kernel, 2 inside the main kernel (pa_decode_opt)."""
+    device buffer unless one is given.  variant: 0 automatic, 1 CUDA cores, 2
+    tensor cores, 3 tensor cores with one KV head per warp (heads_per_cta
+    heads per CTA, 0 = the library's choice).  merge: 0 the library's choice,
+    1 the reduce kernel, 2 inside the main kernel (pa_decode_opt)."""
     NB, Hkv, bs, D = k_cache.shape
     if block_size is not None and block_size != bs:
         raise ValueError(f"block_size {block_size} != cache block size {bs}")
@@ -251,7 +255,7 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
         workspace = _workspace(q.device, need)
     ws_ptr = 0 if workspace is None else _dev(workspace, "workspace")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    opts = pa_decode_opts(int(partition_size), int(variant), int(merge))
+    opts = pa_decode_opts(int(partition_size), int(variant), int(merge), int(heads_per_cta))
     _check(_lib.pa_decode_opt(
         _dev(out, "out", torch.float32), _dev(q, "q", k_cache.dtype), _dev(k_cache, "k_cache"),
         _dev(v_cache, "v_cache", k_cache.dtype), _dev(block_tables, "block_tables", torch.int32),

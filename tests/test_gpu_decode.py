@@ -69,7 +69,7 @@ def test_tiny_workload():
     assert gpu.alloc.stats()["used_blocks"] == 9
 
 
-@pytest.mark.parametrize("variant", [1, 2])
+@pytest.mark.parametrize("variant", [1, 2, 3])
 def test_llama_shaped_reduced(variant):
     wl = workloads.llama(batch=6, lo=1, hi=700, steps=3, num_blocks=512)
     errs, _, _ = run_parity(wl, table_width=48, variant=variant, compare_cache=True)
@@ -184,7 +184,8 @@ def test_variants_and_partitions_agree():
                           steps=1)
     steps = list(wl.steps)
     outs = []
-    for variant, part in ((1, 64), (1, 1024), (2, 64), (2, 512), (2, 1024)):
+    for variant, part in ((1, 64), (1, 1024), (2, 64), (2, 512), (2, 1024), (3, 64), (3, 512),
+                          (3, 1024)):
         r = PagedKVRunner.for_shape(wl.shape, 200, partition_size=part, variant=variant)
         out = None
         for st in steps:

@@ -14,9 +14,10 @@ method can meet, so these cases feed what the workload tests never do:
 * lengths on both sides of the 16-token MMA tile, the 32-token stage and the
   512-token split.
 
-Both decode kernels run every case: variant 1 (CUDA cores, every dtype and
-block size) and variant 2 (tensor cores, 16-bit caches; blocks of 4 rows staged
-by cp.async, larger ones by TMA).
+Every decode kernel runs every case: variant 1 (CUDA cores, every dtype and
+block size), variant 2 (tensor cores, 16-bit caches; blocks of 4 rows staged
+by cp.async, larger ones by TMA) and variant 3 (tensor cores, one KV head per
+warp).
 Tolerances: max-abs 1e-5 for fp32 caches, 3e-3 for bf16 / f16; at logits of
 ~1e3 the fp32 caches add the bound that fp32 rounding of the logits itself
 puts on the output (``_fp32_logit_tolerance``)."""
@@ -98,7 +99,8 @@ def _check(got, exp, dtype, what):
 
 KERNELS = [(1, "f32", 4), (1, "f32", 16), (1, "bf16", 4), (1, "f16", 16),
            (2, "bf16", 4), (2, "f16", 4), (2, "bf16", 8), (2, "bf16", 16), (2, "f16", 32),
-           (2, "bf16", 64)]
+           (2, "bf16", 64), (3, "bf16", 4), (3, "f16", 8), (3, "bf16", 16), (3, "f16", 32),
+           (3, "bf16", 64)]
 
 
 @pytest.mark.parametrize("fill", [float("nan"), float("inf"), float("-inf")])
@@ -195,7 +197,8 @@ def test_zero_and_negative_scale(pa, variant, dtype, bs, scale):
 
 
 @pytest.mark.parametrize("variant,dtype,bs", [(1, "f32", 16), (1, "bf16", 8), (2, "bf16", 16),
-                                              (2, "f16", 8)])
+                                              (2, "f16", 8), (3, "bf16", 16), (3, "f16", 4),
+                                              (3, "bf16", 32)])
 @pytest.mark.parametrize("partition", [64, 512, 1024])
 def test_lengths_around_tiles_stages_and_splits(pa, variant, dtype, bs, partition):
     """Every length from 1 to 70 (tiles of 16, stages of 32 and 64 tokens)
@@ -215,7 +218,7 @@ def test_lengths_around_tiles_stages_and_splits(pa, variant, dtype, bs, partitio
 
 # ---------------------------------------------------------------- split merges
 @pytest.mark.parametrize("variant,dtype,bs", [(1, "f32", 16), (1, "bf16", 4), (2, "bf16", 16),
-                                              (2, "f16", 8)])
+                                              (2, "f16", 8), (3, "bf16", 16), (3, "f16", 8)])
 @pytest.mark.parametrize("partition", [64, 512])
 def test_in_kernel_merge_and_reduce_kernel_agree_with_the_oracle(pa, variant, dtype, bs,
                                                                   partition):
@@ -274,3 +277,22 @@ def test_in_kernel_merge_replays_from_a_cuda_graph(pa):
         exp = attn.paged_decode(qk, kc, vc, tables, lens, scale)
         _check(out.double().cpu().numpy(), exp, "bf16", f"replay {k}")
     del g
+
+
+@pytest.mark.parametrize("heads_per_cta", [1, 2, 4])
+@pytest.mark.parametrize("G,Hkv", [(1, 8), (4, 8), (8, 4), (3, 4)])
+def test_heads_per_cta(pa, heads_per_cta, G, Hkv):
+    """Variant 3 with 1, 2 or 4 KV heads per CTA (one per warp) on every
+    GQA group size the tiles hold, against the oracle."""
+    from oracle import attn
+    D, bs = 128, 16
+    lens = [0, 1, 17, 511, 513, 1600]
+    q, kc, vc, tables, lens = _case(33, lens, G * Hkv, Hkv, D, bs, "bf16", fill=float("nan"))
+    scale = D ** -0.5
+    exp = attn.paged_decode(q, kc, vc, tables, lens, scale)
+    dev = [t.cuda() for t in (q, kc, vc)]
+    out = torch.full(tuple(q.shape), float("nan"), dtype=torch.float32, device="cuda")
+    pa.pa_decode(out, dev[0], dev[1], dev[2], torch.from_numpy(tables).cuda(),
+                 torch.from_numpy(lens).cuda(), scale, variant=3, heads_per_cta=heads_per_cta)
+    torch.cuda.synchronize()
+    _check(out.double().cpu().numpy(), exp, "bf16", f"{heads_per_cta} heads per CTA")

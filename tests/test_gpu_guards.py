@@ -83,8 +83,11 @@ def _unchanged(before, after):
     (torch.float32, 4, 64, 2, [5, 9, 14, 700]),                    # CUDA-core kernel
     (torch.bfloat16, 4, 128, 4, [33, 1025]),
 ])
-def test_decode_writes_only_out_and_its_workspace(dtype, bs, D, G, lens):
+@pytest.mark.parametrize("variant,merge", [(0, 1), (0, 2), (3, 2)])
+def test_decode_writes_only_out_and_its_workspace(dtype, bs, D, G, lens, variant, merge):
     from paged_kv_cache_347_b200 import pagedattn as pa
+    if variant == 3 and dtype == torch.float32:
+        pytest.skip("the tensor-core kernels take 16-bit caches")
     B, Hkv = len(lens), 2
     Hq = G * Hkv
     q, kc, vc, tab, sl = _paged_inputs(B, Hq, Hkv, D, bs, lens, dtype, 3)
@@ -97,7 +100,7 @@ def test_decode_writes_only_out_and_its_workspace(dtype, bs, D, G, lens):
     ws = Guarded(((max(need, 16) + 15) // 16 * 4,), torch.float32)
     before = _snap(qg.t, kg.t, vg.t, tab, sl)
     pa.pa_decode(out.t, qg.t, kg.t, vg.t, tab, sl, 0.125, max_seq_len=max_len,
-                 workspace=ws.t if need else None)
+                 workspace=ws.t if need else None, variant=variant, merge=merge)
     assert out.intact() and ws.intact() and qg.intact() and kg.intact() and vg.intact()
     _unchanged(before, _snap(qg.t, kg.t, vg.t, tab, sl))
     assert torch.isfinite(out.t).all()
