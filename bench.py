@@ -62,6 +62,9 @@ sys.path.insert(0, ROOT)
 import workloads  # noqa: E402
 
 NOMINAL_HBM_GBS = 8000.0
+# pa_decode's default merges split partials with a reduce kernel whenever a
+# sequence has more than one split
+FUSED_MERGE_MAX_SPLITS = 1
 FALLBACK_HBM_GBS = 6650.0
 
 
@@ -322,7 +325,8 @@ class Planned:
         self.step_bytes = [kv_bytes(d.lens, sh.num_kv_heads, sh.head_dim, sh.elem_bytes)
                            for d in self.decodes]
         # kernels each step launches: the copy-on-write copy, the append, the
-        # main decode and, when some sequence has more than one split, the reduce
+        # main decode and, when the longest sequence has more splits than the
+        # library merges inside the main kernel, the reduce
         self.launches_per = []
         for acts in self.plans:
             n = 0
@@ -330,7 +334,8 @@ class Planned:
                 if a.kind == "write":
                     n += (1 if len(a.pairs) else 0) + (1 if a.nrows else 0)
                 else:
-                    n += 1 + (1 if math.ceil(a.max_len / (a.partition or 512)) > 1 else 0)
+                    n += 1 + (1 if math.ceil(a.max_len / (a.partition or 512))
+                              > FUSED_MERGE_MAX_SPLITS else 0)
             self.launches_per.append(n)
 
     def step(self, i: int) -> None:

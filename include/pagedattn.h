@@ -125,9 +125,8 @@ size_t pa_decode_workspace_size(int num_seqs, int num_heads, int head_dim, int m
  *   out[s][h][:] = sum_t softmax(x)_t * v_cache[pb][g][off][:]
  * L_s == 0 gives zeros.  The context is cut into partitions of
  * `partition_size` tokens (512 by default) processed by separate CTAs; their
- * (max, sum, weighted sum) partials are merged inside the kernel by the last
- * CTA of each (sequence, KV head), or by a second kernel when the longest
- * sequence has many partitions (pa_decode_opt).
+ * (max, sum, weighted sum) partials are merged by a second kernel (or, on
+ * request, inside the main kernel: pa_decode_opt).
  *   out           device, float32 [num_seqs][num_heads][head_dim]
  *   q             device, [num_seqs][num_heads][head_dim], `dtype`
  *   k_cache,v_cache device, [num_blocks][num_kv_heads][block_size][head_dim]
@@ -169,10 +168,21 @@ int pa_decode_ex(float *out, const void *q, const void *k_cache, const void *v_c
  *                   2 inside the main kernel: the CTA of a (sequence, KV head)
  *                     to finish last merges that pair's partials, found with
  *                     a ticket word in the workspace (no further launch);
- *                   0 the second when the longest sequence has at most 16
- *                     splits, else the first
+ *                   0 the library's choice: the first (the in-kernel merge
+ *                     costs each split CTA a fence and a ticket round trip
+ *                     before its slot frees, and measured no faster)
  *   heads_per_cta   variant 3 only: KV heads per CTA (1, 2 or 4; 0 = the
  *                   library's choice)
+ *   seq_order       device int32 [num_seqs] or NULL: the order in which the
+ *                   grid takes the sequences, a permutation of 0 .. num_seqs-1
+ *                   (an entry outside that range skips its grid row and
+ *                   sets PA_DEVERR_SEQLEN; a sequence no grid row names is
+ *                   left unwritten, or with several splits merged from
+ *                   stale partials).  The kernels' CTAs start roughly in grid
+ *                   order, so longest first (what pa_step_plan writes and
+ *                   pa_decode_order computes) puts short CTAs at the end of
+ *                   the launch, where they fill the tail; out keeps the
+ *                   batch's order whatever the order given.
  *   reserved        must be 0
  * Variant 3 is the tensor-core kernel with one KV head per consumer warp: a
  * CTA takes heads_per_cta adjacent KV heads of one (sequence, partition),
@@ -189,8 +199,17 @@ typedef struct {
     int variant;
     int merge;
     int heads_per_cta;
+    const int32_t *seq_order;
     int reserved[4];
 } pa_decode_opts;
+
+/*
+ * Longest-first order of a decode batch for pa_decode_opts.seq_order, from
+ * the lengths as the caller knows them on the host: order_out[i] is the
+ * batch row of the i-th longest sequence, ties in batch order.  Host only.
+ *   seq_lens_host  host int32 [num_seqs];  order_out  host int32 [num_seqs]
+ */
+int pa_decode_order(const int32_t *seq_lens_host, int num_seqs, int32_t *order_out);
 
 int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_cache,
                   const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
@@ -205,7 +224,11 @@ int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_
  * decode launches one CTA per (sequence, KV head, partition); when the 512-
  * token default gives between one and two waves of the CTAs the device holds
  * at once, the second wave runs part-empty and the kernel's tail grows.  In
- * that case the result is 1024 if its CTAs fit one wave; otherwise it is 512.
+ * that case the result is 1024 if its CTAs fit one wave.  It is 1024 too when
+ * the longest sequence exceeds 512 tokens and twice the shortest: the rule
+ * assumes the grid takes the sequences longest first (pa_decode_order),
+ * whose short CTAs at the end fill the tail, so that fewer, longer splits
+ * save start-ups and partials.  Otherwise it is 512.
  * (One alternative only: a runtime that keys CUDA graphs on the split length
  * then sees it change rarely as its sequences grow.)
  *   seq_lens_host   host, int32 [num_seqs], each >= 0 (a 0 counts as one CTA)
@@ -458,6 +481,9 @@ int pa_block_tables(const pa_alloc *a, const int64_t *seq_ids, int n_seqs, int32
  *   off_tables  int32 [num_seqs][width]  table rows (entries past a table's
  *                                        length 0), as of the decode event
  *   off_lens    int32 [num_seqs]         lengths, as of the decode event
+ *   off_order   int32 [num_seqs]         the batch rows longest first (ties
+ *                                        in batch order), for
+ *                                        pa_decode_opts.seq_order
  *   bytes       end of the last array
  * The device work of the step then follows the events' order: for each run
  * of consecutive appends its copies, then its rows; the decode at its place
@@ -492,7 +518,7 @@ typedef struct {
     int32_t width;          /* table entries per row */
     int32_t max_seq_len;    /* longest length in the decode batch */
     int32_t events_applied; /* events applied (all of them on success) */
-    int64_t off_slots, off_pairs, off_tables, off_lens, bytes;
+    int64_t off_slots, off_pairs, off_tables, off_lens, off_order, bytes;
 } pa_step_layout;
 
 int pa_step_plan(pa_alloc *a, const int64_t *events, int n_events, const int64_t *decode_ids,

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -116,11 +117,6 @@ static size_t workspace_bytes_for(int num_seqs, int num_heads, int head_dim, int
     return workspace_tickets_offset(num_seqs, num_heads, head_dim, splits) +
            round256((size_t)num_seqs * num_heads * sizeof(unsigned long long));
 }
-
-// Splits up to which pa_decode merges the partials inside the main kernel
-// (the last CTA of each (sequence, KV head) reads them all); beyond it the
-// reduce kernel, whose many CTAs read the partials in parallel, does it.
-constexpr int kFusedMergeMaxSplits = 16;
 
 // A tag per decode call for the in-kernel merge's tickets (never 0).
 static uint32_t next_merge_tag() {
@@ -239,6 +235,8 @@ int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_
         return fail(PA_ERR_UNSUPPORTED, "the tensor-core kernels take bf16/f16 caches");
     for (int r : o.reserved)
         if (r != 0) return fail(PA_ERR_INVALID_ARG, "reserved option fields must be 0");
+    if (reinterpret_cast<uintptr_t>(o.seq_order) & 3u)
+        return fail(PA_ERR_INVALID_ARG, "seq_order must be 4-byte aligned");
     int heads_per_cta = o.heads_per_cta;
     if (heads_per_cta != 0 && variant != 3)
         return fail(PA_ERR_INVALID_ARG, "heads_per_cta is an option of variant 3");
@@ -273,7 +271,10 @@ int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_
     DecodeParams p;
     std::memset(&p, 0, sizeof(p));
     p.out = out;
-    const bool fused = need > 0 && (o.merge == 2 || (o.merge == 0 && splits <= kFusedMergeMaxSplits));
+    // the library's choice is the reduce kernel: merging inside the main
+    // kernel costs every split CTA a fence and a ticket round trip before it
+    // frees its slot, which measured no faster on any workload of the bench
+    const bool fused = need > 0 && o.merge == 2;
     if (need > 0) {
         char *ws = static_cast<char *>(workspace);
         p.part_o = reinterpret_cast<float *>(ws);
@@ -302,6 +303,7 @@ int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_
     p.partition_size = part;
     p.max_splits = splits;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.seq_order = o.seq_order;
 
     // 16-bit caches go to the tensor-core kernel (it needs the cache to fit
     // 2^31 TMA rows); fp32 caches to the CUDA-core kernel.
@@ -378,6 +380,15 @@ int pa_decode_partition_for(const int32_t *seq_lens_host, int num_seqs, int num_
     // the split length sees it change rarely as its sequences grow
     const int64_t n0 = ctas(kDefaultPartition);
     if (n0 > slots && n0 <= 2 * (int64_t)slots && ctas(1024) <= slots) return 1024;
+    // lengths that differ by more than 2x: with the grid taking the sequences
+    // longest first (pa_decode_order), the short CTAs at the end fill the
+    // tail, and fewer, longer splits save start-ups and partials
+    int32_t lo = INT32_MAX, hi = 0;
+    for (int s = 0; s < num_seqs; ++s) {
+        lo = seq_lens_host[s] < lo ? seq_lens_host[s] : lo;
+        hi = seq_lens_host[s] > hi ? seq_lens_host[s] : hi;
+    }
+    if (hi > kDefaultPartition && (int64_t)hi > 2 * (int64_t)lo) return 1024;
     return kDefaultPartition;
 }
 

@@ -25,6 +25,7 @@
 //    sequence's blocks move to a pool of host blocks and back.
 //
 // Pure host code; no CUDA.
+#include <algorithm>
 #include <cstdint>
 #include <climits>
 #include <cstring>
@@ -600,7 +601,8 @@ int pa_step_plan(pa_alloc *a, const int64_t *events, int n_events, const int64_t
     out->off_pairs = a16(8 * n_slots);
     out->off_tables = out->off_pairs + a16(16 * n_appends);
     out->off_lens = out->off_tables + a16(4 * (int64_t)num_seqs * width);
-    out->bytes = out->off_lens + 4 * (int64_t)num_seqs;
+    out->off_order = out->off_lens + a16(4 * (int64_t)num_seqs);
+    out->bytes = out->off_order + 4 * (int64_t)num_seqs;
     if (!stage) return PA_OK;  // size query: nothing applied
     if ((reinterpret_cast<uintptr_t>(stage) & 15u) != 0)
         return pa::fail(PA_ERR_INVALID_ARG, "stage must be 16-byte aligned");
@@ -612,6 +614,7 @@ int pa_step_plan(pa_alloc *a, const int64_t *events, int n_events, const int64_t
     int64_t *pairs = reinterpret_cast<int64_t *>(base + out->off_pairs);
     int32_t *tables = reinterpret_cast<int32_t *>(base + out->off_tables);
     int32_t *lens = reinterpret_cast<int32_t *>(base + out->off_lens);
+    int32_t *order = reinterpret_cast<int32_t *>(base + out->off_order);
 
     int64_t slot_off = 0;
     int npairs = 0;
@@ -667,6 +670,7 @@ int pa_step_plan(pa_alloc *a, const int64_t *events, int n_events, const int64_t
                 int32_t mx = 0;
                 for (int r = 0; r < num_seqs; ++r) mx = lens[r] > mx ? lens[r] : mx;
                 out->max_seq_len = mx;
+                rc = pa_decode_order(lens, num_seqs, order);
             }
         }
         if (rc != PA_OK) {
@@ -683,6 +687,17 @@ int pa_step_plan(pa_alloc *a, const int64_t *events, int n_events, const int64_t
     if (pairs_before) pairs_before[n_events] = npairs;
     out->n_pairs = npairs;
     out->events_applied = n_events;
+    return PA_OK;
+}
+
+int pa_decode_order(const int32_t *seq_lens_host, int num_seqs, int32_t *order_out) {
+    pa::clear_error();
+    if (num_seqs < 0 || (num_seqs > 0 && (!seq_lens_host || !order_out)))
+        return pa::fail(PA_ERR_INVALID_ARG, "bad arguments");
+    for (int i = 0; i < num_seqs; ++i) order_out[i] = i;
+    std::stable_sort(order_out, order_out + num_seqs, [&](int32_t x, int32_t y) {
+        return seq_lens_host[x] > seq_lens_host[y];
+    });
     return PA_OK;
 }
 

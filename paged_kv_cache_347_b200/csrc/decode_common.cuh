@@ -7,6 +7,19 @@
 
 namespace pa {
 
+// Sequence worked on by grid row z: seq_order[z] when the caller gave an
+// order, else z; -1 (PA_DEVERR_SEQLEN raised once) for an entry outside
+// [0, num_seqs).
+__device__ __forceinline__ int seq_of(const DecodeParams &p, int z, bool report) {
+    if (p.seq_order == nullptr) return z;
+    const int s = __ldg(p.seq_order + z);
+    if (s < 0 || s >= p.num_seqs) {
+        if (report) raise_device_error(p.err, PA_DEVERR_SEQLEN);
+        return -1;
+    }
+    return s;
+}
+
 // Length of sequence s, or 0 (with PA_DEVERR_SEQLEN raised once per
 // sequence) when it is negative, above max_seq_len or longer than its table.
 __device__ __forceinline__ int checked_seq_len(const DecodeParams &p, int s, bool report) {
@@ -111,6 +124,7 @@ __device__ __forceinline__ void merge_splits(const DecodeParams &p, int s, int h
         const float2 *ml = reinterpret_cast<const float2 *>(p.part_ml) + u0;
         const float4 *po = reinterpret_cast<const float4 *>(p.part_o + u0 * p.head_dim) + d4;
         float M = -INFINITY;
+#pragma unroll 8
         for (int j = 0; j < nsplit; ++j) M = fmaxf(M, __ldcg(ml + j).x);
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         float den = 0.f;

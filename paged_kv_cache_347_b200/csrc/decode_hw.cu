@@ -100,7 +100,9 @@ __global__ void __launch_bounds__(Cfg<T, D, BS, W, NS>::kThreads)
     // launched as a programmatic dependent of the KV append
     pdl_wait_prior_grid();
 
-    const int split = blockIdx.x, s = blockIdx.z;
+    const int split = blockIdx.x;
+    const int s = seq_of(p, blockIdx.z, split == 0 && blockIdx.y == 0 && threadIdx.x == 0);
+    if (s < 0) return;  // uniform over the CTA, before any barrier
     const int h0 = blockIdx.y * W;  // first KV head of the CTA
     const int L = checked_seq_len(p, s, split == 0 && blockIdx.y == 0 && threadIdx.x == 0);
     const int nsplit = num_splits_for(L, p.partition_size);

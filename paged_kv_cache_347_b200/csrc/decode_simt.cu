@@ -35,7 +35,9 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
     __shared__ float sm_m[NW][GM];
     __shared__ float sm_l[NW][GM];
 
-    const int split = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+    const int split = blockIdx.x, g = blockIdx.y;
+    const int s = seq_of(p, blockIdx.z, split == 0 && g == 0 && threadIdx.x == 0);
+    if (s < 0) return;
     const int L = checked_seq_len(p, s, split == 0 && g == 0 && threadIdx.x == 0);
     const int nsplit = num_splits_for(L, p.partition_size);
     if (split >= nsplit) return;

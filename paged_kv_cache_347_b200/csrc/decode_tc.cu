@@ -120,7 +120,9 @@ __global__ void __launch_bounds__(Cfg<T, D, BS, W, NS>::kThreads)
     // (e.g. the KV append) must be complete before any input is read
     pdl_wait_prior_grid();
 
-    const int split = blockIdx.x, g = blockIdx.y, s = blockIdx.z;
+    const int split = blockIdx.x, g = blockIdx.y;
+    const int s = seq_of(p, blockIdx.z, split == 0 && g == 0 && threadIdx.x == 0);
+    if (s < 0) return;  // uniform over the CTA, before any barrier
     const int L = checked_seq_len(p, s, split == 0 && g == 0 && threadIdx.x == 0);
     const int nsplit = num_splits_for(L, p.partition_size);
     if (split >= nsplit) return;  // uniform over the CTA, before any barrier

@@ -27,6 +27,10 @@ struct DecodeParams {
     // bits the splits of that call done so far.
     unsigned long long *tickets;
     uint32_t tag;
+    // Order in which the grid takes the sequences (grid row z works on
+    // sequence seq_order[z]; null: z itself).  A runtime that knows the
+    // lengths passes longest first, so that the last CTAs to start are short.
+    const int32_t *seq_order;
 };
 
 int num_sms();  // SMs of the current device (cached per device)

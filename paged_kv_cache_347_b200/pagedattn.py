@@ -66,7 +66,7 @@ _sig("pa_decode_partition_for", _i, _vp, _i, _i, _i, _i, _i, _i)
 class pa_decode_opts(ctypes.Structure):
     _fields_ = [("partition_size", ctypes.c_int), ("variant", ctypes.c_int),
                 ("merge", ctypes.c_int), ("heads_per_cta", ctypes.c_int),
-                ("reserved", ctypes.c_int * 4)]
+                ("seq_order", ctypes.c_void_p), ("reserved", ctypes.c_int * 4)]
 
 
 _sig("pa_decode_opt", _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i,
@@ -91,7 +91,19 @@ class pa_step_layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "n_slots", "n_slots_pre", "n_pairs", "n_pairs_pre", "num_seqs", "width",
         "max_seq_len", "events_applied")] + [(n, ctypes.c_int64) for n in (
-            "off_slots", "off_pairs", "off_tables", "off_lens", "bytes")]
+            "off_slots", "off_pairs", "off_tables", "off_lens", "off_order", "bytes")]
+
+
+_sig("pa_decode_order", _i, _vp, _i, _vp)
+
+
+def decode_order(seq_lens) -> np.ndarray:
+    """pa_decode_order: batch rows longest first (ties in batch order)."""
+    lens = np.ascontiguousarray(np.asarray(seq_lens), dtype=np.int32).reshape(-1)
+    out = np.empty(max(lens.size, 1), np.int32)
+    _check(_lib.pa_decode_order(lens.ctypes.data if lens.size else None, lens.size,
+                                out.ctypes.data), "pa_decode_order")
+    return out[:lens.size]
 
 
 _sig("pa_step_plan", _i, _vp, _vp, _i, _vp, _i, _i, _vp, _sz, _vp, _c.POINTER(pa_step_layout))
@@ -228,7 +240,7 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
               block_size: Optional[int] = None, num_kv_heads: Optional[int] = None,
               max_seq_len: Optional[int] = None, workspace: Optional[torch.Tensor] = None,
               partition_size: int = 0, variant: int = 0, merge: int = 0,
-              heads_per_cta: int = 0) -> torch.Tensor:
+              heads_per_cta: int = 0, seq_order: Optional[torch.Tensor] = None) -> torch.Tensor:
     """out float32 [B, Hq, D] <- paged attention of q [B, Hq, D] over the caches.
 
     max_seq_len (a host bound on seq_lens) defaults to the table width times
@@ -236,7 +248,9 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
     device buffer unless one is given.  variant: 0 automatic, 1 CUDA cores, 2
     tensor cores, 3 tensor cores with one KV head per warp (heads_per_cta
     heads per CTA, 0 = the library's choice).  merge: 0 the library's choice,
-    1 the reduce kernel, 2 inside the main kernel (pa_decode_opt)."""
+    1 the reduce kernel, 2 inside the main kernel (pa_decode_opt).  seq_order
+    (int32 [B] on the device, a permutation): the order in which the grid
+    takes the sequences, e.g. longest first (decode_order)."""
     NB, Hkv, bs, D = k_cache.shape
     if block_size is not None and block_size != bs:
         raise ValueError(f"block_size {block_size} != cache block size {bs}")
@@ -255,7 +269,13 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
         workspace = _workspace(q.device, need)
     ws_ptr = 0 if workspace is None else _dev(workspace, "workspace")
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    opts = pa_decode_opts(int(partition_size), int(variant), int(merge), int(heads_per_cta))
+    order = None
+    if seq_order is not None:
+        if seq_order.numel() != B:
+            raise ValueError("seq_order must have one entry per sequence")
+        order = _dev(seq_order, "seq_order", torch.int32)
+    opts = pa_decode_opts(int(partition_size), int(variant), int(merge), int(heads_per_cta),
+                          order)
     _check(_lib.pa_decode_opt(
         _dev(out, "out", torch.float32), _dev(q, "q", k_cache.dtype), _dev(k_cache, "k_cache"),
         _dev(v_cache, "v_cache", k_cache.dtype), _dev(block_tables, "block_tables", torch.int32),

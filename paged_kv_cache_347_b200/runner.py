@@ -82,6 +82,7 @@ class Action:
     cu: Optional[np.ndarray] = None      # prefill: int32 [b + 1] row offsets
     max_q: int = 0
     partition: int = 0                   # decode: split length passed to pa_decode
+    order: Optional[np.ndarray] = None   # decode: int32 [b], rows longest first
     dev: dict = field(default_factory=dict)
 
 
@@ -90,7 +91,7 @@ class PagedKVRunner:
                  head_dim: int, dtype: torch.dtype, scale: float, table_width: int,
                  free_order: Optional[Sequence[int]] = None, max_blocks_per_seq: int = 0,
                  device: str = "cuda", partition_size: int = 0, variant: int = 0,
-                 prefill_variant: int = 0):
+                 prefill_variant: int = 0, longest_first: bool = True):
         self.alloc = pa.BlockAllocator(num_blocks, block_size, free_order, max_blocks_per_seq)
         self.device = torch.device(device)
         dims = (num_blocks, num_kv_heads, block_size, head_dim)
@@ -101,6 +102,8 @@ class PagedKVRunner:
         self.dtype, self.scale, self.width = dtype, scale, table_width
         self.partition_size, self.variant = partition_size, variant
         self.prefill_variant = prefill_variant
+        # decode grids take the batch's sequences longest first (seq_order)
+        self.longest_first = longest_first
         # host-fed steps: two staging slots (page-locked host / device buffer
         # pairs), the event after which each slot's host buffer is free, the
         # event after which each slot's device buffer is free, and the graphs
@@ -191,7 +194,9 @@ class PagedKVRunner:
                                                        self.block_size, self.dtype)
                     acts.append(Action("decode", tables=tables, lens=lens,
                                        max_len=int(lens.max()) if lens.size else 0,
-                                       partition=part))
+                                       partition=part,
+                                       order=pa.decode_order(lens) if self.longest_first
+                                       else None))
                 elif kind == "prefill":
                     sids = [x for x, _ in op[1]]
                     ns = np.array([n for _, n in op[1]], np.int32)
@@ -233,6 +238,8 @@ class PagedKVRunner:
                 a.dev["lens"] = put(a.lens)
                 if a.kind == "prefill":
                     a.dev["cu"] = put(a.cu)
+                elif a.order is not None:
+                    a.dev["order"] = put(a.order)
             elif len(a.pairs):
                 a.dev["pairs"] = put(a.pairs)
 
@@ -269,7 +276,8 @@ class PagedKVRunner:
                     (b, self.num_heads, self.head_dim), dtype=torch.float32, device=self.device)
                 pa.pa_decode(o, q, self.k_cache, self.v_cache, a.dev["tables"], a.dev["lens"],
                              self.scale, max_seq_len=a.max_len,
-                             partition_size=a.partition, variant=self.variant)
+                             partition_size=a.partition, variant=self.variant,
+                             seq_order=a.dev.get("order"))
                 res = o
         return res
 
@@ -369,11 +377,16 @@ class PagedKVRunner:
                 tables = hb[lay.off_tables:lay.off_tables + 4 * b * self.width].view(np.int32)
                 tables = tables.reshape(b, self.width)
                 lens = hb[lay.off_lens:lay.off_lens + 4 * b].view(np.int32)
+                order = hb[lay.off_order:lay.off_order + 4 * b].view(np.int32)
                 d = Action("decode", tables=tables, lens=lens.copy(), max_len=lay.max_seq_len,
-                           partition=self._partition(lens))
+                           partition=self._partition(lens),
+                           order=order if self.longest_first else None)
                 acts.append(d)
                 arrays += [(d, "tables", tables), (d, "lens", lens)]
                 offs += [lay.off_tables, lay.off_lens]
+                if self.longest_first:
+                    arrays.append((d, "order", order))
+                    offs.append(lay.off_order)
         return {"acts": acts, "arrays": arrays, "offs": offs, "bytes": lay.bytes, "slot": slot,
                 "host": host, "dev": devb}
 
@@ -399,6 +412,8 @@ class PagedKVRunner:
                 arrays.append((a, "lens", a.lens))
                 if a.kind == "prefill":
                     arrays.append((a, "cu", a.cu))
+                elif a.order is not None:
+                    arrays.append((a, "order", a.order))
             elif len(a.pairs):
                 arrays.append((a, "pairs", a.pairs))
         offs, total = [], 0

@@ -117,16 +117,22 @@ def _ctas(lens, part, hkv):
     ([1024] * 32, 888),                       # 512 CTAs: one wave, keeps 512
     ([0, 1, 511, 512, 513, 4096, 4097] * 20, 700),
     (list(range(0, 9000, 37)), 1000),
+    ([600, 1300] * 16, 888),                  # longest > 2 x shortest
+    ([600, 1100] * 200, 888),                 # within 2x, many waves: 512
+    ([100, 400] * 64, 888),                   # varied but nothing past 512: 512
 ])
 def test_partition_choice_follows_its_rule(lens, slots):
     """pa_decode_partition_for against its stated rule, evaluated here by
-    brute force: 512 unless 512-token CTAs fill more than one wave and at most
-    two, then 1024 if that fits one wave."""
+    brute force: 1024 when 512-token CTAs fill more than one wave and at most
+    two and 1024-token ones fit one wave, or when the longest sequence is past
+    512 tokens and more than twice the shortest; else 512."""
     from paged_kv_cache_347_b200 import pagedattn as pa
     hkv = 8
     got = pa.decode_partition_for(lens, hkv, 128, 16, torch.bfloat16, slots=slots)
     n0 = _ctas(lens, 512, hkv)
-    want = 1024 if slots < n0 <= 2 * slots and _ctas(lens, 1024, hkv) <= slots else 512
+    waves = slots < n0 <= 2 * slots and _ctas(lens, 1024, hkv) <= slots
+    varied = max(lens) > 512 and max(lens) > 2 * min(lens)
+    want = 1024 if waves or varied else 512
     assert got == want
 
 

@@ -296,3 +296,33 @@ def test_heads_per_cta(pa, heads_per_cta, G, Hkv):
                  torch.from_numpy(lens).cuda(), scale, variant=3, heads_per_cta=heads_per_cta)
     torch.cuda.synchronize()
     _check(out.double().cpu().numpy(), exp, "bf16", f"{heads_per_cta} heads per CTA")
+
+
+@pytest.mark.parametrize("variant", [1, 2, 3])
+def test_dispatch_order_changes_nothing_but_the_schedule(pa, variant):
+    """The grid taking the sequences longest first (seq_order) gives outputs
+    bit-identical to the batch order: each (sequence, head) is computed by the
+    same CTA code over the same tokens.  An entry outside the batch skips its
+    row and raises the length error bit."""
+    Hq, Hkv, D, bs = 16, 4, 128, 16
+    lens = [700, 1, 3000, 0, 64, 1500, 100]   # the last row fits one split
+    q, kc, vc, tables, lens = _case(34, lens, Hq, Hkv, D, bs, "bf16")
+    dev = [t.cuda() for t in (q, kc, vc)]
+    tab, sl = torch.from_numpy(tables).cuda(), torch.from_numpy(lens).cuda()
+    outs = []
+    for order in (None, pa.decode_order(lens)):
+        out = torch.full(tuple(q.shape), float("nan"), dtype=torch.float32, device="cuda")
+        pa.pa_decode(out, dev[0], dev[1], dev[2], tab, sl, D ** -0.5, variant=variant,
+                     seq_order=None if order is None else torch.from_numpy(order).cuda())
+        torch.cuda.synchronize()
+        outs.append(out.cpu())
+    assert torch.equal(outs[0], outs[1])
+    bad = torch.tensor([2, 0, 1, 3, 4, 5, 99], dtype=torch.int32, device="cuda")
+    out = torch.zeros(tuple(q.shape), dtype=torch.float32, device="cuda")
+    pa.device_errors(clear=True)
+    pa.pa_decode(out, dev[0], dev[1], dev[2], tab, sl, D ** -0.5, variant=variant,
+                 seq_order=bad)
+    assert pa.device_errors(clear=True) == ["seqlen"]
+    torch.cuda.synchronize()
+    assert torch.all(out[6] == 0)          # the row no grid row named
+    assert torch.equal(out[:6].cpu(), outs[0][:6])

@@ -101,6 +101,10 @@ def _native_step(nat: pa.BlockAllocator, ops, width):
     pairs = stage[lay.off_pairs:lay.off_pairs + 16 * lay.n_pairs].view(np.int64).reshape(-1, 2)
     tables = stage[lay.off_tables:lay.off_tables + 4 * ids.size * width].view(np.int32)
     lens = stage[lay.off_lens:lay.off_lens + 4 * ids.size].view(np.int32)
+    if code == 0 and ids.size:
+        # the decode's dispatch order: rows longest first, ties in batch order
+        order = stage[lay.off_order:lay.off_order + 4 * ids.size].view(np.int32)
+        assert order.tolist() == np.argsort(-lens.astype(np.int64), kind="stable").tolist()
     return lay, slots, [tuple(int(x) for x in p) for p in pairs], pb, \
         tables.reshape(ids.size, width), lens, code
 
@@ -269,3 +273,10 @@ def test_runner_splits_appends_at_every_other_event():
                             ("write", 7, 8, 4, 8)]
     assert PagedKVRunner.encode_ops([("admit", 3, [1, 2, 3])]) is None
     del r
+
+
+def test_decode_order_is_longest_first_and_stable():
+    assert pa.decode_order([5, 9, 9, 0, 14]).tolist() == [4, 1, 2, 0, 3]
+    assert pa.decode_order([]).tolist() == []
+    r = np.random.default_rng(0).integers(0, 50, size=300)
+    assert pa.decode_order(r).tolist() == np.argsort(-r, kind="stable").tolist()
