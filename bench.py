@@ -136,7 +136,7 @@ DESCR = {
 
 
 def kv_bytes(lens, hkv, d, e) -> int:
-    return int(sum(int(x) for x in lens)) * hkv * d * 2 * e
+    return int(np.asarray(lens, dtype=np.int64).sum()) * hkv * d * 2 * e
 
 
 # ----------------------------------------------------------------- clocks
@@ -363,11 +363,15 @@ _FLUSH = {}
 
 
 def flush_l2(dev) -> None:
-    """Writes 256 MB (twice the 126 MB L2) so that the next kernel starts cold."""
+    """Reads 256 MB (twice the 126 MB L2) so that the next kernel finds none
+    of its data in L2.  A read leaves clean lines, which the next kernel
+    evicts for free; a write would leave ~126 MB of dirty lines for it to
+    write back to HBM in its own time."""
     buf = _FLUSH.get(dev)
     if buf is None:
-        buf = _FLUSH[dev] = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    buf.fill_(1)
+        buf = _FLUSH[dev] = torch.ones(64 << 20, dtype=torch.float32, device=dev)
+        _FLUSH[(dev, "sink")] = torch.empty(1, dtype=torch.float32, device=dev)
+    torch.sum(buf, dim=0, keepdim=True, out=_FLUSH[(dev, "sink")])
 
 
 def time_main_kernel(pl: Planned, n: int, dev) -> dict:

@@ -525,6 +525,35 @@ int pa_step_plan(pa_alloc *a, const int64_t *events, int n_events, const int64_t
                  int num_seqs, int width, void *stage, size_t stage_bytes,
                  int32_t *pairs_before, pa_step_layout *out);
 
+/* ------------------------------------------------------------------------
+ * A host-fed step's device work in one call: the executor a runtime uses
+ * once a step's kernels are a CUDA graph (not from the pages; it is how the
+ * runtime of sanketn26 "Use a runtime that owns the blocks" keeps its host
+ * work per step small).  In order:
+ *   stream_in:  waits for wait_before_in (if non-NULL: e.g. the last use of
+ *               the staging buffer), runs the copies (one cudaMemcpyAsync
+ *               host-to-device each; page-locked sources copy asynchronously),
+ *               records event_in;
+ *   stream_run: waits for event_in and wait_before_run (if non-NULL: e.g. the
+ *               previous output copy of this graph), launches graph_run (a
+ *               cudaGraphExec_t), records event_run;
+ *   stream_out: if graph_out is non-NULL, waits for event_run, launches
+ *               graph_out, records event_out.
+ * Streams are cudaStream_t, events cudaEvent_t, graphs cudaGraphExec_t, all
+ * the caller's.  Returns PA_ERR_CUDA if a call fails (work enqueued before it
+ * stays enqueued), PA_ERR_INVALID_ARG on a NULL event or graph.
+ * ---------------------------------------------------------------------- */
+typedef struct {
+    void *dst;       /* device */
+    const void *src; /* host */
+    size_t bytes;    /* 0 skips the entry */
+} pa_host_copy;
+
+int pa_step_launch(void *stream_in, void *stream_run, void *stream_out,
+                   const pa_host_copy *copies, int n_copies, void *wait_before_in,
+                   void *event_in, void *graph_run, void *wait_before_run, void *event_run,
+                   void *graph_out, void *event_out);
+
 int pa_alloc_stats(const pa_alloc *a, pa_alloc_stats_t *out);
 
 /* Free list from head to tail into out (host int32, up to cap); *n_out =

@@ -551,6 +551,50 @@ int pa_swap_blocks(void *dst_k, void *dst_v, const void *src_k, const void *src_
     return PA_OK;
 }
 
+// One host-fed step's device work in one call (the runtime's step executor):
+// the step's copies in on one stream, its kernels' graph on a second, its
+// output's copy graph on a third, ordered by events.
+int pa_step_launch(void *stream_in, void *stream_run, void *stream_out,
+                   const pa_host_copy *copies, int n_copies, void *wait_before_in,
+                   void *event_in, void *graph_run, void *wait_before_run, void *event_run,
+                   void *graph_out, void *event_out) {
+    clear_error();
+    if (n_copies < 0 || (n_copies > 0 && !copies))
+        return fail(PA_ERR_INVALID_ARG, "bad copy list");
+    if (!event_in || !graph_run || !event_run || (graph_out && !event_out))
+        return fail(PA_ERR_INVALID_ARG, "NULL event or graph");
+    cudaStream_t si = static_cast<cudaStream_t>(stream_in);
+    cudaStream_t sr = static_cast<cudaStream_t>(stream_run);
+    cudaStream_t so = static_cast<cudaStream_t>(stream_out);
+    cudaError_t e = cudaSuccess;
+    if (wait_before_in) e = cudaStreamWaitEvent(si, static_cast<cudaEvent_t>(wait_before_in), 0);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamWaitEvent");
+    for (int i = 0; i < n_copies; ++i) {
+        if (copies[i].bytes == 0) continue;
+        if (!copies[i].dst || !copies[i].src) return fail(PA_ERR_INVALID_ARG, "NULL copy %d", i);
+        e = cudaMemcpyAsync(copies[i].dst, copies[i].src, copies[i].bytes, cudaMemcpyHostToDevice,
+                            si);
+        if (e != cudaSuccess) return cuda_fail(e, "host-to-device copy");
+    }
+    if ((e = cudaEventRecord(static_cast<cudaEvent_t>(event_in), si)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(sr, static_cast<cudaEvent_t>(event_in), 0)) != cudaSuccess)
+        return cuda_fail(e, "event after the copies");
+    if (wait_before_run &&
+        (e = cudaStreamWaitEvent(sr, static_cast<cudaEvent_t>(wait_before_run), 0)) != cudaSuccess)
+        return cuda_fail(e, "cudaStreamWaitEvent");
+    if ((e = cudaGraphLaunch(static_cast<cudaGraphExec_t>(graph_run), sr)) != cudaSuccess)
+        return cuda_fail(e, "kernels' graph launch");
+    if ((e = cudaEventRecord(static_cast<cudaEvent_t>(event_run), sr)) != cudaSuccess)
+        return cuda_fail(e, "cudaEventRecord");
+    if (graph_out) {
+        if ((e = cudaStreamWaitEvent(so, static_cast<cudaEvent_t>(event_run), 0)) != cudaSuccess ||
+            (e = cudaGraphLaunch(static_cast<cudaGraphExec_t>(graph_out), so)) != cudaSuccess ||
+            (e = cudaEventRecord(static_cast<cudaEvent_t>(event_out), so)) != cudaSuccess)
+            return cuda_fail(e, "output copy");
+    }
+    return PA_OK;
+}
+
 int pa_set_profile_events(void *ev_begin, void *ev_end) {
     clear_error();
     t_prof.begin = static_cast<cudaEvent_t>(ev_begin);

@@ -97,6 +97,23 @@ class pa_step_layout(ctypes.Structure):
 _sig("pa_decode_order", _i, _vp, _i, _vp)
 
 
+class pa_host_copy(ctypes.Structure):
+    _fields_ = [("dst", ctypes.c_void_p), ("src", ctypes.c_void_p), ("bytes", ctypes.c_size_t)]
+
+
+_sig("pa_step_launch", _i, _vp, _vp, _vp, _vp, _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp)
+
+
+def step_launch(stream_in: int, stream_run: int, stream_out: int, copies, n_copies: int,
+                wait_before_in: int, event_in: int, graph_run: int, wait_before_run: int,
+                event_run: int, graph_out: int, event_out: int) -> None:
+    """pa_step_launch on raw handles (streams, events, graph execs as ints)."""
+    _check(_lib.pa_step_launch(stream_in, stream_run, stream_out, copies, n_copies,
+                               wait_before_in or None, event_in, graph_run,
+                               wait_before_run or None, event_run, graph_out or None,
+                               event_out or None), "pa_step_launch")
+
+
 def decode_order(seq_lens) -> np.ndarray:
     """pa_decode_order: batch rows longest first (ties in batch order)."""
     lens = np.ascontiguousarray(np.asarray(seq_lens), dtype=np.int32).reshape(-1)

@@ -348,13 +348,22 @@ class PagedKVRunner:
         if enc is None:
             return self._prepare_ops(ops)
         b = int(enc.decode_ids.size)
-        lay = self.alloc.step_layout(enc.events, b, self.width)
         slot = self._next_slot
         self._next_slot = 1 - slot
-        host, devb = self._staging(slot, _a256(lay.bytes) + self._input_bytes(lay.n_slots, b))
+        host, devb = self._staging(slot, 0)
         hb = host.numpy()
         pb = np.empty(enc.events.shape[0] + 1, np.int32)
-        lay = self.alloc.step_plan(enc.events, enc.decode_ids, self.width, hb, pb)
+        try:
+            lay = self.alloc.step_plan(enc.events, enc.decode_ids, self.width, hb, pb)
+        except pa.PagedAttnError as e:
+            need = e.layout.bytes if e.code == -1 else 0
+            if need <= hb.nbytes:
+                raise
+            # too small a buffer is refused before anything is applied: grow,
+            # with room behind the arrays for the step's new rows and queries
+            host, devb = self._staging(slot, _a256(need) + self._input_bytes(e.layout.n_slots, b))
+            hb = host.numpy()
+            lay = self.alloc.step_plan(enc.events, enc.decode_ids, self.width, hb, pb)
         slots = hb[lay.off_slots:lay.off_slots + 8 * lay.n_slots].view(np.int64)
         pairs = hb[lay.off_pairs:lay.off_pairs + 16 * lay.n_pairs].view(np.int64).reshape(-1, 2)
         acts, arrays, offs = [], [], []
@@ -488,19 +497,18 @@ class PagedKVRunner:
 
     def _graph_key(self, prep: dict, k_new: torch.Tensor, q: torch.Tensor):
         acts = prep["acts"]
-        if not self._graphable(acts):
-            return None
         layout = tuple((a.kind, a.nrows, None if a.tables is None else a.tables.shape,
-                        a.partition, self._graph_bound(a.max_len) if a.kind == "decode" else 0)
+                        a.partition, self._graph_bound(a.max_len) if a.kind == "decode" else 0,
+                        a.order is not None)
                        for a in acts)
         return (layout, prep["bytes"], prep["slot"], prep["dev"].data_ptr(),
                 tuple(k_new.shape), tuple(q.shape), k_new.dtype)
 
-    def _input_views(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
-                     q: torch.Tensor):
+    def _input_offsets(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
+                       q: torch.Tensor):
         """Fixed places for the step's new K/V rows and queries in the slot's
-        device buffer, behind its arrays (256-byte aligned; the buffers grow,
-        keeping the arrays, when too small)."""
+        device buffer, behind its arrays (256-byte aligned); the buffers grow,
+        keeping the arrays, when too small."""
         total = prep["bytes"]
         offs, end = [], _a256(total)
         for t in (k_new, v_new, q):
@@ -510,23 +518,14 @@ class PagedKVRunner:
             old = prep["host"]
             prep["host"], prep["dev"] = self._staging(prep["slot"], end)
             prep["host"][:total].copy_(old[:total])
-        devb = prep["dev"]
-        return [devb[off:off + t.nbytes].view(t.dtype).view(t.shape)
-                for off, t in zip(offs, (k_new, v_new, q))]
-
-    def _copy_in(self, prep: dict, ins, k_new, v_new, q) -> None:
-        """The step's inputs to the device, on the current stream: the
-        staging buffer's arrays, then the new rows and queries straight from
-        the caller's (page-locked) tensors."""
-        total = prep["bytes"]
-        if total:
-            prep["dev"][:total].copy_(prep["host"][:total], non_blocking=True)
-        for dst, src in zip(ins, (k_new, v_new, q)):
-            dst.copy_(src, non_blocking=True)
+        return offs
 
     def _capture(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
-                 q: torch.Tensor, ins) -> dict:
+                 q: torch.Tensor, offs) -> dict:
         dec = [a for a in prep["acts"] if a.kind == "decode"][0]
+        devb, host, total = prep["dev"], prep["host"], prep["bytes"]
+        ins = [devb[off:off + t.nbytes].view(t.dtype).view(t.shape)
+               for off, t in zip(offs, (k_new, v_new, q))]
         g = {"out": torch.empty((dec.tables.shape[0], self.num_heads, self.head_dim),
                                 dtype=torch.float32).pin_memory(),
              "in_bytes": sum(t.nbytes for t in (k_new, v_new, q)), "ins": ins}
@@ -546,7 +545,10 @@ class PagedKVRunner:
         side = torch.cuda.Stream(self.device)
         side.wait_stream(torch.cuda.current_stream(self.device))
         with torch.cuda.stream(side):
-            self._copy_in(prep, ins, k_new, v_new, q)
+            if total:
+                devb[:total].copy_(host[:total], non_blocking=True)
+            for dst, src in zip(ins, (k_new, v_new, q)):
+                dst.copy_(src, non_blocking=True)
             body_run()
             body_out()
         side.synchronize()
@@ -558,9 +560,22 @@ class PagedKVRunner:
             with torch.cuda.graph(graph, stream=side, capture_error_mode="thread_local"):
                 body()
             g[name] = graph
-        # events re-recorded at every replay of this layout (made once: the
-        # host side of a replay stays short)
+        g["exec_run"] = g["g_run"].raw_cuda_graph_exec()
+        g["exec_out"] = g["g_out"].raw_cuda_graph_exec()
+        # events re-recorded at every replay of this layout (made, and recorded
+        # once so that they exist, here: the host side of a replay stays short)
         g["ev_in"], g["ev_run"], g["ev_out"] = (torch.cuda.Event() for _ in range(3))
+        with torch.cuda.stream(side):
+            for ev in (g["ev_in"], g["ev_run"], g["ev_out"]):
+                ev.record()
+        side.synchronize()
+        # the copies in: the staging buffer's arrays, then the new rows and
+        # queries (their sources are set per step)
+        c = (pa.pa_host_copy * 4)()
+        c[0].dst, c[0].src, c[0].bytes = devb.data_ptr(), host.data_ptr(), total
+        for i, (off, t) in enumerate(zip(offs, (k_new, v_new, q)), start=1):
+            c[i].dst, c[i].bytes = devb.data_ptr() + off, t.nbytes
+        g["copies"] = c
         g["replayed"] = False
         return g
 
@@ -572,14 +587,14 @@ class PagedKVRunner:
         must stay unchanged until the step's "ready" event."""
         if not self._graphable(prep["acts"]):
             return None
-        ins = self._input_views(prep, k_new, v_new, q)
+        offs = self._input_offsets(prep, k_new, v_new, q)
         key = self._graph_key(prep, k_new, q)
         if key in self._graphs and self._graphs[key] is None:
             return None  # this layout failed to capture before: launch eagerly
         g = self._graphs.get(key)
         if g is None:
             try:
-                g = self._capture(prep, k_new, v_new, q, ins)
+                g = self._capture(prep, k_new, v_new, q, offs)
             except RuntimeError as e:  # capture refused: this layout runs eagerly
                 warnings.warn(f"CUDA graph capture failed, launching eagerly: {e}")
                 self._graphs[key] = None
@@ -594,42 +609,34 @@ class PagedKVRunner:
         if self._s_in is None:
             self._s_in = torch.cuda.Stream(self.device)
             self._s_out = torch.cuda.Stream(self.device)
+            self._s_handles = (self._s_in.cuda_stream, self._s_out.cuda_stream)
         return self._s_in, self._s_out
 
     def replay_graph(self, g: dict, prep: dict) -> dict:
-        """Device half of a graph step.  The copy in runs on a copy stream
-        once the previous step of this staging slot has finished with the
-        slot's device buffer; the kernels run on the current stream after the
-        copy in (and after this layout's previous output has been copied
-        out); the output's copy back runs on a second copy stream.  The
-        output lands in a page-locked tensor owned by the graph, readable once
-        the returned "ready" event has completed (or after wait()) until the
-        next replay of the same layout, which also re-records that event."""
-        cur = torch.cuda.current_stream(self.device)
-        s_in, s_out = self._copy_streams()
+        """Device half of a graph step, one library call (pa_step_launch): the
+        copies in run on a copy stream once the previous step of this staging
+        slot has finished with the slot's device buffer; the kernels' graph
+        runs on the current stream after them (and after this layout's
+        previous output has been copied out); the output's copy graph runs on
+        a second copy stream.  The output lands in a page-locked tensor owned
+        by the graph, readable once the returned "ready" event has completed
+        (or after wait()) until the next replay of the same layout."""
+        self._copy_streams()
+        c = g["copies"]
+        k, v, q = prep["inputs"]
+        c[1].src, c[2].src, c[3].src = k.data_ptr(), v.data_ptr(), q.data_ptr()
         slot = prep["slot"]
-        if self._run_ev[slot] is not None:
-            s_in.wait_event(self._run_ev[slot])
-        torch.cuda.set_stream(s_in)
-        self._copy_in(prep, g["ins"], *prep["inputs"])
-        g["ev_in"].record(s_in)
-        torch.cuda.set_stream(cur)
+        prev = self._run_ev[slot]
+        pa.step_launch(self._s_handles[0], torch.cuda.current_stream(self.device).cuda_stream,
+                       self._s_handles[1], c, 4, prev.cuda_event if prev is not None else 0,
+                       g["ev_in"].cuda_event, g["exec_run"],
+                       g["ev_out"].cuda_event if g["replayed"] else 0, g["ev_run"].cuda_event,
+                       g["exec_out"], g["ev_out"].cuda_event)
         self._stage_ev[slot] = g["ev_in"]  # the host staging buffer is free again after this
-        cur.wait_event(g["ev_in"])
-        if g["replayed"]:
-            cur.wait_event(g["ev_out"])  # the previous output of this layout has left
-        g["g_run"].replay()
-        g["ev_run"].record(cur)
         self._run_ev[slot] = g["ev_run"]
-        s_out.wait_event(g["ev_run"])
-        torch.cuda.set_stream(s_out)
-        g["g_out"].replay()
-        g["ev_out"].record(s_out)
-        torch.cuda.set_stream(cur)
         g["replayed"] = True
-        h2d = prep["bytes"] + g["in_bytes"]
-        return {"h2d": h2d, "d2h": g["out"].nbytes, "acts": prep["acts"], "out": g["out"],
-                "ready": g["ev_out"]}
+        return {"h2d": prep["bytes"] + g["in_bytes"], "d2h": g["out"].nbytes,
+                "acts": prep["acts"], "out": g["out"], "ready": g["ev_out"]}
 
     def launch_graph(self, prep: dict, k_new: torch.Tensor, v_new: torch.Tensor,
                      q: torch.Tensor) -> Optional[dict]:
