@@ -314,7 +314,8 @@ class Planned:
                                                     / max(1, ast["reserved_slots"]), 5)}
         t = time.perf_counter()
         self.plans = [self.runner.plan(st.ops) for st in dec]
-        self.alloc_us = (time.perf_counter() - t) / len(dec) * 1e6
+        self.plan_py_us = (time.perf_counter() - t) / len(dec) * 1e6
+        self.alloc_us = self._step_plan_us(sh, steps)
         for acts in self.plans:
             self.runner.upload(acts)
         self.dev_in = [(st.k_new.to(dev), st.v_new.to(dev), st.q.to(dev)) for st in dec]
@@ -337,6 +338,33 @@ class Planned:
                     n += 1 + (1 if math.ceil(a.max_len / (a.partition or 512))
                               > FUSED_MERGE_MAX_SPLITS else 0)
             self.launches_per.append(n)
+
+    def _step_plan_us(self, sh, steps) -> float:
+        """Host time per decode step of pa_step_plan (the runtime's one call:
+        the step's events applied, slots, table rows, lengths and the
+        longest-first order written into a staging buffer), on a replica of
+        the allocator fed the same events; the events are encoded beforehand,
+        as a runtime keeps them."""
+        from paged_kv_cache_347_b200 import pagedattn as pa
+        from paged_kv_cache_347_b200.runner import PagedKVRunner
+        alloc = pa.BlockAllocator(sh.num_blocks, sh.block_size, sh.free_order)
+        encs = [PagedKVRunner.encode_ops(st.ops) for st in steps]
+        if any(e is None for e in encs):
+            return float("nan")
+        stage = np.zeros(1 << 20, np.uint8)
+
+        def plan(e):
+            nonlocal stage
+            lay = alloc.step_layout(e.events, e.decode_ids.size, self.width)
+            if lay.bytes > stage.nbytes:
+                stage = np.zeros(lay.bytes, np.uint8)
+            alloc.step_plan(e.events, e.decode_ids, self.width, stage)
+
+        plan(encs[0])                                     # the prefill
+        t = time.perf_counter()
+        for e in encs[1:]:
+            alloc.step_plan(e.events, e.decode_ids, self.width, stage)
+        return (time.perf_counter() - t) / max(1, len(encs) - 1) * 1e6
 
     def step(self, i: int) -> None:
         j = i % len(self.plans)
@@ -488,6 +516,9 @@ def run_ours(args, ws, rank, local):
                    "parallelism": f"dp{ws} (independent batches, no collective)",
                    "l2": "inputs larger than L2 (KV cache 1.07 GB per step), no flush",
                    "planned_steps": len(plans), "host_alloc_us_per_step": round(pl.alloc_us, 2),
+                   "host_alloc_note": "pa_step_plan per decode step (events applied, slots, "
+                                      "table rows, lengths, order written)",
+                   "host_plan_op_by_op_us_per_step": round(pl.plan_py_us, 2),
                    "partition_tokens": pl.partitions(),
                    "partition_policy": {-1: "per step, pa_decode_partition_for",
                                         0: "library default"}.get(args.partition, "fixed"),

@@ -478,8 +478,10 @@ int pa_block_tables(const pa_alloc *a, const int64_t *seq_ids, int n_seqs, int32
  *   off_pairs   int64 [n_pairs][2]       copy-on-write (src, dst) pairs, in
  *                                        event order (room for one per append
  *                                        event; n_pairs_pre before the decode)
- *   off_tables  int32 [num_seqs][width]  table rows (entries past a table's
- *                                        length 0), as of the decode event
+ *   off_tables  int32 [num_seqs][width]  table rows as of the decode event;
+ *                                        entries past a table's length are
+ *                                        left as the buffer held them (no
+ *                                        kernel reads them)
  *   off_lens    int32 [num_seqs]         lengths, as of the decode event
  *   off_order   int32 [num_seqs]         the batch rows longest first (ties
  *                                        in batch order), for

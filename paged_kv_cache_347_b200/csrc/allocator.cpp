@@ -665,10 +665,29 @@ int pa_step_plan(pa_alloc *a, const int64_t *events, int n_events, const int64_t
         } else {  // PA_EV_DECODE: the batch's rows as they stand here
             out->n_slots_pre = (int32_t)slot_off;
             out->n_pairs_pre = npairs;
-            rc = pa_block_tables(a, decode_ids, num_seqs, tables, width, lens);
+            // each row's live entries only: the kernels read no entry past a
+            // sequence's last block, so the rest is left as the buffer held it
+            int32_t mx = 0;
+            for (int r = 0; r < num_seqs && rc == PA_OK; ++r) {
+                auto it = a->seqs.find(decode_ids[r]);
+                if (it == a->seqs.end()) {
+                    rc = pa::fail(PA_ERR_UNKNOWN_SEQ, "decode row %d: unknown sequence %lld", r,
+                                  (long long)decode_ids[r]);
+                } else if (it->second.swapped) {
+                    rc = pa::fail(PA_ERR_INVALID_ARG, "decode row %d: sequence %lld is swapped out",
+                                  r, (long long)decode_ids[r]);
+                } else if ((int64_t)it->second.table.size() > width) {
+                    rc = pa::fail(PA_ERR_SEQ_TOO_LONG, "decode row %d: %zu blocks > width %d", r,
+                                  it->second.table.size(), width);
+                } else {
+                    const auto &t = it->second.table;
+                    if (!t.empty())
+                        std::memcpy(tables + (size_t)r * width, t.data(), sizeof(int32_t) * t.size());
+                    lens[r] = (int32_t)it->second.len;
+                    mx = lens[r] > mx ? lens[r] : mx;
+                }
+            }
             if (rc == PA_OK) {
-                int32_t mx = 0;
-                for (int r = 0; r < num_seqs; ++r) mx = lens[r] > mx ? lens[r] : mx;
                 out->max_seq_len = mx;
                 rc = pa_decode_order(lens, num_seqs, order);
             }

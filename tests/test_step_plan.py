@@ -109,6 +109,14 @@ def _native_step(nat: pa.BlockAllocator, ops, width):
         tables.reshape(ids.size, width), lens, code
 
 
+def _same_rows(tab, ref_tab, lens, bs):
+    """Table rows agree on every entry a kernel reads (those below each
+    sequence's block count); the rest is unspecified."""
+    for r, L in enumerate(lens):
+        n = -(-int(L) // bs)
+        assert tab[r, :n].tolist() == ref_tab[r, :n].tolist(), r
+
+
 def _same_state(ref: RefAllocator, nat: pa.BlockAllocator):
     assert nat.free_list() == ref.free_list()
     for b in range(ref.num_blocks):
@@ -137,7 +145,8 @@ def test_workload_steps_bit_exact(name):
         assert pb.tolist() == r_pb, i
         assert lay.events_applied == r_n == len(st.ops)
         if r_tab is not None:
-            assert np.array_equal(tab, r_tab) and np.array_equal(lens, r_lens)
+            assert np.array_equal(lens, r_lens)
+            _same_rows(tab, r_tab, r_lens, sh.block_size)
             assert lay.max_seq_len == int(r_lens.max())
             # the decode splits the step: rows and pairs before it
             k = [j for j, op in enumerate(st.ops) if op[0] == "decode"][0]
@@ -199,7 +208,8 @@ def test_random_event_streams_with_failures(seed):
         if code == 0:
             assert slots.tolist() == r_slots and pairs == r_pairs and pb.tolist() == r_pb
             if r_tab is not None:
-                assert np.array_equal(tab, r_tab) and np.array_equal(lens, r_lens)
+                assert np.array_equal(lens, r_lens)
+                _same_rows(tab, r_tab, r_lens, bs)
         else:
             assert lay.events_applied == r_n, (step, lay.events_applied, r_n)
             assert pb[:r_n].tolist() == r_pb[:r_n]
