@@ -151,3 +151,16 @@ def test_partition_choice_edge_cases():
     with pytest.raises(pa.PagedAttnError):
         pa.decode_partition_for([5], 8, 128, 16, torch.bfloat16, slots=-1)
     assert pa._lib.pa_decode_partition_for(None, 2, 8, 128, 16, 1, 888) == -1
+
+
+def test_step_launch_rejects_bad_arguments_before_any_cuda_call():
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    L = pa._lib
+    # no event or graph
+    assert L.pa_step_launch(None, None, None, None, 0, None, None, None, None, None, None,
+                            None) == -1
+    # a negative copy count, or copies without a list
+    assert L.pa_step_launch(None, None, None, None, -1, None, 1, 1, None, 1, None, None) == -1
+    assert L.pa_step_launch(None, None, None, None, 2, None, 1, 1, None, 1, None, None) == -1
+    # an output graph without its event
+    assert L.pa_step_launch(None, None, None, None, 0, None, 1, 1, None, 1, 1, None) == -1
