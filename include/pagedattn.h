@@ -204,6 +204,32 @@ typedef struct {
 } pa_decode_opts;
 
 /*
+ * A decode step's append and attention in one launch [P1 "Mechanism and
+ * details": a new token goes into its sequence's last block; P3 bullet 3]:
+ * every sequence s appends one token, at position seq_lens[s] - 1, whose K
+ * and V rows are k_new[s] and v_new[s] ([num_seqs][num_kv_heads][head_dim],
+ * `dtype`, device) and whose slot is slot_mapping[s] (device int64); then
+ * out is pa_decode_opt's result over seq_lens[s] tokens, the new one
+ * included.  The CTA of each (sequence, KV head) whose partition holds the
+ * new position writes that head's rows into the caches before it reads the
+ * block (so the step needs no separate pa_reshape_and_cache launch).
+ *   - A slot must be the one the table gives position seq_lens[s] - 1 (as
+ *     the allocator's append returns it); another slot is not written and
+ *     sets PA_DEVERR_SLOT.  A negative slot writes nothing.
+ *   - A copy-on-write copy for the step (pa_copy_blocks) must come before
+ *     this call on the stream; a sequence with seq_lens[s] == 0 appends
+ *     nothing.
+ * Same arguments otherwise, same results and errors as pa_decode_opt.
+ */
+int pa_append_decode(float *out, const void *q, const void *k_new, const void *v_new,
+                     const int64_t *slot_mapping, void *k_cache, void *v_cache,
+                     const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
+                     int num_heads, int num_kv_heads, int head_dim, int block_size,
+                     int max_blocks_per_seq, int num_blocks, int max_seq_len, float scale,
+                     int dtype, void *workspace, size_t workspace_bytes,
+                     const pa_decode_opts *opts, void *stream);
+
+/*
  * Longest-first order of a decode batch for pa_decode_opts.seq_order, from
  * the lengths as the caller knows them on the host: order_out[i] is the
  * batch row of the i-th longest sequence, ties in batch order.  Host only.

@@ -199,6 +199,25 @@ int pa_decode_ex(float *out, const void *q, const void *k_cache, const void *v_c
                          max_seq_len, scale, dtype, workspace, workspace_bytes, &o, stream);
 }
 
+}  // extern "C"
+
+namespace pa {
+// The new tokens of a fused append (pa_append_decode), or none.
+struct AppendArgs {
+    const void *k_new, *v_new;
+    const int64_t *slot_mapping;
+};
+}  // namespace pa
+
+static int decode_impl(float *out, const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
+                       int num_heads, int num_kv_heads, int head_dim, int block_size,
+                       int max_blocks_per_seq, int num_blocks, int max_seq_len, float scale,
+                       int dtype, void *workspace, size_t workspace_bytes,
+                       const pa_decode_opts *opts, const AppendArgs *app, void *stream);
+
+extern "C" {
+
 int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_cache,
                   const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
                   int num_heads, int num_kv_heads, int head_dim, int block_size,
@@ -206,6 +225,40 @@ int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_
                   int dtype, void *workspace, size_t workspace_bytes,
                   const pa_decode_opts *opts, void *stream) {
     clear_error();
+    return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                       max_seq_len, scale, dtype, workspace, workspace_bytes, opts, nullptr,
+                       stream);
+}
+
+int pa_append_decode(float *out, const void *q, const void *k_new, const void *v_new,
+                     const int64_t *slot_mapping, void *k_cache, void *v_cache,
+                     const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
+                     int num_heads, int num_kv_heads, int head_dim, int block_size,
+                     int max_blocks_per_seq, int num_blocks, int max_seq_len, float scale,
+                     int dtype, void *workspace, size_t workspace_bytes,
+                     const pa_decode_opts *opts, void *stream) {
+    clear_error();
+    if (num_seqs > 0 && (!k_new || !v_new || !slot_mapping))
+        return fail(PA_ERR_INVALID_ARG, "NULL new-token pointer");
+    if (num_seqs > 0 && (!aligned16(k_new) || !aligned16(v_new) ||
+                         (reinterpret_cast<uintptr_t>(slot_mapping) & 7u)))
+        return fail(PA_ERR_INVALID_ARG, "misaligned new-token pointer");
+    const AppendArgs app = {k_new, v_new, slot_mapping};
+    return decode_impl(out, q, k_cache, v_cache, block_tables, seq_lens, num_seqs, num_heads,
+                       num_kv_heads, head_dim, block_size, max_blocks_per_seq, num_blocks,
+                       max_seq_len, scale, dtype, workspace, workspace_bytes, opts, &app,
+                       stream);
+}
+
+}  // extern "C"
+
+static int decode_impl(float *out, const void *q, const void *k_cache, const void *v_cache,
+                       const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
+                       int num_heads, int num_kv_heads, int head_dim, int block_size,
+                       int max_blocks_per_seq, int num_blocks, int max_seq_len, float scale,
+                       int dtype, void *workspace, size_t workspace_bytes,
+                       const pa_decode_opts *opts, const AppendArgs *app, void *stream) {
     pa_decode_opts o;
     std::memset(&o, 0, sizeof(o));
     if (opts) o = *opts;
@@ -304,6 +357,11 @@ int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_
     p.max_splits = splits;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.seq_order = o.seq_order;
+    if (app) {
+        p.k_new = app->k_new;
+        p.v_new = app->v_new;
+        p.slot_mapping = app->slot_mapping;
+    }
 
     // 16-bit caches go to the tensor-core kernel (it needs the cache to fit
     // 2^31 TMA rows); fp32 caches to the CUDA-core kernel.
@@ -336,6 +394,8 @@ int pa_decode_opt(float *out, const void *q, const void *k_cache, const void *v_
     }
     return PA_OK;
 }
+
+extern "C" {
 
 int pa_decode_partition_for(const int32_t *seq_lens_host, int num_seqs, int num_kv_heads,
                             int head_dim, int block_size, int dtype, int slots) {

@@ -77,6 +77,43 @@ __device__ __forceinline__ void store_unit(const DecodeParams &p, int s, int h, 
     }
 }
 
+// ---------------------------------------------------------------- fused append
+// The append of mbrenndoerfer.com "Paged Attention > Summary", bullet 3 (a new
+// token's K/V written into its sequence's last block) fused into the decode:
+// the CTA whose split holds position L - 1 writes the new token's rows for
+// KV heads g .. g + nh - 1 before it reads that block.  The slot must be the
+// one the table gives position L - 1; another slot (a caller's mistake that
+// could race with other CTAs' reads) is not written and sets PA_DEVERR_SLOT,
+// and a negative slot means "no write", as for pa_reshape_and_cache.  The
+// lanes of one warp copy 16-byte words; each fences its stores against the
+// async proxy (the TMA loads that follow read the row), and the warp syncs.
+__device__ __forceinline__ void fused_append_rows(const DecodeParams &p, int s, int g, int nh,
+                                                  int L, int elem_bytes, int lane) {
+    const int64_t slot = __ldg(p.slot_mapping + s);
+    if (slot >= 0) {
+        const int pos = L - 1;
+        const int blk = checked_block(p, s, pos / p.block_size);
+        const int64_t want = blk < 0 ? -1 : (int64_t)blk * p.block_size + pos % p.block_size;
+        if (slot != want) {
+            if (lane == 0 && blk >= 0) raise_device_error(p.err, PA_DEVERR_SLOT);
+        } else {
+            const int words = p.head_dim * elem_bytes / 16;  // per row
+            const int64_t b = slot / p.block_size, off = slot % p.block_size;
+            for (int c = lane; c < nh * words; c += 32) {
+                const int h = g + c / words, w = c - (c / words) * words;
+                const int64_t src = ((int64_t)s * p.num_kv_heads + h) * words + w;
+                const int64_t dst = ((b * p.num_kv_heads + h) * p.block_size + off) * words + w;
+                reinterpret_cast<uint4 *>(const_cast<void *>(p.k_cache))[dst] =
+                    __ldg(reinterpret_cast<const uint4 *>(p.k_new) + src);
+                reinterpret_cast<uint4 *>(const_cast<void *>(p.v_cache))[dst] =
+                    __ldg(reinterpret_cast<const uint4 *>(p.v_new) + src);
+            }
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+        }
+    }
+    __syncwarp();
+}
+
 // ---------------------------------------------------------------- in-kernel merge
 // The split-context partials of a (sequence, KV head) can be merged by the
 // main kernel itself: the CTA of that pair to finish last merges them (the

@@ -141,6 +141,9 @@ __global__ void __launch_bounds__(Cfg<T, D, BS, W, NS>::kThreads)
 
     // ------------------------------------------------------------ producer
     if (warp == W) {
+        // the fused append: this split holds the new token of the CTA's heads
+        if (p.k_new != nullptr && L > 0 && split == nsplit - 1)
+            fused_append_rows(p, s, h0, W, L, 2, lane);
         const uint64_t policy = l2_policy_evict_first();
         const uint32_t stage0 = smem_u32(smem);
         if constexpr (C::kAsync) {

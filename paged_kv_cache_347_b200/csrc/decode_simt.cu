@@ -64,6 +64,14 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
 
     const T *kc = static_cast<const T *>(p.k_cache);
     const T *vc = static_cast<const T *>(p.v_cache);
+    if (p.k_new != nullptr) {
+        // the fused append: warp 0 of the CTA holding position L - 1 writes
+        // the new token's rows; the barrier makes them visible to the L2
+        // loads below
+        if (warp == 0 && L > 0 && split == nsplit - 1)
+            fused_append_rows(p, s, g, 1, L, (int)sizeof(T), lane);
+        __syncthreads();
+    }
     float m[GM], l[GM], o[GM][E];
 #pragma unroll
     for (int h = 0; h < GM; ++h) {
@@ -86,8 +94,9 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
                 const int pb = checked_block(p, s, t / bs);
                 if (pb >= 0) {
                     const int64_t row = ((int64_t)pb * Hkv + g) * bs + t % bs;
-                    ku[u] = __ldg(reinterpret_cast<const uint4 *>(kc + row * D + li * E));
-                    vu[u] = __ldg(reinterpret_cast<const uint4 *>(vc + row * D + li * E));
+                    // through L2 (.cg): a row this CTA appended is read back
+                    ku[u] = __ldcg(reinterpret_cast<const uint4 *>(kc + row * D + li * E));
+                    vu[u] = __ldcg(reinterpret_cast<const uint4 *>(vc + row * D + li * E));
                 }
             }
         }

@@ -159,6 +159,10 @@ __global__ void __launch_bounds__(Cfg<T, D, BS, W, NS>::kThreads)
     __syncthreads();
 
     // ------------------------------------------------------------ producer
+    // the fused append: this split holds the new token, whose row the loads
+    // below then read
+    if (warp == W && p.k_new != nullptr && L > 0 && split == nsplit - 1)
+        fused_append_rows(p, s, g, 1, L, 2, lane);
     if (C::kAsync && warp == W) {
         // every lane copies 16-byte chunks of the stage's (block, head) rows
         // into the layout the TMA boxes give (row r of a 1 KB-aligned piece,

@@ -31,6 +31,12 @@ struct DecodeParams {
     // sequence seq_order[z]; null: z itself).  A runtime that knows the
     // lengths passes longest first, so that the last CTAs to start are short.
     const int32_t *seq_order;
+    // Append fused into the decode (null: none): the new token of every
+    // sequence, at position seq_lens[s] - 1, with its K/V rows in
+    // k_new/v_new [B][Hkv][D] and its slot in slot_mapping[B]; the split CTA
+    // holding that position writes its head's rows into the cache first.
+    const void *k_new, *v_new;
+    const int64_t *slot_mapping;
 };
 
 int num_sms();  // SMs of the current device (cached per device)

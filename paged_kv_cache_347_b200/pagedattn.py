@@ -71,6 +71,8 @@ class pa_decode_opts(ctypes.Structure):
 
 _sig("pa_decode_opt", _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i,
      _vp, _sz, _c.POINTER(pa_decode_opts), _vp)
+_sig("pa_append_decode", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
+     _i, _i, _i, _f, _i, _vp, _sz, _c.POINTER(pa_decode_opts), _vp)
 _sig("pa_copy_blocks", _i, _vp, _vp, _vp, _i, _sz, _i, _vp)
 _sig("pa_decode_static", _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f,
      _i, _vp)
@@ -299,6 +301,51 @@ def pa_decode(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cache
         _dev(seq_lens, "seq_lens", torch.int32), B, Hq, Hkv, D, bs, W, NB, int(max_seq_len),
         float(scale), DTYPE_CODE[k_cache.dtype], ws_ptr, ws_bytes, ctypes.byref(opts),
         _stream(q)), "pa_decode")
+    return out
+
+
+def pa_append_decode(out: torch.Tensor, q: torch.Tensor, k_new: torch.Tensor,
+                     v_new: torch.Tensor, slot_mapping: torch.Tensor, k_cache: torch.Tensor,
+                     v_cache: torch.Tensor, block_tables: torch.Tensor, seq_lens: torch.Tensor,
+                     scale: float, max_seq_len: Optional[int] = None,
+                     workspace: Optional[torch.Tensor] = None, partition_size: int = 0,
+                     variant: int = 0, merge: int = 0, heads_per_cta: int = 0,
+                     seq_order: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """pa_append_decode: each sequence's new token (k_new, v_new [B, Hkv, D]
+    at slot_mapping[B], position seq_lens - 1) written into the caches and
+    the decode over seq_lens tokens, in one launch (plus the reduce)."""
+    NB, Hkv, bs, D = k_cache.shape
+    B, Hq, Dq = q.shape
+    if Dq != D or tuple(out.shape) != (B, Hq, D):
+        raise ValueError("q/out shape mismatch")
+    if tuple(k_new.shape) != (B, Hkv, D) or tuple(v_new.shape) != (B, Hkv, D):
+        raise ValueError(f"k_new/v_new must be [{B}, {Hkv}, {D}]")
+    if block_tables.dim() != 2 or block_tables.shape[0] != B or seq_lens.numel() != B or \
+            slot_mapping.numel() != B:
+        raise ValueError("block_tables [B, W], seq_lens [B], slot_mapping [B]")
+    W = block_tables.shape[1]
+    if max_seq_len is None:
+        max_seq_len = W * bs
+    need = decode_workspace_size(B, Hq, D, max_seq_len, partition_size)
+    if workspace is None and need:
+        workspace = _workspace(q.device, need)
+    ws_ptr = 0 if workspace is None else _dev(workspace, "workspace")
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    order = None
+    if seq_order is not None:
+        if seq_order.numel() != B:
+            raise ValueError("seq_order must have one entry per sequence")
+        order = _dev(seq_order, "seq_order", torch.int32)
+    opts = pa_decode_opts(int(partition_size), int(variant), int(merge), int(heads_per_cta),
+                          order)
+    dt = k_cache.dtype
+    _check(_lib.pa_append_decode(
+        _dev(out, "out", torch.float32), _dev(q, "q", dt), _dev(k_new, "k_new", dt),
+        _dev(v_new, "v_new", dt), _dev(slot_mapping, "slot_mapping", torch.int64),
+        _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache", dt),
+        _dev(block_tables, "block_tables", torch.int32), _dev(seq_lens, "seq_lens", torch.int32),
+        B, Hq, Hkv, D, bs, W, NB, int(max_seq_len), float(scale), DTYPE_CODE[dt], ws_ptr,
+        ws_bytes, ctypes.byref(opts), _stream(q)), "pa_append_decode")
     return out
 
 

@@ -83,6 +83,10 @@ class Action:
     max_q: int = 0
     partition: int = 0                   # decode: split length passed to pa_decode
     order: Optional[np.ndarray] = None   # decode: int32 [b], rows longest first
+    ids: Optional[np.ndarray] = None     # write of plain appends: their sequence ids
+    ones: bool = False                   # write: every append was one token
+    fused: bool = False                  # write: its rows go in with the next decode
+    fuse: Optional["Action"] = None      # decode: the write fused into it
     dev: dict = field(default_factory=dict)
 
 
@@ -91,7 +95,8 @@ class PagedKVRunner:
                  head_dim: int, dtype: torch.dtype, scale: float, table_width: int,
                  free_order: Optional[Sequence[int]] = None, max_blocks_per_seq: int = 0,
                  device: str = "cuda", partition_size: int = 0, variant: int = 0,
-                 prefill_variant: int = 0, longest_first: bool = True):
+                 prefill_variant: int = 0, longest_first: bool = True,
+                 fuse_append: bool = True):
         self.alloc = pa.BlockAllocator(num_blocks, block_size, free_order, max_blocks_per_seq)
         self.device = torch.device(device)
         dims = (num_blocks, num_kv_heads, block_size, head_dim)
@@ -104,6 +109,9 @@ class PagedKVRunner:
         self.prefill_variant = prefill_variant
         # decode grids take the batch's sequences longest first (seq_order)
         self.longest_first = longest_first
+        # a decode step's one-token appends go in with the decode
+        # (pa_append_decode) instead of a separate pa_reshape_and_cache
+        self.fuse_append = fuse_append
         # host-fed steps: two staging slots (page-locked host / device buffer
         # pairs), the event after which each slot's host buffer is free, the
         # event after which each slot's device buffer is free, and the graphs
@@ -133,7 +141,7 @@ class PagedKVRunner:
     def plan(self, ops) -> List[Action]:
         acts: List[Action] = []
         row = 0
-        pend = {"slots": [], "pairs": [], "row0": 0, "nrows": 0}
+        pend = {"slots": [], "pairs": [], "row0": 0, "nrows": 0, "ids": None, "ones": False}
 
         def add_rows(slots, pairs, n):
             if pend["nrows"] == 0:
@@ -148,8 +156,9 @@ class PagedKVRunner:
                 pairs = (np.concatenate(pend["pairs"]) if pend["pairs"]
                          else np.empty((0, 2), np.int64))
                 acts.append(Action("write", slots=np.concatenate(pend["slots"]), pairs=pairs,
-                                   row0=pend["row0"], nrows=pend["nrows"]))
-            pend.update(slots=[], pairs=[], nrows=0)
+                                   row0=pend["row0"], nrows=pend["nrows"], ids=pend["ids"],
+                                   ones=pend["ones"]))
+            pend.update(slots=[], pairs=[], nrows=0, ids=None, ones=False)
 
         i = 0
         while i < len(ops):
@@ -163,14 +172,22 @@ class PagedKVRunner:
                     i += 1
                 slots, pairs = self.alloc.batch_append(ids, ns)
                 n = int(sum(ns))
+                plain = pend["nrows"] == 0
                 add_rows(slots.copy(), pairs.copy(), n)
+                if plain:  # a write of plain appends only (so far)
+                    pend["ids"] = np.asarray(ids, np.int64)
+                    pend["ones"] = all(x == 1 for x in ns)
+                else:
+                    pend["ids"] = None
                 row += n
                 continue
             if kind == "append_tokens":
+                pend["ids"] = None
                 slots, pair = self.alloc.seq_append_tokens(op[1], op[2])
                 add_rows(slots.copy(), [pair] if pair else None, len(op[2]))
                 row += len(op[2])
             elif kind == "admit":
+                pend["ids"] = None
                 toks = op[2]
                 c = self.alloc.seq_add_cached(op[1], toks)
                 slots, pair = self.alloc.seq_append_tokens(op[1], toks[c:])
@@ -187,6 +204,7 @@ class PagedKVRunner:
                 elif kind == "free":
                     self.alloc.seq_free(op[1])
                 elif kind == "decode":
+                    dec_ids = np.asarray(op[1], np.int64)
                     tables, lens = self.alloc.block_tables(list(op[1]), self.width)
                     part = self.partition_size
                     if part < 0:
@@ -196,7 +214,7 @@ class PagedKVRunner:
                                        max_len=int(lens.max()) if lens.size else 0,
                                        partition=part,
                                        order=pa.decode_order(lens) if self.longest_first
-                                       else None))
+                                       else None, ids=dec_ids))
                 elif kind == "prefill":
                     sids = [x for x, _ in op[1]]
                     ns = np.array([n for _, n in op[1]], np.int32)
@@ -216,7 +234,20 @@ class PagedKVRunner:
                     raise ValueError(f"unknown op {op!r}")
             i += 1
         flush()
+        self._mark_fusable(acts)
         return acts
+
+    def _mark_fusable(self, acts: List[Action]) -> None:
+        """A write of one-token appends of exactly the decode batch, in its
+        order, right before the decode, goes in with it (pa_append_decode)."""
+        if not self.fuse_append:
+            return
+        for i in range(1, len(acts)):
+            w, d = acts[i - 1], acts[i]
+            if (d.kind == "decode" and w.kind == "write" and w.ones and w.ids is not None
+                    and w.nrows == d.tables.shape[0] and d.ids is not None
+                    and np.array_equal(w.ids, d.ids)):
+                w.fused, d.fuse = True, w
 
     # ------------------------------------------------------------ device side
     def upload(self, acts: List[Action], pin: bool = False) -> None:
@@ -251,7 +282,7 @@ class PagedKVRunner:
             if a.kind == "write":
                 if "pairs" in a.dev:
                     pa.pa_copy_blocks(self.k_cache, self.v_cache, a.dev["pairs"])
-                if a.nrows:
+                if a.nrows and not a.fused:
                     pa.pa_reshape_and_cache(k_new[a.row0:a.row0 + a.nrows],
                                             v_new[a.row0:a.row0 + a.nrows], self.k_cache,
                                             self.v_cache, a.dev["slots"])
@@ -274,10 +305,18 @@ class PagedKVRunner:
                 b = a.tables.shape[0]
                 o = out if out is not None else torch.empty(
                     (b, self.num_heads, self.head_dim), dtype=torch.float32, device=self.device)
-                pa.pa_decode(o, q, self.k_cache, self.v_cache, a.dev["tables"], a.dev["lens"],
-                             self.scale, max_seq_len=a.max_len,
-                             partition_size=a.partition, variant=self.variant,
-                             seq_order=a.dev.get("order"))
+                if a.fuse is not None:
+                    w = a.fuse
+                    pa.pa_append_decode(o, q, k_new[w.row0:w.row0 + b], v_new[w.row0:w.row0 + b],
+                                        w.dev["slots"], self.k_cache, self.v_cache,
+                                        a.dev["tables"], a.dev["lens"], self.scale,
+                                        max_seq_len=a.max_len, partition_size=a.partition,
+                                        variant=self.variant, seq_order=a.dev.get("order"))
+                else:
+                    pa.pa_decode(o, q, self.k_cache, self.v_cache, a.dev["tables"],
+                                 a.dev["lens"], self.scale, max_seq_len=a.max_len,
+                                 partition_size=a.partition, variant=self.variant,
+                                 seq_order=a.dev.get("order"))
                 res = o
         return res
 
@@ -373,8 +412,9 @@ class PagedKVRunner:
             if seg[0] == "write":
                 _, e0, e1, r0, r1 = seg
                 p0, p1 = int(pb[e0]), int(pb[e1])
+                ev = enc.events[e0:e1]
                 w = Action("write", slots=slots[r0:r1], pairs=pairs[p0:p1], row0=r0,
-                           nrows=r1 - r0)
+                           nrows=r1 - r0, ids=ev[:, 1], ones=bool((ev[:, 2] == 1).all()))
                 acts.append(w)
                 if r1 > r0:
                     arrays.append((w, "slots", w.slots))
@@ -389,13 +429,14 @@ class PagedKVRunner:
                 order = hb[lay.off_order:lay.off_order + 4 * b].view(np.int32)
                 d = Action("decode", tables=tables, lens=lens.copy(), max_len=lay.max_seq_len,
                            partition=self._partition(lens),
-                           order=order if self.longest_first else None)
+                           order=order if self.longest_first else None, ids=enc.decode_ids)
                 acts.append(d)
                 arrays += [(d, "tables", tables), (d, "lens", lens)]
                 offs += [lay.off_tables, lay.off_lens]
                 if self.longest_first:
                     arrays.append((d, "order", order))
                     offs.append(lay.off_order)
+        self._mark_fusable(acts)
         return {"acts": acts, "arrays": arrays, "offs": offs, "bytes": lay.bytes, "slot": slot,
                 "host": host, "dev": devb}
 
@@ -499,7 +540,7 @@ class PagedKVRunner:
         acts = prep["acts"]
         layout = tuple((a.kind, a.nrows, None if a.tables is None else a.tables.shape,
                         a.partition, self._graph_bound(a.max_len) if a.kind == "decode" else 0,
-                        a.order is not None)
+                        a.order is not None, a.fused, a.fuse is not None)
                        for a in acts)
         return (layout, prep["bytes"], prep["slot"], prep["dev"].data_ptr(),
                 tuple(k_new.shape), tuple(q.shape), k_new.dtype)
