@@ -6,8 +6,10 @@
 
 One step = one decode step of the workload through every piece of the path:
 the host allocator's slots and tables (a1), the copy-on-write block copy when
-the step has one (a2), the KV append of the new tokens (a3), the paged decode
-main kernel (a4) and the split reduce (a5).  Default workload: the
+the step has one (a2), the KV append of the new tokens (a3, written by the
+decode kernel itself when the step appends one token per decoded sequence:
+pa_append_decode), the paged decode main kernel (a4) and the split reduce
+(a5); the grid takes the sequences longest first.  Default workload: the
 long-context batch (8 sequences x 32768 tokens, 64/8 heads, head_dim 128,
 bf16 KV, block size 16, 512-token splits); each step appends one token per
 sequence and decodes; the last planned step decodes exactly 32768 tokens.
@@ -28,7 +30,10 @@ sequence and decodes; the last planned step decodes exactly 32768 tokens.
   ``--sync-e2e`` waits for each step before launching the next.
 * ``roofline``: the main decode kernel's algorithmic bytes per launch over
   its own CUDA-event time (events recorded by the library around that launch
-  on the launching stream), against the measured HBM copy bandwidth.
+  on the launching stream, L2 flushed by a 256 MB read before each of 32
+  launches), against the measured HBM copy bandwidth.
+* ``configs`` (N = 1): the Llama-8B-shaped, beam and continuous-mix (block
+  16) workloads, each with its step time, main-kernel time and end to end.
 * ``cpu_baseline``: the fp64 oracle on the host cores on a bounded sample of
   the same workload.
 * ``prefill`` (N = 1): the chunked-prefill kernel on 8 x (4096 context +
@@ -325,15 +330,16 @@ class Planned:
         self.decodes = [[a for a in acts if a.kind == "decode"][0] for acts in self.plans]
         self.step_bytes = [kv_bytes(d.lens, sh.num_kv_heads, sh.head_dim, sh.elem_bytes)
                            for d in self.decodes]
-        # kernels each step launches: the copy-on-write copy, the append, the
-        # main decode and, when the longest sequence has more splits than the
+        # kernels each step launches: the copy-on-write copy, the append
+        # (unless the decode writes the step's new tokens itself), the main
+        # decode and, when the longest sequence has more splits than the
         # library merges inside the main kernel, the reduce
         self.launches_per = []
         for acts in self.plans:
             n = 0
             for a in acts:
                 if a.kind == "write":
-                    n += (1 if len(a.pairs) else 0) + (1 if a.nrows else 0)
+                    n += (1 if len(a.pairs) else 0) + (1 if a.nrows and not a.fused else 0)
                 else:
                     n += 1 + (1 if math.ceil(a.max_len / (a.partition or 512))
                               > FUSED_MERGE_MAX_SPLITS else 0)
