@@ -216,29 +216,34 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback 6.65 TB/s"
 
 
-DECODE_SOURCES = ("decode_tc.cu", "decode_common.cuh", "common.cuh", "launch.h")
+# the main decode kernel of each variant: its name and its sources
+DECODE_KERNELS = {1: ("decode_simt_kernel", "decode_simt.cu"),
+                  2: ("decode_tc_kernel", "decode_tc.cu"),
+                  3: ("decode_hw_kernel", "decode_hw.cu")}
+COMMON_SOURCES = ("decode_common.cuh", "common.cuh", "launch.h")
 
 
-def decode_source_hash() -> str:
-    """First 16 hex digits of the sha256 of the main decode kernel's sources."""
+def decode_source_hash(variant: int) -> str:
+    """First 16 hex digits of the sha256 of a decode kernel's sources."""
     h = hashlib.sha256()
-    for name in DECODE_SOURCES:
+    for name in (DECODE_KERNELS[variant][1],) + COMMON_SOURCES:
         with open(os.path.join(ROOT, "paged_kv_cache_347_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def traffic_from_profile(workload: str, alg_bytes_per_launch: float):
+def traffic_from_profile(workload: str, variant: int, alg_bytes_per_launch: float):
     """DRAM bytes (read + write) per launch of the main decode kernel, from
     the committed ncu summary, if it was taken on the kernel's sources as they
     are now (else None).  A summary taken on a smaller case of the workload
     is scaled to a full launch by the ratio of algorithmic bytes, which
     holds while traffic grows in proportion to the tokens read."""
-    path = os.path.join(ROOT, "profiles", f"decode_tc_{workload}.json")
+    name = DECODE_KERNELS[variant][0]
+    path = os.path.join(ROOT, "profiles", f"{name}_{workload}.json")
     try:
         with open(path) as f:
             prof = json.load(f)
-        h = decode_source_hash()
+        h = decode_source_hash(variant)
     except (OSError, ValueError):
         return None
     if prof.get("kernel_src_sha256_16") != h:
@@ -425,7 +430,8 @@ def time_main_kernel(pl: Planned, n: int, dev) -> dict:
         if i >= 2:
             pa.set_profile_events(*evs[i - 2])
         pa.pa_decode(pl.out, q, r.k_cache, r.v_cache, d.dev["tables"], d.dev["lens"], r.scale,
-                     max_seq_len=d.max_len, partition_size=d.partition, variant=r.variant)
+                     max_seq_len=d.max_len, partition_size=d.partition, variant=d.variant,
+                     heads_per_cta=d.hpc, seq_order=d.dev.get("order"))
         if i >= 2:
             pa.set_profile_events(None, None)
             alg.append(pl.alg_bytes(j))
@@ -434,14 +440,15 @@ def time_main_kernel(pl: Planned, n: int, dev) -> dict:
     return {"us": us, "alg": alg}
 
 
-def roofline_of(main: dict, peak: float, peak_src: str, traffic) -> dict:
+def roofline_of(main: dict, peak: float, peak_src: str, traffic,
+                kernel: str = "decode_tc_kernel") -> dict:
     us = np.asarray(main["us"])
     per_launch = float(np.mean(main["alg"]))
     # bytes over time launch by launch, averaged: the launches differ in size
     achieved = float(np.sum(main["alg"]) / np.sum(us) / 1e3)
     return {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": traffic,
-            "kernel": "pa_decode main (decode_tc_kernel)", "peak_source": peak_src,
+            "kernel": f"pa_decode main ({kernel})", "peak_source": peak_src,
             "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
             "main_us_per_launch": round(float(us.mean()), 2),
             "main_us_median": round(float(np.median(us)), 2),
@@ -502,8 +509,9 @@ def run_ours(args, ws, rank, local):
     ms_per_step = elapsed_max / args.steps * 1e3
 
     peak, peak_src = hbm_peak()
-    traffic = traffic_from_profile(args.workload, float(np.mean(main["alg"])))
-    roof = roofline_of(main, peak, peak_src, traffic)
+    variant = pl.decodes[-1].variant or (1 if sh.dtype == "f32" else 2)
+    traffic = traffic_from_profile(args.workload, variant, float(np.mean(main["alg"])))
+    roof = roofline_of(main, peak, peak_src, traffic, DECODE_KERNELS[variant][0])
 
     # end to end through the public API with host buffers
     e2e = run_e2e(args, sh, pl.width, seed, pl.prefill, dev, ws)
@@ -526,8 +534,10 @@ def run_ours(args, ws, rank, local):
                                       "table rows, lengths, order written)",
                    "host_plan_op_by_op_us_per_step": round(pl.plan_py_us, 2),
                    "partition_tokens": pl.partitions(),
-                   "partition_policy": {-1: "per step, pa_decode_partition_for",
+                   "partition_policy": {-1: "per step, pa_decode_choose",
                                         0: "library default"}.get(args.partition, "fixed"),
+                   "kernels": sorted({DECODE_KERNELS[d.variant or 2][0] for d in pl.decodes}),
+                   "dispatch": "longest first; one-token appends fused into the decode",
                    "allocator_after_prefill": pl.alloc_info},
         "roofline": roof, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
     }
@@ -587,7 +597,8 @@ def measure_config(name: str, args, dev, peak: float) -> dict:
     torch.cuda.synchronize()
     step_us = [b_.elapsed_time(e_) * 1e3 for b_, e_ in evs]
     main = time_main_kernel(pl, 16, dev)
-    roof = roofline_of(main, peak, "", None)
+    variant = pl.decodes[-1].variant or 2
+    roof = roofline_of(main, peak, "", None, DECODE_KERNELS[variant][0])
     sh = pl.sh
     e2e_args = argparse.Namespace(**vars(args))
     e2e_args.workload, e2e_args.steps, e2e_args.e2e_steps, e2e_args.batch = name, n_e2e, n_e2e, 0
@@ -598,6 +609,7 @@ def measure_config(name: str, args, dev, peak: float) -> dict:
            "us_per_step": round(mean_step, 2),
            "kv_GBs_step": round(kv / (mean_step * 1e-6 * n_steps) / 1e9, 1),
            "main_us": roof["main_us_per_launch"], "main_GBs": roof["achieved"],
+           "kernels": sorted({DECODE_KERNELS[d.variant or 2][0] for d in pl.decodes}),
            "main_frac_of_peak": roof["frac"], "main_timed_launches": roof["timed_launches"],
            "partition_tokens": pl.partitions(),
            "tokens_per_s": round(pl.b / (mean_step * 1e-6), 1),

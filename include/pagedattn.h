@@ -230,6 +230,28 @@ int pa_append_decode(float *out, const void *q, const void *k_new, const void *v
                      const pa_decode_opts *opts, void *stream);
 
 /*
+ * The kernel, split length and heads per CTA for a decode batch, from the
+ * lengths as the caller knows them on the host; fills opts->partition_size,
+ * ->variant and ->heads_per_cta and leaves the other fields.  Measured on
+ * B200 (one GPU of this library's workloads, grids taking the sequences
+ * longest first):
+ *   - fp32 caches: the CUDA-core kernel, pa_decode_partition_for's split;
+ *   - 16-bit caches, block size 8 or 16, an even KV head count, and a step
+ *     that reads at least ~322 times the 512 KB one two-head CTA of 512
+ *     tokens reads (~170 MB at D 128): variant 3 with two KV heads per CTA
+ *     and 512-token splits.  Such a CTA cannot stream faster than ~18 GB/s
+ *     from its ring, so it needs ~29 us; when the whole read takes longer
+ *     than that at HBM speed, its fewer start-ups and the absent merge across
+ *     warps win (Llama-8B-shaped 60.4 -> 58.4 us, long context 173 -> 171
+ *     us, continuous mix 58.4 -> 52.2 us late in its run); below it, the
+ *     one-head CTAs' parallelism wins (beam search: 29.7 us against 35.8);
+ *   - otherwise variant 2 with pa_decode_partition_for's split.
+ * slots as for pa_decode_partition_for.  Host only.
+ */
+int pa_decode_choose(const int32_t *seq_lens_host, int num_seqs, int num_kv_heads,
+                     int head_dim, int block_size, int dtype, int slots, pa_decode_opts *opts);
+
+/*
  * Longest-first order of a decode batch for pa_decode_opts.seq_order, from
  * the lengths as the caller knows them on the host: order_out[i] is the
  * batch row of the i-th longest sequence, ties in batch order.  Host only.

@@ -452,6 +452,37 @@ int pa_decode_partition_for(const int32_t *seq_lens_host, int num_seqs, int num_
     return kDefaultPartition;
 }
 
+int pa_decode_choose(const int32_t *seq_lens_host, int num_seqs, int num_kv_heads,
+                     int head_dim, int block_size, int dtype, int slots, pa_decode_opts *opts) {
+    clear_error();
+    if (!opts) return fail(PA_ERR_INVALID_ARG, "NULL opts");
+    const int part = pa_decode_partition_for(seq_lens_host, num_seqs, num_kv_heads, head_dim,
+                                             block_size, dtype, slots);
+    if (part < 0) return part;
+    opts->partition_size = part;
+    opts->variant = dtype == PA_F32 ? 1 : 2;
+    opts->heads_per_cta = 0;
+    if (dtype == PA_F32 || num_kv_heads % 2 != 0 || (block_size != 8 && block_size != 16))
+        return PA_OK;
+    // A CTA of two KV heads over 512 tokens carries 512 KB at D 128 (16-bit)
+    // and streams at most ~18 GB/s from its 32 KB ring, ~29 us; it pays off
+    // (no merge across warps, half the start-ups) when the step's whole read
+    // takes at least that long at the HBM's ~5.8 TB/s, i.e. when the step
+    // reads at least ~322 such CTA loads' worth of bytes; below, the
+    // one-head CTAs' parallelism wins.
+    int64_t tokens = 0;
+    for (int s = 0; s < num_seqs; ++s) tokens += seq_lens_host[s];
+    const int64_t token_bytes = (int64_t)head_dim * 2 * 2;     // K + V of one head, 16-bit
+    const int64_t total = tokens * num_kv_heads * token_bytes;
+    const int64_t cta = (int64_t)kDefaultPartition * 2 * token_bytes;
+    if (total >= 322 * cta) {
+        opts->variant = 3;
+        opts->heads_per_cta = 2;
+        opts->partition_size = kDefaultPartition;
+    }
+    return PA_OK;
+}
+
 int pa_decode(float *out, const void *q, const void *k_cache, const void *v_cache,
               const int32_t *block_tables, const int32_t *seq_lens, int num_seqs,
               int num_heads, int num_kv_heads, int head_dim, int block_size,

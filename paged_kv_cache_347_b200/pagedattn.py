@@ -71,6 +71,20 @@ class pa_decode_opts(ctypes.Structure):
 
 _sig("pa_decode_opt", _i, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i,
      _vp, _sz, _c.POINTER(pa_decode_opts), _vp)
+_sig("pa_decode_choose", _i, _vp, _i, _i, _i, _i, _i, _i, _c.POINTER(pa_decode_opts))
+
+
+def decode_choose(seq_lens, num_kv_heads: int, head_dim: int, block_size: int, dtype,
+                  slots: int = 0) -> Tuple[int, int, int]:
+    """pa_decode_choose: (partition_size, variant, heads_per_cta) for a batch
+    of these host lengths."""
+    lens = np.ascontiguousarray(np.asarray(seq_lens), dtype=np.int32).reshape(-1)
+    code = DTYPE_CODE[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    o = pa_decode_opts()
+    _check(_lib.pa_decode_choose(lens.ctypes.data if lens.size else None, lens.size,
+                                 num_kv_heads, head_dim, block_size, code, slots,
+                                 ctypes.byref(o)), "pa_decode_choose")
+    return o.partition_size, o.variant, o.heads_per_cta
 _sig("pa_append_decode", _i, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i,
      _i, _i, _i, _f, _i, _vp, _sz, _c.POINTER(pa_decode_opts), _vp)
 _sig("pa_copy_blocks", _i, _vp, _vp, _vp, _i, _sz, _i, _vp)

@@ -17,9 +17,13 @@ runner turns a step into device actions in two phases:
   ``pa_reshape_and_cache``, and for a decode ``pa_decode``; all on the
   current stream, nothing synchronised.
 
-``partition_size`` 0 keeps pa_decode's 512-token splits; -1 picks, for each
-decode, pa_decode_partition_for's length from the batch's lengths (longer
-splits when 512 would leave a part-empty second wave of CTAs).
+Each decode's kernel and split length: with ``partition_size`` -1 (the
+default) and ``variant`` 0, pa_decode_choose's from the batch's lengths
+(variant 3 with two KV heads per CTA on steps that read enough, else variant
+2 with pa_decode_partition_for's split); a fixed ``partition_size`` (0 is
+pa_decode's 512) or ``variant`` is kept as given.  The grid takes the batch
+longest first, and a step's one-token appends go in with the decode
+(pa_append_decode), unless ``longest_first`` / ``fuse_append`` are off.
 
 ``run`` does both for one step, moving the host arrays to the device on the
 way.  Planning ahead lets a caller stage a whole run of steps in device
@@ -82,6 +86,8 @@ class Action:
     cu: Optional[np.ndarray] = None      # prefill: int32 [b + 1] row offsets
     max_q: int = 0
     partition: int = 0                   # decode: split length passed to pa_decode
+    variant: int = 0                     # decode: kernel (0 = pa_decode's own choice)
+    hpc: int = 0                         # decode: KV heads per CTA (variant 3)
     order: Optional[np.ndarray] = None   # decode: int32 [b], rows longest first
     ids: Optional[np.ndarray] = None     # write of plain appends: their sequence ids
     ones: bool = False                   # write: every append was one token
@@ -94,7 +100,7 @@ class PagedKVRunner:
     def __init__(self, num_blocks: int, block_size: int, num_heads: int, num_kv_heads: int,
                  head_dim: int, dtype: torch.dtype, scale: float, table_width: int,
                  free_order: Optional[Sequence[int]] = None, max_blocks_per_seq: int = 0,
-                 device: str = "cuda", partition_size: int = 0, variant: int = 0,
+                 device: str = "cuda", partition_size: int = -1, variant: int = 0,
                  prefill_variant: int = 0, longest_first: bool = True,
                  fuse_append: bool = True):
         self.alloc = pa.BlockAllocator(num_blocks, block_size, free_order, max_blocks_per_seq)
@@ -206,13 +212,10 @@ class PagedKVRunner:
                 elif kind == "decode":
                     dec_ids = np.asarray(op[1], np.int64)
                     tables, lens = self.alloc.block_tables(list(op[1]), self.width)
-                    part = self.partition_size
-                    if part < 0:
-                        part = pa.decode_partition_for(lens, self.num_kv_heads, self.head_dim,
-                                                       self.block_size, self.dtype)
+                    part, var, hpc = self._choose(lens)
                     acts.append(Action("decode", tables=tables, lens=lens,
                                        max_len=int(lens.max()) if lens.size else 0,
-                                       partition=part,
+                                       partition=part, variant=var, hpc=hpc,
                                        order=pa.decode_order(lens) if self.longest_first
                                        else None, ids=dec_ids))
                 elif kind == "prefill":
@@ -311,12 +314,13 @@ class PagedKVRunner:
                                         w.dev["slots"], self.k_cache, self.v_cache,
                                         a.dev["tables"], a.dev["lens"], self.scale,
                                         max_seq_len=a.max_len, partition_size=a.partition,
-                                        variant=self.variant, seq_order=a.dev.get("order"))
+                                        variant=a.variant, heads_per_cta=a.hpc,
+                                        seq_order=a.dev.get("order"))
                 else:
                     pa.pa_decode(o, q, self.k_cache, self.v_cache, a.dev["tables"],
                                  a.dev["lens"], self.scale, max_seq_len=a.max_len,
-                                 partition_size=a.partition, variant=self.variant,
-                                 seq_order=a.dev.get("order"))
+                                 partition_size=a.partition, variant=a.variant,
+                                 heads_per_cta=a.hpc, seq_order=a.dev.get("order"))
                 res = o
         return res
 
@@ -427,8 +431,9 @@ class PagedKVRunner:
                 tables = tables.reshape(b, self.width)
                 lens = hb[lay.off_lens:lay.off_lens + 4 * b].view(np.int32)
                 order = hb[lay.off_order:lay.off_order + 4 * b].view(np.int32)
+                part, var, hpc = self._choose(lens)
                 d = Action("decode", tables=tables, lens=lens.copy(), max_len=lay.max_seq_len,
-                           partition=self._partition(lens),
+                           partition=part, variant=var, hpc=hpc,
                            order=order if self.longest_first else None, ids=enc.decode_ids)
                 acts.append(d)
                 arrays += [(d, "tables", tables), (d, "lens", lens)]
@@ -440,12 +445,19 @@ class PagedKVRunner:
         return {"acts": acts, "arrays": arrays, "offs": offs, "bytes": lay.bytes, "slot": slot,
                 "host": host, "dev": devb}
 
-    def _partition(self, lens: np.ndarray) -> int:
-        part = self.partition_size
-        if part < 0:
-            part = pa.decode_partition_for(lens, self.num_kv_heads, self.head_dim,
-                                           self.block_size, self.dtype)
-        return part
+    def _choose(self, lens: np.ndarray):
+        """(split length, kernel, KV heads per CTA) of a decode: the runner's
+        fixed choices, else the library's for these lengths
+        (pa_decode_choose / pa_decode_partition_for)."""
+        part, var = self.partition_size, self.variant
+        if part >= 0:
+            return part, var, 0
+        if var == 0:
+            return pa.decode_choose(lens, self.num_kv_heads, self.head_dim, self.block_size,
+                                    self.dtype)
+        part = pa.decode_partition_for(lens, self.num_kv_heads, self.head_dim,
+                                       self.block_size, self.dtype)
+        return part, var, 0
 
     def _prepare_ops(self, ops) -> dict:
         """prepare() for steps pa_step_plan does not take: plan op by op,
@@ -539,7 +551,8 @@ class PagedKVRunner:
     def _graph_key(self, prep: dict, k_new: torch.Tensor, q: torch.Tensor):
         acts = prep["acts"]
         layout = tuple((a.kind, a.nrows, None if a.tables is None else a.tables.shape,
-                        a.partition, self._graph_bound(a.max_len) if a.kind == "decode" else 0,
+                        a.partition, a.variant, a.hpc,
+                        self._graph_bound(a.max_len) if a.kind == "decode" else 0,
                         a.order is not None, a.fused, a.fuse is not None)
                        for a in acts)
         return (layout, prep["bytes"], prep["slot"], prep["dev"].data_ptr(),

@@ -164,3 +164,28 @@ def test_step_launch_rejects_bad_arguments_before_any_cuda_call():
     assert L.pa_step_launch(None, None, None, None, 2, None, 1, 1, None, 1, None, None) == -1
     # an output graph without its event
     assert L.pa_step_launch(None, None, None, None, 0, None, 1, 1, None, 1, 1, None) == -1
+
+
+def test_decode_choice_follows_its_rule():
+    """pa_decode_choose: two-head CTAs of variant 3 with 512-token splits once
+    a step reads at least 322 x 512 KB (D 128, 16-bit), else variant 2 with
+    pa_decode_partition_for's split; fp32 takes the CUDA-core kernel."""
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    bf = torch.bfloat16
+    # 8 x 32768 tokens x 8 heads x 512 B = 1.07 GB
+    assert pa.decode_choose([32768] * 8, 8, 128, 16, bf, slots=888) == (512, 3, 2)
+    # 16 beams of ~2300 tokens: 151 MB < 322 x 512 KB
+    assert pa.decode_choose([2300] * 16, 8, 128, 16, bf, slots=888) == (512, 2, 0)
+    # just on either side of the threshold
+    need = 322 * 512 * 2 * 512          # bytes
+    per_token = 8 * 512                 # 8 KV heads x 512 B
+    assert pa.decode_choose([need // per_token], 8, 128, 16, bf, slots=888)[1] == 3
+    assert pa.decode_choose([need // per_token - 1], 8, 128, 16, bf, slots=888)[1] == 2
+    # block sizes other than 8 and 16, odd KV head counts, fp32
+    assert pa.decode_choose([32768] * 8, 8, 128, 32, bf, slots=888)[1] == 2
+    assert pa.decode_choose([32768] * 8, 7, 128, 16, bf, slots=888)[1] == 2
+    assert pa.decode_choose([32768] * 8, 8, 128, 16, torch.float32, slots=888)[1:] == (1, 0)
+    # variant 2 keeps pa_decode_partition_for's split
+    lens = [600, 1300] * 16
+    assert pa.decode_choose(lens, 8, 128, 32, bf, slots=888) == (
+        pa.decode_partition_for(lens, 8, 128, 32, bf, slots=888), 2, 0)
