@@ -853,13 +853,24 @@ def study_blocksize(args):
         d = [a for a in acts if a.kind == "decode"][0]
         o = torch.empty(dev[2].shape, dtype=torch.float32, device="cuda")
         r.execute(acts, *dev)
+        # pa_decode's plain launch (variant 2, batch order, 512-token splits),
+        # and the runner's choice (kernel, split, longest first)
         ms = _events_ms(lambda: pa.pa_decode(o, dev[2], r.k_cache, r.v_cache, d.dev["tables"],
                                              d.dev["lens"], r.scale, max_seq_len=d.max_len),
                         reps=20)
+        ms_c = _events_ms(lambda: pa.pa_decode(o, dev[2], r.k_cache, r.v_cache, d.dev["tables"],
+                                               d.dev["lens"], r.scale, max_seq_len=d.max_len,
+                                               partition_size=d.partition, variant=d.variant,
+                                               heads_per_cta=d.hpc,
+                                               seq_order=d.dev.get("order")), reps=20)
         kvb = kv_bytes(d.lens, 8, 128, 2)
         st = r.alloc.stats()
         out["rows"].append({"block_size": bs, "decode_us": round(ms * 1e3, 2),
                             "kv_GBs": round(kvb / ms / 1e6, 1),
+                            "chosen_decode_us": round(ms_c * 1e3, 2),
+                            "chosen_kv_GBs": round(kvb / ms_c / 1e6, 1),
+                            "chosen": {"kernel": DECODE_KERNELS[d.variant or 2][0],
+                                       "partition": d.partition, "heads_per_cta": d.hpc},
                             "kernel": "tensor-core, " + ("cp.async" if bs < 8 else "TMA"),
                             "reserved_slots": st["reserved_slots"],
                             "logical_tokens": st["logical_tokens"],
