@@ -624,8 +624,118 @@ def measure_config(name: str, args, dev, peak: float) -> dict:
     return out
 
 
+def _chunks(enc, max_new: int):
+    """A step's events cut into pieces of at most max_new appended tokens
+    (a long append split across pieces; appends stay in order, so the rows
+    of each piece are the next slice of the step's K/V rows).  Yields
+    (events, first row, end row)."""
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    cur, rows, r0 = [], 0, 0
+    for code, x, y in enc.events.tolist():
+        if code != pa.EV_APPEND:
+            cur.append((code, x, y))
+            continue
+        while y > 0:
+            take = min(y, max_new - rows)
+            cur.append((code, x, take))
+            rows += take
+            y -= take
+            if rows == max_new:
+                yield np.asarray(cur, np.int64).reshape(-1, 3), r0, r0 + rows
+                cur, r0, rows = [], r0 + rows, 0
+    if cur:
+        yield np.asarray(cur, np.int64).reshape(-1, 3), r0, r0 + rows
+
+
+def _decode_lens(sh, encs, width):
+    """Each step's decode lengths, from the same events replayed on a host
+    replica of the allocator (for the byte count of the metric)."""
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    alloc = pa.BlockAllocator(sh.num_blocks, sh.block_size, sh.free_order)
+    stage = np.zeros(1 << 16, np.uint8)
+    out = []
+    for enc in encs:
+        lay = alloc.step_layout(enc.events, enc.decode_ids.size, width)
+        if lay.bytes > stage.nbytes:
+            stage = np.zeros(lay.bytes, np.uint8)
+        lay = alloc.step_plan(enc.events, enc.decode_ids, width, stage)
+        b = enc.decode_ids.size
+        out.append(stage[lay.off_lens:lay.off_lens + 4 * b].view(np.int32).copy())
+    return out
+
+
+def run_e2e_runtime(args, sh, width, seed, dev, ws):
+    """Live steps through the native runtime (pa_runtime: one library call
+    per step -- the allocator's events, the decode's choice, the copies in,
+    the kernels from a CUDA graph, the output's copy back), inputs in
+    page-locked host memory, every output read one step behind."""
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    from paged_kv_cache_347_b200.runner import PagedKVRunner
+    n = max(1, min(args.steps, args.e2e_steps))
+    w = min(args.warmup, 3)
+    wl, _ = make_workload(args.workload, n + w, seed, args.batch)
+    steps = list(wl.steps)
+    dt = {"f32": torch.float32, "bf16": torch.bfloat16, "f16": torch.float16}[sh.dtype]
+    dims = (sh.num_blocks, sh.num_kv_heads, sh.block_size, sh.head_dim)
+    kc = torch.zeros(dims, dtype=dt, device=dev)
+    vc = torch.zeros_like(kc)
+    # a step's host inputs: its events as arrays (the form a runtime keeps
+    # them in), new K/V rows and queries in page-locked memory
+    encs = [PagedKVRunner.encode_ops(st.ops) for st in steps]
+    lens = _decode_lens(sh, encs, width)
+    b = steps[1].q.shape[0]
+    max_new = max(16384, max(st.k_new.shape[0] for st in steps[1:]))
+    rt = pa.Runtime(kc, vc, sh.num_heads, width, b, max_new, sh.scale, sh.free_order)
+    k0, v0 = steps[0].k_new.pin_memory(), steps[0].v_new.pin_memory()
+    none = np.empty(0, np.int64)
+    for ev, r0, r1 in _chunks(encs[0], max_new):      # the prefill, untimed
+        rt.wait_event(rt.step(ev, none, k0[r0:r1], v0[r0:r1], None, None))
+    rt.wait()
+    host = [(encs[i], steps[i].k_new.pin_memory(), steps[i].v_new.pin_memory(),
+             steps[i].q.pin_memory()) for i in range(1, len(steps))]
+    outs = [torch.empty((b, sh.num_heads, sh.head_dim), dtype=torch.float32).pin_memory()
+            for _ in range(2)]
+
+    def loop(first, count):
+        pending = []
+        for i in range(first, first + count):
+            enc, k, v, q = host[i]
+            pending.append(rt.step(enc.events, enc.decode_ids, k, v, q, outs[i & 1]))
+            if len(pending) > 1:
+                rt.wait_event(pending.pop(0))
+        for ev in pending:
+            rt.wait_event(ev)
+
+    loop(0, w)
+    st0 = rt.stats()
+    barrier(ws)
+    t = time.perf_counter()
+    loop(w, n)
+    el = time.perf_counter() - t
+    st1 = rt.stats()
+    kv = sum(kv_bytes(lens[1 + i], sh.num_kv_heads, sh.head_dim, sh.elem_bytes)
+             for i in range(w, w + n))
+    h2d = sum(host[i][1].nbytes + host[i][2].nbytes + host[i][3].nbytes
+              for i in range(w, w + n)) / n
+    el, total = aggregate(el, float(kv), ws, dev)
+    return {"value": round(total / el / 1e9, 1), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(outs[0].nbytes),
+            "steps": n, "us_per_step": round(el / n * 1e6, 2),
+            "graph_replayed_steps": st1["replays"] - st0["replays"],
+            "path": "pa_runtime (one library call per step)",
+            "h2d_note": "new K/V rows and queries counted; the step's arrays (slots, table "
+                        "rows, lengths, order) cross in the same copy stream",
+            "outputs_read": "one step behind the launches"}
+
+
 def run_e2e(args, sh, width, seed, prefill, dev, ws):
-    """Live steps through the public API (PagedKVRunner prepare / stage_graph
+    if not args.e2e_python:
+        return run_e2e_runtime(args, sh, width, seed, dev, ws)
+    return run_e2e_python(args, sh, width, seed, prefill, dev, ws)
+
+
+def run_e2e_python(args, sh, width, seed, prefill, dev, ws):
+    """Live steps through the Python runner (PagedKVRunner prepare / stage_graph
     / replay_graph, or launch when a step has no graph form): host allocator,
     inputs copied from pinned host memory, every output copied back to pinned
     host memory and waited for, one step behind the launches unless
@@ -953,6 +1063,8 @@ def main():
                     help="e2e: wait for each step's output before launching the next")
     ap.add_argument("--no-prefill", action="store_true",
                     help="skip the chunked-prefill line added to the N = 1 bench output")
+    ap.add_argument("--e2e-python", action="store_true",
+                    help="e2e through the Python runner instead of the native runtime")
     ap.add_argument("--no-graph", action="store_true",
                     help="e2e: launch every step eagerly instead of replaying CUDA graphs")
     ap.add_argument("--cpu-budget", type=float, default=15.0)

@@ -26,7 +26,8 @@
  *     error, pa_last_error() gives a message for the calling thread.
  *   - Device pointers are plain CUDA device addresses owned by the caller
  *     (e.g. allocated by PyTorch); the library allocates no device memory and
- *     keeps no pointer after a call returns.  Host pointers are plain host
+ *     keeps no pointer after a call returns (except a pa_runtime, which owns
+ *     its buffers and keeps the caches it is given: see "Runtime").  Host pointers are plain host
  *     memory owned by the caller.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Device
  *     work is enqueued on it and the call returns without synchronising;
@@ -603,6 +604,67 @@ int pa_step_launch(void *stream_in, void *stream_run, void *stream_out,
                    const pa_host_copy *copies, int n_copies, void *wait_before_in,
                    void *event_in, void *graph_run, void *wait_before_run, void *event_run,
                    void *graph_out, void *event_out);
+
+/* ------------------------------------------------------------------------
+ * Runtime: a decode runtime around the calls above, one call per host-fed
+ * step (the pages leave tables and allocation to a runtime that owns them:
+ * sanketn26 "PagedAttention", "Use a runtime that owns the blocks").
+ *
+ * pa_rt_create makes one for caller-owned caches k_cache, v_cache ([NB][Hkv]
+ * [bs][D], `dtype`, device, left as they are) with its own allocator
+ * (free_order as for pa_alloc_create).  Unlike the rest of the library it
+ * owns device memory: two staging buffers (arrays + the largest step's new
+ * K/V rows and queries), the split workspace, two output buffers, plus two
+ * page-locked host buffers, three non-blocking streams and its CUDA graphs;
+ * pa_rt_destroy waits for its streams and frees them.
+ *
+ * pa_rt_step takes a step's events as pa_step_plan does (decode_ids: the
+ * decode batch), its new K/V rows k_new, v_new (host, [n new tokens][Hkv][D],
+ * in event order), its queries q (host, [num_seqs][Hq][D]) and a host output
+ * buffer out (float32 [num_seqs][Hq][D]); host buffers should be page-locked
+ * (the copies are asynchronous).  It applies the events (pa_step_plan),
+ * chooses the decode (pa_decode_choose, longest first; one-token appends of
+ * exactly the decode batch go in with it, pa_append_decode), copies the
+ * step's inputs in on one stream, runs its kernels on another (from a CUDA
+ * graph of the step's layout once that layout has run once; steps with
+ * copy-on-write copies run directly) and copies the output out on a third.
+ * It returns at once; *ready (if non-NULL) receives a cudaEvent_t that
+ * completes once out holds the step's output and the inputs have been read.
+ * Steps alternate between two staging slots: a step's host work (this call)
+ * overlaps the previous step's kernels, and the call waits only for the copy
+ * in of the step two back.  Keep the inputs unchanged and do not read out
+ * until *ready completes.
+ *   - Limits: num_seqs <= max_batch, new tokens <= max_new_tokens, table rows
+ *     of table_width entries; beyond them PA_ERR_INVALID_ARG before anything
+ *     is applied.  Errors of pa_step_plan are returned as it returns them.
+ *   - A CUDA error part-way leaves the runtime's allocator ahead of its
+ *     device work: destroy the runtime.
+ * pa_rt_wait synchronises the runtime's streams; pa_event_wait waits for an
+ * event (e.g. *ready); pa_rt_allocator gives its allocator (for queries and
+ * for ops the events do not cover); pa_rt_stats counts steps, graph replays
+ * and captures.
+ * ---------------------------------------------------------------------- */
+typedef struct pa_runtime pa_runtime;
+
+typedef struct {
+    int num_blocks, block_size, num_heads, num_kv_heads, head_dim, dtype;
+    int table_width;         /* table entries per decode row */
+    int max_batch;           /* decode rows per step */
+    int max_new_tokens;      /* appended tokens per step */
+    int max_blocks_per_seq;  /* the allocator's bound, 0 = none */
+    float scale;
+} pa_runtime_config;
+
+int pa_rt_create(pa_runtime **out, const pa_runtime_config *cfg, void *k_cache, void *v_cache,
+                 const int32_t *free_order);
+void pa_rt_destroy(pa_runtime *rt);
+pa_alloc *pa_rt_allocator(pa_runtime *rt);
+int pa_rt_step(pa_runtime *rt, const int64_t *events, int n_events, const int64_t *decode_ids,
+               int num_seqs, const void *k_new, const void *v_new, const void *q, float *out,
+               void **ready);
+int pa_rt_wait(pa_runtime *rt);
+int pa_event_wait(void *event);
+int pa_rt_stats(const pa_runtime *rt, int64_t *steps, int64_t *replays, int64_t *captures);
 
 int pa_alloc_stats(const pa_alloc *a, pa_alloc_stats_t *out);
 

@@ -140,6 +140,22 @@ def decode_order(seq_lens) -> np.ndarray:
 
 
 _sig("pa_step_plan", _i, _vp, _vp, _i, _vp, _i, _i, _vp, _sz, _vp, _c.POINTER(pa_step_layout))
+
+
+class pa_runtime_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in (
+        "num_blocks", "block_size", "num_heads", "num_kv_heads", "head_dim", "dtype",
+        "table_width", "max_batch", "max_new_tokens", "max_blocks_per_seq")] + [
+        ("scale", ctypes.c_float)]
+
+
+_sig("pa_rt_create", _i, _c.POINTER(_vp), _c.POINTER(pa_runtime_config), _vp, _vp, _vp)
+_sig("pa_rt_destroy", None, _vp)
+_sig("pa_rt_allocator", _vp, _vp)
+_sig("pa_rt_step", _i, _vp, _vp, _i, _vp, _i, _vp, _vp, _vp, _vp, _c.POINTER(_vp))
+_sig("pa_rt_wait", _i, _vp)
+_sig("pa_event_wait", _i, _vp)
+_sig("pa_rt_stats", _i, _vp, _vp, _vp, _vp)
 EV_ADD, EV_FREE, EV_FORK, EV_APPEND, EV_DECODE = 1, 2, 3, 4, 5
 _sig("pa_alloc_free_list", _i, _vp, _vp, _i, _vp)
 _sig("pa_alloc_refcount", _i, _vp, _i)
@@ -470,8 +486,18 @@ def _np_ptr(a: np.ndarray) -> int:
 class BlockAllocator:
     """Handle on the C++ host allocator (pa_alloc_*, pa_seq_*)."""
 
+    @classmethod
+    def view(cls, handle: int, num_blocks: int, block_size: int) -> "BlockAllocator":
+        """A handle on an allocator someone else owns (a pa_runtime's)."""
+        self = cls.__new__(cls)
+        self._h = ctypes.c_void_p(handle)
+        self._owned = False
+        self.num_blocks, self.block_size = num_blocks, block_size
+        return self
+
     def __init__(self, num_blocks: int, block_size: int,
                  free_order: Optional[Sequence[int]] = None, max_blocks_per_seq: int = 0):
+        self._owned = True
         self._h = ctypes.c_void_p()
         fo = None
         if free_order is not None:
@@ -488,7 +514,7 @@ class BlockAllocator:
         # bound at definition time: at interpreter shutdown the module globals
         # (ctypes among them) may already be None
         h = getattr(self, "_h", None)
-        if h is not None and h.value:
+        if h is not None and h.value and getattr(self, "_owned", True):
             _destroy(h)
             self._h = _null()
 
@@ -628,3 +654,61 @@ class BlockAllocator:
     def seq_swap_in(self, seq_id: int) -> np.ndarray:
         """(host block, device block) pairs, in logical order."""
         return self._swap(_lib.pa_seq_swap_in, "pa_seq_swap_in", seq_id)
+
+
+# ----------------------------------------------------------------- runtime
+class Runtime:
+    """pa_runtime: one C call per host-fed decode step over caller-owned
+    caches (see pagedattn.h, "Runtime").  Host tensors passed to step()
+    should be page-locked; the step's output is in ``out`` once the returned
+    event has completed (wait_event)."""
+
+    def __init__(self, k_cache: torch.Tensor, v_cache: torch.Tensor, num_heads: int,
+                 table_width: int, max_batch: int, max_new_tokens: int, scale: float,
+                 free_order: Optional[Sequence[int]] = None, max_blocks_per_seq: int = 0):
+        NB, Hkv, bs, D = k_cache.shape
+        self.k_cache, self.v_cache = k_cache, v_cache   # kept alive with the runtime
+        self.cfg = pa_runtime_config(NB, bs, num_heads, Hkv, D, DTYPE_CODE[k_cache.dtype],
+                                     table_width, max_batch, max_new_tokens, max_blocks_per_seq,
+                                     scale)
+        fo = None
+        if free_order is not None:
+            fo = np.ascontiguousarray(free_order, dtype=np.int32)
+        self._h = ctypes.c_void_p()
+        _check(_lib.pa_rt_create(ctypes.byref(self._h), ctypes.byref(self.cfg),
+                                 _dev(k_cache, "k_cache"), _dev(v_cache, "v_cache", k_cache.dtype),
+                                 None if fo is None else _np_ptr(fo)), "pa_rt_create")
+        self.alloc = BlockAllocator.view(_lib.pa_rt_allocator(self._h), NB, bs)
+        self._ready = ctypes.c_void_p()
+
+    def __del__(self, _destroy=_lib.pa_rt_destroy, _null=ctypes.c_void_p):
+        h = getattr(self, "_h", None)
+        if h is not None and h.value:
+            _destroy(h)
+            self._h = _null()
+
+    def step(self, events: np.ndarray, decode_ids: np.ndarray, k_new: Optional[torch.Tensor],
+             v_new: Optional[torch.Tensor], q: Optional[torch.Tensor],
+             out: Optional[torch.Tensor]) -> int:
+        """One step; returns its "ready" event (a cudaEvent_t as an int)."""
+        rc = _lib.pa_rt_step(self._h, events.ctypes.data, events.shape[0],
+                             decode_ids.ctypes.data if decode_ids.size else None, decode_ids.size,
+                             None if k_new is None else k_new.data_ptr(),
+                             None if v_new is None else v_new.data_ptr(),
+                             None if q is None else q.data_ptr(),
+                             None if out is None else out.data_ptr(), ctypes.byref(self._ready))
+        if rc != 0:
+            raise PagedAttnError(rc, "pa_rt_step")
+        return self._ready.value
+
+    @staticmethod
+    def wait_event(event: int) -> None:
+        _check(_lib.pa_event_wait(event), "pa_event_wait")
+
+    def wait(self) -> None:
+        _check(_lib.pa_rt_wait(self._h), "pa_rt_wait")
+
+    def stats(self) -> dict:
+        v = [ctypes.c_int64() for _ in range(3)]
+        _check(_lib.pa_rt_stats(self._h, *(ctypes.addressof(x) for x in v)), "pa_rt_stats")
+        return {"steps": v[0].value, "replays": v[1].value, "captures": v[2].value}
