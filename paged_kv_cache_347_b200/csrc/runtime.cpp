@@ -351,8 +351,12 @@ int pa_rt_step(pa_runtime *rt, const int64_t *events, int n_events, const int64_
     const bool graphable = lay.n_pairs == 0 && decode_at >= 0 && num_seqs > 0;
     std::vector<int64_t> key;
     if (graphable) {
-        key = {s, lay.n_slots, num_seqs, opts.partition_size, opts.variant, opts.heads_per_cta,
-               max_len, (int64_t)rt->acts.size()};
+        // everything the captured launches take: the array offsets (they
+        // follow the events' counts), the decode's choice and bound, and the
+        // actions' row ranges and fusion
+        key = {s, lay.n_slots, num_seqs, lay.off_pairs, lay.off_tables, lay.off_lens,
+               lay.off_order, opts.partition_size, opts.variant, opts.heads_per_cta, max_len,
+               (int64_t)rt->acts.size()};
         for (const Act &a : rt->acts) {
             key.push_back(a.kind);
             key.push_back(a.r0);
