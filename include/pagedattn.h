@@ -234,20 +234,22 @@ int pa_append_decode(float *out, const void *q, const void *k_new, const void *v
  * The kernel, split length and heads per CTA for a decode batch, from the
  * lengths as the caller knows them on the host; fills opts->partition_size,
  * ->variant and ->heads_per_cta and leaves the other fields.  Measured on
- * B200 (one GPU of this library's workloads, grids taking the sequences
- * longest first):
+ * B200 with the grid taking the sequences longest first:
  *   - fp32 caches: the CUDA-core kernel, pa_decode_partition_for's split;
- *   - 16-bit caches, block size 8 or 16, an even KV head count, and a step
- *     that reads at least ~322 times the 512 KB one two-head CTA of 512
- *     tokens reads (~170 MB at D 128): variant 3 with two KV heads per CTA
- *     and 512-token splits.  Such a CTA cannot stream faster than ~18 GB/s
- *     from its ring, so it needs ~29 us; when the whole read takes longer
- *     than that at HBM speed, its fewer start-ups and the absent merge across
- *     warps win (Llama-8B-shaped 60.4 -> 58.4 us, long context 173 -> 171
- *     us, continuous mix 58.4 -> 52.2 us late in its run); below it, the
- *     one-head CTAs' parallelism wins (beam search: 29.7 us against 35.8);
+ *   - 16-bit caches, block size 8 or 16, an even KV head count: variant 3
+ *     with two KV heads per CTA (it matched or beat variant 2 on every batch
+ *     measured, once its split fits the batch), and the split by the waves
+ *     of CTAs it makes: the largest of 1024, 768, 640, 512, 384, 256 tokens
+ *     whose CTAs ((num_kv_heads / 2) x the splits of each sequence) fill
+ *     between 0.6 and 1 wave of `slots`; if even 1024 needs more than a wave,
+ *     512; if even 256 fills less than 0.6 of one, 256.  (Beam search, 16
+ *     sequences of ~2070 tokens: 256, 25.6 us against 29.7 for variant 2 at
+ *     512; Llama-8B-shaped: 512, 58.4 us against 60.4; 64 such sequences:
+ *     1024, 101.3 us against 107.6 at 512's 1.4 waves; long context and the
+ *     continuous mix: 512.)
  *   - otherwise variant 2 with pa_decode_partition_for's split.
- * slots as for pa_decode_partition_for.  Host only.
+ * slots: CTAs resident at once; 0 asks the device (the chosen kernel's
+ * occupancy times the SM count).  Host only.
  */
 int pa_decode_choose(const int32_t *seq_lens_host, int num_seqs, int num_kv_heads,
                      int head_dim, int block_size, int dtype, int slots, pa_decode_opts *opts);

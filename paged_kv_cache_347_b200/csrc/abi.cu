@@ -464,22 +464,45 @@ int pa_decode_choose(const int32_t *seq_lens_host, int num_seqs, int num_kv_head
     opts->heads_per_cta = 0;
     if (dtype == PA_F32 || num_kv_heads % 2 != 0 || (block_size != 8 && block_size != 16))
         return PA_OK;
-    // A CTA of two KV heads over 512 tokens carries 512 KB at D 128 (16-bit)
-    // and streams at most ~18 GB/s from its 32 KB ring, ~29 us; it pays off
-    // (no merge across warps, half the start-ups) when the step's whole read
-    // takes at least that long at the HBM's ~5.8 TB/s, i.e. when the step
-    // reads at least ~322 such CTA loads' worth of bytes; below, the
-    // one-head CTAs' parallelism wins.
-    int64_t tokens = 0;
-    for (int s = 0; s < num_seqs; ++s) tokens += seq_lens_host[s];
-    const int64_t token_bytes = (int64_t)head_dim * 2 * 2;     // K + V of one head, 16-bit
-    const int64_t total = tokens * num_kv_heads * token_bytes;
-    const int64_t cta = (int64_t)kDefaultPartition * 2 * token_bytes;
-    if (total >= 322 * cta) {
-        opts->variant = 3;
-        opts->heads_per_cta = 2;
-        opts->partition_size = kDefaultPartition;
+    // Two KV heads per CTA, one per warp (variant 3), with the split chosen
+    // by the waves of CTAs it makes: the largest split whose CTAs fill
+    // between 0.6 and 1 wave of the CTAs the device holds at once (one wave,
+    // every CTA streaming from the start, none so long that its ring's rate
+    // bounds the launch); if even 1024-token splits need more than a wave,
+    // 512 (several waves, short CTAs to balance them); if even 256-token
+    // splits fill less than 0.6 of a wave, 256 (the most parallelism).
+    if (slots == 0) {
+        static std::atomic<int> cache[kMaxDevices][2][2][2];
+        const int dev = current_device();
+        if (dev < 0 || dev >= kMaxDevices) return fail(PA_ERR_CUDA, "no CUDA device");
+        std::atomic<int> &c = cache[dev][dtype == PA_F16][head_dim == 128][block_size == 16];
+        int per_sm = c.load(std::memory_order_relaxed);
+        if (per_sm <= 0) {
+            per_sm = decode_hw2_resident_per_sm(dtype, head_dim, block_size);
+            if (per_sm <= 0) return fail(PA_ERR_CUDA, "occupancy query failed");
+            c.store(per_sm, std::memory_order_relaxed);
+        }
+        slots = per_sm * num_sms();
     }
+    auto ctas = [&](int p) {
+        int64_t n = 0;
+        for (int s = 0; s < num_seqs; ++s)
+            n += seq_lens_host[s] <= p ? 1 : (seq_lens_host[s] + p - 1) / p;
+        return n * (num_kv_heads / 2);
+    };
+    static const int kSplits[] = {1024, 768, 640, 512, 384, 256};
+    int chosen = 0;
+    for (int p : kSplits) {
+        const int64_t n = ctas(p);
+        if (10 * n >= 6 * (int64_t)slots && n <= slots) {
+            chosen = p;
+            break;
+        }
+    }
+    if (chosen == 0) chosen = ctas(1024) > slots ? kDefaultPartition : 256;
+    opts->variant = 3;
+    opts->heads_per_cta = 2;
+    opts->partition_size = chosen;
     return PA_OK;
 }
 

@@ -464,6 +464,43 @@ static cudaError_t launch_d(const DecodeParams &p, int W, const CUtensorMap &mk,
 
 }  // namespace hw
 
+namespace hw {
+// CTAs of an instance resident per SM (its shared-memory attribute set first,
+// as launch_inst does), or -1.
+template <typename T, int D, int BS, int W>
+static int resident_w() {
+    constexpr int kStage = 2 * (D / 64) * W * (BS < 16 ? 16 : BS) * kRowBytes;
+    constexpr int NS = kStage >= 32768 ? 2 : (32768 / kStage < 4 ? 32768 / kStage : 4);
+    using C = Cfg<T, D, BS, W, NS>;
+    if (cudaFuncSetAttribute(decode_hw_kernel<T, D, BS, W, NS>,
+                             cudaFuncAttributeMaxDynamicSharedMemorySize, C::kDynSmem) != cudaSuccess)
+        return -1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, decode_hw_kernel<T, D, BS, W, NS>,
+                                                      C::kThreads, C::kDynSmem) != cudaSuccess)
+        return -1;
+    return n;
+}
+template <typename T, int D>
+static int resident_d(int block_size) {
+    switch (block_size) {
+    case 8: return resident_w<T, D, 8, 2>();
+    case 16: return resident_w<T, D, 16, 2>();
+    default: return -1;
+    }
+}
+}  // namespace hw
+
+int decode_hw2_resident_per_sm(int dtype, int head_dim, int block_size) {
+    if (dtype != PA_BF16 && dtype != PA_F16) return -1;
+    if (head_dim != 64 && head_dim != 128) return -1;
+    if (dtype == PA_BF16)
+        return head_dim == 128 ? hw::resident_d<__nv_bfloat16, 128>(block_size)
+                               : hw::resident_d<__nv_bfloat16, 64>(block_size);
+    return head_dim == 128 ? hw::resident_d<__half, 128>(block_size)
+                           : hw::resident_d<__half, 64>(block_size);
+}
+
 cudaError_t launch_decode_hw(const DecodeParams &p, int dtype, int heads_per_cta,
                              cudaStream_t stream) {
     if (dtype != PA_BF16 && dtype != PA_F16) return cudaErrorNotSupported;

@@ -66,6 +66,9 @@ cudaError_t launch_decode_tc(const DecodeParams &p, int dtype, cudaStream_t stre
 // 64) heads per CTA.  cudaErrorNotSupported for shapes it does not cover.
 cudaError_t launch_decode_hw(const DecodeParams &p, int dtype, int heads_per_cta,
                              cudaStream_t stream);
+// CTAs of that kernel with two KV heads per CTA resident per SM (block size 8
+// or 16), or -1
+int decode_hw2_resident_per_sm(int dtype, int head_dim, int block_size);
 // CTAs of the tensor-core decode kernel for this shape resident per SM, or -1
 int decode_tc_resident_per_sm(int dtype, int head_dim, int block_size);
 

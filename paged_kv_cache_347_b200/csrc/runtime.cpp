@@ -190,8 +190,9 @@ int pa_rt_create(pa_runtime **out, const pa_runtime_config *cfg, void *k_cache, 
     rt->off_q = rt->off_v + rt->kv_cap;
     rt->slot_bytes = rt->off_q + rt->q_cap;
     rt->out_bytes = (size_t)c.max_batch * c.num_heads * c.head_dim * sizeof(float);
+    // partials for the shortest split pa_decode_choose picks (256 tokens)
     rt->ws_bytes = pa_decode_workspace_size(c.max_batch, c.num_heads, c.head_dim,
-                                            c.table_width * c.block_size, 512);
+                                            c.table_width * c.block_size, 256);
     cudaError_t e = cudaGetDevice(&rt->dev);
     for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
         e = cudaHostAlloc(reinterpret_cast<void **>(&rt->host[i]), rt->arrays_cap,

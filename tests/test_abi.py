@@ -4,6 +4,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 import torch
 
@@ -166,26 +167,46 @@ def test_step_launch_rejects_bad_arguments_before_any_cuda_call():
     assert L.pa_step_launch(None, None, None, None, 0, None, 1, 1, None, 1, 1, None) == -1
 
 
-def test_decode_choice_follows_its_rule():
-    """pa_decode_choose: two-head CTAs of variant 3 with 512-token splits once
-    a step reads at least 322 x 512 KB (D 128, 16-bit), else variant 2 with
-    pa_decode_partition_for's split; fp32 takes the CUDA-core kernel."""
+def _choice_by_rule(lens, hkv, slots):
+    """pa_decode_choose's rule for two-head CTAs, evaluated here by brute force."""
+    def ctas(p):
+        return (hkv // 2) * sum(1 if L <= p else -(-L // p) for L in lens)
+    for p in (1024, 768, 640, 512, 384, 256):
+        if 0.6 * slots <= ctas(p) <= slots:
+            return p
+    return 512 if ctas(1024) > slots else 256
+
+
+@pytest.mark.parametrize("lens", [
+    [32768] * 8,                                   # many waves at any split: 512
+    [2070] * 16,                                   # beam-shaped: 256
+    list(np.random.default_rng(1).integers(512, 4097, 32)),    # Llama-8B-shaped
+    list(np.random.default_rng(2).integers(512, 4097, 64)),
+    [150] * 256,                                   # 1024 one-split CTAs: 512
+    [100, 30],                                     # tiny: 256
+    [0, 1, 511, 512, 513, 4096, 4097] * 20,
+])
+def test_decode_choice_follows_its_rule(lens):
+    """pa_decode_choose: for 16-bit caches with block size 8 or 16 and an even
+    KV head count, two-head CTAs (variant 3) with the split the wave rule
+    gives; otherwise variant 2 (fp32: 1) with pa_decode_partition_for's split."""
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    lens = [int(x) for x in lens]
+    bf = torch.bfloat16
+    for bs in (8, 16):
+        assert pa.decode_choose(lens, 8, 128, bs, bf, slots=888) == (
+            _choice_by_rule(lens, 8, 888), 3, 2)
+    for bs in (4, 32, 64):
+        assert pa.decode_choose(lens, 8, 128, bs, bf, slots=888) == (
+            pa.decode_partition_for(lens, 8, 128, bs, bf, slots=888), 2, 0)
+    assert pa.decode_choose(lens, 7, 128, 16, bf, slots=888)[1:] == (2, 0)
+    assert pa.decode_choose(lens, 8, 128, 16, torch.float32, slots=888)[1:] == (1, 0)
+
+
+def test_decode_choice_on_the_bench_shapes():
     from paged_kv_cache_347_b200 import pagedattn as pa
     bf = torch.bfloat16
-    # 8 x 32768 tokens x 8 heads x 512 B = 1.07 GB
     assert pa.decode_choose([32768] * 8, 8, 128, 16, bf, slots=888) == (512, 3, 2)
-    # 16 beams of ~2300 tokens: 151 MB < 322 x 512 KB
-    assert pa.decode_choose([2300] * 16, 8, 128, 16, bf, slots=888) == (512, 2, 0)
-    # just on either side of the threshold
-    need = 322 * 512 * 2 * 512          # bytes
-    per_token = 8 * 512                 # 8 KV heads x 512 B
-    assert pa.decode_choose([need // per_token], 8, 128, 16, bf, slots=888)[1] == 3
-    assert pa.decode_choose([need // per_token - 1], 8, 128, 16, bf, slots=888)[1] == 2
-    # block sizes other than 8 and 16, odd KV head counts, fp32
-    assert pa.decode_choose([32768] * 8, 8, 128, 32, bf, slots=888)[1] == 2
-    assert pa.decode_choose([32768] * 8, 7, 128, 16, bf, slots=888)[1] == 2
-    assert pa.decode_choose([32768] * 8, 8, 128, 16, torch.float32, slots=888)[1:] == (1, 0)
-    # variant 2 keeps pa_decode_partition_for's split
-    lens = [600, 1300] * 16
-    assert pa.decode_choose(lens, 8, 128, 32, bf, slots=888) == (
-        pa.decode_partition_for(lens, 8, 128, 32, bf, slots=888), 2, 0)
+    assert pa.decode_choose([2070] * 16, 8, 128, 16, bf, slots=888) == (256, 3, 2)
+    llama = [int(x) for x in np.random.default_rng(1).integers(512, 4097, 32)]
+    assert pa.decode_choose(llama, 8, 128, 16, bf, slots=888) == (512, 3, 2)
