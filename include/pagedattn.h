@@ -238,15 +238,15 @@ int pa_append_decode(float *out, const void *q, const void *k_new, const void *v
  *   - fp32 caches: the CUDA-core kernel, pa_decode_partition_for's split;
  *   - 16-bit caches, block size 8 or 16, an even KV head count: variant 3
  *     with two KV heads per CTA (it matched or beat variant 2 on every batch
- *     measured, once its split fits the batch), and the split by the waves
- *     of CTAs it makes: the largest of 1024, 768, 640, 512, 384, 256 tokens
- *     whose CTAs ((num_kv_heads / 2) x the splits of each sequence) fill
- *     between 0.6 and 1 wave of `slots`; if even 1024 needs more than a wave,
- *     512; if even 256 fills less than 0.6 of one, 256.  (Beam search, 16
- *     sequences of ~2070 tokens: 256, 25.6 us against 29.7 for variant 2 at
- *     512; Llama-8B-shaped: 512, 58.4 us against 60.4; 64 such sequences:
- *     1024, 101.3 us against 107.6 at 512's 1.4 waves; long context and the
- *     continuous mix: 512.)
+ *     measured, once its split fits the batch), and the split by the share
+ *     of a wave it fills: the shortest of 256, 384, 512, 640, 768, 1024
+ *     tokens whose CTAs ((num_kv_heads / 2) x the splits of each sequence)
+ *     fill at most 0.85 of `slots`; if even 1024 fills more, 1024 when its
+ *     CTAs fit in `slots`, else 512.  (Measured as first-to-last CTA spans:
+ *     beam search, 16 sequences of ~2070 tokens: 256; Llama-8B-shaped, 32
+ *     sequences of U[512, 4096]: 512, 48.8 us against 49.6 at 384 (0.95 of a
+ *     wave) and 50.6 at 640; 64 such sequences: 1024, within 1.3% of the best
+ *     split; long context and the continuous mix: 512.)
  *   - otherwise variant 2 with pa_decode_partition_for's split.
  * slots: CTAs resident at once; 0 asks the device (the chosen kernel's
  * occupancy times the SM count).  Host only.

@@ -465,12 +465,12 @@ int pa_decode_choose(const int32_t *seq_lens_host, int num_seqs, int num_kv_head
     if (dtype == PA_F32 || num_kv_heads % 2 != 0 || (block_size != 8 && block_size != 16))
         return PA_OK;
     // Two KV heads per CTA, one per warp (variant 3), with the split chosen
-    // by the waves of CTAs it makes: the largest split whose CTAs fill
-    // between 0.6 and 1 wave of the CTAs the device holds at once (one wave,
-    // every CTA streaming from the start, none so long that its ring's rate
-    // bounds the launch); if even 1024-token splits need more than a wave,
-    // 512 (several waves, short CTAs to balance them); if even 256-token
-    // splits fill less than 0.6 of a wave, 256 (the most parallelism).
+    // by the share of a wave of resident CTAs it fills: the shortest split
+    // whose CTAs fill at most 0.85 of the CTAs the device holds at once (as
+    // many concurrent streams as fit in one wave with some slack, each CTA
+    // short enough that the last ones do not bound the launch); if even
+    // 1024-token splits fill more, 1024 when they still fit one wave, else
+    // 512 (several waves, short CTAs to balance them).
     if (slots == 0) {
         static std::atomic<int> cache[kMaxDevices][2][2][2];
         const int dev = current_device();
@@ -490,16 +490,15 @@ int pa_decode_choose(const int32_t *seq_lens_host, int num_seqs, int num_kv_head
             n += seq_lens_host[s] <= p ? 1 : (seq_lens_host[s] + p - 1) / p;
         return n * (num_kv_heads / 2);
     };
-    static const int kSplits[] = {1024, 768, 640, 512, 384, 256};
+    static const int kSplits[] = {256, 384, 512, 640, 768, 1024};  // fill falls as p grows
     int chosen = 0;
     for (int p : kSplits) {
-        const int64_t n = ctas(p);
-        if (10 * n >= 6 * (int64_t)slots && n <= slots) {
+        if (20 * ctas(p) <= 17 * (int64_t)slots) {
             chosen = p;
             break;
         }
     }
-    if (chosen == 0) chosen = ctas(1024) > slots ? kDefaultPartition : 256;
+    if (chosen == 0) chosen = ctas(1024) <= slots ? 1024 : kDefaultPartition;
     opts->variant = 3;
     opts->heads_per_cta = 2;
     opts->partition_size = chosen;

@@ -186,37 +186,165 @@ __global__ void __launch_bounds__(kSimtThreads) decode_simt_kernel(DecodeParams 
     }
 }
 
-// Merge of the split partials: one CTA per (query head, sequence) with more
-// than one split.  out = sum_x 2^(m_x - M) o_x / sum_x 2^(m_x - M) l_x with
-// M = max_x m_x (m in log2 units).  The partials were just written by the main
-// kernel and are read from L2, so the kernel is latency-bound: the weights go
-// to shared memory in one pass, then each thread owns 4 consecutive d of one
-// group of splits (kReduceThreads / (D/4) groups) and keeps its float4 loads
-// independent so they are all in flight at once.
-constexpr int kReduceThreads = 256;
-constexpr int kReduceMaxSplits = 2048;
+// Merge of the split partials of each (sequence, query head) -- a unit:
+// out = sum_x 2^(m_x - M) o_x / sum_x 2^(m_x - M) l_x with M = max_x m_x (m in
+// log2 units).  The partials were just written by the main kernel and are read
+// from L2, so the kernel is latency-bound: a unit takes `wpu` warps (1, 2 or
+// 4, from the longest sequence's split count), each warp's lanes own 4
+// consecutive d of a row (two rows per load when D = 64), and every lane
+// issues the loads of up to 8 of its rows -- partial and (m, l) together --
+// before it uses any, keeping a running maximum across batches of rows.  The
+// warps of a unit then leave their sums in shared memory, and the last of
+// them to count itself in (a shared-memory counter) combines them.
+constexpr int kReduceThreads = 256;  // 8 warps
+constexpr int kReduceBatch = 8;      // rows a lane has in flight
 
-__global__ void __launch_bounds__(kReduceThreads) decode_reduce_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kReduceThreads, 4) decode_reduce_kernel(DecodeParams p, int wpu) {
     // launched as a programmatic dependent of the main kernel: wait for its
     // partials to be complete and visible
+    pdl_wait_prior_grid();
+    __shared__ float4 acc_s[kReduceThreads / 32][32];
+    __shared__ float2 md_s[kReduceThreads / 32];
+    __shared__ int arrived[kReduceThreads / 32];  // per unit (first warp's slot)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x < kReduceThreads / 32) arrived[threadIdx.x] = 0;
+    __syncthreads();
+    const int64_t unit = (int64_t)blockIdx.x * (kReduceThreads / 32 / wpu) + warp / wpu;
+    const int wsub = warp % wpu;
+    // both exits below are taken by all the warps of a unit or by none
+    if (unit >= (int64_t)p.num_seqs * p.num_heads) return;
+    const int s = (int)(unit / p.num_heads);
+    const int L = checked_seq_len(p, s, false);
+    const int nsplit = num_splits_for(L, p.partition_size);
+    if (nsplit <= 1) return;
+    const int D4 = p.head_dim >> 2;  // 32 or 16
+    const int rpl = 32 / D4;         // rows one warp-wide load covers: 1 or 2
+    const int sub = lane / D4, c4 = lane - sub * D4;
+    const int stride = wpu * rpl;    // between a lane's consecutive rows
+    const int64_t u0 = unit * p.max_splits;
+    const float2 *ml = reinterpret_cast<const float2 *>(p.part_ml) + u0;
+    const float4 *po = reinterpret_cast<const float4 *>(p.part_o) + u0 * D4 + c4;
+
+    float M = -INFINITY, den = 0.f;  // warp-uniform
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    // rows of this warp in a batch: x0 + sub + k * stride (k < kReduceBatch);
+    // lane j < kReduceBatch * rpl loads (m, l) of row k = j / rpl, sub = j % rpl
+    // and the lanes holding that row take its weight by a shuffle.  The loop
+    // bound is the same for every lane of the warp (the shuffles need all).
+    const int j_sub = lane % rpl, j_k = lane / rpl;
+    for (int x0 = wsub * rpl; x0 < nsplit; x0 += kReduceBatch * stride) {
+        float4 v_o[kReduceBatch];
+#pragma unroll
+        for (int k = 0; k < kReduceBatch; ++k) {
+            const int x = x0 + sub + k * stride;
+            v_o[k] = x < nsplit ? __ldg(po + (int64_t)x * D4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        const int xj = x0 + j_sub + j_k * stride;
+        const float2 mlj = j_k < kReduceBatch && xj < nsplit ? __ldg(ml + xj)
+                                                             : make_float2(-INFINITY, 0.f);
+        float bm = mlj.x;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, off));
+        const float mn = fmaxf(M, bm);
+        const float a = M == -INFINITY ? 0.f : exp2f(M - mn);
+        const float wj = mlj.x == -INFINITY ? 0.f : exp2f(mlj.x - mn);
+        float dj = wj * mlj.y;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) dj += __shfl_xor_sync(0xffffffffu, dj, off);
+        den = fmaf(den, a, dj);
+        acc.x *= a;
+        acc.y *= a;
+        acc.z *= a;
+        acc.w *= a;
+#pragma unroll
+        for (int k = 0; k < kReduceBatch; ++k) {
+            const float w = __shfl_sync(0xffffffffu, wj, k * rpl + sub);
+            acc.x = fmaf(w, v_o[k].x, acc.x);
+            acc.y = fmaf(w, v_o[k].y, acc.y);
+            acc.z = fmaf(w, v_o[k].z, acc.z);
+            acc.w = fmaf(w, v_o[k].w, acc.w);
+        }
+        M = mn;
+    }
+    if (rpl == 2) {  // the two half-warps held different rows of the same d
+        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, 16);
+        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, 16);
+        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, 16);
+        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, 16);
+    }
+    float4 *dst = reinterpret_cast<float4 *>(p.out + unit * p.head_dim) + c4;
+    if (wpu == 1) {
+        if (lane < D4) {
+            const float inv = den > 0.f ? 1.f / den : 0.f;
+            *dst = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+        }
+        return;
+    }
+    if (lane < D4) acc_s[warp][c4] = acc;
+    if (lane == 0) md_s[warp] = make_float2(M, den);
+    __threadfence_block();
+    __syncwarp();
+    const int w0 = warp - wsub;  // the unit's first warp
+    int last = 0;
+    if (lane == 0) last = atomicAdd(&arrived[w0], 1) == wpu - 1;
+    last = __shfl_sync(0xffffffffu, last, 0);
+    if (!last) return;
+    __threadfence_block();
+    if (lane < D4) {
+        float mt = -INFINITY;
+        for (int w = 0; w < wpu; ++w) mt = fmaxf(mt, md_s[w0 + w].x);
+        float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+        float d = 0.f;
+        for (int w = 0; w < wpu; ++w) {
+            const float2 md = md_s[w0 + w];
+            const float sc = md.x == -INFINITY ? 0.f : exp2f(md.x - mt);
+            const float4 v = acc_s[w0 + w][c4];
+            d = fmaf(sc, md.y, d);
+            t.x = fmaf(sc, v.x, t.x);
+            t.y = fmaf(sc, v.y, t.y);
+            t.z = fmaf(sc, v.z, t.z);
+            t.w = fmaf(sc, v.w, t.w);
+        }
+        const float inv = d > 0.f ? 1.f / d : 0.f;
+        *dst = make_float4(t.x * inv, t.y * inv, t.z * inv, t.w * inv);
+    }
+}
+
+// The same merge for many splits (more than a warp's batch of rows times 4
+// warps): one CTA per unit, whose threads own (a group of splits, 4
+// consecutive d); the first batch of each thread's partial rows is loaded
+// before the weights are formed from the (m, l) pairs, so both loads are in
+// flight together.
+constexpr int kWideMaxSplits = 2048;
+
+__global__ void __launch_bounds__(kReduceThreads) decode_reduce_wide_kernel(DecodeParams p) {
     pdl_wait_prior_grid();
     const int h = blockIdx.x, s = blockIdx.y;
     const int L = checked_seq_len(p, s, false);
     const int nsplit = num_splits_for(L, p.partition_size);
     if (nsplit <= 1) return;
-    __shared__ float w_s[kReduceMaxSplits];
+    __shared__ float w_s[kWideMaxSplits];
     __shared__ float red[kReduceThreads / 32];
     __shared__ float4 part[kReduceThreads];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
     const int64_t u0 = ((int64_t)s * p.num_heads + h) * p.max_splits;
     const float2 *ml = reinterpret_cast<const float2 *>(p.part_ml + 2 * u0);
-
+    const int D4 = p.head_dim / 4;
+    const int groups = kReduceThreads / D4;
+    const int grp = tid / D4, c4 = tid - grp * D4;
+    const float4 *po = reinterpret_cast<const float4 *>(p.part_o + u0 * p.head_dim) + c4;
+    float4 v[kReduceBatch];
+#pragma unroll
+    for (int k = 0; k < kReduceBatch; ++k) {
+        const int x = grp + k * groups;
+        v[k] = x < nsplit ? __ldg(po + (int64_t)x * D4) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     // max of the split maxima
     float M = -INFINITY;
     for (int x = tid; x < nsplit; x += kReduceThreads) {
-        const float2 v = __ldg(ml + x);
-        w_s[x] = v.x;
-        M = fmaxf(M, v.x);
+        const float2 t = __ldg(ml + x);
+        w_s[x] = t.x;
+        M = fmaxf(M, t.x);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
@@ -229,7 +357,7 @@ __global__ void __launch_bounds__(kReduceThreads) decode_reduce_kernel(DecodePar
     // weights and the denominator
     float den = 0.f;
     for (int x = tid; x < nsplit; x += kReduceThreads) {
-        const float wgt = exp2f(w_s[x] - M);
+        const float wgt = w_s[x] == -INFINITY ? 0.f : exp2f(w_s[x] - M);
         w_s[x] = wgt;
         den = fmaf(wgt, __ldg(ml + x).y, den);
     }
@@ -237,45 +365,35 @@ __global__ void __launch_bounds__(kReduceThreads) decode_reduce_kernel(DecodePar
     for (int off = 16; off > 0; off >>= 1) den += __shfl_xor_sync(0xffffffffu, den, off);
     if (lane == 0) red[wid] = den;
     __syncthreads();
-
-    // numerator: thread = (group of splits, 4 consecutive d)
-    const int D4 = p.head_dim / 4;
-    const int groups = kReduceThreads / D4;
-    const int grp = tid / D4, c4 = tid - grp * D4;
-    const float4 *po = reinterpret_cast<const float4 *>(p.part_o + u0 * p.head_dim) + c4;
+    // numerator: the rows in flight, then any further ones
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    int x = grp;
-    for (; x + 7 * groups < nsplit; x += 8 * groups) {
-        float4 v[8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) v[k] = __ldg(po + (int64_t)(x + k * groups) * D4);
-#pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            const float wgt = w_s[x + k * groups];
-            acc.x = fmaf(wgt, v[k].x, acc.x);
-            acc.y = fmaf(wgt, v[k].y, acc.y);
-            acc.z = fmaf(wgt, v[k].z, acc.z);
-            acc.w = fmaf(wgt, v[k].w, acc.w);
-        }
+    for (int k = 0; k < kReduceBatch; ++k) {
+        const int x = grp + k * groups;
+        const float wgt = x < nsplit ? w_s[x] : 0.f;
+        acc.x = fmaf(wgt, v[k].x, acc.x);
+        acc.y = fmaf(wgt, v[k].y, acc.y);
+        acc.z = fmaf(wgt, v[k].z, acc.z);
+        acc.w = fmaf(wgt, v[k].w, acc.w);
     }
-    for (; x < nsplit; x += groups) {
-        const float4 v = __ldg(po + (int64_t)x * D4);
+    for (int x = grp + kReduceBatch * groups; x < nsplit; x += groups) {
+        const float4 t = __ldg(po + (int64_t)x * D4);
         const float wgt = w_s[x];
-        acc.x = fmaf(wgt, v.x, acc.x);
-        acc.y = fmaf(wgt, v.y, acc.y);
-        acc.z = fmaf(wgt, v.z, acc.z);
-        acc.w = fmaf(wgt, v.w, acc.w);
+        acc.x = fmaf(wgt, t.x, acc.x);
+        acc.y = fmaf(wgt, t.y, acc.y);
+        acc.z = fmaf(wgt, t.z, acc.z);
+        acc.w = fmaf(wgt, t.w, acc.w);
     }
     part[tid] = acc;
     __syncthreads();
     if (tid < D4) {
         float4 tot = part[tid];
         for (int gq = 1; gq < groups; ++gq) {
-            const float4 v = part[gq * D4 + tid];
-            tot.x += v.x;
-            tot.y += v.y;
-            tot.z += v.z;
-            tot.w += v.w;
+            const float4 t = part[gq * D4 + tid];
+            tot.x += t.x;
+            tot.y += t.y;
+            tot.z += t.z;
+            tot.w += t.w;
         }
         float dsum = 0.f;
 #pragma unroll
@@ -318,8 +436,17 @@ cudaError_t launch_decode_simt(const DecodeParams &p, int dtype, cudaStream_t st
 
 cudaError_t launch_decode_reduce(const DecodeParams &p, cudaStream_t stream) {
     if (p.max_splits <= 1 || p.num_seqs == 0) return cudaSuccess;
+    // warps per (sequence, query head): enough that a lane holds at most one
+    // batch of rows of the longest sequence's splits; beyond 4, the wide form
+    const int rpl = 128 / p.head_dim;
+    int wpu = 1;
+    while (wpu < 8 && wpu * rpl * kReduceBatch < p.max_splits) wpu *= 2;
+    const bool wide = wpu == 8;
+    const int64_t units = (int64_t)p.num_seqs * p.num_heads;
+    const int64_t per_cta = kReduceThreads / 32 / wpu;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.num_heads, p.num_seqs);
+    cfg.gridDim = wide ? dim3(p.num_heads, p.num_seqs)
+                       : dim3((unsigned)((units + per_cta - 1) / per_cta));
     cfg.blockDim = dim3(kReduceThreads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
@@ -328,7 +455,8 @@ cudaError_t launch_decode_reduce(const DecodeParams &p, cudaStream_t stream) {
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, decode_reduce_kernel, p);
+    if (wide) return cudaLaunchKernelEx(&cfg, decode_reduce_wide_kernel, p);
+    return cudaLaunchKernelEx(&cfg, decode_reduce_kernel, p, wpu);
 }
 
 }  // namespace pa

@@ -30,6 +30,7 @@
 #include <mutex>
 
 #include "decode_common.cuh"
+#include "prefill_common.cuh"
 
 namespace pa {
 namespace pf {
@@ -125,7 +126,7 @@ __global__ void __launch_bounds__(kThreads) prefill_tc_kernel(
             prefetch_tensormap(&tmap_k);
             prefetch_tensormap(&tmap_v);
         }
-        const uint64_t policy = l2_policy_evict_first();
+        const uint64_t policy = l2_policy_evict_normal();
         int issued = 0;
         for (int i = 0; i < nstages; ++i) {
             // the stage's table entries, one per lane, gathered in lane 0

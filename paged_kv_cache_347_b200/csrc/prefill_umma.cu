@@ -38,6 +38,7 @@
 #include <type_traits>
 
 #include "decode_common.cuh"
+#include "prefill_common.cuh"
 #include "umma.cuh"
 
 namespace pa {
@@ -203,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         const bool is_k = warp == 8;
         const CUtensorMap *map = is_k ? &tmap_k : &tmap_v;
         if (lane == 0) prefetch_tensormap(map);
-        const uint64_t policy = l2_policy_evict_first();
+        const uint64_t policy = l2_policy_evict_normal();
         const uint32_t ring = is_k ? k_s : v_s, full = is_k ? k_full : v_full,
                        empty = is_k ? k_empty : v_empty;
         const int nslots = is_k ? NK : NV;

@@ -171,14 +171,15 @@ def _choice_by_rule(lens, hkv, slots):
     """pa_decode_choose's rule for two-head CTAs, evaluated here by brute force."""
     def ctas(p):
         return (hkv // 2) * sum(1 if L <= p else -(-L // p) for L in lens)
-    for p in (1024, 768, 640, 512, 384, 256):
-        if 0.6 * slots <= ctas(p) <= slots:
+    for p in (256, 384, 512, 640, 768, 1024):
+        if ctas(p) <= 0.85 * slots:
             return p
-    return 512 if ctas(1024) > slots else 256
+    return 1024 if ctas(1024) <= slots else 512
 
 
 @pytest.mark.parametrize("lens", [
     [32768] * 8,                                   # many waves at any split: 512
+    [32768] * 6,                                   # 1024-token splits: 0.86 of a wave
     [2070] * 16,                                   # beam-shaped: 256
     list(np.random.default_rng(1).integers(512, 4097, 32)),    # Llama-8B-shaped
     list(np.random.default_rng(2).integers(512, 4097, 64)),
