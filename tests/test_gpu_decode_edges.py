@@ -79,13 +79,13 @@ def _case(seed, lens, Hq, Hkv, D, bs, dtype, q_scale=1.0, fill=None):
     return q, kc, vc, tables, np.asarray(lens, np.int32)
 
 
-def _run(pa, q, kc, vc, tables, lens, scale, variant, partition=0):
+def _run(pa, q, kc, vc, tables, lens, scale, variant, partition=0, max_seq_len=None):
     dev = [t.cuda() for t in (q, kc, vc)]
     tab = torch.from_numpy(tables).cuda()
     sl = torch.from_numpy(lens).cuda()
     out = torch.full(tuple(q.shape), float("nan"), dtype=torch.float32, device="cuda")
     pa.pa_decode(out, dev[0], dev[1], dev[2], tab, sl, scale, partition_size=partition,
-                 variant=variant)
+                 variant=variant, max_seq_len=max_seq_len)
     torch.cuda.synchronize()
     return out.double().cpu().numpy()
 
@@ -217,6 +217,32 @@ def test_lengths_around_tiles_stages_and_splits(pa, variant, dtype, bs, partitio
 
 
 # ---------------------------------------------------------------- split merges
+@pytest.mark.parametrize("variant,dtype,bs", [(1, "f32", 16), (2, "bf16", 16), (3, "f16", 8)])
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("max_splits", [2, 8, 9, 16, 17, 32, 33, 64, 65, 130])
+def test_every_form_of_the_split_reduce(pa, variant, dtype, bs, D, max_splits):
+    """The reduce gives a (sequence, query head) 1, 2 or 4 warps, or a whole
+    CTA, from the longest sequence's split count and the rows a warp-wide
+    load covers (one at D 128, two at D 64); its lanes batch 8 rows at a
+    time.  64-token splits and a longest sequence of exactly ``max_splits``
+    splits put every form and both sides of each boundary under test, next
+    to shorter sequences (one split, none, a split edge) in the same batch."""
+    from oracle import attn
+    Hq, Hkv = 8, 2
+    part = 64
+    top = max_splits * part
+    lens = [0, 1, part - 1, part, part + 1, max(1, top - part - 5), top - 3, top]
+    q, kc, vc, tables, lens = _case(31 + max_splits, lens, Hq, Hkv, D, bs, dtype,
+                                    fill=float("nan"))
+    scale = D ** -0.5
+    exp = attn.paged_decode(q, kc, vc, tables, lens, scale)
+    # the bound is the longest length, so the launch has exactly max_splits
+    got = _run(pa, q, kc, vc, tables, lens, scale, variant, partition=part,
+               max_seq_len=int(lens.max()))
+    _check(got, exp, dtype, f"variant {variant} D {D} splits {max_splits}")
+    assert np.all(got[0] == 0.0)
+
+
 @pytest.mark.parametrize("variant,dtype,bs", [(1, "f32", 16), (1, "bf16", 4), (2, "bf16", 16),
                                               (2, "f16", 8), (3, "bf16", 16), (3, "f16", 8)])
 @pytest.mark.parametrize("partition", [64, 512])
