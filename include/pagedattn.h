@@ -326,9 +326,13 @@ int pa_prefill(float *out, const void *q, const void *k_cache, const void *v_cac
  *   1  the mma.sync kernel: 64 (token, head) rows per CTA, accumulators in
  *      registers;
  *   2  the tcgen05 kernel: 128 rows per CTA; Q, S = Q K^T, P and O = P V held
- *      in tensor memory, the MMAs issued by two threads.
+ *      in tensor memory, the MMAs issued by two threads;
+ *   3  the same kernel persistent: one CTA per SM walks its share of the
+ *      128-row tiles (in the order of kernel 2's grid), the
+ *      next tile's Q going into a second TMEM buffer and its first products
+ *      starting while the current tile's output is written.
  * Same arguments, results (within fp32 rounding) and errors as pa_prefill;
- * another variant returns PA_ERR_INVALID_ARG.  Both kernels need all of a
+ * another variant returns PA_ERR_INVALID_ARG.  All kernels need all of a
  * sequence's table entries for positions < L_s to be valid blocks (an entry
  * outside [0, num_blocks) reads as zeros and sets PA_DEVERR_TABLE).
  */

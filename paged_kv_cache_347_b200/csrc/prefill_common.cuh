@@ -15,4 +15,13 @@ __device__ __forceinline__ uint64_t l2_policy_evict_normal() {
     return p;
 }
 
+// One 32-byte store of 8 floats (sm_100): a whole L2 sector per lane, half
+// the transactions of two 16-byte stores.  ptr must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(float *ptr, const float (&v)[8]) {
+    asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr),
+                 "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]),
+                 "f"(v[7])
+                 : "memory");
+}
+
 }  // namespace pa

@@ -34,6 +34,8 @@
 // (bounded) for their copies, warp 0 waits for the MMAs and frees the TMEM.
 #include <math.h>
 
+#include <algorithm>
+#include <climits>
 #include <mutex>
 #include <type_traits>
 
@@ -62,8 +64,8 @@ struct Cfg {
     static constexpr int kXchOffset = kVOffset + NV * kStageBytes;  // float [2][2][128]
     static constexpr int kBarOffset = kXchOffset + 2 * 2 * kM * 4;
     // k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] s_full[2] p_full[2] pv_done[2]
-    // q_full mma_done xchg[4]
-    static constexpr int kNumBars = 2 * NK + 2 * NV + 6 + 2 + 4;
+    // q_full[2] o_free mma_done xchg[4]
+    static constexpr int kNumBars = 2 * NK + 2 * NV + 6 + 4 + 4;
     static constexpr int kTmemSlot = kBarOffset + kNumBars * 8;
     static constexpr int kAbortOffset = kTmemSlot + 16;
     static constexpr int kSmemBytes = kAbortOffset + 16;
@@ -72,7 +74,7 @@ struct Cfg {
     static_assert(kDynSmem <= 227 * 1024, "shared memory");
     static_assert(kKeys % BS == 0 && kBlocksPerStage <= 32, "block size");
     static_assert(D == 64 || D == 128, "head size");
-    static_assert(kColO + D <= kColQ && kColQ + D / 2 <= kTmemCols, "tensor memory");
+    static_assert(kColO + D <= kColQ && kColQ + D <= kTmemCols, "tensor memory: two Q buffers");
 };
 
 // A bounded mbarrier wait taken by a whole warp, with one outcome for all
@@ -125,7 +127,60 @@ template <> struct PSplit<__half> {
     }
 };
 
-template <typename T, int D, int BS, int NK, int NV>
+// What a CTA needs of one token tile: its sequence and KV head, where its
+// rows start, how many keys it attends to.
+struct Tile {
+    int s, g, q0, tok0, ntok, pos0, nkeys, nstages, nblk;
+};
+
+// Tile u of the launch.  One tile per CTA: the 3-D grid, token tiles that
+// attend to the most keys first within a (sequence, KV head).  Persistent:
+// the same order as a list (sequence, then KV head, then token tile, longest
+// first), CTA c taking tiles c, c + gridDim.x, ...: the CTAs at work at any
+// time hold the tiles of a few (sequence, KV head) pairs, which share their
+// K/V through L2, and each CTA's tiles mix long and short ones.  Every role
+// of the CTA calls
+// this with the same u and gets the same answer; false: nothing to do
+// (an empty tile, or a sequence whose lengths break the bounds, which
+// `report` records).
+template <int BS, bool kPersist>
+__device__ __forceinline__ bool describe_tile(const PrefillParams &p, int u, bool report,
+                                              Tile &t) {
+    const int TQ = p.tokens_per_cta;
+    const int X = (p.max_q_len + TQ - 1) / TQ;  // token tiles per (sequence, KV head)
+    int qt, g, s;
+    if constexpr (kPersist) {
+        qt = X - 1 - u % X;
+        g = (u / X) % p.num_kv_heads;
+        s = u / (X * p.num_kv_heads);
+    } else {
+        qt = gridDim.x - 1 - blockIdx.x;
+        g = blockIdx.y;
+        s = blockIdx.z;
+    }
+    const int q0 = __ldg(p.cu_q + s);
+    const int n = __ldg(p.cu_q + s + 1) - q0;
+    const int L = __ldg(p.seq_lens + s);
+    if (n < 0 || n > L || L > p.max_seq_len || n > p.max_q_len ||
+        (int64_t)(L + BS - 1) / BS > p.max_blocks_per_seq) {
+        if (report && qt == 0 && g == 0) raise_device_error(p.err, PA_DEVERR_SEQLEN);
+        return false;
+    }
+    const int tok0 = qt * TQ;
+    if (tok0 >= n) return false;
+    t.s = s;
+    t.g = g;
+    t.q0 = q0;
+    t.tok0 = tok0;
+    t.ntok = min(TQ, n - tok0);
+    t.pos0 = L - n + tok0;
+    t.nkeys = t.pos0 + t.ntok;
+    t.nstages = (t.nkeys + kKeys - 1) / kKeys;
+    t.nblk = (t.nkeys + BS - 1) / BS;
+    return true;
+}
+
+template <typename T, int D, int BS, int NK, int NV, bool kPersist>
 __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
     const PrefillParams p) {
@@ -136,25 +191,17 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
 
     pdl_wait_prior_grid();
 
-    // later token tiles attend to more keys: hand them out first
-    const int qt = gridDim.x - 1 - blockIdx.x, g = blockIdx.y, s = blockIdx.z;
     const int G = p.num_heads / p.num_kv_heads;
     const int TQ = p.tokens_per_cta;  // 128 / G
-    const int q0 = __ldg(p.cu_q + s);
-    const int n = __ldg(p.cu_q + s + 1) - q0;
-    const int L = __ldg(p.seq_lens + s);
-    if (n < 0 || n > L || L > p.max_seq_len || n > p.max_q_len ||
-        (int64_t)(L + BS - 1) / BS > p.max_blocks_per_seq) {
-        if (qt == 0 && g == 0 && threadIdx.x == 0) raise_device_error(p.err, PA_DEVERR_SEQLEN);
-        return;
+    const int ntiles =
+        kPersist ? ((p.max_q_len + TQ - 1) / TQ) * p.num_kv_heads * p.num_seqs : 1;
+    const int u0 = kPersist ? (int)blockIdx.x : 0;
+    const int ustep = kPersist ? (int)gridDim.x : 1;
+    if constexpr (!kPersist) {
+        Tile t;
+        // uniform over the CTA, before any barrier or TMEM use
+        if (!describe_tile<BS, false>(p, 0, threadIdx.x == 0, t)) return;
     }
-    const int tok0 = qt * TQ;
-    if (tok0 >= n) return;  // uniform, before any barrier or TMEM use
-    const int ntok = min(TQ, n - tok0);
-    const int pos0 = L - n + tok0;
-    const int nkeys = pos0 + ntok;
-    const int nstages = (nkeys + kKeys - 1) / kKeys;
-    const int nblk = (nkeys + BS - 1) / BS;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     const uint32_t sbase = smem_u32(smem);
@@ -162,8 +209,8 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     const uint32_t bar0 = sbase + C::kBarOffset;
     const uint32_t k_full = bar0, k_empty = k_full + 8 * NK, v_full = k_empty + 8 * NK,
                    v_empty = v_full + 8 * NV, s_full = v_empty + 8 * NV, p_full = s_full + 16,
-                   pv_done = p_full + 16, q_full = pv_done + 16, mma_done = q_full + 8,
-                   xchg = mma_done + 8;
+                   pv_done = p_full + 16, q_full = pv_done + 16, o_free = q_full + 16,
+                   mma_done = o_free + 8, xchg = mma_done + 8;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kAbortOffset);
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + C::kTmemSlot);
 
@@ -176,15 +223,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
             mbar_init(v_full + 8 * i, 1);
             mbar_init(v_empty + 8 * i, 1);
         }
-        // s_full, p_full and pv_done once per S buffer: stage i+1 can run ahead
-        // of a waiter on stage i, stage i+2 never can
+        // s_full, p_full and pv_done once per S buffer, q_full once per Q
+        // buffer: a phase is never waited on two completions behind
         for (int b = 0; b < 2; ++b) {
             mbar_init(s_full + 8 * b, 1);
             mbar_init(p_full + 8 * b, kSoftmaxThreads);
             mbar_init(pv_done + 8 * b, 1);
+            mbar_init(q_full + 8 * b, kSoftmaxThreads);
         }
-        mbar_init(q_full, kSoftmaxThreads);
-        mbar_init(mma_done, 2);  // both issuing threads
+        mbar_init(o_free, kSoftmaxThreads);  // a tile's O read out of TMEM
+        mbar_init(mma_done, 2);              // both issuing threads
         for (int q = 0; q < 4; ++q) mbar_init(xchg + 8 * q, 64);
         *abort_flag = 0;
         fence_mbarrier_init();
@@ -199,7 +247,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     const uint32_t tmem = *tmem_slot;
 
     // ------------------------------------------------------------ producers
-    // warp 8 loads the K stages, warp 9 the V stages, each at its own pace
+    // warp 8 loads the K stages, warp 9 the V stages, each at its own pace;
+    // the ring runs on across the CTA's tiles (gi counts stages over all of
+    // them)
     if (warp == 8 || warp == 9) {
         const bool is_k = warp == 8;
         const CUtensorMap *map = is_k ? &tmap_k : &tmap_v;
@@ -208,41 +258,50 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         const uint32_t ring = is_k ? k_s : v_s, full = is_k ? k_full : v_full,
                        empty = is_k ? k_empty : v_empty;
         const int nslots = is_k ? NK : NV;
-        int issued = 0;
-        for (int i = 0; i < nstages; ++i) {
-            const int slot = i % nslots;
-            const int jb = i * C::kBlocksPerStage;
-            const int jn = min(C::kBlocksPerStage, nblk - jb);
-            // lane j < jn holds the physical block of the stage's j-th table entry
-            int blk = -1;
-            if (lane < jn) {
-                const int b = checked_block_row(p.block_tables, p.max_blocks_per_seq, p.num_blocks,
-                                                p.err, s, jb + lane);
-                blk = b < 0 ? p.num_blocks : b;  // out of range: the copy reads the fill value
-            }
-            int stop = 0;
-            if (lane == 0 && i >= nslots &&
-                !mbar_wait_bounded(empty + 8 * slot, ((i / nslots) - 1) & 1, abort_flag))
-                stop = 1;
-            if (__shfl_sync(0xffffffffu, stop, 0)) break;
-            if (lane == 0) mbar_arrive_expect_tx(full + 8 * slot, (uint32_t)(jn * 2 * BS * D));
-            __syncwarp();
-            if (blk >= 0) {
-                const uint32_t dst = ring + slot * C::kStageBytes + lane * BS * kRowBytes;
-                const int y = (blk * p.num_kv_heads + g) * BS;
+        int gi = 0;  // stages issued
+        bool stop = false;
+        for (int u = u0; !stop && u < ntiles; u += ustep) {
+            Tile t;
+            if (!describe_tile<BS, kPersist>(p, u, false, t)) continue;
+            for (int i = 0; i < t.nstages; ++i) {
+                const int slot = gi % nslots;
+                const int jb = i * C::kBlocksPerStage;
+                const int jn = min(C::kBlocksPerStage, t.nblk - jb);
+                // lane j < jn holds the physical block of the stage's j-th table entry
+                int blk = -1;
+                if (lane < jn) {
+                    const int b = checked_block_row(p.block_tables, p.max_blocks_per_seq,
+                                                    p.num_blocks, p.err, t.s, jb + lane);
+                    blk = b < 0 ? p.num_blocks : b;  // out of range: the copy reads the fill value
+                }
+                int quit = 0;
+                if (lane == 0 && gi >= nslots &&
+                    !mbar_wait_bounded(empty + 8 * slot, ((gi / nslots) - 1) & 1, abort_flag))
+                    quit = 1;
+                if (__shfl_sync(0xffffffffu, quit, 0)) {
+                    stop = true;
+                    break;
+                }
+                if (lane == 0) mbar_arrive_expect_tx(full + 8 * slot, (uint32_t)(jn * 2 * BS * D));
+                __syncwarp();
+                if (blk >= 0) {
+                    const uint32_t dst = ring + slot * C::kStageBytes + lane * BS * kRowBytes;
+                    const int y = (blk * p.num_kv_heads + t.g) * BS;
 #pragma unroll
-                for (int pc = 0; pc < C::kPieces; ++pc)
-                    tma_load_2d(dst + pc * C::kKVPiece, map, pc * 64, y, full + 8 * slot, policy);
+                    for (int pc = 0; pc < C::kPieces; ++pc)
+                        tma_load_2d(dst + pc * C::kKVPiece, map, pc * 64, y, full + 8 * slot,
+                                    policy);
+                }
+                ++gi;
             }
-            issued = i + 1;
         }
         if (lane == 0) {
-            if (issued < nstages) {
+            if (stop) {
                 raise_device_error(p.err, PA_DEVERR_TIMEOUT);
                 *abort_flag = 1;
             }
             // wait (bounded) for the copies still in flight
-            for (int i = max(0, issued - nslots); i < issued; ++i)
+            for (int i = max(0, gi - nslots); i < gi; ++i)
                 mbar_wait_bounded(full + 8 * (i % nslots), (i / nslots) & 1, nullptr);
         }
         return;
@@ -252,65 +311,79 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     // Warp 10 issues the S MMAs, warp 11 the PV MMAs, each from one thread, so
     // that neither waits behind the other's barrier checks.  MMAs of two
     // threads are not ordered against each other: S(i+2) overwrites the TMEM
-    // columns PV(i) reads, so the S thread waits for PV(i) to complete.
+    // columns PV(i) reads, so the S thread waits for PV(i) to complete.  Stage
+    // indices (gi) and tile indices (tp) run on across the CTA's tiles: a
+    // tile's Q sits in TMEM buffer tp % 2, and its first PV, which starts O
+    // afresh, waits until the softmax warps have read out the previous tile's O.
     if (warp == 10 || warp == 11) {
         if (lane == 0) {
             constexpr uint32_t fmt = StoreT<T>::kCode == PA_BF16 ? 1u : 0u;
-            bool ok = mbar_wait_bounded(q_full, 0, abort_flag);
-            umma::fence_after_sync();
-            if (warp == 10) {
-                constexpr uint32_t idesc_s = umma::idesc_f16(fmt, kM, kKeys, 0);
-#pragma unroll 1
-                for (int i = 0; ok && i < nstages; ++i) {
-                    // S(i) = Q . K_i^T into S buffer i % 2, once PV(i-2) has read it
-                    const int slot = i % NK;
-                    if (i >= 2 && !mbar_wait_bounded(pv_done + 8 * (i & 1), ((i >> 1) - 1) & 1,
-                                                     abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    if (!mbar_wait_bounded(k_full + 8 * slot, (i / NK) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
+            bool ok = true;
+            int gi = 0, tp = 0;
+            for (int u = u0; ok && u < ntiles; u += ustep) {
+                Tile t;
+                if (!describe_tile<BS, kPersist>(p, u, false, t)) continue;
+                if (warp == 10) {
+                    constexpr uint32_t idesc_s = umma::idesc_f16(fmt, kM, kKeys, 0);
+                    ok = mbar_wait_bounded(q_full + 8 * (tp & 1), (tp >> 1) & 1, abort_flag);
                     umma::fence_after_sync();
-                    // K rows: 8-row groups 1 KB apart; descriptors advance by (bytes >> 4)
-                    const uint64_t b0 = umma::smem_desc_sw128(k_s + slot * C::kStageBytes, 16, 1024);
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t ka = ((kk >> 2) * C::kKVPiece + (kk & 3) * 32) >> 4;
-                        umma::mma_f16_ts(tmem + (i & 1) * kKeys, tmem + kColQ + 8 * kk, b0 + ka,
-                                         idesc_s, kk > 0);
-                    }
-                    umma::commit(s_full + 8 * (i & 1));
-                    umma::commit(k_empty + 8 * slot);
-                }
-            } else {
-                constexpr uint32_t idesc_o = umma::idesc_f16(fmt, kM, D, 1);
+                    const uint32_t qcol = tmem + kColQ + (tp & 1) * (D / 2);
 #pragma unroll 1
-                for (int i = 0; ok && i < nstages; ++i) {
-                    // O += P_i . V_i once the softmax has written P_i
-                    const int slot = i % NV;
-                    if (!mbar_wait_bounded(p_full + 8 * (i & 1), (i >> 1) & 1, abort_flag) ||
-                        !mbar_wait_bounded(v_full + 8 * slot, (i / NV) & 1, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    umma::fence_after_sync();
-                    // V rows: 8-row groups 1 KB apart, 64-column pieces 16 KB apart
-                    const uint64_t b0 = umma::smem_desc_sw128(v_s + slot * C::kStageBytes,
-                                                              C::kKVPiece, 1024);
-                    const uint32_t pb = tmem + (i & 1) * kKeys;
+                    for (int i = 0; ok && i < t.nstages; ++i, ++gi) {
+                        // S(gi) = Q . K^T into S buffer gi % 2, once PV(gi-2) has read it
+                        const int slot = gi % NK;
+                        if (gi >= 2 && !mbar_wait_bounded(pv_done + 8 * (gi & 1),
+                                                          ((gi >> 1) - 1) & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        if (!mbar_wait_bounded(k_full + 8 * slot, (gi / NK) & 1, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        umma::fence_after_sync();
+                        // K rows: 8-row groups 1 KB apart; descriptors advance by (bytes >> 4)
+                        const uint64_t b0 =
+                            umma::smem_desc_sw128(k_s + slot * C::kStageBytes, 16, 1024);
 #pragma unroll
-                    for (int j = 0; j < kKeys / 16; ++j) {  // keys 16j..16j+15
-                        const uint64_t b = b0 + ((j * 16 * kRowBytes) >> 4);
-                        umma::mma_f16_ts(tmem + kColO, pb + 16 * j, b, idesc_o,
-                                         (i > 0 || j > 0) ? 1u : 0u);
-                        umma::mma_f16_ts(tmem + kColO, pb + 16 * j + 8, b, idesc_o, 1u);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t ka = ((kk >> 2) * C::kKVPiece + (kk & 3) * 32) >> 4;
+                            umma::mma_f16_ts(tmem + (gi & 1) * kKeys, qcol + 8 * kk, b0 + ka,
+                                             idesc_s, kk > 0);
+                        }
+                        umma::commit(s_full + 8 * (gi & 1));
+                        umma::commit(k_empty + 8 * slot);
                     }
-                    umma::commit(pv_done + 8 * (i & 1));
-                    umma::commit(v_empty + 8 * slot);
+                } else {
+                    constexpr uint32_t idesc_o = umma::idesc_f16(fmt, kM, D, 1);
+#pragma unroll 1
+                    for (int i = 0; ok && i < t.nstages; ++i, ++gi) {
+                        // O += P(gi) . V(gi) once the softmax has written P(gi)
+                        const int slot = gi % NV;
+                        if (!mbar_wait_bounded(p_full + 8 * (gi & 1), (gi >> 1) & 1, abort_flag) ||
+                            !mbar_wait_bounded(v_full + 8 * slot, (gi / NV) & 1, abort_flag) ||
+                            (i == 0 && tp > 0 &&
+                             !mbar_wait_bounded(o_free, (tp - 1) & 1, abort_flag))) {
+                            ok = false;
+                            break;
+                        }
+                        umma::fence_after_sync();
+                        // V rows: 8-row groups 1 KB apart, 64-column pieces 16 KB apart
+                        const uint64_t b0 = umma::smem_desc_sw128(v_s + slot * C::kStageBytes,
+                                                                  C::kKVPiece, 1024);
+                        const uint32_t pb = tmem + (gi & 1) * kKeys;
+#pragma unroll
+                        for (int j = 0; j < kKeys / 16; ++j) {  // keys 16j..16j+15
+                            const uint64_t b = b0 + ((j * 16 * kRowBytes) >> 4);
+                            umma::mma_f16_ts(tmem + kColO, pb + 16 * j, b, idesc_o,
+                                             (i > 0 || j > 0) ? 1u : 0u);
+                            umma::mma_f16_ts(tmem + kColO, pb + 16 * j + 8, b, idesc_o, 1u);
+                        }
+                        umma::commit(pv_done + 8 * (gi & 1));
+                        umma::commit(v_empty + 8 * slot);
+                    }
                 }
+                ++tp;
             }
             if (!ok) {
                 raise_device_error(p.err, PA_DEVERR_TIMEOUT);
@@ -325,37 +398,42 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     const int quarter = warp & 3, half = warp >> 2;
     const int r = quarter * 32 + lane;  // row == TMEM lane
     const int tl = r / G, hh = r - tl * G;
-    const bool valid = r < TQ * G && tl < ntok;
-    const int qp = valid ? pos0 + tl : nkeys - 1;
-    // stages i < n_fast end at or before the first chunk token: no mask there
-    const int n_fast = min(nstages, (pos0 + 1) / kKeys);
-    const int64_t qrow = ((int64_t)(q0 + tok0 + tl) * p.num_heads + g * G + hh) * D;
     const uint32_t lane_base = tmem + ((uint32_t)(quarter * 32) << 16);
     // S is computed with sign(scale) folded into Q (a sign-bit flip, exact),
     // so that the logit scale applied below is non-negative
     const uint32_t qflip = p.scale_log2 < 0.f ? 0x80008000u : 0u;
     const float sl2 = fabsf(p.scale_log2);
-    {
-        // the Q row into TMEM, two elements per column: for D 128 each half
-        // of the row's threads writes 32 columns, for D 64 the first writes all
-        if (D == 128 || half == 0) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.q) + qrow) +
-                               half * (D == 128 ? 8 : 0);
-            uint32_t w[32];
+    // the tile's row: the row's last key position, the tile's key count
+    int qp = 0, nkeys = 0;
+    // The Q row of a tile, two elements per 32-bit word: for D 128 each half
+    // of the row's threads takes 32 words, for D 64 the first takes all.
+    // Loaded into registers first, so that the loads of the next tile's Q
+    // can be in flight while the current tile's output is written.
+    const bool q_writer = D == 128 || half == 0;
+    const bool out32 = (reinterpret_cast<uintptr_t>(p.out) & 31u) == 0;
+    auto load_q = [&](const Tile &t, uint32_t (&w)[32]) {
+        const bool ok_row = r < TQ * G && tl < t.ntok;
+        const int64_t row = ((int64_t)(t.q0 + t.tok0 + tl) * p.num_heads + t.g * G + hh) * D;
+        const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const T *>(p.q) + row) +
+                           half * (D == 128 ? 8 : 0);
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint4 v = valid ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-                w[4 * c] = v.x ^ qflip;
-                w[4 * c + 1] = v.y ^ qflip;
-                w[4 * c + 2] = v.z ^ qflip;
-                w[4 * c + 3] = v.w ^ qflip;
-            }
-            umma::st32(lane_base + kColQ + half * 32, w);
+        for (int c = 0; c < 8; ++c) {
+            uint4 v = ok_row && q_writer ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            w[4 * c] = v.x ^ qflip;
+            w[4 * c + 1] = v.y ^ qflip;
+            w[4 * c + 2] = v.z ^ qflip;
+            w[4 * c + 3] = v.w ^ qflip;
+        }
+    };
+    // into TMEM buffer b, then counted on that buffer's q_full barrier
+    auto store_q = [&](uint32_t (&w)[32], int b) {
+        if (q_writer) {
+            umma::st32(lane_base + kColQ + b * (D / 2) + half * 32, w);
             umma::wait_st();
         }
         umma::fence_before_sync();
-        mbar_arrive(q_full);
-    }
+        mbar_arrive(q_full + 8 * b);
+    };
     float *xch = reinterpret_cast<float *>(smem + C::kXchOffset);  // [parity][half][row]
     const uint32_t my_xchg = xchg + 8 * quarter;
     int xp = 0;  // exchanges so far (the same sequence for both threads of a row)
@@ -371,11 +449,11 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     float m = -INFINITY, l = 0.f;
     // One stage.  Stages reaching beyond the first chunk token run the
     // masked body, every earlier stage the unmasked one.
-    auto stage = [&](int i, auto masked_c) __attribute__((always_inline)) -> bool {
+    auto stage = [&](int i, int gi, auto masked_c) __attribute__((always_inline)) -> bool {
         constexpr bool kMasked = decltype(masked_c)::value;
-        if (!warp_wait(s_full + 8 * (i & 1), (i >> 1) & 1, abort_flag)) return false;
+        if (!warp_wait(s_full + 8 * (gi & 1), (gi >> 1) & 1, abort_flag)) return false;
         umma::fence_after_sync();
-        const uint32_t hcol = lane_base + (i & 1) * kKeys + half * 64;  // this thread's S / P
+        const uint32_t hcol = lane_base + (gi & 1) * kKeys + half * 64;  // this thread's S / P
         const int last = qp - (i * kKeys + half * 64);  // the row's last key in the half
         uint32_t sr[2][32];
         umma::ld32(hcol, sr[0]);
@@ -445,7 +523,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         }
         if (__any_sync(0xffffffffu, rescale)) {  // warp-collective TMEM access
             // O must hold PV up to stage i-1 before it is rescaled
-            if (i > 0 && !warp_wait(pv_done + 8 * ((i - 1) & 1), ((i - 1) >> 1) & 1, abort_flag))
+            if (i > 0 && !warp_wait(pv_done + 8 * ((gi - 1) & 1), ((gi - 1) >> 1) & 1, abort_flag))
                 return false;
             umma::fence_after_sync();
 #pragma unroll
@@ -464,9 +542,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
                 // last stage: V rows past the last key hold stale or unwritten
                 // data; zero them so that their zero weights give exact zeros.
                 // The wait only orders these stores after the stage's copies.
-                if (!warp_wait(v_full + 8 * (i % NV), (i / NV) & 1, abort_flag)) return false;
+                if (!warp_wait(v_full + 8 * (gi % NV), (gi / NV) & 1, abort_flag)) return false;
                 const int first = nkeys - i * kKeys;  // rows [first, 128)
-                uint8_t *vst = smem + C::kVOffset + (i % NV) * C::kStageBytes;
+                uint8_t *vst = smem + C::kVOffset + (gi % NV) * C::kStageBytes;
                 for (int idx = threadIdx.x; idx < (kKeys - first) * C::kPieces * 8;
                      idx += kSoftmaxThreads) {
                     const int row = first + idx / (C::kPieces * 8);
@@ -479,37 +557,93 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         }
         umma::wait_st();
         umma::fence_before_sync();
-        mbar_arrive(p_full + 8 * (i & 1));
+        mbar_arrive(p_full + 8 * (gi & 1));
         return true;
     };
+    // The CTA's tiles in turn.  Between two tiles: the next tile's Q loads go
+    // out, the last PV of the tile is waited for, the next Q goes into the
+    // other TMEM buffer (so the S thread can start the next tile while this
+    // one's output is written), O is read out and o_free counted, and the
+    // output is normalised and stored.
     bool ok = true;
-    int i = 0;
-    for (; ok && i < n_fast; ++i) ok = stage(i, std::false_type{});
-    for (; ok && i < nstages; ++i) ok = stage(i, std::true_type{});
-    float other = 0.f;
-    if (ok)
-        ok = warp_wait(pv_done + 8 * ((nstages - 1) & 1), ((nstages - 1) >> 1) & 1, abort_flag) &&
+    int gi = 0, tp = 0;  // stages and tiles done, the same counts as the MMA threads'
+    Tile t;
+    int u = u0;
+    bool have = false;
+    for (; !have && u < ntiles; u += have ? 0 : ustep)
+        have = describe_tile<BS, kPersist>(p, u, threadIdx.x == 0, t);
+    if (have) {
+        uint32_t w[32];
+        load_q(t, w);
+        store_q(w, 0);
+    }
+    while (have && ok) {
+        const bool valid = r < TQ * G && tl < t.ntok;
+        qp = valid ? t.pos0 + tl : t.nkeys - 1;
+        nkeys = t.nkeys;
+        // stages i < n_fast end at or before the first chunk token: no mask there
+        const int n_fast = min(t.nstages, (t.pos0 + 1) / kKeys);
+        m = -INFINITY;
+        l = 0.f;
+        int i = 0;
+        for (; ok && i < n_fast; ++i) ok = stage(i, gi + i, std::false_type{});
+        for (; ok && i < t.nstages; ++i) ok = stage(i, gi + i, std::true_type{});
+        if (!ok) break;
+        const int glast = gi + t.nstages - 1;
+        gi += t.nstages;
+        // the next tile, if any
+        Tile nt;
+        bool have_next = false;
+        int un = u + ustep;
+        for (; !have_next && un < ntiles; un += have_next ? 0 : ustep)
+            have_next = describe_tile<BS, kPersist>(p, un, threadIdx.x == 0, nt);
+        uint32_t w[32];
+        if (have_next) load_q(nt, w);
+        float other = 0.f;
+        ok = warp_wait(pv_done + 8 * (glast & 1), (glast >> 1) & 1, abort_flag) &&
              exchange(l, other);
-    if (ok) {
+        if (!ok) break;
         umma::fence_after_sync();
+        if (have_next) store_q(w, (tp + 1) & 1);
         const float lt = l + other;
         const float inv = lt > 0.f ? 1.f / lt : 0.f;
+        const int64_t qrow = ((int64_t)(t.q0 + t.tok0 + tl) * p.num_heads + t.g * G + hh) * D;
         float *dst = p.out + qrow + half * (D / 2);
+        // O out of TMEM a 32-column chunk at a time, normalised and stored;
+        // each lane writes its own row: 32-byte stores when out allows them
+        // (whole sectors), else 16-byte ones
 #pragma unroll
         for (int cb = 0; cb < D / 64; ++cb) {
             uint32_t o[32];
             umma::ld32(lane_base + kColO + half * (D / 2) + 32 * cb, o);
             umma::wait_ld();
-            if (valid) {
+            if (cb == D / 64 - 1) {
+                // O is out of TMEM: the next tile's first PV may start it afresh
+                umma::fence_before_sync();
+                mbar_arrive(o_free);
+            }
+            if (valid && out32) {
+#pragma unroll
+                for (int e = 0; e < 32; e += 8) {
+                    float v8[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) v8[k] = __uint_as_float(o[e + k]) * inv;
+                    st_global_v8(dst + cb * 32 + e, v8);
+                }
+            } else if (valid) {
 #pragma unroll
                 for (int e = 0; e < 32; e += 4)
-                    *reinterpret_cast<float4 *>(dst + cb * 32 + e) =
-                        make_float4(__uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
-                                    __uint_as_float(o[e + 2]) * inv,
-                                    __uint_as_float(o[e + 3]) * inv);
+                    *reinterpret_cast<float4 *>(dst + cb * 32 + e) = make_float4(
+                        __uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
+                        __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
             }
         }
-    } else if (lane == 0) {
+        ++tp;
+        t = nt;
+        u = un;
+        have = have_next;
+    }
+    if (!ok && lane == 0) {
         raise_device_error(p.err, PA_DEVERR_TIMEOUT);
         *abort_flag = 1;  // the other warps stop waiting
     }
@@ -525,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     pdl_launch_dependents();
 }
 
-template <typename T, int D, int BS>
+template <typename T, int D, int BS, bool kPersist>
 static cudaError_t launch_inst(const PrefillParams &p, const CUtensorMap &mk,
                                const CUtensorMap &mv, cudaStream_t stream) {
     constexpr int NK = D == 128 ? 3 : 6, NV = D == 128 ? 3 : 6;
@@ -536,14 +670,24 @@ static cudaError_t launch_inst(const PrefillParams &p, const CUtensorMap &mk,
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[dev], [&] {
-        attr_err[dev] = cudaFuncSetAttribute(prefill_umma_kernel<T, D, BS, NK, NV>,
+        attr_err[dev] = cudaFuncSetAttribute(prefill_umma_kernel<T, D, BS, NK, NV, kPersist>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kDynSmem);
     });
     if (attr_err[dev] != cudaSuccess) return attr_err[dev];
+    const int tiles_x = (p.max_q_len + p.tokens_per_cta - 1) / p.tokens_per_cta;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((p.max_q_len + p.tokens_per_cta - 1) / p.tokens_per_cta, p.num_kv_heads,
-                       p.num_seqs);
+    if constexpr (kPersist) {
+        // one CTA per SM (shared memory and TMEM allow no more), each walking
+        // its share of the tile list
+        const int64_t tiles = (int64_t)tiles_x * p.num_kv_heads * p.num_seqs;
+        if (tiles > INT_MAX) return cudaErrorInvalidValue;
+        const int sms = num_sms();
+        if (sms <= 0) return cudaErrorInvalidDevice;
+        cfg.gridDim = dim3((unsigned)std::min<int64_t>(tiles, sms));
+    } else {
+        cfg.gridDim = dim3(tiles_x, p.num_kv_heads, p.num_seqs);
+    }
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = C::kDynSmem;
     cfg.stream = stream;
@@ -552,24 +696,32 @@ static cudaError_t launch_inst(const PrefillParams &p, const CUtensorMap &mk,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_umma_kernel<T, D, BS, NK, NV>, mk, mv, p);
+    return cudaLaunchKernelEx(&cfg, prefill_umma_kernel<T, D, BS, NK, NV, kPersist>, mk, mv, p);
 }
 
-template <typename T, int D>
+template <typename T, int D, bool kPersist>
 static cudaError_t launch_d(const PrefillParams &p, const CUtensorMap &mk, const CUtensorMap &mv,
                             cudaStream_t stream) {
     switch (p.block_size) {
-    case 8: return launch_inst<T, D, 8>(p, mk, mv, stream);
-    case 16: return launch_inst<T, D, 16>(p, mk, mv, stream);
-    case 32: return launch_inst<T, D, 32>(p, mk, mv, stream);
-    case 64: return launch_inst<T, D, 64>(p, mk, mv, stream);
+    case 8: return launch_inst<T, D, 8, kPersist>(p, mk, mv, stream);
+    case 16: return launch_inst<T, D, 16, kPersist>(p, mk, mv, stream);
+    case 32: return launch_inst<T, D, 32, kPersist>(p, mk, mv, stream);
+    case 64: return launch_inst<T, D, 64, kPersist>(p, mk, mv, stream);
     default: return cudaErrorNotSupported;
     }
 }
 
+template <typename T, int D>
+static cudaError_t launch_p(const PrefillParams &p, bool persistent, const CUtensorMap &mk,
+                            const CUtensorMap &mv, cudaStream_t stream) {
+    return persistent ? launch_d<T, D, true>(p, mk, mv, stream)
+                      : launch_d<T, D, false>(p, mk, mv, stream);
+}
+
 }  // namespace pu
 
-cudaError_t launch_prefill_umma(const PrefillParams &p, int dtype, cudaStream_t stream) {
+cudaError_t launch_prefill_umma(const PrefillParams &p, int dtype, bool persistent,
+                                cudaStream_t stream) {
     if (p.num_seqs == 0 || p.max_q_len == 0) return cudaSuccess;
     const int64_t rows = (int64_t)p.num_blocks * p.num_kv_heads * p.block_size;
     CUtensorMap mk, mv;
@@ -577,10 +729,10 @@ cudaError_t launch_prefill_umma(const PrefillParams &p, int dtype, cudaStream_t 
         !make_cache_tensor_map(&mv, p.v_cache, dtype, p.head_dim, rows, p.block_size))
         return cudaErrorInvalidValue;
     if (dtype == PA_BF16)
-        return p.head_dim == 128 ? pu::launch_d<__nv_bfloat16, 128>(p, mk, mv, stream)
-                                 : pu::launch_d<__nv_bfloat16, 64>(p, mk, mv, stream);
-    return p.head_dim == 128 ? pu::launch_d<__half, 128>(p, mk, mv, stream)
-                             : pu::launch_d<__half, 64>(p, mk, mv, stream);
+        return p.head_dim == 128 ? pu::launch_p<__nv_bfloat16, 128>(p, persistent, mk, mv, stream)
+                                 : pu::launch_p<__nv_bfloat16, 64>(p, persistent, mk, mv, stream);
+    return p.head_dim == 128 ? pu::launch_p<__half, 128>(p, persistent, mk, mv, stream)
+                             : pu::launch_p<__half, 64>(p, persistent, mk, mv, stream);
 }
 
 }  // namespace pa

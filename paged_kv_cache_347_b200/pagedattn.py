@@ -385,7 +385,8 @@ def pa_prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cach
                variant: int = 0) -> torch.Tensor:
     """Causal attention of each sequence's last n_s tokens (rows cu_q_lens[s]..
     cu_q_lens[s+1] of q [total, Hq, D]) over its paged context; out float32.
-    variant: 0 automatic, 1 the mma.sync kernel, 2 the tcgen05 kernel."""
+    variant: 0 automatic, 1 the mma.sync kernel, 2 the tcgen05 kernel, 3 the tcgen05
+    kernel persistent (one CTA per SM over a share of the tiles)."""
     NB, Hkv, bs, D = k_cache.shape
     total, Hq, Dq = q.shape
     if Dq != D or tuple(out.shape) != (total, Hq, D):

@@ -281,8 +281,9 @@ def test_preempted_sequence_swaps_out_and_back_and_decodes_on():
 
 
 # ---------------------------------------------------------------- chunked prefill
-# prefill_variant 1 = mma.sync kernel, 2 = tcgen05 kernel (TMEM accumulators)
-@pytest.mark.parametrize("pv", [1, 2])
+# prefill_variant 1 = mma.sync kernel, 2 = tcgen05 kernel (TMEM accumulators),
+# 3 = the tcgen05 kernel persistent (one CTA per SM walking its share of the tiles)
+@pytest.mark.parametrize("pv", [1, 2, 3])
 @pytest.mark.parametrize("dtype,Hq,Hkv,D,bs", [("bf16", 32, 8, 128, 16), ("f16", 8, 8, 64, 8),
                                                ("bf16", 16, 2, 128, 32), ("bf16", 6, 2, 64, 64),
                                                ("f16", 12, 2, 128, 16), ("bf16", 7, 7, 128, 8)])
@@ -294,7 +295,7 @@ def test_chunked_prefill_matches_oracle(dtype, Hq, Hkv, D, bs, pv):
     assert len(errs) == 2 and max(errs) <= TOL[dtype], errs
 
 
-@pytest.mark.parametrize("pv", [1, 2])
+@pytest.mark.parametrize("pv", [1, 2, 3])
 def test_chunk_covering_the_whole_sequence_and_single_tokens(pv):
     wl = workloads.chunked_prefill(batch=6, ctx_lo=0, ctx_hi=0, chunk_lo=1, chunk_hi=130,
                                    num_blocks=512, chunks=3)
@@ -302,7 +303,7 @@ def test_chunk_covering_the_whole_sequence_and_single_tokens(pv):
     assert max(errs) <= TOL["bf16"], errs
 
 
-@pytest.mark.parametrize("pv", [1, 2])
+@pytest.mark.parametrize("pv", [1, 2, 3])
 def test_prefill_long_context(pv):
     """Chunks of 512-1024 rows after 2k-6k tokens of context: many 64-key
     stages per CTA, several CTAs per sequence, ragged last CTA and stage."""
@@ -313,7 +314,7 @@ def test_prefill_long_context(pv):
     assert max(errs) <= TOL["bf16"], errs
 
 
-@pytest.mark.parametrize("pv", [1, 2])
+@pytest.mark.parametrize("pv", [1, 2, 3])
 @pytest.mark.parametrize("dtype", ["bf16", "f16"])
 @pytest.mark.parametrize("scale", [-0.2, 0.0, 0.5])
 def test_prefill_any_finite_scale(pv, dtype, scale):
@@ -441,7 +442,7 @@ def test_steps_read_one_step_behind_match_the_oracle():
         assert err <= TOL["bf16"], (i, kinds[i], err)
 
 
-@pytest.mark.parametrize("pv", [1, 2])
+@pytest.mark.parametrize("pv", [1, 2, 3])
 @pytest.mark.parametrize("dtype,Hq,Hkv,D,bs,ctx,chunk_lo,chunk_hi", [
     ("bf16", 16, 4, 128, 16, 300, 0, 3),     # empty chunks next to 1-3-token ones (seed 11)
     ("bf16", 10, 2, 128, 16, 500, 1, 300),   # G = 5: 25 tokens x 5 heads + 3 idle rows per tile
@@ -456,7 +457,21 @@ def test_prefill_edge_shapes(pv, dtype, Hq, Hkv, D, bs, ctx, chunk_lo, chunk_hi)
     assert len(errs) == 2 and max(errs) <= TOL[dtype], errs
 
 
-@pytest.mark.parametrize("pv", [1, 2])
+@pytest.mark.parametrize("pv", [2, 3])
+def test_prefill_many_tiles_per_cta(pv):
+    """Forty sequences with chunks of 0 to 300 tokens after 0 to 700 tokens of
+    context: ~800 token tiles (many of them empty) for 148 persistent CTAs,
+    so every CTA walks several tiles of different sequences and lengths, with
+    empty ones skipped between them, in both of its Q buffers."""
+    wl = workloads.chunked_prefill(seed=13, batch=40, ctx_lo=0, ctx_hi=700, chunk_lo=0,
+                                   chunk_hi=300, num_heads=16, num_kv_heads=4, head_dim=128,
+                                   dtype="bf16", block_size=16,
+                                   num_blocks=40 * (700 + 600) // 16 + 64, chunks=2)
+    errs, _, _ = run_parity(wl, table_width=(700 + 600) // 16 + 2, prefill_variant=pv)
+    assert len(errs) == 2 and max(errs) <= TOL["bf16"], errs
+
+
+@pytest.mark.parametrize("pv", [1, 2, 3])
 def test_prefill_full_study_size_sampled(pv):
     """The prefill study's first workload at full size (8 sequences, 4096
     tokens of context + a 1024-token chunk, 32/8 heads, D 128, bf16, bs 16),
@@ -469,7 +484,7 @@ def test_prefill_full_study_size_sampled(pv):
     assert len(errs) == 1 and max(errs) <= TOL["bf16"], errs
 
 
-@pytest.mark.parametrize("pv", [1, 2])
+@pytest.mark.parametrize("pv", [1, 2, 3])
 def test_prefill_bad_table_entry_is_reported(pv):
     """A table entry outside [0, num_blocks) is read as zeros and sets the
     "table" device error bit; the other sequences still match the oracle."""

@@ -120,7 +120,7 @@ def test_static_decode_writes_only_out():
     assert not pa.device_errors()
 
 
-@pytest.mark.parametrize("variant", [1, 2])
+@pytest.mark.parametrize("variant", [1, 2, 3])
 @pytest.mark.parametrize("G", [4, 7])
 def test_prefill_writes_only_out(variant, G):
     from paged_kv_cache_347_b200 import pagedattn as pa
