@@ -552,7 +552,7 @@ def run_ours(args, ws, rank, local):
     if rank == 0 and ws == 1 and not args.no_prefill:
         # the chunked-prefill kernel (tensor-core bound), timed apart from the
         # decode steps above
-        mma_sync, tc = prefill_rows(4096, 1024)
+        mma_sync, tc, persistent = prefill_rows(4096, 1024)
         peak_tf, peak_tf_src = _bf16_peak_tflops()
         res["prefill"] = {
             "workload": "chunked prefill: 8 x (4096 context + 1024-token chunk), 32/8 heads, "
@@ -561,7 +561,7 @@ def run_ours(args, ws, rank, local):
             "roofline": {"bound": "tensor", "achieved": tc["tflops"], "peak": peak_tf,
                          "unit": "TFLOP/s", "frac": tc["frac_of_bf16_peak"],
                          "flops_per_launch": tc["flops_per_launch"], "peak_source": peak_tf_src},
-            "mma_sync_kernel_ms": mma_sync["ms"],
+            "mma_sync_kernel_ms": mma_sync["ms"], "persistent_kernel_ms": persistent["ms"],
             "max_abs_diff_vs_mma_sync": tc["max_abs_diff_vs_mma_sync"]}
     if rank == 0 and ws == 1 and not args.no_cpu:
         smp = OracleSampler(args.workload, seed)
@@ -1051,9 +1051,10 @@ def _bf16_peak_tflops():
 
 
 def prefill_rows(ctx: int, chunk: int, batch: int = 8):
-    """Both prefill kernels on one chunked-prefill workload (32/8 heads, D 128,
-    bf16, bs 16): CUDA-event ms over 20 launches each, the definition's FLOPs
-    (4 * D * Hq per (row, attended key)) and the kernels' full-size agreement."""
+    """The prefill kernels (mma.sync, tcgen05, tcgen05 persistent) on one
+    chunked-prefill workload (32/8 heads, D 128, bf16, bs 16): CUDA-event ms
+    over 20 launches each, the definition's FLOPs (4 * D * Hq per (row,
+    attended key)) and the kernels' full-size agreement."""
     from paged_kv_cache_347_b200 import pagedattn as pa
     from paged_kv_cache_347_b200.runner import PagedKVRunner
     wl = workloads.chunked_prefill(batch=batch, ctx_lo=ctx, ctx_hi=ctx, chunk_lo=chunk,
@@ -1071,7 +1072,7 @@ def prefill_rows(ctx: int, chunk: int, batch: int = 8):
     flops = 4.0 * 128 * 32 * sum(ctx + i + 1 for i in range(chunk)) * batch
     peak, _ = _bf16_peak_tflops()
     rows = []
-    for variant, kernel in ((1, "mma.sync"), (2, "tcgen05")):
+    for variant, kernel in ((1, "mma.sync"), (2, "tcgen05"), (3, "tcgen05 persistent")):
         ms = _events_ms(lambda: pa.pa_prefill(o, dev[2], r.k_cache, r.v_cache, a.dev["tables"],
                                               a.dev["lens"], a.dev["cu"], r.scale,
                                               max_q_len=a.max_q, max_seq_len=a.max_len,
@@ -1083,7 +1084,7 @@ def prefill_rows(ctx: int, chunk: int, batch: int = 8):
                "flops_per_launch": flops}
         if variant == 1:
             first = o.clone()
-        else:  # both kernels compute the same rows at full size
+        else:  # the kernels compute the same rows at full size
             row["max_abs_diff_vs_mma_sync"] = float((o - first).abs().max())
         rows.append(row)
     del r
