@@ -6,8 +6,10 @@
 // details"): row r of a sequence's chunk, at position L - n + r, attends to
 // positions 0..L-n+r through the block table.
 //
-// CTA = 128 (token, query head) rows: 128/G chunk tokens of one KV head g of
-// one sequence, walking the context in stages of 128 keys.  Twelve warps:
+// Tile = 128 (token, query head) rows: 128/G chunk tokens of one KV head g of
+// one sequence, walking the context in stages of 128 keys.  A CTA takes one
+// tile, or (the persistent form) one CTA per SM walks every gridDim-th tile,
+// with stage and tile counters running on across tiles.  Twelve warps:
 //   * warps 0-7, softmax: warp w serves TMEM lanes 32 (w % 4) .. +31 (the
 //     rows) and keys 64 (w / 4) .. +63 of each stage, so each row has two
 //     threads, which agree its maximum through shared memory.  A thread reads
@@ -24,10 +26,15 @@
 //     S is double-buffered, so the softmax of stage i+1 can start as soon as
 //     it ends stage i; S(i+2), which overwrites the columns PV(i) reads, is
 //     issued once PV(i) has completed.
+// Between two tiles the softmax warps put the next tile's Q into the other Q
+// buffer as soon as the tile's last PV is done (the S thread can start the
+// next tile), read O out of TMEM and count it on o_free (the next tile's
+// first PV starts O afresh), then normalise and store the rows.
 // TMEM (512 columns): S/P buffers [0,128) and [128,256), O [256,256+D),
-// Q [384,384+D/2).  In P, key block j (keys 16j..16j+15) holds its high parts
-// in columns 16j..16j+7 and its remainders in 16j+8..16j+15, two keys per
-// column; Q holds two elements of a row per column.
+// two Q buffers [384,384+D/2) and [384+D/2,384+D).  In P, key block j (keys
+// 16j..16j+15) holds its high parts in columns 16j..16j+7 and its remainders
+// in 16j+8..16j+15, two keys per column; Q holds two elements of a row per
+// column.
 //
 // Every wait is bounded (~2 s); on a timeout the CTA records
 // PA_DEVERR_TIMEOUT, the other warps stop waiting, the producers wait
