@@ -143,6 +143,35 @@ def test_prefill_writes_only_out(variant, G):
     assert not pa.device_errors()
 
 
+@pytest.mark.parametrize("variant", [2, 3])
+def test_prefill_output_16_byte_aligned(variant):
+    """The tcgen05 kernels write a row with 32-byte stores when out is
+    32-byte aligned and fall back to 16-byte ones when it is only 16-byte
+    aligned: an out that starts 16 bytes into a buffer gets the same bits as
+    an aligned one, and the 16 bytes before it and the tail stay untouched."""
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    G, Hkv, D, bs = 4, 2, 128, 16
+    lens, chunks = [300, 1000, 129], [300, 77, 1]
+    B = len(lens)
+    _, kc, vc, tab, sl = _paged_inputs(B, G * Hkv, Hkv, D, bs, lens, torch.bfloat16, 9)
+    T = sum(chunks)
+    g = torch.Generator(device="cuda").manual_seed(10)
+    q = torch.randn(T, G * Hkv, D, generator=g, device="cuda").to(torch.bfloat16)
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(chunks)]), dtype=torch.int32, device="cuda")
+    n = T * G * Hkv * D
+    aligned = torch.empty(n, dtype=torch.float32, device="cuda")
+    buf = torch.full((n + 8,), float("nan"), dtype=torch.float32, device="cuda")
+    shifted = buf[4:4 + n]                      # 16 bytes past a 256-byte boundary
+    assert shifted.data_ptr() % 32 == 16
+    for o in (aligned, shifted):
+        pa.pa_prefill(o.view(T, G * Hkv, D), q, kc, vc, tab, sl, cu, 0.088,
+                      max_q_len=max(chunks), max_seq_len=tab.shape[1] * bs, variant=variant)
+    torch.cuda.synchronize()
+    assert torch.equal(aligned.view(torch.int32), shifted.view(torch.int32))
+    assert torch.isnan(buf[:4]).all() and torch.isnan(buf[4 + n:]).all()
+    assert not pa.device_errors()
+
+
 @pytest.mark.parametrize("dtype,bs,D", [(torch.bfloat16, 16, 128), (torch.float32, 4, 64),
                                         (torch.float16, 64, 64)])
 def test_append_writes_only_its_slots(dtype, bs, D):
