@@ -490,9 +490,11 @@ def run_ours(args, ws, rank, local):
         total_bytes += pl.step_bytes[(args.warmup + i) % len(plans)]
         launches += pl.launches_per[(args.warmup + i) % len(plans)]
     timed = torch.cuda.CUDAGraph()
+    keep = []  # every split workspace a captured step writes stays allocated
     with torch.cuda.graph(timed, capture_error_mode="thread_local"):
         for i in range(args.steps):
             pl.step(args.warmup + i)
+            keep.append(pa.cached_workspace(dev))
     timed.replay()
     torch.cuda.synchronize()
 
@@ -510,7 +512,7 @@ def run_ours(args, ws, rank, local):
     timed.replay()
     t_end.record()
     torch.cuda.synchronize()
-    del timed
+    del timed, keep
     # the main kernel alone, after the steps (its own launches, not counted
     # in gpu_launches); still inside the clock record
     main = time_main_kernel(pl, max(16, args.main_launches), dev)
