@@ -100,6 +100,23 @@ static int splits_for(int max_seq_len, int partition) {
     return max_seq_len <= 0 ? 1 : (int)(((int64_t)max_seq_len + partition - 1) / partition);
 }
 
+// CTAs of the two-head variant-3 kernel resident at once on the current
+// device (its occupancy, asked once per device and shape, times the SMs), or
+// a negative status.
+static int hw2_slots(int dtype, int head_dim, int block_size) {
+    static std::atomic<int> cache[kMaxDevices][2][2][2];
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return fail(PA_ERR_CUDA, "no CUDA device");
+    std::atomic<int> &c = cache[dev][dtype == PA_F16][head_dim == 128][block_size == 16];
+    int per_sm = c.load(std::memory_order_relaxed);
+    if (per_sm <= 0) {
+        per_sm = decode_hw2_resident_per_sm(dtype, head_dim, block_size);
+        if (per_sm <= 0) return fail(PA_ERR_CUDA, "occupancy query failed");
+        c.store(per_sm, std::memory_order_relaxed);
+    }
+    return per_sm * num_sms();
+}
+
 static size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Workspace: part_o [B][Hq][S][D] float, part_ml [B][Hq][S][2] float, then
@@ -262,7 +279,8 @@ static int decode_impl(float *out, const void *q, const void *k_cache, const voi
     pa_decode_opts o;
     std::memset(&o, 0, sizeof(o));
     if (opts) o = *opts;
-    const int partition_size = o.partition_size, variant = o.variant;
+    const int partition_size = o.partition_size;
+    int variant = o.variant;
     if (o.merge < 0 || o.merge > 2) return fail(PA_ERR_INVALID_ARG, "merge %d", o.merge);
     int rc = check_shape(num_kv_heads, head_dim, block_size, dtype);
     if (rc) return rc;
@@ -377,6 +395,20 @@ static int decode_impl(float *out, const void *q, const void *k_cache, const voi
         e = cudaEventRecord(prof.begin, st);
         if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     }
+    // The automatic choice for 16-bit caches: two KV heads per CTA, one per
+    // warp (variant 3), where the kernel exists for the block size and its
+    // grid (every split of the longest length, empty ones included) fills at
+    // least one wave of resident CTAs; else the tensor-core kernel with its
+    // CTA per KV head, twice as many CTAs for a thin batch.
+    if (variant == 0 && tc_ok && (block_size == 8 || block_size == 16) &&
+        num_kv_heads % 2 == 0) {
+        const int slots = hw2_slots(dtype, head_dim, block_size);
+        if (slots < 0) return slots;
+        if ((int64_t)p.max_splits * (num_kv_heads / 2) * num_seqs >= slots) {
+            variant = 3;
+            heads_per_cta = 2;
+        }
+    }
     if (variant == 3)
         e = launch_decode_hw(p, dtype, heads_per_cta, st);
     else if ((variant == 0 && tc_ok) || variant == 2)
@@ -472,17 +504,8 @@ int pa_decode_choose(const int32_t *seq_lens_host, int num_seqs, int num_kv_head
     // 1024-token splits fill more, 1024 when they still fit one wave, else
     // 512 (several waves, short CTAs to balance them).
     if (slots == 0) {
-        static std::atomic<int> cache[kMaxDevices][2][2][2];
-        const int dev = current_device();
-        if (dev < 0 || dev >= kMaxDevices) return fail(PA_ERR_CUDA, "no CUDA device");
-        std::atomic<int> &c = cache[dev][dtype == PA_F16][head_dim == 128][block_size == 16];
-        int per_sm = c.load(std::memory_order_relaxed);
-        if (per_sm <= 0) {
-            per_sm = decode_hw2_resident_per_sm(dtype, head_dim, block_size);
-            if (per_sm <= 0) return fail(PA_ERR_CUDA, "occupancy query failed");
-            c.store(per_sm, std::memory_order_relaxed);
-        }
-        slots = per_sm * num_sms();
+        slots = hw2_slots(dtype, head_dim, block_size);
+        if (slots < 0) return slots;
     }
     auto ctas = [&](int p) {
         int64_t n = 0;
