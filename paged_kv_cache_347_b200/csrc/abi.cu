@@ -388,13 +388,6 @@ static int decode_impl(float *out, const void *q, const void *k_cache, const voi
                        rows + (int64_t)(num_kv_heads + 1) * block_size < (int64_t(1) << 31);
     if (variant >= 2 && !tc_ok)
         return fail(PA_ERR_UNSUPPORTED, "cache too large for the tensor-core kernels");
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const ProfileEvents prof = t_prof;
-    cudaError_t e;
-    if (prof.begin && prof.end) {
-        e = cudaEventRecord(prof.begin, st);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
-    }
     // The automatic choice for 16-bit caches: two KV heads per CTA, one per
     // warp (variant 3), where the kernel exists for the block size and its
     // grid (every split of the longest length, empty ones included) fills at
@@ -408,6 +401,13 @@ static int decode_impl(float *out, const void *q, const void *k_cache, const voi
             variant = 3;
             heads_per_cta = 2;
         }
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const ProfileEvents prof = t_prof;
+    cudaError_t e;
+    if (prof.begin && prof.end) {
+        e = cudaEventRecord(prof.begin, st);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaEventRecord");
     }
     if (variant == 3)
         e = launch_decode_hw(p, dtype, heads_per_cta, st);
