@@ -329,9 +329,9 @@ static int decode_impl(float *out, const void *q, const void *k_cache, const voi
         (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
         return fail(PA_ERR_INVALID_ARG, "misaligned pointer");
     const int splits = splits_for(max_seq_len, part);
-    if (splits > 2048)
-        return fail(PA_ERR_UNSUPPORTED, "max_seq_len %d needs %d splits of %d tokens (max 2048)",
-                    max_seq_len, splits, part);
+    if (splits > kMaxSplits)
+        return fail(PA_ERR_UNSUPPORTED, "max_seq_len %d needs %d splits of %d tokens (max %d)",
+                    max_seq_len, splits, part, kMaxSplits);
     const size_t need = workspace_bytes_for(num_seqs, num_heads, head_dim, splits);
     if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
         return fail(PA_ERR_INVALID_ARG, "workspace of %zu bytes needed, %zu given", need,

@@ -315,15 +315,13 @@ __global__ void __launch_bounds__(kReduceThreads, 4) decode_reduce_kernel(Decode
 // consecutive d); the first batch of each thread's partial rows is loaded
 // before the weights are formed from the (m, l) pairs, so both loads are in
 // flight together.
-constexpr int kWideMaxSplits = 2048;
-
 __global__ void __launch_bounds__(kReduceThreads) decode_reduce_wide_kernel(DecodeParams p) {
     pdl_wait_prior_grid();
     const int h = blockIdx.x, s = blockIdx.y;
     const int L = checked_seq_len(p, s, false);
     const int nsplit = num_splits_for(L, p.partition_size);
     if (nsplit <= 1) return;
-    __shared__ float w_s[kWideMaxSplits];
+    __shared__ float w_s[kMaxSplits];
     __shared__ float red[kReduceThreads / 32];
     __shared__ float4 part[kReduceThreads];
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;

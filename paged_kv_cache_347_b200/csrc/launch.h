@@ -7,6 +7,11 @@
 
 namespace pa {
 
+// Most splits one decode call may have (max_seq_len / partition_size,
+// rounded up): the wide split reduce keeps one weight per split in shared
+// memory, and the entry points reject a call that would need more.
+constexpr int kMaxSplits = 2048;
+
 // Everything a decode kernel needs; passed by value.
 struct DecodeParams {
     float *out;        // [B][Hq][D]
