@@ -570,7 +570,7 @@ def run_ours(args, ws, rank, local):
     if rank == 0 and ws == 1 and not args.no_prefill:
         # the chunked-prefill kernel (tensor-core bound), timed apart from the
         # decode steps above
-        mma_sync, tc, persistent = prefill_rows(4096, 1024)
+        mma_sync, tc, persistent, p16 = prefill_rows(4096, 1024)
         peak_tf, peak_tf_src = _bf16_peak_tflops()
         res["prefill"] = {
             "workload": "chunked prefill: 8 x (4096 context + 1024-token chunk), 32/8 heads, "
@@ -580,7 +580,14 @@ def run_ours(args, ws, rank, local):
                          "unit": "TFLOP/s", "frac": tc["frac_of_bf16_peak"],
                          "flops_per_launch": tc["flops_per_launch"], "peak_source": peak_tf_src},
             "mma_sync_kernel_ms": mma_sync["ms"], "persistent_kernel_ms": persistent["ms"],
-            "max_abs_diff_vs_mma_sync": tc["max_abs_diff_vs_mma_sync"]}
+            "max_abs_diff_vs_mma_sync": tc["max_abs_diff_vs_mma_sync"],
+            "one_fp16_p": {
+                "variant": 4, "ms": p16["ms"], "tflops": p16["tflops"],
+                "frac": p16["frac_of_bf16_peak"],
+                "max_abs_diff_vs_mma_sync": p16["max_abs_diff_vs_mma_sync"],
+                "note": "opt-in: each weight rounded once to fp16 (within 2^-11, against "
+                        "2^-14 for the default's high part + remainder), half the P.V "
+                        "products; the bf16 V stages converted to fp16 in shared memory"}}
     if rank == 0 and ws == 1 and not args.no_cpu:
         smp = OracleSampler(args.workload, seed)
         nb, secs, pairs = smp.run(args.cpu_budget)
@@ -1069,8 +1076,8 @@ def _bf16_peak_tflops():
 
 
 def prefill_rows(ctx: int, chunk: int, batch: int = 8):
-    """The prefill kernels (mma.sync, tcgen05, tcgen05 persistent) on one
-    chunked-prefill workload (32/8 heads, D 128, bf16, bs 16): CUDA-event ms
+    """The prefill kernels (mma.sync, tcgen05, tcgen05 persistent, tcgen05 with
+    one fp16 P) on one chunked-prefill workload (32/8 heads, D 128, bf16, bs 16): CUDA-event ms
     over 20 launches each, the definition's FLOPs (4 * D * Hq per (row,
     attended key)) and the kernels' full-size agreement."""
     from paged_kv_cache_347_b200 import pagedattn as pa
@@ -1090,7 +1097,8 @@ def prefill_rows(ctx: int, chunk: int, batch: int = 8):
     flops = 4.0 * 128 * 32 * sum(ctx + i + 1 for i in range(chunk)) * batch
     peak, _ = _bf16_peak_tflops()
     rows = []
-    for variant, kernel in ((1, "mma.sync"), (2, "tcgen05"), (3, "tcgen05 persistent")):
+    for variant, kernel in ((1, "mma.sync"), (2, "tcgen05"), (3, "tcgen05 persistent"),
+                            (4, "tcgen05, one fp16 P")):
         ms = _events_ms(lambda: pa.pa_prefill(o, dev[2], r.k_cache, r.v_cache, a.dev["tables"],
                                               a.dev["lens"], a.dev["cu"], r.scale,
                                               max_q_len=a.max_q, max_seq_len=a.max_len,

@@ -78,6 +78,8 @@ typedef enum {
 #define PA_DEVERR_SLOT 0x4u    /* slot >= num_blocks * block_size             */
 #define PA_DEVERR_PAIR 0x8u    /* copy pair block outside [0, num_blocks)     */
 #define PA_DEVERR_TIMEOUT 0x10u/* a pipeline wait gave up after ~2 s          */
+#define PA_DEVERR_RANGE 0x20u  /* prefill variant 4, bf16 cache: a V value    */
+                               /* beyond the fp16 range (non-finite rows)      */
 
 /* Message of the last failed call on this thread ("" if none). */
 const char *pa_last_error(void);
@@ -339,11 +341,24 @@ int pa_prefill(float *out, const void *q, const void *k_cache, const void *v_cac
  *   3  the same kernel persistent: one CTA per SM walks its share of the
  *      128-row tiles (in the order of kernel 2's grid), the
  *      next tile's Q going into a second TMEM buffer and its first products
- *      starting while the current tile's output is written.
- * Same arguments, results (within fp32 rounding) and errors as pa_prefill;
- * another variant returns PA_ERR_INVALID_ARG.  All kernels need all of a
- * sequence's table entries for positions < L_s to be valid blocks (an entry
- * outside [0, num_blocks) reads as zeros and sets PA_DEVERR_TABLE).
+ *      starting while the current tile's output is written;
+ *   4  kernel 2 with the weights P entering the P V product as one fp16 per
+ *      weight (kernels 1-3 carry a 16-bit high part and its remainder, two
+ *      products): half the P V work.  A bf16 cache's V stages are converted
+ *      to fp16 in shared memory by a fourth warpgroup (512 threads).  Each
+ *      weight is then within 2^-11 of its value (2^-25 absolute below
+ *      2^-14), against 2^-14 for kernels 2 and 3, so the output error bound
+ *      grows to about 2^-11 * max|v|: within 3e-3 while |v| <= 6.  A bf16 V
+ *      value of magnitude 65536 or more (beyond the fp16 range) makes its
+ *      tile's rows non-finite and sets PA_DEVERR_RANGE; f16 caches have no
+ *      such case.  Measured on 8 x (4096 + 1024) rows, 32/8 heads, D 128:
+ *      0.733 ms vs 0.788 (bf16) and 0.683 vs 0.803 (f16) in 20-launch
+ *      bursts, 11-18% faster in one-second loops at the power cap.
+ * Same arguments, results (within the stated rounding) and errors as
+ * pa_prefill; another variant returns PA_ERR_INVALID_ARG.  All kernels need
+ * all of a sequence's table entries for positions < L_s to be valid blocks
+ * (an entry outside [0, num_blocks) reads as zeros and sets
+ * PA_DEVERR_TABLE).
  */
 int pa_prefill_ex(float *out, const void *q, const void *k_cache, const void *v_cache,
                   const int32_t *block_tables, const int32_t *seq_lens, const int32_t *cu_q_lens,

@@ -554,8 +554,8 @@ int pa_prefill_ex(float *out, const void *q, const void *k_cache, const void *v_
                   int max_blocks_per_seq, int num_blocks, int max_q_len, int max_seq_len,
                   float scale, int dtype, int variant, void *stream) {
     clear_error();
-    if (variant < 0 || variant > 3)
-        return fail(PA_ERR_INVALID_ARG, "prefill variant %d not in {0, 1, 2, 3}", variant);
+    if (variant < 0 || variant > 4)
+        return fail(PA_ERR_INVALID_ARG, "prefill variant %d not in {0, 1, 2, 3, 4}", variant);
     if (variant == 0) variant = kPrefillDefault;
     int rc = check_shape(num_kv_heads, head_dim, block_size, dtype);
     if (rc) return rc;
@@ -610,7 +610,7 @@ int pa_prefill_ex(float *out, const void *q, const void *k_cache, const void *v_
     p.tokens_per_cta = (variant >= 2 ? 128 : 64) / G;
     p.scale_log2 = scale * 1.4426950408889634f;
     const cudaStream_t st = static_cast<cudaStream_t>(stream);
-    cudaError_t e = variant >= 2 ? launch_prefill_umma(p, dtype, variant == 3, st)
+    cudaError_t e = variant >= 2 ? launch_prefill_umma(p, dtype, variant - 2, st)
                                  : launch_prefill_tc(p, dtype, st);
     if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
     return PA_OK;

@@ -98,10 +98,11 @@ struct PrefillParams {
 };
 // mma.sync kernel: 64 (token, head) rows per CTA, accumulators in registers.
 cudaError_t launch_prefill_tc(const PrefillParams &p, int dtype, cudaStream_t stream);
-// tcgen05 kernel: 128 rows per CTA, S and O accumulated in TMEM; persistent:
-// one CTA per SM walking a share of the token tiles, each tile's start
-// overlapping the previous tile's end.
-cudaError_t launch_prefill_umma(const PrefillParams &p, int dtype, bool persistent,
+// tcgen05 kernel: 128 rows per CTA, S and O accumulated in TMEM.  form 0:
+// one tile per CTA; 1 (persistent): one CTA per SM walking a share of the
+// token tiles, each tile's start overlapping the previous tile's end; 2: one
+// tile per CTA with P entering the PV product as one fp16 per weight.
+cudaError_t launch_prefill_umma(const PrefillParams &p, int dtype, int form,
                                 cudaStream_t stream);
 
 // One CTA waiting, bounded, on an mbarrier phase nothing completes (selftest.cu).

@@ -36,6 +36,15 @@
 // in 16j+8..16j+15, two keys per column; Q holds two elements of a row per
 // column.
 //
+// The one-fp16-P form (kP16): each weight is rounded once to fp16, the
+// words of a thread's 64 keys taking the first 32 of its S columns (key
+// block j of the tile at column 64 (j / 4) + 8 (j % 4)), and PV(i) is one
+// MMA per key block with P and V both f16.  Against a bf16 cache a fourth
+// warpgroup (warps 12-15) rewrites each landed V stage in place as fp16
+// (and zeroes the rows past the tile's last key) before the PV thread may
+// read it; a V value beyond the fp16 range turns infinite there, which the
+// epilogue finds in the output and reports as PA_DEVERR_RANGE.
+//
 // Every wait is bounded (~2 s); on a timeout the CTA records
 // PA_DEVERR_TIMEOUT, the other warps stop waiting, the producers wait
 // (bounded) for their copies, warp 0 waits for the MMAs and frees the TMEM.
@@ -57,6 +66,11 @@ constexpr int kM = 128;               // rows per CTA
 constexpr int kKeys = 128;            // keys per stage
 constexpr int kSoftmaxThreads = 256;  // 8 warps, two threads per row
 constexpr int kThreads = kSoftmaxThreads + 128;  // + K, V producers, S, PV issuers
+// + one warpgroup converting the V stages of a bf16 cache to fp16 (one-fp16-P form)
+constexpr int kConvThreads = 128;
+__host__ __device__ constexpr int threads_for(bool conv) {
+    return conv ? kThreads + kConvThreads : kThreads;
+}
 constexpr int kTmemCols = 512;
 constexpr int kColO = 256, kColQ = 384;
 constexpr int kRowBytes = 128;        // one 64-element piece of a 16-bit row
@@ -71,8 +85,8 @@ struct Cfg {
     static constexpr int kXchOffset = kVOffset + NV * kStageBytes;  // float [2][2][128]
     static constexpr int kBarOffset = kXchOffset + 2 * 2 * kM * 4;
     // k_full[NK] k_empty[NK] v_full[NV] v_empty[NV] s_full[2] p_full[2] pv_done[2]
-    // q_full[2] o_free mma_done xchg[4]
-    static constexpr int kNumBars = 2 * NK + 2 * NV + 6 + 4 + 4;
+    // q_full[2] o_free mma_done xchg[4] v_conv[NV]
+    static constexpr int kNumBars = 2 * NK + 3 * NV + 6 + 4 + 4;
     static constexpr int kTmemSlot = kBarOffset + kNumBars * 8;
     static constexpr int kAbortOffset = kTmemSlot + 16;
     static constexpr int kSmemBytes = kAbortOffset + 16;
@@ -134,6 +148,15 @@ template <> struct PSplit<__half> {
     }
 };
 
+// Two bf16 values (one 32-bit word, the lower element in the low half) as
+// two fp16 values in the same places: each widened to fp32 (exact), then
+// rounded to the nearest fp16.  Exact for magnitudes in [2^-14, 65504];
+// smaller ones keep 2^-24 absolute precision, 65536 and above become
+// infinite.
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+    return Mma<__half>::pack(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
 // What a CTA needs of one token tile: its sequence and KV head, where its
 // rows start, how many keys it attends to.
 struct Tile {
@@ -187,11 +210,13 @@ __device__ __forceinline__ bool describe_tile(const PrefillParams &p, int u, boo
     return true;
 }
 
-template <typename T, int D, int BS, int NK, int NV, bool kPersist>
-__global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
-    const __grid_constant__ CUtensorMap tmap_k, const __grid_constant__ CUtensorMap tmap_v,
-    const PrefillParams p) {
+template <typename T, int D, int BS, int NK, int NV, bool kPersist, bool kP16>
+__global__ void __launch_bounds__(threads_for(kP16 && std::is_same<T, __nv_bfloat16>::value), 1)
+    prefill_umma_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                        const __grid_constant__ CUtensorMap tmap_v, const PrefillParams p) {
     using C = Cfg<D, BS, NK, NV>;
+    // one fp16 P against a bf16 cache: V converted to fp16 in shared memory
+    constexpr bool kConv = kP16 && std::is_same<T, __nv_bfloat16>::value;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -217,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     const uint32_t k_full = bar0, k_empty = k_full + 8 * NK, v_full = k_empty + 8 * NK,
                    v_empty = v_full + 8 * NV, s_full = v_empty + 8 * NV, p_full = s_full + 16,
                    pv_done = p_full + 16, q_full = pv_done + 16, o_free = q_full + 16,
-                   mma_done = o_free + 8, xchg = mma_done + 8;
+                   mma_done = o_free + 8, xchg = mma_done + 8, v_conv = xchg + 32;
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + C::kAbortOffset);
     volatile uint32_t *tmem_slot = reinterpret_cast<volatile uint32_t *>(smem + C::kTmemSlot);
 
@@ -241,6 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         mbar_init(o_free, kSoftmaxThreads);  // a tile's O read out of TMEM
         mbar_init(mma_done, 2);              // both issuing threads
         for (int q = 0; q < 4; ++q) mbar_init(xchg + 8 * q, 64);
+        for (int i = 0; i < NV; ++i) mbar_init(v_conv + 8 * i, kConvThreads);
         *abort_flag = 0;
         fence_mbarrier_init();
     }
@@ -314,6 +340,74 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         return;
     }
 
+    // ------------------------------------------------------------ V converters
+    // (bf16 cache, one-fp16-P form) warps 12-15, one per SM sub-partition:
+    // each V stage, once landed, is rewritten in place as fp16 (the 128-byte
+    // swizzle moves 16-byte chunks within a row only, so a chunk converts
+    // where it lies), rows past the tile's last key as zeros, and counted on
+    // v_conv before the PV MMA reads it.
+    if constexpr (kConv) {
+        if (warp >= 12) {
+            const int ct = threadIdx.x - kThreads;  // 0..127
+            constexpr int kChunks = C::kPieces * kKeys * 8;  // 16-byte chunks per V stage
+            static_assert(kChunks % kConvThreads == 0 && C::kKVPiece == kKeys * 8 * 16,
+                          "V stage: whole chunks per converter thread, contiguous pieces");
+            int gi = 0;
+            bool ok = true;
+            for (int u = u0; ok && u < ntiles; u += ustep) {
+                Tile t;
+                if (!describe_tile<BS, kPersist>(p, u, false, t)) continue;
+                for (int i = 0; i < t.nstages; ++i, ++gi) {
+                    const int slot = gi % NV;
+                    if (!warp_wait(v_full + 8 * slot, (gi / NV) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const int first = min(kKeys, t.nkeys - i * kKeys);  // rows >= first: zeros
+                    // the stage's pieces are contiguous: chunk idx lies idx * 16 bytes
+                    // in, in row (idx % 1024) / 8 of its piece
+                    uint4 *a = reinterpret_cast<uint4 *>(smem + C::kVOffset +
+                                                         slot * C::kStageBytes) + ct;
+                    constexpr int kPer = kChunks / kConvThreads;
+                    if (first == kKeys) {
+                        uint4 w[kPer];
+#pragma unroll
+                        for (int k = 0; k < kPer; ++k) w[k] = a[k * kConvThreads];
+#pragma unroll
+                        for (int k = 0; k < kPer; ++k) {
+                            w[k].x = bf16x2_to_f16x2(w[k].x);
+                            w[k].y = bf16x2_to_f16x2(w[k].y);
+                            w[k].z = bf16x2_to_f16x2(w[k].z);
+                            w[k].w = bf16x2_to_f16x2(w[k].w);
+                            a[k * kConvThreads] = w[k];
+                        }
+                    } else {
+#pragma unroll 4
+                        for (int k = 0; k < kPer; ++k) {
+                            const int row = ((ct + k * kConvThreads) & (kKeys * 8 - 1)) >> 3;
+                            uint4 w = make_uint4(0u, 0u, 0u, 0u);
+                            if (row < first) {
+                                w = a[k * kConvThreads];
+                                w.x = bf16x2_to_f16x2(w.x);
+                                w.y = bf16x2_to_f16x2(w.y);
+                                w.z = bf16x2_to_f16x2(w.z);
+                                w.w = bf16x2_to_f16x2(w.w);
+                            }
+                            a[k * kConvThreads] = w;
+                        }
+                    }
+                    umma::fence_proxy_async_smem();  // visible to the tensor core's reads
+                    mbar_arrive(v_conv + 8 * slot);
+                }
+            }
+            if (!ok && lane == 0) {
+                raise_device_error(p.err, PA_DEVERR_TIMEOUT);
+                *abort_flag = 1;
+            }
+            return;
+        }
+    }
+
     // ------------------------------------------------------------ MMA issuers
     // Warp 10 issues the S MMAs, warp 11 the PV MMAs, each from one thread, so
     // that neither waits behind the other's barrier checks.  MMAs of two
@@ -362,13 +456,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
                         umma::commit(k_empty + 8 * slot);
                     }
                 } else {
-                    constexpr uint32_t idesc_o = umma::idesc_f16(fmt, kM, D, 1);
+                    // P as one fp16 per weight: P and V both f16
+                    constexpr uint32_t idesc_o = umma::idesc_f16(kP16 ? 0u : fmt, kM, D, 1);
 #pragma unroll 1
                     for (int i = 0; ok && i < t.nstages; ++i, ++gi) {
                         // O += P(gi) . V(gi) once the softmax has written P(gi)
                         const int slot = gi % NV;
+                        // a bf16 V stage is read once the converters are done with it
+                        const uint32_t v_ready = kConv ? v_conv : v_full;
                         if (!mbar_wait_bounded(p_full + 8 * (gi & 1), (gi >> 1) & 1, abort_flag) ||
-                            !mbar_wait_bounded(v_full + 8 * slot, (gi / NV) & 1, abort_flag) ||
+                            !mbar_wait_bounded(v_ready + 8 * slot, (gi / NV) & 1, abort_flag) ||
                             (i == 0 && tp > 0 &&
                              !mbar_wait_bounded(o_free, (tp - 1) & 1, abort_flag))) {
                             ok = false;
@@ -382,9 +479,16 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
 #pragma unroll
                         for (int j = 0; j < kKeys / 16; ++j) {  // keys 16j..16j+15
                             const uint64_t b = b0 + ((j * 16 * kRowBytes) >> 4);
-                            umma::mma_f16_ts(tmem + kColO, pb + 16 * j, b, idesc_o,
-                                             (i > 0 || j > 0) ? 1u : 0u);
-                            umma::mma_f16_ts(tmem + kColO, pb + 16 * j + 8, b, idesc_o, 1u);
+                            if constexpr (kP16) {
+                                // block j in the columns of the half of the keys it
+                                // belongs to: (j / 4) * 64 + (j % 4) * 8
+                                umma::mma_f16_ts(tmem + kColO, pb + (j >> 2) * 64 + (j & 3) * 8, b,
+                                                 idesc_o, (i > 0 || j > 0) ? 1u : 0u);
+                            } else {
+                                umma::mma_f16_ts(tmem + kColO, pb + 16 * j, b, idesc_o,
+                                                 (i > 0 || j > 0) ? 1u : 0u);
+                                umma::mma_f16_ts(tmem + kColO, pb + 16 * j + 8, b, idesc_o, 1u);
+                            }
                         }
                         umma::commit(pv_done + 8 * (gi & 1));
                         umma::commit(v_empty + 8 * slot);
@@ -502,6 +606,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         // takes key block q / 16 of the chunk, high parts in its first 8
         // columns, remainders in the next 8 (over the chunk's own S columns)
         uint64_t acc[2] = {pk(0.f, 0.f), pk(0.f, 0.f)};
+        // (the one-fp16 form: the pair's word goes to column 16c + e of the
+        // thread's own S columns, so that its 64 keys take the first 32)
+        [[maybe_unused]] uint32_t p16[32];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
             uint32_t(&w)[32] = sr[c];
@@ -515,13 +622,20 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
                 }
                 const float p0 = umma::ex2(y0), p1 = umma::ex2(y1);
                 acc[e & 1] = add2(acc[e & 1], pk(p0, p1));
-                PSplit<T>::run(p0, p1, w[2 * e], w[2 * e + 1]);
+                if constexpr (kP16)
+                    p16[16 * c + e] = Mma<__half>::pack(p0, p1);
+                else
+                    PSplit<T>::run(p0, p1, w[2 * e], w[2 * e + 1]);
             }
-            uint32_t pw[32];
+            if constexpr (!kP16) {
+                uint32_t pw[32];
 #pragma unroll
-            for (int q = 0; q < 32; ++q) pw[q] = w[2 * ((q >> 4) * 8 + (q & 7)) + ((q >> 3) & 1)];
-            umma::st32(hcol + 32 * c, pw);
+                for (int q = 0; q < 32; ++q)
+                    pw[q] = w[2 * ((q >> 4) * 8 + (q & 7)) + ((q >> 3) & 1)];
+                umma::st32(hcol + 32 * c, pw);
+            }
         }
+        if constexpr (kP16) umma::st32(hcol, p16);
         {
             float a0, a1, b0, b1;
             upk(acc[0], a0, a1);
@@ -544,7 +658,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
                 umma::st32(col, o);
             }
         }
-        if constexpr (kMasked) {
+        if constexpr (kMasked && !kConv) {  // (the converters zero them in that form)
             if (i * kKeys + kKeys > nkeys) {
                 // last stage: V rows past the last key hold stale or unwritten
                 // data; zero them so that their zero weights give exact zeros.
@@ -619,11 +733,18 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
         // O out of TMEM a 32-column chunk at a time, normalised and stored;
         // each lane writes its own row: 32-byte stores when out allows them
         // (whole sectors), else 16-byte ones
+        [[maybe_unused]] uint32_t nonfinite = 0u;
 #pragma unroll
         for (int cb = 0; cb < D / 64; ++cb) {
             uint32_t o[32];
             umma::ld32(lane_base + kColO + half * (D / 2) + 32 * cb, o);
             umma::wait_ld();
+            if constexpr (kConv) {
+                // a V value beyond the fp16 range became infinite in the
+                // conversion and reaches every row of the tile
+#pragma unroll
+                for (int e = 0; e < 32; ++e) nonfinite |= (~o[e] & 0x7f800000u) == 0u;
+            }
             if (cb == D / 64 - 1) {
                 // O is out of TMEM: the next tile's first PV may start it afresh
                 umma::fence_before_sync();
@@ -644,6 +765,9 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
                         __uint_as_float(o[e]) * inv, __uint_as_float(o[e + 1]) * inv,
                         __uint_as_float(o[e + 2]) * inv, __uint_as_float(o[e + 3]) * inv);
             }
+        }
+        if constexpr (kConv) {
+            if (valid && nonfinite) raise_device_error(p.err, PA_DEVERR_RANGE);
         }
         ++tp;
         t = nt;
@@ -666,7 +790,7 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_umma_kernel(
     pdl_launch_dependents();
 }
 
-template <typename T, int D, int BS, bool kPersist>
+template <typename T, int D, int BS, bool kPersist, bool kP16>
 static cudaError_t launch_inst(const PrefillParams &p, const CUtensorMap &mk,
                                const CUtensorMap &mv, cudaStream_t stream) {
     constexpr int NK = D == 128 ? 3 : 6, NV = D == 128 ? 3 : 6;
@@ -677,7 +801,7 @@ static cudaError_t launch_inst(const PrefillParams &p, const CUtensorMap &mk,
     cudaGetDevice(&dev);
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::call_once(once[dev], [&] {
-        attr_err[dev] = cudaFuncSetAttribute(prefill_umma_kernel<T, D, BS, NK, NV, kPersist>,
+        attr_err[dev] = cudaFuncSetAttribute(prefill_umma_kernel<T, D, BS, NK, NV, kPersist, kP16>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::kDynSmem);
     });
@@ -695,7 +819,7 @@ static cudaError_t launch_inst(const PrefillParams &p, const CUtensorMap &mk,
     } else {
         cfg.gridDim = dim3(tiles_x, p.num_kv_heads, p.num_seqs);
     }
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(threads_for(kP16 && std::is_same<T, __nv_bfloat16>::value));
     cfg.dynamicSmemBytes = C::kDynSmem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -703,31 +827,35 @@ static cudaError_t launch_inst(const PrefillParams &p, const CUtensorMap &mk,
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, prefill_umma_kernel<T, D, BS, NK, NV, kPersist>, mk, mv, p);
+    return cudaLaunchKernelEx(&cfg, prefill_umma_kernel<T, D, BS, NK, NV, kPersist, kP16>, mk, mv,
+                              p);
 }
 
-template <typename T, int D, bool kPersist>
+template <typename T, int D, bool kPersist, bool kP16>
 static cudaError_t launch_d(const PrefillParams &p, const CUtensorMap &mk, const CUtensorMap &mv,
                             cudaStream_t stream) {
     switch (p.block_size) {
-    case 8: return launch_inst<T, D, 8, kPersist>(p, mk, mv, stream);
-    case 16: return launch_inst<T, D, 16, kPersist>(p, mk, mv, stream);
-    case 32: return launch_inst<T, D, 32, kPersist>(p, mk, mv, stream);
-    case 64: return launch_inst<T, D, 64, kPersist>(p, mk, mv, stream);
+    case 8: return launch_inst<T, D, 8, kPersist, kP16>(p, mk, mv, stream);
+    case 16: return launch_inst<T, D, 16, kPersist, kP16>(p, mk, mv, stream);
+    case 32: return launch_inst<T, D, 32, kPersist, kP16>(p, mk, mv, stream);
+    case 64: return launch_inst<T, D, 64, kPersist, kP16>(p, mk, mv, stream);
     default: return cudaErrorNotSupported;
     }
 }
 
+// form 0: one tile per CTA; 1: persistent; 2: one tile per CTA, P as one
+// fp16 per weight (a bf16 cache's V stages converted to fp16)
 template <typename T, int D>
-static cudaError_t launch_p(const PrefillParams &p, bool persistent, const CUtensorMap &mk,
+static cudaError_t launch_p(const PrefillParams &p, int form, const CUtensorMap &mk,
                             const CUtensorMap &mv, cudaStream_t stream) {
-    return persistent ? launch_d<T, D, true>(p, mk, mv, stream)
-                      : launch_d<T, D, false>(p, mk, mv, stream);
+    if (form == 1) return launch_d<T, D, true, false>(p, mk, mv, stream);
+    if (form == 2) return launch_d<T, D, false, true>(p, mk, mv, stream);
+    return launch_d<T, D, false, false>(p, mk, mv, stream);
 }
 
 }  // namespace pu
 
-cudaError_t launch_prefill_umma(const PrefillParams &p, int dtype, bool persistent,
+cudaError_t launch_prefill_umma(const PrefillParams &p, int dtype, int form,
                                 cudaStream_t stream) {
     if (p.num_seqs == 0 || p.max_q_len == 0) return cudaSuccess;
     const int64_t rows = (int64_t)p.num_blocks * p.num_kv_heads * p.block_size;
@@ -736,10 +864,10 @@ cudaError_t launch_prefill_umma(const PrefillParams &p, int dtype, bool persiste
         !make_cache_tensor_map(&mv, p.v_cache, dtype, p.head_dim, rows, p.block_size))
         return cudaErrorInvalidValue;
     if (dtype == PA_BF16)
-        return p.head_dim == 128 ? pu::launch_p<__nv_bfloat16, 128>(p, persistent, mk, mv, stream)
-                                 : pu::launch_p<__nv_bfloat16, 64>(p, persistent, mk, mv, stream);
-    return p.head_dim == 128 ? pu::launch_p<__half, 128>(p, persistent, mk, mv, stream)
-                             : pu::launch_p<__half, 64>(p, persistent, mk, mv, stream);
+        return p.head_dim == 128 ? pu::launch_p<__nv_bfloat16, 128>(p, form, mk, mv, stream)
+                                 : pu::launch_p<__nv_bfloat16, 64>(p, form, mk, mv, stream);
+    return p.head_dim == 128 ? pu::launch_p<__half, 128>(p, form, mk, mv, stream)
+                             : pu::launch_p<__half, 64>(p, form, mk, mv, stream);
 }
 
 }  // namespace pa

@@ -30,7 +30,8 @@ DTYPE_CODE = {torch.float32: PA_F32, torch.bfloat16: PA_BF16, torch.float16: PA_
 STATUS = {0: "PA_OK", -1: "PA_ERR_INVALID_ARG", -2: "PA_ERR_UNSUPPORTED",
           -3: "PA_ERR_OUT_OF_BLOCKS", -4: "PA_ERR_UNKNOWN_SEQ", -5: "PA_ERR_CUDA",
           -6: "PA_ERR_DEVICE_BOUNDS", -7: "PA_ERR_SEQ_TOO_LONG"}
-DEVERR = {0x1: "table", 0x2: "seqlen", 0x4: "slot", 0x8: "pair", 0x10: "timeout"}
+DEVERR = {0x1: "table", 0x2: "seqlen", 0x4: "slot", 0x8: "pair", 0x10: "timeout",
+          0x20: "range"}
 
 _c = ctypes
 _vp, _i, _i64, _sz, _f = _c.c_void_p, _c.c_int, _c.c_int64, _c.c_size_t, _c.c_float
@@ -386,7 +387,10 @@ def pa_prefill(out: torch.Tensor, q: torch.Tensor, k_cache: torch.Tensor, v_cach
     """Causal attention of each sequence's last n_s tokens (rows cu_q_lens[s]..
     cu_q_lens[s+1] of q [total, Hq, D]) over its paged context; out float32.
     variant: 0 automatic, 1 the mma.sync kernel, 2 the tcgen05 kernel, 3 the tcgen05
-    kernel persistent (one CTA per SM over a share of the tiles)."""
+    kernel persistent (one CTA per SM over a share of the tiles), 4 the tcgen05
+    kernel with P as one fp16 per weight (half the P.V products; each weight
+    within 2^-11 instead of 2^-14; a bf16 V value beyond the fp16 range sets
+    the "range" device error)."""
     NB, Hkv, bs, D = k_cache.shape
     total, Hq, Dq = q.shape
     if Dq != D or tuple(out.shape) != (total, Hq, D):

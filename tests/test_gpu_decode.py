@@ -295,6 +295,77 @@ def test_chunked_prefill_matches_oracle(dtype, Hq, Hkv, D, bs, pv):
     assert len(errs) == 2 and max(errs) <= TOL[dtype], errs
 
 
+# prefill_variant 4: the tcgen05 kernel with P entering the PV product as one
+# fp16 per weight (a bf16 cache's V stages converted to fp16 in shared memory)
+@pytest.mark.parametrize("dtype,Hq,Hkv,D,bs", [("f16", 8, 8, 64, 8), ("f16", 12, 2, 128, 16),
+                                               ("bf16", 32, 8, 128, 16), ("bf16", 6, 2, 64, 64),
+                                               ("bf16", 7, 7, 128, 32), ("bf16", 16, 2, 128, 8),
+                                               ("f16", 32, 8, 128, 16)])
+def test_chunked_prefill_one_fp16_p_matches_oracle(dtype, Hq, Hkv, D, bs):
+    wl = workloads.chunked_prefill(batch=5, ctx_lo=0, ctx_hi=400, chunk_lo=1, chunk_hi=200,
+                                   num_heads=Hq, num_kv_heads=Hkv, head_dim=D, dtype=dtype,
+                                   block_size=bs, num_blocks=4096 // bs * 2, chunks=2)
+    errs, _, _ = run_parity(wl, table_width=1000 // bs + 2, prefill_variant=4)
+    assert len(errs) == 2 and max(errs) <= TOL[dtype], errs
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_prefill_one_fp16_p_long_context_sampled(dtype):
+    """Variant 4 on the prefill study's first shape (8 x (4096 + 1024),
+    32/8 heads, D 128, bs 16): 64 sampled (row, head) pairs."""
+    wl = workloads.chunked_prefill(batch=8, ctx_lo=4096, ctx_hi=4096, chunk_lo=1024,
+                                   chunk_hi=1024, dtype=dtype,
+                                   num_blocks=8 * (4096 + 1024) // 16 + 64)
+    errs, _, _ = run_parity(wl, table_width=(4096 + 1024) // 16 + 2, sample=64,
+                            prefill_variant=4)
+    assert len(errs) == 1 and max(errs) <= TOL[dtype], errs
+
+
+def test_prefill_one_fp16_p_edge_shapes():
+    """Variant 4: empty chunks beside 1-3-token ones, and G = 5 with idle rows."""
+    for Hq, Hkv, ctx, lo, hi in ((16, 4, 300, 0, 3), (10, 2, 500, 1, 300)):
+        wl = workloads.chunked_prefill(seed=11, batch=6, ctx_lo=ctx // 2, ctx_hi=ctx,
+                                       chunk_lo=lo, chunk_hi=hi, num_heads=Hq, num_kv_heads=Hkv,
+                                       head_dim=128, dtype="bf16", block_size=16,
+                                       num_blocks=6 * (ctx + 2 * hi) // 16 + 64, chunks=2)
+        errs, _, _ = run_parity(wl, table_width=(ctx + 2 * hi) // 16 + 2, prefill_variant=4)
+        assert len(errs) == 2 and max(errs) <= TOL["bf16"], errs
+
+
+def test_prefill_one_fp16_p_reports_values_beyond_fp16():
+    """A bf16 V value of 1e5 has no fp16 counterpart: variant 4 sets the
+    "range" device error bit (its tile's rows are not finite); variant 2
+    computes the same call within tolerance of the oracle."""
+    from oracle import attn
+    pa = _pa()
+    pa.device_errors()
+    g = torch.Generator().manual_seed(5)
+    Hkv, G, D, bs, L, n = 2, 4, 128, 16, 200, 40
+    nb = (L + bs - 1) // bs
+    kc = torch.randn(nb, Hkv, bs, D, generator=g).to(torch.bfloat16)
+    vc = torch.randn(nb, Hkv, bs, D, generator=g).to(torch.bfloat16)
+    vc[3, 1, 5, 7] = 1e5
+    q = torch.randn(n, Hkv * G, D, generator=g).to(torch.bfloat16)
+    tab = torch.arange(nb, dtype=torch.int32).view(1, nb)
+    sl = torch.tensor([L], dtype=torch.int32)
+    cu = torch.tensor([0, n], dtype=torch.int32)
+    exp = attn.paged_prefill(q, kc, vc, tab.numpy(), sl.numpy(), cu.numpy(), 0.088)
+    out = torch.empty(n, Hkv * G, D, dtype=torch.float32, device="cuda")
+    args = (q.cuda(), kc.cuda(), vc.cuda(), tab.cuda(), sl.cuda(), cu.cuda(), 0.088)
+    pa.pa_prefill(out, *args[:6], args[6], max_q_len=n, variant=4)
+    assert pa.device_errors() == ["range"]
+    got = out.double().cpu().numpy()
+    assert not np.isfinite(got[:, G:, 7]).any()  # KV head 1's rows, that column
+    assert float(np.abs(got[:, :G] - exp[:, :G]).max()) <= 3e-3  # KV head 0: unaffected
+    pa.pa_prefill(out, *args[:6], args[6], max_q_len=n, variant=2)
+    assert pa.device_errors() == []
+    got = out.double().cpu().numpy()
+    assert float(np.abs(got[:, :G] - exp[:, :G]).max()) <= 3e-3
+    # variant 2 carries P to within 2^-14 of each weight: an error bound
+    # proportional to the largest |v|
+    assert float(np.abs(got[:, G:] - exp[:, G:]).max()) <= 2.0 ** -13 * 1e5
+
+
 @pytest.mark.parametrize("pv", [1, 2, 3])
 def test_chunk_covering_the_whole_sequence_and_single_tokens(pv):
     wl = workloads.chunked_prefill(batch=6, ctx_lo=0, ctx_hi=0, chunk_lo=1, chunk_hi=130,

@@ -120,7 +120,7 @@ def test_static_decode_writes_only_out():
     assert not pa.device_errors()
 
 
-@pytest.mark.parametrize("variant", [1, 2, 3])
+@pytest.mark.parametrize("variant", [1, 2, 3, 4])
 @pytest.mark.parametrize("G", [4, 7])
 def test_prefill_writes_only_out(variant, G):
     from paged_kv_cache_347_b200 import pagedattn as pa
@@ -143,7 +143,7 @@ def test_prefill_writes_only_out(variant, G):
     assert not pa.device_errors()
 
 
-@pytest.mark.parametrize("variant", [2, 3])
+@pytest.mark.parametrize("variant", [2, 3, 4])
 def test_prefill_output_16_byte_aligned(variant):
     """The tcgen05 kernels write a row with 32-byte stores when out is
     32-byte aligned and fall back to 16-byte ones when it is only 16-byte
