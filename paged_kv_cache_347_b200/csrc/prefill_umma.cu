@@ -36,10 +36,12 @@
 // in 16j+8..16j+15, two keys per column; Q holds two elements of a row per
 // column.
 //
-// The one-fp16-P form (kP16): each weight is rounded once to fp16, the
-// words of a thread's 64 keys taking the first 32 of its S columns (key
-// block j of the tile at column 64 (j / 4) + 8 (j % 4)), and PV(i) is one
-// MMA per key block with P and V both f16.  Against a bf16 cache a fourth
+// The one-fp16-P form (kP16, one tile per CTA): each weight is rounded once
+// to fp16, and P takes 64 columns of its own, [448, 512) (free with a single
+// Q buffer; key block j at 448 + 8 j, a thread's 64 keys in 32 of them), so
+// S(i+2) waits only until the softmax has read S(i), and the softmax waits
+// for PV(i-1) to have read P(i-1) before it writes P(i).  PV(i) is one MMA
+// per key block with P and V both f16.  Against a bf16 cache a fourth
 // warpgroup (warps 12-15) rewrites each landed V stage in place as fp16
 // (and zeroes the rows past the tile's last key) before the PV thread may
 // read it; a V value beyond the fp16 range turns infinite there, which the
@@ -73,6 +75,9 @@ __host__ __device__ constexpr int threads_for(bool conv) {
 }
 constexpr int kTmemCols = 512;
 constexpr int kColO = 256, kColQ = 384;
+// the one-fp16-P form (one tile per CTA, so one Q buffer): P in columns of
+// its own, [448, 512), key block j at kColP + 8 j
+constexpr int kColP = 448;
 constexpr int kRowBytes = 128;        // one 64-element piece of a 16-bit row
 
 template <int D, int BS, int NK, int NV>
@@ -217,6 +222,9 @@ __global__ void __launch_bounds__(threads_for(kP16 && std::is_same<T, __nv_bfloa
     using C = Cfg<D, BS, NK, NV>;
     // one fp16 P against a bf16 cache: V converted to fp16 in shared memory
     constexpr bool kConv = kP16 && std::is_same<T, __nv_bfloat16>::value;
+    static_assert(!(kP16 && kPersist), "the one-fp16-P form takes one tile per CTA");
+    static_assert(!kP16 || (kColQ + D / 2 <= kColP && kColP + kKeys / 2 <= kTmemCols),
+                  "tensor memory: P columns beside the one Q buffer");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -433,7 +441,9 @@ __global__ void __launch_bounds__(threads_for(kP16 && std::is_same<T, __nv_bfloa
                     for (int i = 0; ok && i < t.nstages; ++i, ++gi) {
                         // S(gi) = Q . K^T into S buffer gi % 2, once PV(gi-2) has read it
                         const int slot = gi % NK;
-                        if (gi >= 2 && !mbar_wait_bounded(pv_done + 8 * (gi & 1),
+                        // (with P in columns of its own, once the softmax has read
+                        // S(gi-2): it arrives on p_full after that)
+                        if (gi >= 2 && !mbar_wait_bounded((kP16 ? p_full : pv_done) + 8 * (gi & 1),
                                                           ((gi >> 1) - 1) & 1, abort_flag)) {
                             ok = false;
                             break;
@@ -475,15 +485,13 @@ __global__ void __launch_bounds__(threads_for(kP16 && std::is_same<T, __nv_bfloa
                         // V rows: 8-row groups 1 KB apart, 64-column pieces 16 KB apart
                         const uint64_t b0 = umma::smem_desc_sw128(v_s + slot * C::kStageBytes,
                                                                   C::kKVPiece, 1024);
-                        const uint32_t pb = tmem + (gi & 1) * kKeys;
+                        [[maybe_unused]] const uint32_t pb = tmem + (gi & 1) * kKeys;
 #pragma unroll
                         for (int j = 0; j < kKeys / 16; ++j) {  // keys 16j..16j+15
                             const uint64_t b = b0 + ((j * 16 * kRowBytes) >> 4);
                             if constexpr (kP16) {
-                                // block j in the columns of the half of the keys it
-                                // belongs to: (j / 4) * 64 + (j % 4) * 8
-                                umma::mma_f16_ts(tmem + kColO, pb + (j >> 2) * 64 + (j & 3) * 8, b,
-                                                 idesc_o, (i > 0 || j > 0) ? 1u : 0u);
+                                umma::mma_f16_ts(tmem + kColO, tmem + kColP + 8 * j, b, idesc_o,
+                                                 (i > 0 || j > 0) ? 1u : 0u);
                             } else {
                                 umma::mma_f16_ts(tmem + kColO, pb + 16 * j, b, idesc_o,
                                                  (i > 0 || j > 0) ? 1u : 0u);
@@ -635,7 +643,13 @@ __global__ void __launch_bounds__(threads_for(kP16 && std::is_same<T, __nv_bfloa
                 umma::st32(hcol + 32 * c, pw);
             }
         }
-        if constexpr (kP16) umma::st32(hcol, p16);
+        if constexpr (kP16) {
+            // P(gi) goes where P(gi-1) was: once PV(gi-1) has read it
+            if (i > 0 && !warp_wait(pv_done + 8 * ((gi - 1) & 1), ((gi - 1) >> 1) & 1, abort_flag))
+                return false;
+            umma::fence_after_sync();
+            umma::st32(lane_base + kColP + half * 32, p16);
+        }
         {
             float a0, a1, b0, b1;
             upk(acc[0], a0, a1);
