@@ -32,6 +32,16 @@ def test_library_exports_every_declared_symbol():
     assert pa.version() >= 10000
 
 
+def test_binding_names_every_device_error_bit():
+    """The binding's names for the device error word cover exactly the bits
+    the header defines."""
+    from paged_kv_cache_347_b200 import pagedattn as pa
+    src = open(os.path.join(ROOT, "include", "pagedattn.h")).read()
+    bits = {int(v, 16): n.lower()
+            for n, v in re.findall(r"#define PA_DEVERR_([A-Z]+)\s+(0x[0-9a-fA-F]+)u", src)}
+    assert bits == pa.DEVERR
+
+
 def test_checks_before_any_device_work():
     from paged_kv_cache_347_b200 import pagedattn as pa
     L = pa._lib
