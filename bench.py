@@ -1119,7 +1119,7 @@ def prefill_rows(ctx: int, chunk: int, batch: int = 8):
 
 
 def study_prefill(args):
-    """Chunked prefill, both kernels: 8 sequences x (4096 context + 1024
+    """Chunked prefill, every kernel: 8 sequences x (4096 context + 1024
     chunk), (0 + 4096), (16384 + 512); 32/8 heads, D 128, bf16, bs 16."""
     from paged_kv_cache_347_b200 import pagedattn as pa
     res = {"study": "prefill", "rows": []}
