@@ -655,7 +655,9 @@ int pa_step_launch(void *stream_in, void *stream_run, void *stream_out,
  * (the copies are asynchronous).  It applies the events (pa_step_plan),
  * chooses the decode (pa_decode_choose, longest first; one-token appends of
  * exactly the decode batch go in with it, pa_append_decode), copies the
- * step's inputs in on one stream, runs its kernels on another (from a CUDA
+ * step's inputs in on one stream (the new rows and the queries first: they
+ * need nothing from the plan, so the host link carries them while the host
+ * plans; then the step's arrays), runs its kernels on another (from a CUDA
  * graph of the step's layout once that layout has run once; steps with
  * copy-on-write copies run directly) and copies the output out on a third.
  * It returns at once; *ready (if non-NULL) receives a cudaEvent_t that
@@ -666,7 +668,9 @@ int pa_step_launch(void *stream_in, void *stream_run, void *stream_out,
  * until *ready completes.
  *   - Limits: num_seqs <= max_batch, new tokens <= max_new_tokens, table rows
  *     of table_width entries; beyond them PA_ERR_INVALID_ARG before anything
- *     is applied.  Errors of pa_step_plan are returned as it returns them.
+ *     is applied.  Errors of pa_step_plan are returned as it returns them; a
+ *     call that fails after its input copies were enqueued waits for them
+ *     before it returns, so the caller may reuse its buffers at once.
  *   - A CUDA error part-way leaves the runtime's allocator ahead of its
  *     device work: destroy the runtime.
  * pa_rt_wait synchronises the runtime's streams; pa_event_wait waits for an

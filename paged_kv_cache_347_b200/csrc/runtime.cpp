@@ -6,14 +6,16 @@
 // This one owns the allocator, two staging slots (page-locked host memory
 // and a device buffer each), the split workspace, two device output buffers,
 // three streams and a cache of CUDA graphs.  A step:
-//   1. pa_step_plan applies the step's events and writes slots, copy pairs,
+//   1. on the copy-in stream: the new K/V rows and the queries go to fixed
+//      places of the slot's device buffer (they need nothing from the plan,
+//      so the host link carries them while the host plans);
+//   2. pa_step_plan applies the step's events and writes slots, copy pairs,
 //      table rows, lengths and the longest-first order into the slot's host
 //      buffer;
-//   2. pa_decode_choose picks the decode's kernel and split from the lengths;
+//   3. pa_decode_choose picks the decode's kernel and split from the lengths;
 //      a run of one-token appends of exactly the decode batch, right before
-//      the decode, goes in with it (pa_append_decode);
-//   3. on the copy-in stream: the arrays, the new K/V rows and the queries go
-//      to fixed places of the slot's device buffer;
+//      the decode, goes in with it (pa_append_decode); the arrays follow the
+//      rows on the copy-in stream;
 //   4. on the run stream: the step's kernels, replayed from a CUDA graph
 //      captured for its layout (steps with copy-on-write copies, or a layout
 //      seen for the first time, launch directly; a new layout is captured
@@ -273,14 +275,36 @@ int pa_rt_step(pa_runtime *rt, const int64_t *events, int n_events, const int64_
     const int s = rt->next;
     rt->next ^= 1;
     cudaError_t e;
+    // The new K/V rows and the queries go in first: they come from the
+    // caller's buffers to fixed places of the slot's device buffer and need
+    // nothing from the plan, so the host link starts on them while the host
+    // plans.  The slot's device buffer is rewritten once its previous
+    // kernels are done with it.
+    const size_t row = (size_t)c.num_kv_heads * c.head_dim * rt->elem;
+    const size_t qb = (size_t)num_seqs * c.num_heads * c.head_dim * rt->elem;
+    if ((rt->used[s] && (e = cudaStreamWaitEvent(rt->s_in, rt->ev_run[s], 0)) != cudaSuccess) ||
+        (n_slots > 0 &&
+         ((e = cudaMemcpyAsync(rt->devb[s] + rt->off_k, k_new, n_slots * row,
+                               cudaMemcpyHostToDevice, rt->s_in)) != cudaSuccess ||
+          (e = cudaMemcpyAsync(rt->devb[s] + rt->off_v, v_new, n_slots * row,
+                               cudaMemcpyHostToDevice, rt->s_in)) != cudaSuccess)) ||
+        (qb > 0 && (e = cudaMemcpyAsync(rt->devb[s] + rt->off_q, q, qb, cudaMemcpyHostToDevice,
+                                        rt->s_in)) != cudaSuccess))
+        return cuda_err(e, "copy in");
+    // (from here on, a failing call first lets those copies finish, so that
+    // the caller may reuse its buffers once the call has returned)
+    auto fail_after_copies = [&](int code) {
+        cudaStreamSynchronize(rt->s_in);
+        return code;
+    };
     // the slot's host buffer is free once its previous copy in has run
     if (rt->used[s] && (e = cudaEventSynchronize(rt->ev_in[s])) != cudaSuccess)
-        return cuda_err(e, "waiting for the staging buffer");
+        return fail_after_copies(cuda_err(e, "waiting for the staging buffer"));
     rt->pairs_before.resize((size_t)n_events + 1);
     pa_step_layout lay;
     int rc = pa_step_plan(rt->alloc, events, n_events, decode_ids, num_seqs, c.table_width,
                           rt->host[s], rt->arrays_cap, rt->pairs_before.data(), &lay);
-    if (rc != PA_OK) return rc;
+    if (rc != PA_OK) return fail_after_copies(rc);
     // device actions in event order
     rt->acts.clear();
     int decode_at = -1;
@@ -320,31 +344,20 @@ int pa_rt_step(pa_runtime *rt, const int64_t *events, int n_events, const int64_
         const int32_t *lens = reinterpret_cast<const int32_t *>(rt->host[s] + lay.off_lens);
         rc = pa_decode_choose(lens, num_seqs, c.num_kv_heads, c.head_dim, c.block_size, c.dtype,
                               0, &opts);
-        if (rc != PA_OK) return rc;
+        if (rc != PA_OK) return fail_after_copies(rc);
         // a power-of-two bound on the lengths (at least 512, at most the
         // table's capacity) keeps a graph's grid fixed while steps change little
         max_len = 512;
         while (max_len < lay.max_seq_len) max_len *= 2;
         max_len = std::min(max_len, c.table_width * c.block_size);
     }
-    // copies in: the slot's device buffer is rewritten once its previous
-    // kernels are done with it
-    const size_t row = (size_t)c.num_kv_heads * c.head_dim * rt->elem;
-    const size_t qb = (size_t)num_seqs * c.num_heads * c.head_dim * rt->elem;
-    if (rt->used[s] && (e = cudaStreamWaitEvent(rt->s_in, rt->ev_run[s], 0)) != cudaSuccess)
-        return cuda_err(e, "ordering the copy in");
+    // the step's arrays (slots, pairs, table rows, lengths, order) follow
+    // the rows on the copy-in stream; the kernels wait for all of it
     if ((e = cudaMemcpyAsync(rt->devb[s], rt->host[s], lay.bytes, cudaMemcpyHostToDevice,
                              rt->s_in)) != cudaSuccess ||
-        (n_slots > 0 &&
-         ((e = cudaMemcpyAsync(rt->devb[s] + rt->off_k, k_new, n_slots * row,
-                               cudaMemcpyHostToDevice, rt->s_in)) != cudaSuccess ||
-          (e = cudaMemcpyAsync(rt->devb[s] + rt->off_v, v_new, n_slots * row,
-                               cudaMemcpyHostToDevice, rt->s_in)) != cudaSuccess)) ||
-        (qb > 0 && (e = cudaMemcpyAsync(rt->devb[s] + rt->off_q, q, qb, cudaMemcpyHostToDevice,
-                                        rt->s_in)) != cudaSuccess) ||
         (e = cudaEventRecord(rt->ev_in[s], rt->s_in)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(rt->s_run, rt->ev_in[s], 0)) != cudaSuccess)
-        return cuda_err(e, "copy in");
+        return fail_after_copies(cuda_err(e, "copy in"));
     // the slot's output buffer is rewritten once its previous copy out is done
     if (rt->used[s] && (e = cudaStreamWaitEvent(rt->s_run, rt->ev_out[s], 0)) != cudaSuccess)
         return cuda_err(e, "ordering the output");
