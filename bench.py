@@ -588,6 +588,14 @@ def run_ours(args, ws, rank, local):
                 "note": "opt-in: each weight rounded once to fp16 (within 2^-11, against "
                         "2^-14 for the default's high part + remainder), half the P.V "
                         "products; the bf16 V stages converted to fp16 in shared memory"}}
+        # the same workload with an f16 cache, where the one-fp16-P form needs
+        # no conversion of V
+        t2, t4 = prefill_rows(4096, 1024, dtype="f16",
+                              variants=((2, "tcgen05"), (4, "tcgen05, one fp16 P")))
+        res["prefill"]["f16_cache"] = {
+            "tcgen05_ms": t2["ms"], "one_fp16_p_ms": t4["ms"], "one_fp16_p_tflops": t4["tflops"],
+            "one_fp16_p_frac": t4["frac_of_bf16_peak"],
+            "max_abs_diff_one_fp16_p_vs_tcgen05": t4["max_abs_diff_vs_tcgen05"]}
     if rank == 0 and ws == 1 and not args.no_cpu:
         smp = OracleSampler(args.workload, seed)
         nb, secs, pairs = smp.run(args.cpu_budget)
@@ -1075,7 +1083,9 @@ def _bf16_peak_tflops():
         return 1590.0, "fallback 1.59 PFLOP/s"
 
 
-def prefill_rows(ctx: int, chunk: int, batch: int = 8):
+def prefill_rows(ctx: int, chunk: int, batch: int = 8, dtype: str = "bf16",
+                 variants=((1, "mma.sync"), (2, "tcgen05"), (3, "tcgen05 persistent"),
+                           (4, "tcgen05, one fp16 P"))):
     """The prefill kernels (mma.sync, tcgen05, tcgen05 persistent, tcgen05 with
     one fp16 P) on one chunked-prefill workload (32/8 heads, D 128, bf16, bs 16): CUDA-event ms
     over 20 launches each, the definition's FLOPs (4 * D * Hq per (row,
@@ -1083,7 +1093,8 @@ def prefill_rows(ctx: int, chunk: int, batch: int = 8):
     from paged_kv_cache_347_b200 import pagedattn as pa
     from paged_kv_cache_347_b200.runner import PagedKVRunner
     wl = workloads.chunked_prefill(batch=batch, ctx_lo=ctx, ctx_hi=ctx, chunk_lo=chunk,
-                                   chunk_hi=chunk, num_blocks=batch * (ctx + chunk) // 16 + 64)
+                                   chunk_hi=chunk, dtype=dtype,
+                                   num_blocks=batch * (ctx + chunk) // 16 + 64)
     steps = list(wl.steps)
     r = PagedKVRunner.for_shape(wl.shape, (ctx + chunk) // 16 + 2)
     r.run(steps[0])
@@ -1097,21 +1108,22 @@ def prefill_rows(ctx: int, chunk: int, batch: int = 8):
     flops = 4.0 * 128 * 32 * sum(ctx + i + 1 for i in range(chunk)) * batch
     peak, _ = _bf16_peak_tflops()
     rows = []
-    for variant, kernel in ((1, "mma.sync"), (2, "tcgen05"), (3, "tcgen05 persistent"),
-                            (4, "tcgen05, one fp16 P")):
+    first = None
+    for variant, kernel in variants:
         ms = _events_ms(lambda: pa.pa_prefill(o, dev[2], r.k_cache, r.v_cache, a.dev["tables"],
                                               a.dev["lens"], a.dev["cu"], r.scale,
                                               max_q_len=a.max_q, max_seq_len=a.max_len,
                                               variant=variant), reps=20)
         tf = flops / (ms * 1e-3) / 1e12
         row = {"kernel": kernel, "context": ctx, "chunk": chunk, "batch": batch,
-               "ms": round(ms, 3), "tflops": round(tf, 1),
+               "dtype": dtype, "ms": round(ms, 3), "tflops": round(tf, 1),
                "frac_of_bf16_peak": round(tf / peak, 4), "peak_tflops": peak,
                "flops_per_launch": flops}
-        if variant == 1:
-            first = o.clone()
+        if first is None:
+            first, first_kernel = o.clone(), kernel
         else:  # the kernels compute the same rows at full size
-            row["max_abs_diff_vs_mma_sync"] = float((o - first).abs().max())
+            row[f"max_abs_diff_vs_{first_kernel.replace('.', '_').replace(' ', '_')}"] = \
+                float((o - first).abs().max())
         rows.append(row)
     del r
     torch.cuda.empty_cache()
