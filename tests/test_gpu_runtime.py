@@ -103,3 +103,37 @@ def test_limits_are_refused_before_anything_is_applied(pa):
         rt.step(ev, np.array([0, 1, 2], np.int64), None, None,
                 torch.zeros(3, 2, 64).pin_memory(), torch.zeros(3, 2, 64).pin_memory())
     assert rt.alloc.free_list() == before
+
+
+def test_a_step_failing_in_its_plan_leaves_the_runtime_usable(pa):
+    """A step whose appends need more blocks than are free fails in the
+    allocator after its new rows were already on their way in: the call
+    returns PA_ERR_OUT_OF_BLOCKS once those copies are done, the allocator is
+    as before, and the next step decodes over exactly the rows appended by
+    the steps that succeeded (checked against softmax(q K^T * scale) V in
+    float64)."""
+    NB, bs, D, Hq = 16, 4, 64, 2
+    kc = torch.zeros((NB, 1, bs, D), device="cuda")
+    vc = torch.zeros_like(kc)
+    scale = 0.125
+    rt = pa.Runtime(kc, vc, Hq, 4, 2, 128, scale)
+    g = torch.Generator().manual_seed(3)
+    rows = lambda n: torch.randn(n, 1, D, generator=g).pin_memory()
+    k1, v1 = rows(8), rows(8)
+    ev = np.array([[pa.EV_ADD, 1, 0], [pa.EV_APPEND, 1, 8]], np.int64)
+    rt.wait_event(rt.step(ev, np.empty(0, np.int64), k1, v1, None, None))
+    before = rt.alloc.free_list()
+    ev = np.array([[pa.EV_APPEND, 1, 100]], np.int64)                    # 25 blocks, 14 free
+    with pytest.raises(pa.PagedAttnError) as err:
+        rt.step(ev, np.empty(0, np.int64), rows(100), rows(100), None, None)
+    assert err.value.code == -3                                          # PA_ERR_OUT_OF_BLOCKS
+    assert rt.alloc.free_list() == before
+    k2, v2, q = rows(1), rows(1), torch.randn(1, Hq, D, generator=g).pin_memory()
+    out = torch.empty(1, Hq, D).pin_memory()
+    ev = np.array([[pa.EV_APPEND, 1, 1], [pa.EV_DECODE, 0, 0]], np.int64)
+    rt.wait_event(rt.step(ev, np.array([1], np.int64), k2, v2, q, out))
+    rt.wait()
+    K = torch.cat([k1, k2])[:, 0].double()
+    V = torch.cat([v1, v2])[:, 0].double()
+    w = torch.softmax(q[0].double() @ K.T * scale, dim=-1)
+    assert float((out[0].double() - w @ V).abs().max()) <= TOL["f32"]
