@@ -614,8 +614,8 @@ __global__ void __launch_bounds__(threads_for(kP16 && std::is_same<T, __nv_bfloa
         // takes key block q / 16 of the chunk, high parts in its first 8
         // columns, remainders in the next 8 (over the chunk's own S columns)
         uint64_t acc[2] = {pk(0.f, 0.f), pk(0.f, 0.f)};
-        // (the one-fp16 form: the pair's word goes to column 16c + e of the
-        // thread's own S columns, so that its 64 keys take the first 32)
+        // (the one-fp16 form: the pair's word is word 16c + e of the thread's
+        // 32 P columns, kColP + 32 half: key block j of the tile at kColP + 8 j)
         [[maybe_unused]] uint32_t p16[32];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
